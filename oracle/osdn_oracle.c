@@ -1,0 +1,167 @@
+/*
+ * OSDN oracle: a plain, slow, token-by-token CPU recurrence in float64.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product path (the CUDA library and
+ * its Python binding) links, imports or calls this file. Only the tests, the
+ * smoke check and the benchmark's CPU-baseline leg use it. It shares no code,
+ * header, table or helper with the CUDA kernels.
+ *
+ * What it computes (page "OSDN: Improving Delta Rule with Provable Online
+ * Preconditioning in Linear Attention", gist.science technical summary):
+ *
+ *   Section 1 (problem statement): per-token regression loss
+ *       f_t(S) = 1/2 || S k_t - v_t ||^2,   S in R^{dv x dk}.
+ *   Section 2.1 (algebraic equivalence): right-preconditioned step
+ *       S_t = S_{t-1} - beta_t grad f_t(S_{t-1}) D_t,  D_t = diag(d_t),
+ *   which equals the write-side scaled key form
+ *       S_t = S_{t-1} + beta_t (v_t - S_{t-1} k_t) (d_t (.) k_t)^T.
+ *   The read/erase key stays k_t; only the write key is scaled.
+ *   Output o_t = S_t q_t (read after the write, no 1/sqrt(dk) scale).
+ *   Section 2.2 (decoupled hypergradient): closed form
+ *       h_t(d) = ((1 - beta_t <d, k_t^2>)^2 - 1) / (2 ||k_t||^2),
+ *   gradient  grad_d h_t(d) = -beta_t (1 - beta_t <d, k_t^2>) k_t^2 / ||k_t||^2.
+ *   Section 2.3 (APF): d_{t+1} = r_t d_t - eta grad_d h_t(d_t)
+ *       = r_t d_t + eta beta_t (1 - beta_t <d_t, k_t^2>) k_t^2 / ||k_t||^2.
+ *
+ * Readings fixed here (the pages leave them open):
+ *   - online gradient DESCENT on h (the page writes "+ eta grad h"; descent is
+ *     what "OGD on h" means and what drives beta <d, k^2> toward the gated
+ *     Newton condition beta <d*, k^2> = 1 of Theorem 5.2);
+ *   - no projection step after the APF update (the recurrence stays affine);
+ *   - play-then-update: token t writes with d_t, and d_1 = d0;
+ *   - r_t is an input per (token, head); r == NULL means APF off (r == 1);
+ *   - ||k_t||^2 == 0 skips the gradient term (h is undefined there).
+ */
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int B, T, H, dk, dv;
+    double eta;
+    const double *q, *k, *v, *beta, *r, *d0, *S0;
+    double *out, *S_final, *d_final;
+    int unit_begin, unit_end;
+} oracle_job;
+
+/* One token of the recurrence for one (sequence, head). S is dv x dk
+ * row-major, d has dk entries; both are updated in place. o receives dv
+ * values. e and a are scratch of dv and dk entries. */
+static void oracle_token(int dk, int dv, double eta, double *S, double *d,
+                         const double *q, const double *k, const double *v,
+                         double beta, double r, double *o, double *e, double *a)
+{
+    double n = 0.0, s = 0.0;
+    for (int i = 0; i < dk; ++i) {
+        a[i] = k[i] * k[i];           /* k_t^2, elementwise */
+        n += a[i];                    /* ||k_t||^2 */
+        s += d[i] * a[i];             /* <d_t, k_t^2> with the pre-update d */
+    }
+    /* residual e = S_{t-1} k_t - v_t (gradient of f_t is e k_t^T) */
+    for (int row = 0; row < dv; ++row) {
+        double acc = 0.0;
+        const double *Srow = S + (size_t)row * dk;
+        for (int i = 0; i < dk; ++i) acc += Srow[i] * k[i];
+        e[row] = acc - v[row];
+    }
+    /* S_t = S_{t-1} - beta e (d (.) k)^T */
+    for (int row = 0; row < dv; ++row) {
+        double *Srow = S + (size_t)row * dk;
+        double be = beta * e[row];
+        for (int i = 0; i < dk; ++i) Srow[i] -= be * (d[i] * k[i]);
+    }
+    /* o_t = S_t q_t */
+    for (int row = 0; row < dv; ++row) {
+        double acc = 0.0;
+        const double *Srow = S + (size_t)row * dk;
+        for (int i = 0; i < dk; ++i) acc += Srow[i] * q[i];
+        o[row] = acc;
+    }
+    /* d_{t+1} = r d_t + eta beta (1 - beta s) k^2 / ||k||^2 */
+    double x = 0.0;
+    if (n > 0.0) x = eta * beta * (1.0 - beta * s) / n;
+    for (int i = 0; i < dk; ++i) d[i] = r * d[i] + x * a[i];
+}
+
+static void *oracle_worker(void *arg)
+{
+    oracle_job *J = (oracle_job *)arg;
+    const int dk = J->dk, dv = J->dv, T = J->T, H = J->H;
+    double *S = (double *)malloc(sizeof(double) * (size_t)dv * dk);
+    double *d = (double *)malloc(sizeof(double) * (size_t)dk);
+    double *e = (double *)malloc(sizeof(double) * (size_t)dv);
+    double *a = (double *)malloc(sizeof(double) * (size_t)dk);
+    for (int u = J->unit_begin; u < J->unit_end; ++u) {
+        const int b = u / H, h = u % H;
+        if (J->S0) memcpy(S, J->S0 + (size_t)u * dv * dk, sizeof(double) * (size_t)dv * dk);
+        else memset(S, 0, sizeof(double) * (size_t)dv * dk);
+        if (J->d0) memcpy(d, J->d0 + (size_t)u * dk, sizeof(double) * (size_t)dk);
+        else for (int i = 0; i < dk; ++i) d[i] = 1.0;
+        for (int t = 0; t < T; ++t) {
+            const size_t tok = ((size_t)b * T + t) * H + h;  /* [B, T, H] */
+            oracle_token(dk, dv, J->eta, S, d,
+                         J->q + tok * dk, J->k + tok * dk, J->v + tok * dv,
+                         J->beta[tok], J->r ? J->r[tok] : 1.0,
+                         J->out + tok * dv, e, a);
+        }
+        if (J->S_final) memcpy(J->S_final + (size_t)u * dv * dk, S, sizeof(double) * (size_t)dv * dk);
+        if (J->d_final) memcpy(J->d_final + (size_t)u * dk, d, sizeof(double) * (size_t)dk);
+    }
+    free(S); free(d); free(e); free(a);
+    return NULL;
+}
+
+/* Forward over a whole sequence batch.
+ * q, k: [B, T, H, dk]; v, out: [B, T, H, dv]; beta, r: [B, T, H] (r may be NULL);
+ * d0: [B, H, dk] (NULL = ones); S0: [B, H, dv, dk] (NULL = zeros);
+ * S_final: [B, H, dv, dk], d_final: [B, H, dk] (either may be NULL).
+ * The (b, h) units are independent; nthreads host threads share them.
+ * Returns 0, or -1 on bad sizes. */
+int osdn_oracle_fwd(int B, int T, int H, int dk, int dv, double eta,
+                    const double *q, const double *k, const double *v,
+                    const double *beta, const double *r,
+                    const double *d0, const double *S0,
+                    double *out, double *S_final, double *d_final,
+                    int nthreads)
+{
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    const int units = B * H;
+    if (units == 0) return 0;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > units) nthreads = units;
+    oracle_job *jobs = (oracle_job *)calloc((size_t)nthreads, sizeof(oracle_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int w = 0; w < nthreads; ++w) {
+        oracle_job J = {B, T, H, dk, dv, eta, q, k, v, beta, r, d0, S0,
+                        out, S_final, d_final,
+                        (int)((long long)units * w / nthreads),
+                        (int)((long long)units * (w + 1) / nthreads)};
+        jobs[w] = J;
+    }
+    for (int w = 1; w < nthreads; ++w) pthread_create(&th[w], NULL, oracle_worker, &jobs[w]);
+    oracle_worker(&jobs[0]);
+    for (int w = 1; w < nthreads; ++w) pthread_join(th[w], NULL);
+    free(jobs); free(th);
+    return 0;
+}
+
+/* One decode token for every (b, h): q, k [B, H, dk]; v, out [B, H, dv];
+ * beta, r [B, H] (r may be NULL); S [B, H, dv, dk] and d [B, H, dk] updated
+ * in place. Same arithmetic as one step of osdn_oracle_fwd. */
+int osdn_oracle_step(int B, int H, int dk, int dv, double eta,
+                     const double *q, const double *k, const double *v,
+                     const double *beta, const double *r,
+                     double *S, double *d, double *out)
+{
+    if (B < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    double *e = (double *)malloc(sizeof(double) * (size_t)dv);
+    double *a = (double *)malloc(sizeof(double) * (size_t)dk);
+    for (int u = 0; u < B * H; ++u) {
+        oracle_token(dk, dv, eta, S + (size_t)u * dv * dk, d + (size_t)u * dk,
+                     q + (size_t)u * dk, k + (size_t)u * dk, v + (size_t)u * dv,
+                     beta[u], r ? r[u] : 1.0, out + (size_t)u * dv, e, a);
+    }
+    free(e); free(a);
+    return 0;
+}
