@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Throughput of the OSDN chunkwise forward on B200: tokens/s, TFLOP/s and the
+fraction of the HBM / bf16 roofline.
+
+One step = one osdn_fwd over the whole workload (phase 1 preconditioner scan +
+phase 2 chunked delta rule) with inputs resident in HBM. Default workload: the
+1.3B-shaped layer (B=8, H=16, T=4096, dk=dv=128, C=64, bf16, APF on, shifted key
+statistics). Inputs (q, k, v: 403 MB) are larger than the 126 MB L2, so no
+flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own full workload (independent sequences;
+no collective on the data path), so scaling is weak; the step time is the max
+over ranks. ``--impl reference`` times the float64 CPU oracle on a bounded
+sample of the same workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from preconditioned_delta_rule_token_b200 import workloads as W  # noqa: E402
+
+FLOPS_PER_TOKEN_HEAD = None   # set from the workload (6 dk dv + C (3 dk + 2 dv))
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {"340m": W.LAYER_340M, "1p3b": W.LAYER_1P3B, "long": W.LONG_RECALL}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="1p3b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops_per_token_head(w):
+    return 6 * w.dk * w.dv + w.chunk * (3 * w.dk + 2 * w.dv)
+
+
+def elem(w):
+    return 2 if w.dtype == W.BF16 else 4
+
+
+def path_bytes(w, with_S0=False, with_d0=False):
+    """Algorithmic bytes of the whole forward: read q, k, v, beta (+ r), write out;
+    per (b, h) write final S and d (read S0, d0 when given)."""
+    e = elem(w)
+    per_tok = (2 * w.dk + 2 * w.dv) * e + e + (e if w.apf else 0)
+    per_unit = 4 * (w.dv * w.dk + w.dk) + (4 * w.dv * w.dk if with_S0 else 0) + (4 * w.dk if with_d0 else 0)
+    return w.B * w.T * w.H * per_tok + w.B * w.H * per_unit
+
+
+def scan_bytes(w):
+    """Phase 1: read k, beta (+ r), write the scaled keys; write final d (d0 read: ones here)."""
+    e = elem(w)
+    return w.B * w.T * w.H * (2 * w.dk * e + e + (e if w.apf else 0)) + w.B * w.H * 4 * w.dk
+
+
+def chunk_bytes(w):
+    """Phase 2: read q, k, scaled keys, v, beta, write out; write final S."""
+    e = elem(w)
+    return w.B * w.T * w.H * ((3 * w.dk + 2 * w.dv) * e + e) + w.B * w.H * 4 * w.dv * w.dk
+
+
+def source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {
+    "chunk": ["preconditioned_delta_rule_token_b200/csrc/chunk_ffma.cuh",
+              "preconditioned_delta_rule_token_b200/csrc/common.cuh"],
+    "scan": ["preconditioned_delta_rule_token_b200/csrc/scan_seq.cuh",
+             "preconditioned_delta_rule_token_b200/csrc/common.cuh"],
+}
+
+
+def ncu_traffic(kernel, workload_name):
+    """DRAM bytes per launch from a committed ncu capture (profiles/traffic.txt),
+    only if the kernel source is unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = source_sha(KERNEL_SOURCES[kernel])
+    with open(path) as fh:
+        for line in fh:
+            parts = line.split("\t")
+            if len(parts) >= 4 and not line.startswith("#"):
+                if parts[0] == kernel and parts[1] == sha and parts[2] == workload_name:
+                    return float(parts[3])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken during the timed region."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device, enabled=True):
+        self.proc = None
+        self.samples = []
+        if not enabled:
+            return
+        sel = []
+        try:
+            uuid = torch.cuda.get_device_properties(device).uuid
+            sel = ["-i", "GPU-" + str(uuid)]
+        except Exception:
+            sel = []
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "100"] + sel, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                self.samples.append(dict(sm=float(f[2]), smax=float(f[3]), power=float(f[4]),
+                                         hw=f[6], hwt=f[7], swt=f[8], pcap=f[9]))
+            except ValueError:
+                continue
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = set()
+        for s in self.samples:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if s[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s["sm"] for s in self.samples),
+                "sm_max_mhz": max(s["smax"] for s in self.samples), "reasons": sorted(reasons),
+                "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, seconds=12.0, max_units=None):
+    """Time the float64 oracle on a bounded sample of workload w: the first n
+    (b, h) units over the full sequence, n sized from a short calibration run
+    so the sample takes about `seconds`. Returns (tokens/s, description, cores)."""
+    import oracle
+    cores = cpu_cores()
+    inp = W.make_forward_inputs(w)
+    f = W.to_f64
+    units = [(b, h) for b in range(w.B) for h in range(w.H)]
+
+    def run(n, T):
+        sel = units[:n]
+        q = f(inp["q"])[:, :T]
+        k = f(inp["k"])[:, :T]
+        v = f(inp["v"])[:, :T]
+        be = f(inp["beta"])[:, :T]
+        r = None if inp["r"] is None else f(inp["r"])[:, :T]
+        # gather the sampled units as B = n sequences of one head
+
+        def pick4(x):
+            return None if x is None else np.ascontiguousarray(np.stack([x[b, :, h] for (b, h) in sel])[:, :, None])
+        t0 = time.perf_counter()
+        oracle.fwd(pick4(q), pick4(k), pick4(v), pick4(be), pick4(r), None, None, eta=w.eta, nthreads=cores)
+        return time.perf_counter() - t0
+
+    Tc = min(w.T, 256)
+    nc = min(len(units), cores)
+    tcal = run(nc, Tc)
+    per_unit_token = tcal * min(nc, cores) / (nc * Tc)         # core-seconds per unit-token
+    n = int(seconds * cores / (per_unit_token * w.T))
+    n = max(1, min(len(units) if max_units is None else max_units, n))
+    el = run(n, w.T)
+    tokens = n * w.T / w.H                                       # layer tokens (all H heads) equivalent
+    desc = "%d of %d (b,h) units x full T=%d (%.1f s); tokens counted as units*T/H" % (n, len(units), w.T, el)
+    return tokens / el, desc, cores
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    cores = cpu_cores()
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    times, toks = [], []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        tps, desc, cores = oracle_sample(w, seconds=budget)
+        if i >= args.warmup:
+            toks.append(tps)
+    value = statistics.median(toks)
+    line = {"impl": "reference", "metric": "OSDN chunkwise fwd tokens/s", "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, world):
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
+            "apf": w.apf, "eta": w.eta, "structure": w.structure, "global_batch": w.B * world, "seq_len": w.T,
+            "parallelism": "dp%d (independent sequences per rank)" % world,
+            "l2": "inputs larger than L2 (q,k,v %.0f MB > 126 MB); no flush" % (
+                w.B * w.T * w.H * (2 * w.dk + w.dv) * elem(w) / 1e6)}
+
+
+def run_ours(args, world, rank, local):
+    import preconditioned_delta_rule_token_b200 as pk
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    if rank:
+        import dataclasses
+        w = dataclasses.replace(w, seed=w.seed + 1000 * rank)
+    inp = W.make_forward_inputs(w)
+    g = {k: None if v is None else v.to(dev) for k, v in inp.items()}
+    g["d0"] = None            # d0 = ones (the library's default), as in the workload
+    p = pk.make_params(w.B, w.T, w.H, w.dk, w.dv, g["k"].dtype, w.eta, w.chunk)
+    out = torch.empty((w.B, w.T, w.H, w.dv), dtype=g["k"].dtype, device=dev)
+    Sf = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+    df = torch.empty((w.B, w.H, w.dk), dtype=torch.float32, device=dev)
+    ws = torch.empty(pk.osdn_fwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        pk.osdn_fwd_scan(p, g["k"], g["beta"], g["r"], None, df, ws, stream)
+        if ev is not None:
+            ev.record(stream)
+        pk.osdn_fwd_chunk(p, g["q"], g["k"], g["v"], g["beta"], None, out, Sf, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev, enabled=not args.no_clocks)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step(ev[i][1])
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    clocks.stop()
+    assert pk.osdn_sync_status(stream) == 0
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    scan_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    chunk_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    ms = total_ms / args.steps
+    if world > 1:
+        t = torch.tensor([ms, scan_ms, chunk_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, scan_ms, chunk_ms = t.tolist()
+
+    # end-to-end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {k: None if v is None else v.pin_memory() for k, v in inp.items() if k in ("q", "k", "v", "beta", "r")}
+        dbuf = {k: None if v is None else torch.empty_like(v, device=dev) for k, v in host.items()}
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_S = torch.empty(Sf.shape, dtype=Sf.dtype).pin_memory()
+        h_d = torch.empty(df.shape, dtype=df.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+        d2h = sum(t.numel() * t.element_size() for t in (h_out, h_S, h_d))
+
+        def e2e_step():
+            for k_, v_ in host.items():
+                if v_ is not None:
+                    dbuf[k_].copy_(v_, non_blocking=True)
+            pk.osdn_fwd(p, dbuf["q"], dbuf["k"], dbuf["v"], dbuf["beta"], dbuf["r"], None, None, out, Sf, df, ws,
+                        stream)
+            h_out.copy_(out, non_blocking=True)
+            h_S.copy_(Sf, non_blocking=True)
+            h_d.copy_(df, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = t.item()
+        e2e = {"value": world * w.B * w.T / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tf_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    F = flops_per_token_head(w) * w.B * w.T * w.H
+    t_roof = max(F / (tf_peak * 1e12), path_bytes(w) / (hbm * 1e9))
+    kernels = {
+        "chunk": dict(ms=chunk_ms, bytes=chunk_bytes(w), name="osdn chunk kernel (phase 2)"),
+        "scan": dict(ms=scan_ms, bytes=scan_bytes(w), name="osdn scan kernel (phase 1)"),
+    }
+    dom = max(kernels, key=lambda k_: kernels[k_]["ms"])
+    kd = kernels[dom]
+    achieved = kd["bytes"] / (kd["ms"] / 1e3) / 1e9
+    traffic = ncu_traffic(dom, args.workload)
+    line = {
+        "metric": "OSDN chunkwise fwd tokens/s", "value": world * w.B * w.T / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == W.BF16
+        else "f32", "data": "synthetic", "config": config_of(w, world),
+        "tflops": world * F / (ms / 1e3) / 1e12,
+        "path_roofline": {"t_roofline_us": t_roof * 1e6, "frac": t_roof / (ms / 1e3), "bound": "hbm" if
+                          path_bytes(w) / (hbm * 1e9) >= F / (tf_peak * 1e12) else "tensor",
+                          "bytes": path_bytes(w), "flops": F, "peak_kind": peak_kind},
+        "roofline": {"kernel": kd["name"], "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic, "algorithmic_bytes": kd["bytes"],
+                     "launch_ms": kd["ms"], "peak_kind": peak_kind + " hbm_gbs"},
+        "kernels_ms": {k_: v_["ms"] for k_, v_ in kernels.items()},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": t_wall,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        v_, desc, cores = oracle_sample(w, seconds=12.0)
+        line["cpu_baseline"] = {"value": v_, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,148 @@
+/*
+ * osdn.h - C ABI of libosdn.so: the Online Scaled DeltaNet (OSDN) forward and
+ * single-token decode on NVIDIA B200 (sm_100a).
+ *
+ * Method: "OSDN: Improving Delta Rule with Provable Online Preconditioning in
+ * Linear Attention" (gist.science technical summary).
+ *   section 2.1: S_t = S_{t-1} + beta_t (v_t - S_{t-1} k_t) (d_t (.) k_t)^T,
+ *                o_t = S_t q_t, S in R^{dv x dk}; the read/erase key is k_t,
+ *                the write key is the scaled key d_t (.) k_t;
+ *   section 2.2: the preconditioner step uses only k_t and beta_t;
+ *   section 2.3: d_{t+1} = r_t d_t + eta beta_t (1 - beta_t <d_t, k_t^2>)
+ *                k_t^2 / ||k_t||^2   (APF; r == 1 when APF is off).
+ * Readings of points the pages leave open: the preconditioner step is a
+ * descent step on the hypergradient surrogate; no projection follows it;
+ * token t writes with d_t (d_1 = d0); ||k_t|| = 0 skips the step; no
+ * normalisation or 1/sqrt(dk) scale is applied to q or k inside the op.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *     never allocates device memory and never frees anything.
+ *   - Layouts are dense row-major (last dimension contiguous):
+ *       q, k   [B, T, H, dk]     v, out [B, T, H, dv]
+ *       beta, r [B, T, H]
+ *       d (d0, final_d) [B, H, dk] fp32     S (S0, final_S) [B, H, dv, dk] fp32
+ *     For osdn_step, T is absent: q, k [B, H, dk]; v, out [B, H, dv];
+ *     beta, r [B, H].
+ *   - q, k, v, beta, r and out share one element type (osdn_params.dtype);
+ *     S and d are always fp32. Every pointer must be 16-byte aligned.
+ *   - Work is enqueued on the caller's CUDA stream (cudaStream_t passed as
+ *     void*, NULL = legacy default stream) and returns without a host sync.
+ *   - Return value: OSDN_OK or an OSDN_ERR_* code; nothing aborts. A
+ *     human-readable message for the calling thread's last error is available
+ *     from osdn_get_last_error().
+ *   - Supported sizes: dk, dv in {64, 128}; chunk = 64; B, H >= 1; T >= 0
+ *     (T = 0 copies the initial state to the final state).
+ */
+#ifndef OSDN_H
+#define OSDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define OSDN_ABI_VERSION 1
+
+enum {
+    OSDN_OK = 0,
+    OSDN_ERR_INVALID_ARG = 1,   /* NULL required pointer, bad size, misalignment */
+    OSDN_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. dk = 96) */
+    OSDN_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    OSDN_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up */
+};
+
+typedef enum { OSDN_BF16 = 0, OSDN_FP32 = 1 } osdn_dtype;
+
+typedef struct {
+    uint32_t struct_size;   /* must be sizeof(osdn_params): ABI versioning */
+    int32_t B;              /* sequences */
+    int32_t T;              /* tokens per sequence (ignored by osdn_step) */
+    int32_t H;              /* heads */
+    int32_t dk;             /* key / query width */
+    int32_t dv;             /* value width */
+    int32_t chunk;          /* chunk length C of the chunkwise form; 64 */
+    int32_t dtype;          /* osdn_dtype of q, k, v, beta, r, out */
+    float eta;              /* hypergradient step size of the preconditioner */
+} osdn_params;
+
+/* Bytes of device workspace osdn_fwd needs for these parameters (written to
+ * *bytes). The workspace holds the scaled write keys d_t (.) k_t in the input
+ * dtype plus a small status block; it is scratch owned by the caller, needs no
+ * initialisation, and may be reused by the next call on the same stream.
+ * Returns OSDN_OK, OSDN_ERR_INVALID_ARG or OSDN_ERR_UNSUPPORTED. */
+int osdn_fwd_workspace_size(const osdn_params *p, size_t *bytes);
+
+/* Chunkwise-parallel OSDN forward over T tokens for every (b, h).
+ *   Phase 1 (preconditioner scan, section 2.2 "two phases"): d_t for every
+ *   token from k, beta, r and d0; the scaled write keys d_t (.) k_t go to the
+ *   workspace; d after the last token goes to final_d.
+ *   Phase 2 (chunked delta rule with the scaled write key, section 2.1): per
+ *   chunk of C tokens, A = strict_tril(diag(beta) K Kw^T),
+ *   T = (I + A)^{-1}, U = T diag(beta) (V - K S^T),
+ *   O = Q S^T + tril(Q Kw^T) U, S <- S + U^T Kw (Kw = scaled write keys).
+ * r == NULL: APF off (r == 1). d0 == NULL: d0 = ones. S0 == NULL: S0 = 0.
+ * final_S, final_d may be NULL (not written). out may not be NULL when T > 0.
+ * workspace must hold osdn_fwd_workspace_size() bytes (16-byte aligned).
+ * Errors: OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED, OSDN_ERR_CUDA. */
+int osdn_fwd(const osdn_params *p,
+             const void *q, const void *k, const void *v,
+             const void *beta, const void *r,
+             const float *d0, const float *S0,
+             void *out, float *final_S, float *final_d,
+             void *workspace, size_t workspace_bytes,
+             void *cuda_stream);
+
+/* Phase 1 of osdn_fwd alone: the preconditioner scan. Reads k, beta, r and
+ * d0; writes the scaled write keys d_t (.) k_t into the workspace and d after
+ * the last token into final_d (nullable). Same arguments and rules as
+ * osdn_fwd. osdn_fwd == osdn_fwd_scan then osdn_fwd_chunk on one stream. */
+int osdn_fwd_scan(const osdn_params *p,
+                  const void *k, const void *beta, const void *r,
+                  const float *d0, float *final_d,
+                  void *workspace, size_t workspace_bytes,
+                  void *cuda_stream);
+
+/* Phase 2 of osdn_fwd alone: the chunked delta rule with the scaled write
+ * keys that a preceding osdn_fwd_scan with the same parameters left in the
+ * workspace (ordered before this call on the stream). Writes out and
+ * final_S (nullable). Same arguments and rules as osdn_fwd. */
+int osdn_fwd_chunk(const osdn_params *p,
+                   const void *q, const void *k, const void *v, const void *beta,
+                   const float *S0, void *out, float *final_S,
+                   const void *workspace, size_t workspace_bytes,
+                   void *cuda_stream);
+
+/* One recurrent decode token for every (b, h), in place (constant memory):
+ *   k~ = d (.) k;  S <- S + beta (v - S k) k~^T;  out = S q (after the write);
+ *   d <- r d + eta beta (1 - beta <d, k^2>) k^2 / ||k||^2 (pre-update d).
+ * p->T is ignored. S [B, H, dv, dk] and d [B, H, dk] are read and written.
+ * r == NULL: APF off. Errors: OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED,
+ * OSDN_ERR_CUDA. */
+int osdn_step(const osdn_params *p,
+              const void *q, const void *k, const void *v,
+              const void *beta, const void *r,
+              float *S, float *d, void *out,
+              void *cuda_stream);
+
+/* Waits for the work queued on cuda_stream, then reports whether any bounded
+ * device-side wait of the library's kernels gave up since the last call
+ * (OSDN_ERR_TIMEOUT) and clears that flag. Returns OSDN_OK when none did,
+ * OSDN_ERR_CUDA when the stream itself reports an error. This is the only
+ * entry point that synchronises the host. */
+int osdn_sync_status(void *cuda_stream);
+
+/* Message describing the calling thread's most recent error ("" if none).
+ * The string is owned by the library and valid until the thread's next call. */
+const char *osdn_get_last_error(void);
+
+/* OSDN_ABI_VERSION of the loaded library. */
+int osdn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OSDN_H */

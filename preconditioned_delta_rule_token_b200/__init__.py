@@ -1,0 +1,52 @@
+"""OSDN (Online Scaled DeltaNet) forward and decode on B200 (sm_100a).
+
+The compute lives in ``libosdn.so`` (CUDA kernels behind the C ABI of
+``include/osdn.h``); this package is its ctypes binding plus two convenience
+wrappers that allocate outputs and workspace with PyTorch:
+
+    out, S, d = forward(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2)
+    o = step(q, k, v, beta, S, d, r=None, eta=1e-2)      # S, d updated in place
+
+All tensors must be CUDA tensors; there is no CPU path.
+"""
+from __future__ import annotations
+
+import torch
+
+from ._binding import (OSDN_BF16, OSDN_ERR_CUDA, OSDN_ERR_INVALID_ARG, OSDN_ERR_TIMEOUT, OSDN_ERR_UNSUPPORTED,
+                       OSDN_FP32, OSDN_OK, LIB_PATH, OsdnError, build, get_last_error, make_params, osdn_fwd,
+                       osdn_fwd_chunk, osdn_fwd_scan,
+                       osdn_fwd_workspace_size, osdn_params, osdn_step, osdn_sync_status)
+
+__all__ = ["forward", "step", "osdn_fwd", "osdn_fwd_scan", "osdn_fwd_chunk", "osdn_step", "osdn_fwd_workspace_size", "osdn_sync_status",
+           "osdn_params", "make_params", "get_last_error", "OsdnError", "build", "LIB_PATH",
+           "OSDN_OK", "OSDN_ERR_INVALID_ARG", "OSDN_ERR_UNSUPPORTED", "OSDN_ERR_CUDA", "OSDN_ERR_TIMEOUT",
+           "OSDN_BF16", "OSDN_FP32"]
+
+
+def forward(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, chunk=64, workspace=None, stream=None):
+    """OSDN forward. q, k [B,T,H,dk]; v [B,T,H,dv]; beta, r [B,T,H] (bf16 or fp32,
+    one dtype); d0 [B,H,dk] and S0 [B,H,dv,dk] fp32 or None.
+    Returns (out [B,T,H,dv], final_S [B,H,dv,dk] fp32, final_d [B,H,dk] fp32)."""
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    p = make_params(B, T, H, dk, dv, k.dtype, eta, chunk)
+    dev = k.device
+    out = torch.empty((B, T, H, dv), dtype=k.dtype, device=dev)
+    final_S = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    final_d = torch.empty((B, H, dk), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(osdn_fwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    osdn_fwd(p, q, k, v, beta, r, d0, S0, out, final_S, final_d, workspace, stream)
+    return out, final_S, final_d
+
+
+def step(q, k, v, beta, S, d, r=None, eta=1e-2, stream=None):
+    """One decode token for every (b, h): q, k [B,H,dk]; v [B,H,dv]; beta, r [B,H];
+    S [B,H,dv,dk] and d [B,H,dk] fp32, updated in place. Returns out [B,H,dv]."""
+    B, H, dk = k.shape
+    dv = v.shape[-1]
+    p = make_params(B, 1, H, dk, dv, k.dtype, eta)
+    out = torch.empty((B, H, dv), dtype=k.dtype, device=k.device)
+    osdn_step(p, q, k, v, beta, r, S, d, out, stream)
+    return out

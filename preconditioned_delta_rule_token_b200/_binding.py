@@ -1,0 +1,168 @@
+"""ctypes binding of libosdn.so (argument marshalling only).
+
+Every arithmetic step runs in the library's CUDA kernels; this module checks
+tensors, builds the ``osdn_params`` block and passes raw device pointers and
+the current CUDA stream. It raises if the library is missing or the tensors
+are not on a CUDA device: there is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_ROOT = os.path.dirname(_PKG)
+_CSRC = os.path.join(_PKG, "csrc")
+_INCLUDE = os.path.join(_ROOT, "include")
+LIB_PATH = os.path.join(_PKG, "libosdn.so")
+
+OSDN_OK, OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED, OSDN_ERR_CUDA, OSDN_ERR_TIMEOUT = range(5)
+OSDN_BF16, OSDN_FP32 = 0, 1
+
+NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+              "-Xcompiler", "-fPIC", "-shared", "-cudart", "static", "--expt-relaxed-constexpr"]
+
+
+class osdn_params(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("B", ctypes.c_int32), ("T", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("dk", ctypes.c_int32), ("dv", ctypes.c_int32),
+                ("chunk", ctypes.c_int32), ("dtype", ctypes.c_int32), ("eta", ctypes.c_float)]
+
+
+class OsdnError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__("osdn error %d: %s" % (code, msg))
+        self.code = code
+
+
+def _sources():
+    return sorted(os.path.join(_CSRC, f) for f in os.listdir(_CSRC) if f.endswith((".cu", ".cuh")))
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile libosdn.so in-tree for sm_100a with nvcc."""
+    deps = _sources() + [os.path.join(_INCLUDE, "osdn.h")]
+    if not force and os.path.exists(LIB_PATH):
+        if os.path.getmtime(LIB_PATH) >= max(os.path.getmtime(p) for p in deps):
+            return LIB_PATH
+    tmp = LIB_PATH + ".tmp%d" % os.getpid()
+    cmd = ["nvcc"] + NVCC_FLAGS + ["-I", _INCLUDE, "-I", _CSRC, "-o", tmp, os.path.join(_CSRC, "osdn_api.cu")]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    subprocess.check_call(cmd)
+    os.replace(tmp, LIB_PATH)
+    return LIB_PATH
+
+
+def build_if_missing() -> str:
+    return build(force=False)
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library (raises if it was never built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OsdnError(OSDN_ERR_UNSUPPORTED, "libosdn.so is not built (run __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        P = ctypes.POINTER(osdn_params)
+        L.osdn_fwd_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+        L.osdn_fwd_workspace_size.restype = ctypes.c_int
+        L.osdn_fwd.argtypes = [P] + [vp] * 10 + [vp, sz, vp]
+        L.osdn_fwd.restype = ctypes.c_int
+        L.osdn_fwd_scan.argtypes = [P] + [vp] * 5 + [vp, sz, vp]
+        L.osdn_fwd_scan.restype = ctypes.c_int
+        L.osdn_fwd_chunk.argtypes = [P] + [vp] * 7 + [vp, sz, vp]
+        L.osdn_fwd_chunk.restype = ctypes.c_int
+        L.osdn_step.argtypes = [P] + [vp] * 8 + [vp]
+        L.osdn_step.restype = ctypes.c_int
+        L.osdn_sync_status.argtypes = [vp]
+        L.osdn_sync_status.restype = ctypes.c_int
+        L.osdn_get_last_error.argtypes = []
+        L.osdn_get_last_error.restype = ctypes.c_char_p
+        L.osdn_abi_version.argtypes = []
+        L.osdn_abi_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def get_last_error() -> str:
+    return lib().osdn_get_last_error().decode()
+
+
+def _check(rc):
+    if rc != OSDN_OK:
+        raise OsdnError(rc, get_last_error())
+
+
+def make_params(B, T, H, dk, dv, dtype, eta, chunk=64) -> osdn_params:
+    p = osdn_params()
+    p.struct_size = ctypes.sizeof(osdn_params)
+    p.B, p.T, p.H, p.dk, p.dv, p.chunk = int(B), int(T), int(H), int(dk), int(dv), int(chunk)
+    p.dtype = OSDN_BF16 if dtype == torch.bfloat16 else OSDN_FP32
+    p.eta = float(eta)
+    return p
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise OsdnError(OSDN_ERR_INVALID_ARG, "tensor is not on a CUDA device (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise OsdnError(OSDN_ERR_INVALID_ARG, "tensor is not contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def osdn_fwd_workspace_size(params: osdn_params) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().osdn_fwd_workspace_size(ctypes.byref(params), ctypes.byref(n)))
+    return n.value
+
+
+def osdn_fwd(params, q, k, v, beta, r, d0, S0, out, final_S, final_d, workspace, stream=None):
+    """Raw C-ABI call: every tensor preallocated by the caller (device memory)."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().osdn_fwd(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(d0), _ptr(S0),
+                          _ptr(out), _ptr(final_S), _ptr(final_d), _ptr(workspace), ctypes.c_size_t(ws_bytes),
+                          _stream(stream)))
+
+
+def _ws_bytes(workspace):
+    return 0 if workspace is None else workspace.numel() * workspace.element_size()
+
+
+def osdn_fwd_scan(params, k, beta, r, d0, final_d, workspace, stream=None):
+    """Raw C-ABI call of phase 1 (preconditioner scan into the workspace)."""
+    _check(lib().osdn_fwd_scan(ctypes.byref(params), _ptr(k), _ptr(beta), _ptr(r), _ptr(d0), _ptr(final_d),
+                               _ptr(workspace), ctypes.c_size_t(_ws_bytes(workspace)), _stream(stream)))
+
+
+def osdn_fwd_chunk(params, q, k, v, beta, S0, out, final_S, workspace, stream=None):
+    """Raw C-ABI call of phase 2 (chunked delta rule reading the workspace)."""
+    _check(lib().osdn_fwd_chunk(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(out),
+                                _ptr(final_S), _ptr(workspace), ctypes.c_size_t(_ws_bytes(workspace)),
+                                _stream(stream)))
+
+
+def osdn_step(params, q, k, v, beta, r, S, d, out, stream=None):
+    """Raw C-ABI call: one decode token for every (b, h); S and d updated in place."""
+    _check(lib().osdn_step(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(S), _ptr(d),
+                           _ptr(out), _stream(stream)))
+
+
+def osdn_sync_status(stream=None) -> int:
+    return lib().osdn_sync_status(_stream(stream))

@@ -1,0 +1,288 @@
+// Host side of libosdn.so: argument checks, workspace layout and kernel
+// launches behind the C ABI declared in include/osdn.h.  Nothing here
+// allocates device memory or synchronises the host (except osdn_sync_status).
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <initializer_list>
+#include <string>
+
+#include "osdn.h"
+
+#include "chunk_ffma.cuh"
+#include "scan_seq.cuh"
+#include "step.cuh"
+
+namespace {
+
+thread_local std::string t_last_error;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(OSDN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t elem_size(int dtype) { return dtype == OSDN_BF16 ? 2 : 4; }
+
+// Common checks of the parameter block. need_T: the forward (T used).
+int check_params(const osdn_params* p, bool need_T) {
+    if (!p) return fail(OSDN_ERR_INVALID_ARG, "params is NULL");
+    if (p->struct_size != sizeof(osdn_params))
+        return fail(OSDN_ERR_INVALID_ARG, "params.struct_size is %u, expected %zu (ABI mismatch)",
+                    p->struct_size, sizeof(osdn_params));
+    if (p->B < 1 || p->H < 1) return fail(OSDN_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", p->B, p->H);
+    if (need_T && p->T < 0) return fail(OSDN_ERR_INVALID_ARG, "T must be >= 0 (got %d)", p->T);
+    if (p->dtype != OSDN_BF16 && p->dtype != OSDN_FP32)
+        return fail(OSDN_ERR_INVALID_ARG, "unknown dtype %d", p->dtype);
+    if (p->dk <= 0 || p->dv <= 0) return fail(OSDN_ERR_INVALID_ARG, "dk and dv must be positive");
+    if ((p->dk != 64 && p->dk != 128) || (p->dv != 64 && p->dv != 128))
+        return fail(OSDN_ERR_UNSUPPORTED, "dk, dv must be 64 or 128 (got %d, %d)", p->dk, p->dv);
+    if (need_T && p->chunk != 64) return fail(OSDN_ERR_UNSUPPORTED, "chunk must be 64 (got %d)", p->chunk);
+    if (!(p->eta == p->eta)) return fail(OSDN_ERR_INVALID_ARG, "eta is NaN");
+    const double tokens = (double)p->B * (double)(need_T ? p->T : 1) * (double)p->H;
+    if (tokens * (double)(p->dk > p->dv ? p->dk : p->dv) > 9.0e18)
+        return fail(OSDN_ERR_INVALID_ARG, "tensor sizes overflow 64-bit indexing");
+    if ((double)p->B * p->H > 2147483647.0) return fail(OSDN_ERR_INVALID_ARG, "B * H exceeds the grid limit");
+    return OSDN_OK;
+}
+
+struct WorkspaceLayout {
+    size_t kw_off, kw_bytes, total;
+};
+
+WorkspaceLayout layout_of(const osdn_params* p) {
+    WorkspaceLayout L;
+    L.kw_off = 0;
+    L.kw_bytes = (size_t)p->B * (size_t)p->T * (size_t)p->H * (size_t)p->dk * elem_size(p->dtype);
+    L.total = round_up(L.kw_bytes, 256);
+    if (L.total == 0) L.total = 256;
+    return L;
+}
+
+__global__ void fill_ones_kernel(float* x, size_t n) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        x[i] = 1.f;
+}
+
+int copy_initial_state(const osdn_params* p, const float* d0, const float* S0, float* final_S, float* final_d,
+                       bool want_S, bool want_d, cudaStream_t st) {
+    const size_t units = (size_t)p->B * p->H;
+    cudaError_t e;
+    if (want_S && final_S) {
+        const size_t bytes = units * p->dv * p->dk * sizeof(float);
+        e = S0 ? cudaMemcpyAsync(final_S, S0, bytes, cudaMemcpyDeviceToDevice, st)
+               : cudaMemsetAsync(final_S, 0, bytes, st);
+        if (e != cudaSuccess) return cuda_fail(e, "initial state copy");
+    }
+    if (want_d && final_d) {
+        const size_t n = units * p->dk;
+        if (d0) {
+            e = cudaMemcpyAsync(final_d, d0, n * sizeof(float), cudaMemcpyDeviceToDevice, st);
+        } else {
+            const size_t blocks = (n + 255) / 256;
+            fill_ones_kernel<<<(unsigned)(blocks > 1024 ? 1024 : blocks), 256, 0, st>>>(final_d, n);
+            e = cudaGetLastError();
+        }
+        if (e != cudaSuccess) return cuda_fail(e, "initial preconditioner copy");
+    }
+    return OSDN_OK;
+}
+
+// Phase 1: preconditioner scan -> scaled write keys (workspace) and final d.
+template <typename Tin>
+int launch_scan(const osdn_params* p, const Tin* k, const Tin* beta, const Tin* r, const float* d0, float* final_d,
+                Tin* kw, cudaStream_t st) {
+    if (p->T == 0) return copy_initial_state(p, d0, nullptr, nullptr, final_d, false, true, st);
+    const int units = p->B * p->H;
+    const dim3 grid((units + 3) / 4);
+    if (p->dk == 128)
+        osdn::scan_seq_kernel<128, Tin><<<grid, 128, 0, st>>>(k, beta, r, d0, kw, final_d, p->B, p->T, p->H, p->eta);
+    else
+        osdn::scan_seq_kernel<64, Tin><<<grid, 128, 0, st>>>(k, beta, r, d0, kw, final_d, p->B, p->T, p->H, p->eta);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    return OSDN_OK;
+}
+
+// Phase 2: chunkwise delta rule with the scaled write key.
+template <typename Tin>
+int launch_chunk(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, const Tin* beta, const float* S0,
+                 Tin* out, float* final_S, const Tin* kw, cudaStream_t st) {
+    if (p->T == 0) return copy_initial_state(p, nullptr, S0, final_S, nullptr, true, false, st);
+    const int units = p->B * p->H;
+    constexpr int DVT = 64;
+    const dim3 grid(units, p->dv / DVT);
+    cudaError_t e;
+    if (p->dk == 128) {
+        auto kern = osdn::chunk_ffma_kernel<128, DVT, Tin>;
+        const size_t smem = osdn::FfmaSmem<128, DVT>::kBytes;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return cuda_fail(e, "chunk kernel attribute");
+        kern<<<grid, 256, smem, st>>>(q, k, kw, v, beta, S0, out, final_S, p->B, p->T, p->H, p->dv);
+    } else {
+        auto kern = osdn::chunk_ffma_kernel<64, DVT, Tin>;
+        const size_t smem = osdn::FfmaSmem<64, DVT>::kBytes;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return cuda_fail(e, "chunk kernel attribute");
+        kern<<<grid, 256, smem, st>>>(q, k, kw, v, beta, S0, out, final_S, p->B, p->T, p->H, p->dv);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "chunk launch");
+    return OSDN_OK;
+}
+
+// Pointer and workspace checks shared by the forward entry points.
+int check_fwd_args(const osdn_params* p, std::initializer_list<const void*> required,
+                   std::initializer_list<const void*> all, const void* workspace, size_t ws_bytes) {
+    if (p->T > 0) {
+        for (const void* x : required)
+            if (!x) return fail(OSDN_ERR_INVALID_ARG, "a required pointer (q, k, v, beta, out) is NULL");
+        if (!workspace) return fail(OSDN_ERR_INVALID_ARG, "workspace is NULL");
+    }
+    for (const void* x : all)
+        if (x && !aligned16(x)) return fail(OSDN_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
+    if (workspace && !aligned16(workspace)) return fail(OSDN_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
+    const size_t need = layout_of(p).total;
+    if (p->T > 0 && ws_bytes < need)
+        return fail(OSDN_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+    return OSDN_OK;
+}
+
+template <typename Tin>
+int launch_step(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, const Tin* beta, const Tin* r,
+                float* S, float* d, Tin* out, cudaStream_t st) {
+    const unsigned units = (unsigned)(p->B * p->H);
+    if (p->dk == 128 && p->dv == 128) osdn::step_kernel<128, 128, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta);
+    else if (p->dk == 128) osdn::step_kernel<128, 64, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta);
+    else if (p->dv == 128) osdn::step_kernel<64, 128, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta);
+    else osdn::step_kernel<64, 64, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "step launch");
+    return OSDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int osdn_abi_version(void) { return OSDN_ABI_VERSION; }
+
+const char* osdn_get_last_error(void) { return t_last_error.c_str(); }
+
+int osdn_fwd_workspace_size(const osdn_params* p, size_t* bytes) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    if (!bytes) return fail(OSDN_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = layout_of(p).total;
+    return OSDN_OK;
+}
+
+int osdn_fwd(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
+             const float* d0, const float* S0, void* out, float* final_S, float* final_d, void* workspace,
+             size_t workspace_bytes, void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    rc = check_fwd_args(p, {q, k, v, beta, out}, {q, k, v, beta, r, d0, S0, out, final_S, final_d}, workspace,
+                        workspace_bytes);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    char* ws = reinterpret_cast<char*>(workspace);
+    const size_t kw_off = layout_of(p).kw_off;
+    if (p->dtype == OSDN_BF16) {
+        using T = __nv_bfloat16;
+        T* kw = (T*)(ws ? ws + kw_off : nullptr);
+        rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
+        if (rc) return rc;
+        return launch_chunk<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S, kw, st);
+    }
+    using T = float;
+    T* kw = (T*)(ws ? ws + kw_off : nullptr);
+    rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
+    if (rc) return rc;
+    return launch_chunk<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S, kw, st);
+}
+
+int osdn_fwd_scan(const osdn_params* p, const void* k, const void* beta, const void* r, const float* d0,
+                  float* final_d, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    rc = check_fwd_args(p, {k, beta}, {k, beta, r, d0, final_d}, workspace, workspace_bytes);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    char* ws = reinterpret_cast<char*>(workspace) + layout_of(p).kw_off;
+    if (p->dtype == OSDN_BF16) {
+        using T = __nv_bfloat16;
+        return launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, (T*)ws, st);
+    }
+    return launch_scan<float>(p, (const float*)k, (const float*)beta, (const float*)r, d0, final_d, (float*)ws, st);
+}
+
+int osdn_fwd_chunk(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta,
+                   const float* S0, void* out, float* final_S, const void* workspace, size_t workspace_bytes,
+                   void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    rc = check_fwd_args(p, {q, k, v, beta, out}, {q, k, v, beta, S0, out, final_S}, workspace, workspace_bytes);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    const char* ws = reinterpret_cast<const char*>(workspace) + layout_of(p).kw_off;
+    if (p->dtype == OSDN_BF16) {
+        using T = __nv_bfloat16;
+        return launch_chunk<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S,
+                               (const T*)ws, st);
+    }
+    return launch_chunk<float>(p, (const float*)q, (const float*)k, (const float*)v, (const float*)beta, S0,
+                               (float*)out, final_S, (const float*)ws, st);
+}
+
+int osdn_step(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
+              float* S, float* d, void* out, void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, false);
+    if (rc) return rc;
+    if (!q || !k || !v || !beta || !S || !d || !out)
+        return fail(OSDN_ERR_INVALID_ARG, "q, k, v, beta, S, d and out must not be NULL");
+    const void* ptrs[] = {q, k, v, beta, r, S, d, out};
+    for (const void* x : ptrs)
+        if (x && !aligned16(x)) return fail(OSDN_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    if (p->dtype == OSDN_BF16) {
+        using T = __nv_bfloat16;
+        return launch_step<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)r, S, d, (T*)out, st);
+    }
+    return launch_step<float>(p, (const float*)q, (const float*)k, (const float*)v, (const float*)beta,
+                              (const float*)r, S, d, (float*)out, st);
+}
+
+int osdn_sync_status(void* cuda_stream) {
+    t_last_error.clear();
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    unsigned int status = 0, zero = 0;
+    if ((e = cudaMemcpyFromSymbol(&status, osdn::g_osdn_status, sizeof(status))) != cudaSuccess)
+        return cuda_fail(e, "status read");
+    if (status && (e = cudaMemcpyToSymbol(osdn::g_osdn_status, &zero, sizeof(zero))) != cudaSuccess)
+        return cuda_fail(e, "status clear");
+    if (status & osdn::kStatusTimeout) return fail(OSDN_ERR_TIMEOUT, "a bounded device-side wait gave up");
+    return OSDN_OK;
+}
+
+}  // extern "C"

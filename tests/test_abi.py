@@ -1,0 +1,84 @@
+"""The C-ABI library: it builds, loads without a GPU, exports every entry
+point declared in include/osdn.h, and rejects bad arguments on the host
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(osdn_\w+)\s*\(", text))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("osdn_fwd", "osdn_step", "osdn_fwd_workspace_size", "osdn_get_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(osdn_lib):
+    lib = ctypes.CDLL(osdn_lib.LIB_PATH)
+    for name in sorted(_declared_functions()):
+        assert hasattr(lib, name), name
+    assert lib.osdn_abi_version() == 1
+
+
+def _params(osdn_lib, **kw):
+    import torch
+    a = dict(B=2, T=100, H=3, dk=128, dv=64, dtype=torch.bfloat16, eta=1e-2, chunk=64)
+    a.update(kw)
+    return osdn_lib.make_params(**a)
+
+
+def test_workspace_size_and_argument_checks(osdn_lib):
+    L = osdn_lib.lib()
+    n = ctypes.c_size_t(0)
+    p = _params(osdn_lib)
+    assert L.osdn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    assert n.value >= 2 * 100 * 3 * 128 * 2 and n.value % 256 == 0
+    bad = _params(osdn_lib)
+    bad.struct_size = 8
+    assert L.osdn_fwd_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == osdn_lib.OSDN_ERR_INVALID_ARG
+    assert "struct_size" in osdn_lib.get_last_error()
+    for kw, code in ((dict(dk=96), osdn_lib.OSDN_ERR_UNSUPPORTED), (dict(chunk=32), osdn_lib.OSDN_ERR_UNSUPPORTED),
+                     (dict(B=0), osdn_lib.OSDN_ERR_INVALID_ARG), (dict(T=-1), osdn_lib.OSDN_ERR_INVALID_ARG),
+                     (dict(eta=float("nan")), osdn_lib.OSDN_ERR_INVALID_ARG)):
+        p = _params(osdn_lib, **kw)
+        assert L.osdn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == code, kw
+        assert osdn_lib.get_last_error() != ""
+
+
+def test_null_and_misaligned_pointers_are_rejected_on_the_host(osdn_lib):
+    L = osdn_lib.lib()
+    p = _params(osdn_lib)
+    fake = ctypes.c_void_p(1 << 20)             # never dereferenced: checks fail first
+    rc = L.osdn_fwd(ctypes.byref(p), None, fake, fake, fake, None, None, None, fake, None, None, fake,
+                    ctypes.c_size_t(1 << 30), None)
+    assert rc == osdn_lib.OSDN_ERR_INVALID_ARG and "NULL" in osdn_lib.get_last_error()
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    rc = L.osdn_fwd(ctypes.byref(p), fake, odd, fake, fake, None, None, None, fake, None, None, fake,
+                    ctypes.c_size_t(1 << 30), None)
+    assert rc == osdn_lib.OSDN_ERR_INVALID_ARG and "aligned" in osdn_lib.get_last_error()
+    rc = L.osdn_fwd(ctypes.byref(p), fake, fake, fake, fake, None, None, None, fake, None, None, fake,
+                    ctypes.c_size_t(16), None)
+    assert rc == osdn_lib.OSDN_ERR_INVALID_ARG and "workspace" in osdn_lib.get_last_error()
+    rc = L.osdn_step(ctypes.byref(p), fake, fake, fake, fake, None, None, fake, fake, None)
+    assert rc == osdn_lib.OSDN_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(osdn_lib):
+    import torch
+    import preconditioned_delta_rule_token_b200 as pk
+    x = torch.zeros((1, 4, 1, 64), dtype=torch.bfloat16)
+    with pytest.raises(pk.OsdnError):
+        pk.forward(x, x, x, torch.zeros((1, 4, 1), dtype=torch.bfloat16))

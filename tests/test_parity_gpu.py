@@ -1,0 +1,203 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 CPU oracle
+on the same seeded inputs.
+
+Metric: max over (b, h) slices of max|gpu - oracle| / max|oracle|, separately
+for out, final S and final d. Bar: 2e-2 for bf16 inputs with fp32
+accumulation, 1e-4 in fp32 mode. Full-size workloads are checked on sampled
+(b, h) units that the oracle recomputes alone (units are independent).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from preconditioned_delta_rule_token_b200 import workloads as W
+from tests._util import BF16_TOL, FP32_TOL, slice_rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(x):
+    return None if x is None else x.cuda()
+
+
+def _run_gpu(inp, eta, chunk=64):
+    import preconditioned_delta_rule_token_b200 as pk
+    out, S, d = pk.forward(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["beta"]), _dev(inp["r"]),
+                           _dev(inp["d0"]), _dev(inp["S0"]), eta=eta, chunk=chunk)
+    assert pk.osdn_sync_status() == 0
+    return out.float().cpu().numpy(), S.cpu().numpy(), d.cpu().numpy()
+
+
+def _unit(inp, b, h):
+    """Inputs of one (b, h) unit as a B = H = 1 problem (float64)."""
+    f = W.to_f64
+    sl4 = lambda x: None if x is None else f(x)[b:b + 1, :, h:h + 1]
+    sl3 = lambda x: None if x is None else f(x)[b:b + 1, :, h:h + 1]
+    return dict(q=sl4(inp["q"]), k=sl4(inp["k"]), v=sl4(inp["v"]), beta=sl3(inp["beta"]), r=sl3(inp["r"]),
+                d0=None if inp["d0"] is None else f(inp["d0"])[b:b + 1, h:h + 1],
+                S0=None if inp["S0"] is None else f(inp["S0"])[b:b + 1, h:h + 1])
+
+
+def _oracle(inp, eta):
+    f = W.to_f64
+    return oracle.fwd(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["beta"]), f(inp["r"]), f(inp["d0"]),
+                      f(inp["S0"]), eta=eta)
+
+
+def _errs(gpu, ref):
+    return (slice_rel_err(gpu[0], ref[0], (0, 2)), slice_rel_err(gpu[1], ref[1], (0, 1)),
+            slice_rel_err(gpu[2], ref[2], (0, 1)))
+
+
+SMALL = [
+    # dtype, B, H, T, dk, dv, apf, eta, d0, S0
+    (W.FP32, 1, 1, 256, 64, 64, True, 1e-2, "ones", "zeros"),
+    (W.FP32, 2, 3, 65, 128, 128, True, 1.0, "uniform", "normal"),
+    (W.FP32, 2, 2, 130, 128, 64, False, 0.0, "uniform", "normal"),
+    (W.FP32, 1, 3, 1, 64, 128, True, 1e-2, "ones", "normal"),
+    (W.BF16, 2, 3, 200, 128, 128, True, 1e-2, "uniform", "normal"),
+    (W.BF16, 2, 3, 63, 128, 128, False, 1.0, "uniform", "zeros"),
+    (W.BF16, 1, 2, 129, 64, 64, True, 0.0, "ones", "normal"),
+    (W.BF16, 3, 1, 192, 128, 64, True, 1e-2, "uniform", "normal"),
+    (W.BF16, 1, 2, 64, 64, 128, False, 1e-2, "ones", "zeros"),
+    (W.BF16, 2, 2, 1, 128, 128, True, 1.0, "uniform", "normal"),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "%s-B%dH%dT%d-dk%ddv%d-apf%d-eta%g-%s-%s" % c)
+def test_small_cases_full_oracle(case):
+    dtype, B, H, T, dk, dv, apf, eta, d0, S0 = case
+    w = W.Workload("small", B, H, T, dk, dv, 64, dtype, apf, "gaussian", eta=eta, seed=100 + T + dk, d0=d0, S0=S0)
+    inp = W.make_forward_inputs(w)
+    errs = _errs(_run_gpu(inp, eta), _oracle(inp, eta))
+    tol = FP32_TOL if dtype == W.FP32 else BF16_TOL
+    assert max(errs) <= tol, errs
+
+
+def test_tiny_fp32_workload():
+    w = W.TINY_FP32
+    inp = W.make_forward_inputs(w)
+    errs = _errs(_run_gpu(inp, w.eta), _oracle(inp, w.eta))
+    assert max(errs) <= FP32_TOL, errs
+
+
+@pytest.mark.parametrize("w,units", [
+    (W.LAYER_340M, [(0, 0), (3, 5), (7, 7)]),
+    (W.LAYER_1P3B, [(0, 0), (5, 11), (7, 15)]),
+    (W.LONG_RECALL, [(0, 0), (0, 15)]),
+], ids=["340M", "1.3B", "long"])
+def test_full_size_workloads_on_sampled_units(w, units):
+    inp = W.make_forward_inputs(w)
+    out, S, d = _run_gpu(inp, w.eta)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(S)) and np.all(np.isfinite(d))
+    for (b, h) in units:
+        u = _unit(inp, b, h)
+        ref = oracle.fwd(u["q"], u["k"], u["v"], u["beta"], u["r"], u["d0"], u["S0"], eta=w.eta)
+        got = (out[b:b + 1, :, h:h + 1], S[b:b + 1, h:h + 1], d[b:b + 1, h:h + 1])
+        errs = _errs(got, ref)
+        assert max(errs) <= BF16_TOL, (b, h, errs)
+
+
+def test_zero_tokens_returns_initial_state():
+    import preconditioned_delta_rule_token_b200 as pk
+    w = W.Workload("t0", 2, 2, 0, 128, 128, 64, W.BF16, True, d0="uniform", S0="normal", seed=5)
+    inp = W.make_forward_inputs(w)
+    out, S, d = pk.forward(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["beta"]), _dev(inp["r"]),
+                           _dev(inp["d0"]), _dev(inp["S0"]), eta=w.eta)
+    torch.cuda.synchronize()
+    assert out.numel() == 0
+    assert torch.equal(S.cpu(), inp["S0"]) and torch.equal(d.cpu(), inp["d0"])
+    out, S, d = pk.forward(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["beta"]), None, None, None)
+    torch.cuda.synchronize()
+    assert torch.all(S == 0) and torch.all(d == 1)
+
+
+@pytest.mark.parametrize("dtype", [W.FP32, W.BF16])
+def test_continuation_equals_one_forward(dtype):
+    """Checkpoint/resume: forward over T1 then over T2 from the carried (S, d)
+    equals one forward over T1 + T2 (T1 not a multiple of the chunk)."""
+    import preconditioned_delta_rule_token_b200 as pk
+    w = W.Workload("cont", 2, 2, 150, 128, 128, 64, dtype, True, d0="uniform", S0="normal", eta=0.5, seed=6)
+    inp = W.make_forward_inputs(w)
+    g = {k_: _dev(v_) for k_, v_ in inp.items()}
+    o_full, S_full, d_full = pk.forward(g["q"], g["k"], g["v"], g["beta"], g["r"], g["d0"], g["S0"], eta=w.eta)
+    T1 = 77
+    part = lambda x, a, b: x[:, a:b].contiguous()
+    o1, S1, d1 = pk.forward(part(g["q"], 0, T1), part(g["k"], 0, T1), part(g["v"], 0, T1), part(g["beta"], 0, T1),
+                            part(g["r"], 0, T1), g["d0"], g["S0"], eta=w.eta)
+    o2, S2, d2 = pk.forward(part(g["q"], T1, 150), part(g["k"], T1, 150), part(g["v"], T1, 150),
+                            part(g["beta"], T1, 150), part(g["r"], T1, 150), d1, S1, eta=w.eta)
+    torch.cuda.synchronize()
+    tol = FP32_TOL if dtype == W.FP32 else BF16_TOL
+    ref = _oracle(inp, w.eta)
+    got = (torch.cat([o1, o2], 1).float().cpu().numpy(), S2.cpu().numpy(), d2.cpu().numpy())
+    assert max(_errs(got, ref)) <= tol
+    full = (o_full.float().cpu().numpy(), S_full.cpu().numpy(), d_full.cpu().numpy())
+    assert max(_errs(got, full)) <= tol
+
+
+@pytest.mark.parametrize("dtype", [W.FP32, W.BF16])
+def test_decode_steps_equal_forward(dtype):
+    """T calls of the single-token step equal one forward over the same tokens."""
+    import preconditioned_delta_rule_token_b200 as pk
+    w = W.Workload("dec", 2, 3, 40, 128, 128, 64, dtype, True, d0="uniform", S0="normal", eta=0.3, seed=7)
+    inp = W.make_forward_inputs(w)
+    g = {k_: _dev(v_) for k_, v_ in inp.items()}
+    S = g["S0"].clone()
+    d = g["d0"].clone()
+    outs = []
+    for t in range(w.T):
+        outs.append(pk.step(g["q"][:, t].contiguous(), g["k"][:, t].contiguous(), g["v"][:, t].contiguous(),
+                            g["beta"][:, t].contiguous(), S, d, r=g["r"][:, t].contiguous(), eta=w.eta))
+    torch.cuda.synchronize()
+    got = (torch.stack(outs, 1).float().cpu().numpy(), S.cpu().numpy(), d.cpu().numpy())
+    ref = _oracle(inp, w.eta)
+    tol = FP32_TOL if dtype == W.FP32 else BF16_TOL
+    assert max(_errs(got, ref)) <= tol
+
+
+def test_decode_workload_sampled_units():
+    """Decode workload: B = 256 sequences x H = 16 heads, 1024 single-token calls
+    from S0 ~ N(0, 0.02^2); sampled heads recomputed by the oracle step by step."""
+    import preconditioned_delta_rule_token_b200 as pk
+    w = W.DECODE
+    st = W.make_decode_state(w)
+    S = st["S0"].cuda()
+    d = st["d0"].cuda()
+    units = [(0, 0), (17, 3), (128, 9), (255, 15)]
+    So = {u: np.ascontiguousarray(W.to_f64(st["S0"][u[0]:u[0] + 1, u[1]:u[1] + 1])) for u in units}
+    do = {u: np.ascontiguousarray(W.to_f64(st["d0"][u[0]:u[0] + 1, u[1]:u[1] + 1])) for u in units}
+    worst = 0.0
+    for t in range(w.steps):
+        tok = W.make_decode_token(w, t)
+        o = pk.step(tok["q"].cuda(), tok["k"].cuda(), tok["v"].cuda(), tok["beta"].cuda(), S, d,
+                    r=_dev(tok["r"]), eta=w.eta)
+        check = (t % 128 == 127) or t == w.steps - 1
+        oc = o.float().cpu().numpy() if check else None
+        for (b, h) in units:
+            f = lambda x: None if x is None else W.to_f64(x)[b:b + 1, h:h + 1]
+            ro = oracle.step(f(tok["q"]), f(tok["k"]), f(tok["v"]), f(tok["beta"]), So[(b, h)], do[(b, h)],
+                             r=f(tok["r"]), eta=w.eta)
+            if check:
+                worst = max(worst, slice_rel_err(oc[b:b + 1, h:h + 1], ro, (0, 1)))
+    Sc, dc = S.cpu().numpy(), d.cpu().numpy()
+    for (b, h) in units:
+        worst = max(worst, slice_rel_err(Sc[b:b + 1, h:h + 1], So[(b, h)], (0, 1)),
+                    slice_rel_err(dc[b:b + 1, h:h + 1], do[(b, h)], (0, 1)))
+    assert worst <= BF16_TOL, worst
+
+
+def test_gpu_preconditioner_is_decoupled_from_values_and_queries():
+    """Section 2.2's decoupling on the GPU path: final d does not depend on v or q."""
+    import preconditioned_delta_rule_token_b200 as pk
+    w = W.Workload("dec2", 2, 2, 100, 128, 128, 64, W.BF16, True, d0="uniform", eta=0.5, seed=8)
+    inp = W.make_forward_inputs(w)
+    g = {k_: _dev(v_) for k_, v_ in inp.items()}
+    _, _, d1 = pk.forward(g["q"], g["k"], g["v"], g["beta"], g["r"], g["d0"], None, eta=w.eta)
+    _, _, d2 = pk.forward(torch.randn_like(g["q"]), g["k"], torch.randn_like(g["v"]), g["beta"], g["r"], g["d0"],
+                          None, eta=w.eta)
+    torch.cuda.synchronize()
+    assert torch.equal(d1, d2)
