@@ -127,6 +127,36 @@ int osdn_step(const osdn_params *p,
               float *S, float *d, void *out,
               void *cuda_stream);
 
+/* Largest scratch osdn_fwd_noalloc can use: B * T * H * dk * element size
+ * (2 bytes for bf16, 4 for fp32) must not exceed this. */
+#define OSDN_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* osdn_fwd without a workspace argument, for callers that cannot allocate
+ * device memory at call time. Examples: a plugin or extension whose device
+ * memory is owned and budgeted by a host framework, or a latency-critical
+ * loop that must not enter the CUDA allocator, which can synchronise the
+ * device. The pages describe no such variant; the method has no counterpart
+ * of it. Arguments and results are those of osdn_fwd.
+ *
+ * The scaled write keys go to one fixed scratch array inside the library
+ * (OSDN_NOALLOC_SCRATCH_BYTES of device memory that every GPU which loads the
+ * library keeps until the process exits). The library calls no cudaMalloc or
+ * cudaFree for it. The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture. Every call uses the same array, and the
+ * scan overwrites every scratch entry the chunk phase reads, so stale contents
+ * from an earlier call are never used. Two calls that overlap on the GPU (for
+ * example on two streams) race on the array: order them on one stream.
+ * Errors: those of osdn_fwd; OSDN_ERR_INVALID_ARG when the scratch needed
+ * exceeds OSDN_NOALLOC_SCRATCH_BYTES; OSDN_ERR_CUDA when the address lookup
+ * fails. */
+int osdn_fwd_noalloc(const osdn_params *p,
+                     const void *q, const void *k, const void *v,
+                     const void *beta, const void *r,
+                     const float *d0, const float *S0,
+                     void *out, float *final_S, float *final_d,
+                     void *cuda_stream);
+
 /* Waits for the work queued on cuda_stream, then reports whether any bounded
  * device-side wait of the library's kernels gave up since the last call
  * (OSDN_ERR_TIMEOUT) and clears that flag. Returns OSDN_OK when none did,

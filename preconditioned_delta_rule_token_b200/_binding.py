@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libosdn.so")
 
 OSDN_OK, OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED, OSDN_ERR_CUDA, OSDN_ERR_TIMEOUT = range(5)
 OSDN_BF16, OSDN_FP32 = 0, 1
+OSDN_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared", "-cudart", "static", "--expt-relaxed-constexpr"]
@@ -81,6 +82,8 @@ def lib():
         L.osdn_fwd_scan.restype = ctypes.c_int
         L.osdn_fwd_chunk.argtypes = [P] + [vp] * 7 + [vp, sz, vp]
         L.osdn_fwd_chunk.restype = ctypes.c_int
+        L.osdn_fwd_noalloc.argtypes = [P] + [vp] * 10 + [vp]
+        L.osdn_fwd_noalloc.restype = ctypes.c_int
         L.osdn_step.argtypes = [P] + [vp] * 8 + [vp]
         L.osdn_step.restype = ctypes.c_int
         L.osdn_sync_status.argtypes = [vp]
@@ -156,6 +159,13 @@ def osdn_fwd_chunk(params, q, k, v, beta, S0, out, final_S, workspace, stream=No
     _check(lib().osdn_fwd_chunk(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(out),
                                 _ptr(final_S), _ptr(workspace), ctypes.c_size_t(_ws_bytes(workspace)),
                                 _stream(stream)))
+
+
+def osdn_fwd_noalloc(params, q, k, v, beta, r, d0, S0, out, final_S, final_d, stream=None):
+    """Raw C-ABI call of the forward that takes no workspace: the library uses
+    its own fixed scratch array (see OSDN_NOALLOC_SCRATCH_BYTES in osdn.h)."""
+    _check(lib().osdn_fwd_noalloc(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(d0),
+                                  _ptr(S0), _ptr(out), _ptr(final_S), _ptr(final_d), _stream(stream)))
 
 
 def osdn_step(params, q, k, v, beta, r, S, d, out, stream=None):

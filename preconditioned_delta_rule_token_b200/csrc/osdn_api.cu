@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <initializer_list>
+#include <mutex>
 #include <string>
 
 #include "osdn.h"
@@ -174,6 +175,32 @@ int launch_step(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, 
     return OSDN_OK;
 }
 
+// Scratch for osdn_fwd_noalloc: a fixed array in device memory, sized by
+// OSDN_NOALLOC_SCRATCH_BYTES. In host code the symbol is only a handle; its
+// device address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[OSDN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set up on first use).
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(OSDN_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the scratch array");
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return OSDN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -250,6 +277,39 @@ int osdn_fwd_chunk(const osdn_params* p, const void* q, const void* k, const voi
     }
     return launch_chunk<float>(p, (const float*)q, (const float*)k, (const float*)v, (const float*)beta, S0,
                                (float*)out, final_S, (const float*)ws, st);
+}
+
+int osdn_fwd_noalloc(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta,
+                     const void* r, const float* d0, const float* S0, void* out, float* final_S, float* final_d,
+                     void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    const size_t need = layout_of(p).kw_bytes;
+    if (need > (size_t)OSDN_NOALLOC_SCRATCH_BYTES)
+        return fail(OSDN_ERR_INVALID_ARG, "scratch needed (%zu bytes) exceeds OSDN_NOALLOC_SCRATCH_BYTES (%zu bytes)",
+                    need, (size_t)OSDN_NOALLOC_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    if (p->T > 0) {
+        rc = noalloc_scratch(&scratch);
+        if (rc) return rc;
+    }
+    rc = check_fwd_args(p, {q, k, v, beta, out}, {q, k, v, beta, r, d0, S0, out, final_S, final_d}, scratch,
+                        (size_t)OSDN_NOALLOC_SCRATCH_BYTES);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    if (p->dtype == OSDN_BF16) {
+        using T = __nv_bfloat16;
+        T* kw = (T*)scratch;
+        rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
+        if (rc) return rc;
+        return launch_chunk<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S, kw, st);
+    }
+    float* kw = (float*)scratch;
+    rc = launch_scan<float>(p, (const float*)k, (const float*)beta, (const float*)r, d0, final_d, kw, st);
+    if (rc) return rc;
+    return launch_chunk<float>(p, (const float*)q, (const float*)k, (const float*)v, (const float*)beta, S0,
+                               (float*)out, final_S, kw, st);
 }
 
 int osdn_step(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
