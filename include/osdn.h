@@ -164,6 +164,14 @@ int osdn_fwd_noalloc(const osdn_params *p,
  * entry point that synchronises the host. */
 int osdn_sync_status(void *cuda_stream);
 
+/* Diagnostics: upper bound, in nanoseconds, on any single device-side wait
+ * (mbarrier) of kernels launched after this call; 0 restores the default
+ * (4 s). A wait that reaches it makes its CTA stop early (after letting its
+ * own copies and MMAs in flight finish), and osdn_sync_status() then reports
+ * OSDN_ERR_TIMEOUT; the results of that call are undefined. Meant for tests
+ * of the failure path; process-wide, not thread-safe against launches. */
+void osdn_set_wait_limit_ns(unsigned long long ns);
+
 /* Message describing the calling thread's most recent error ("" if none).
  * The string is owned by the library and valid until the thread's next call. */
 const char *osdn_get_last_error(void);

@@ -69,8 +69,11 @@ def lib():
     """The loaded library (raises if it was never built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise OsdnError(OSDN_ERR_UNSUPPORTED, "libosdn.so is not built (run __graft_entry__.build())")
+        try:
+            build(force=False)          # rebuild in-tree when a source is newer than the library
+        except (OSError, subprocess.CalledProcessError) as exc:
+            if not os.path.exists(LIB_PATH):
+                raise OsdnError(OSDN_ERR_UNSUPPORTED, "libosdn.so is not built and nvcc failed: %s" % exc)
         L = ctypes.CDLL(LIB_PATH)
         vp, sz = ctypes.c_void_p, ctypes.c_size_t
         P = ctypes.POINTER(osdn_params)

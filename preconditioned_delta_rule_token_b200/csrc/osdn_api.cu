@@ -1,17 +1,22 @@
 // Host side of libosdn.so: argument checks, workspace layout and kernel
 // launches behind the C ABI declared in include/osdn.h.  Nothing here
 // allocates device memory or synchronises the host (except osdn_sync_status).
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <initializer_list>
 #include <mutex>
 #include <string>
+#include <type_traits>
 
 #include "osdn.h"
 
 #include "chunk_ffma.cuh"
+#include "chunk_tc.cuh"
 #include "scan_seq.cuh"
 #include "step.cuh"
 
@@ -103,6 +108,60 @@ int copy_initial_state(const osdn_params* p, const float* d0, const float* S0, f
     return OSDN_OK;
 }
 
+// Upper bound on any single device-side wait of the tensor-core kernels.
+std::atomic<unsigned long long> g_wait_limit_ns{4000000000ull};
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 4-D bf16 tensor map over [B, T, H, width] (dims listed innermost first), box
+// {box0, 1, 64 tokens, 1}. The token dimension is its own dimension, so a box
+// that runs past T reads zeros instead of the next sequence.
+int make_token_map(CUtensorMap* m, const void* base, int B, int T, int H, int width, int box0,
+                   CUtensorMapSwizzle swizzle) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(OSDN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t dims[4] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)width * 2, (cuuint64_t)H * width * 2, (cuuint64_t)T * H * width * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)box0, 1, 64, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(OSDN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return OSDN_OK;
+}
+
+// Phase 2 on the tensor cores: bf16, dk = dv = 128.
+int launch_chunk_tc(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                    const __nv_bfloat16* beta, const float* S0, __nv_bfloat16* out, float* final_S,
+                    const __nv_bfloat16* kw, cudaStream_t st) {
+    CUtensorMap mq, mk, mkw, mv;
+    int rc;
+    if ((rc = make_token_map(&mq, q, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    if ((rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    if ((rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    if ((rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
+    auto kern = osdn::chunk_tc_kernel<0>;
+    const size_t smem = osdn::TcSmem::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk kernel attribute");
+    kern<<<p->B * p->H, 128, smem, st>>>(mq, mk, mkw, mv, beta, S0, out, final_S, p->B, p->T, p->H,
+                                         g_wait_limit_ns.load());
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core chunk launch");
+    return OSDN_OK;
+}
+
 // Phase 1: preconditioner scan -> scaled write keys (workspace) and final d.
 template <typename Tin>
 int launch_scan(const osdn_params* p, const Tin* k, const Tin* beta, const Tin* r, const float* d0, float* final_d,
@@ -124,6 +183,9 @@ template <typename Tin>
 int launch_chunk(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, const Tin* beta, const float* S0,
                  Tin* out, float* final_S, const Tin* kw, cudaStream_t st) {
     if (p->T == 0) return copy_initial_state(p, nullptr, S0, final_S, nullptr, true, false, st);
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
+        if (p->dk == 128 && p->dv == 128) return launch_chunk_tc(p, q, k, v, beta, S0, out, final_S, kw, st);
+    }
     const int units = p->B * p->H;
     constexpr int DVT = 64;
     const dim3 grid(units, p->dv / DVT);
@@ -206,6 +268,8 @@ int noalloc_scratch(void** out) {
 extern "C" {
 
 int osdn_abi_version(void) { return OSDN_ABI_VERSION; }
+
+void osdn_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns ? ns : 4000000000ull); }
 
 const char* osdn_get_last_error(void) { return t_last_error.c_str(); }
 
