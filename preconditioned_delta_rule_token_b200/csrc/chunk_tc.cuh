@@ -19,7 +19,8 @@
 // bf16 operands in 128-byte-swizzled shared memory (TMA-filled for Q, K, Kw;
 // written by the CTA for S, Xh, U, T, P), fp32 accumulators in TMEM. The
 // state S stays in TMEM for the whole sequence; its bf16 copy for MMA2 is
-// refreshed once per chunk. T = (I + A)^{-1} is solved on CUDA cores in fp32.
+// refreshed once per chunk. T = (I + A)^{-1} is a blocked 16 x 16 inverse on CUDA cores (fp32 diagonal
+// blocks, mma.sync tf32 block products).
 //
 // One CTA (128 threads = the 128 TMEM lanes) owns one (sequence, head).
 // Thread i owns TMEM lane i: row v = i of S, U^T and O^T; in the epilogues of
@@ -29,6 +30,7 @@
 // leaves after a bounded drain, releasing its TMEM.
 #pragma once
 #include "tc_ptx.cuh"
+#include "tril_inv.cuh"
 
 namespace osdn {
 
@@ -40,9 +42,9 @@ struct TcSmem {
     static constexpr uint32_t XU = 98304;             // Xh^T, then U^T: [128 v][64 t] bf16
     static constexpr uint32_t TB = 114688;            // T [64 t][64 j] bf16
     static constexpr uint32_t PB = 122880;            // P [64 t][64 j] bf16
-    static constexpr int LDF = 65;                    // fp32 row stride of A and T
-    static constexpr uint32_t AF = 131072;            // A fp32 [64][65]
-    static constexpr uint32_t TF = AF + 64 * LDF * 4;  // T fp32 [64][65]
+    static constexpr int LDF = tri::LD;               // fp32 row stride of A and T
+    static constexpr uint32_t AF = 131072;            // A fp32 [64][LDF]
+    static constexpr uint32_t TF = AF + 64 * LDF * 4;  // T fp32 [64][LDF]
     static constexpr uint32_t BETA = TF + 64 * LDF * 4;
     static constexpr uint32_t BAR = BETA + 256;       // tma_bar, mma_bar, tmem base address
     static constexpr uint32_t END = BAR + 64;
@@ -239,23 +241,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         __syncthreads();
 
-        // (4) T = (I + A)^{-1} by column-wise forward substitution (fp32):
-        //     T[j][j] = 1, T[t][j] = -sum_{m=j}^{t-1} A[t][m] T[m][j]; two threads per column.
-        {
-            const int j = tid >> 1, part = tid & 1;
-            for (int t = part; t < j; t += 2) TF[t * L::LDF + j] = 0.f;
-            if (part == 0) TF[j * L::LDF + j] = 1.f;
-            __syncwarp();
-            for (int t = 1; t < C; ++t) {
-                float s = 0.f;
-                if (t > j)
-                    for (int m = j + part; m < t; m += 2) s = fmaf(AF[t * L::LDF + m], TF[m * L::LDF + j], s);
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                if (t > j && part == 0) TF[t * L::LDF + j] = -s;
-                __syncwarp();
-            }
-        }
-        __syncthreads();
+        // (4) T = (I + A)^{-1}: blocked 16 x 16 inverse (fp32 diagonal blocks, tf32 block products)
+        tri::tril_inv64(AF, TF, warp, tid & 31, [] { __syncthreads(); });
         if (tid < C) {   // T -> bf16 K-major swizzled (B operand of MMA3)
             const int t = tid;
 #pragma unroll

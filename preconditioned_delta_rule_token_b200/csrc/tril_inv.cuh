@@ -1,0 +1,153 @@
+// Inverse of a 64 x 64 unit lower-triangular matrix, T = (I + A)^{-1}, with A
+// strictly lower (the UT/WY transform of the chunkwise delta rule, and the
+// same transform in the chunk form of the preconditioner recurrence).
+//
+// Blocked in 16 x 16 blocks (block indices 0..3):
+//   level 0: T_ii = (I + A_ii)^{-1} by forward substitution, one warp per block;
+//   level 1: T_10 = -T_11 A_10 T_00 and T_32 = -T_33 A_32 T_22
+//            (the two 32 x 32 diagonal blocks are then complete);
+//   level 2: X = A_[23][01] T_[01]  (the 32 x 32 lower-left block, 4 warps);
+//   level 3: T_[23][01] = -T_[23] X.
+// The 16 x 16 x 16 block products run on mma.sync m16n8k8 with tf32 inputs
+// and fp32 accumulation; the diagonal blocks are exact fp32 FFMA.
+// Executed by the 128 threads (4 warps) of one group; sync() must be a barrier
+// over exactly those threads. A and T are fp32 in shared memory with row
+// stride LD (68 keeps the fragment loads free of bank conflicts); T may not
+// alias A. On return T holds the full 64 x 64 inverse (zeros above the
+// diagonal) and every thread of the group has passed a final sync().
+#pragma once
+#include "common.cuh"
+
+namespace osdn {
+namespace tri {
+
+constexpr int LD = 68;
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void mma_tf32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// c += X Y for 16 x 16 blocks X (row-major at X, stride LD) and Y; one warp.
+// c[nh] holds output columns nh*8 .. nh*8+7 in the m16n8 accumulator layout.
+__device__ __forceinline__ void blk_mma(float (&c)[2][4], const float* X, const float* Y, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const int k0 = ks * 8;
+        const uint32_t a0 = to_tf32(X[g * LD + k0 + t]);
+        const uint32_t a1 = to_tf32(X[(g + 8) * LD + k0 + t]);
+        const uint32_t a2 = to_tf32(X[g * LD + k0 + t + 4]);
+        const uint32_t a3 = to_tf32(X[(g + 8) * LD + k0 + t + 4]);
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+            const uint32_t b0 = to_tf32(Y[(k0 + t) * LD + nh * 8 + g]);
+            const uint32_t b1 = to_tf32(Y[(k0 + t + 4) * LD + nh * 8 + g]);
+            mma_tf32(c[nh], a0, a1, a2, a3, b0, b1);
+        }
+    }
+}
+
+__device__ __forceinline__ void blk_zero(float (&c)[2][4]) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) c[i][j] = 0.f;
+}
+
+// Store s * c into the 16 x 16 block at D (stride LD).
+__device__ __forceinline__ void blk_store(float* D, const float (&c)[2][4], float s, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        D[g * LD + nh * 8 + 2 * t] = s * c[nh][0];
+        D[g * LD + nh * 8 + 2 * t + 1] = s * c[nh][1];
+        D[(g + 8) * LD + nh * 8 + 2 * t] = s * c[nh][2];
+        D[(g + 8) * LD + nh * 8 + 2 * t + 1] = s * c[nh][3];
+    }
+}
+
+template <class Sync>
+__device__ __forceinline__ void tril_inv64(const float* A, float* T, int warp, int lane, Sync sync) {
+    auto blkA = [&](int i, int j) { return A + (i * 16) * LD + j * 16; };
+    auto blkT = [&](int i, int j) { return T + (i * 16) * LD + j * 16; };
+
+    {   // level 0: diagonal block `warp`, lane j (< 16) owns column j; zero the rest of the block row
+        const int j = lane & 15, o = warp * 16;
+        float c[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) c[t] = (t == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int t = 1; t < 16; ++t) {
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < t; m += 2) {
+                s0 = fmaf(A[(o + t) * LD + o + m], c[m], s0);
+                if (m + 1 < t) s1 = fmaf(A[(o + t) * LD + o + m + 1], c[m + 1], s1);
+            }
+            if (t > j) c[t] = -(s0 + s1);
+        }
+        if (lane < 16) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) T[(o + t) * LD + o + j] = c[t];
+        }
+        // zeros above the diagonal blocks: row block `warp`, column blocks > warp
+        for (int idx = lane; idx < 16 * 48; idx += 32) {
+            const int r = idx / 48, cc = idx % 48;
+            if (o + 16 + cc < 64) T[(o + r) * LD + o + 16 + cc] = 0.f;
+        }
+    }
+    sync();
+    // level 1: warps 0 and 1 build T_10 and T_32 (two products each, through a block of T as scratch)
+    if (warp < 2) {
+        const int i = warp * 2 + 1, j = warp * 2;     // (1,0) or (3,2)
+        float c[2][4];
+        blk_zero(c);
+        blk_mma(c, blkA(i, j), blkT(j, j), lane);     // W = A_ij T_jj
+        blk_store(blkT(i, j), c, 1.f, lane);
+        __syncwarp();
+        blk_zero(c);
+        blk_mma(c, blkT(i, i), blkT(i, j), lane);     // T_ii W
+        __syncwarp();
+        blk_store(blkT(i, j), c, -1.f, lane);
+    }
+    sync();
+    // level 2: X_ab = sum_m A_am T_mb for a in {2,3}, b in {0,1} (m in {0,1}, T_01 = 0)
+    {
+        const int a = 2 + (warp >> 1), bb = warp & 1;
+        float c[2][4];
+        blk_zero(c);
+        if (bb == 0) {
+            blk_mma(c, blkA(a, 0), blkT(0, 0), lane);
+            blk_mma(c, blkA(a, 1), blkT(1, 0), lane);
+        } else {
+            blk_mma(c, blkA(a, 1), blkT(1, 1), lane);
+        }
+        blk_store(blkT(a, bb), c, 1.f, lane);
+    }
+    sync();
+    // level 3: T_ab = -(T_a2 X_2b + T_a3 X_3b), T_23 = 0; all products read X before any write
+    {
+        const int a = 2 + (warp >> 1), bb = warp & 1;
+        float c[2][4];
+        blk_zero(c);
+        blk_mma(c, blkT(a, 2), blkT(2, bb), lane);
+        if (a == 3) blk_mma(c, blkT(3, 3), blkT(3, bb), lane);
+        sync();
+        blk_store(blkT(a, bb), c, -1.f, lane);
+    }
+    sync();
+}
+
+}  // namespace tri
+}  // namespace osdn
