@@ -44,7 +44,7 @@ WORKLOADS = {"340m": W.LAYER_340M, "1p3b": W.LAYER_1P3B, "long": W.LONG_RECALL}
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="1p3b")
@@ -100,11 +100,10 @@ def source_sha(files):
     return h.hexdigest()[:16]
 
 
-KERNEL_SOURCES = {
-    "chunk": ["preconditioned_delta_rule_token_b200/csrc/chunk_ffma.cuh",
-              "preconditioned_delta_rule_token_b200/csrc/common.cuh"],
-    "scan": ["preconditioned_delta_rule_token_b200/csrc/scan_seq.cuh",
-             "preconditioned_delta_rule_token_b200/csrc/common.cuh"],
+_CSRC = "preconditioned_delta_rule_token_b200/csrc/"
+KERNEL_SOURCES = {   # the sources each timed kernel is built from (bf16, dk = dv = 128 path)
+    "chunk": [_CSRC + f for f in ("chunk_tc.cuh", "tc_ptx.cuh", "tril_inv.cuh", "common.cuh")],
+    "scan": [_CSRC + f for f in ("scan_tc.cuh", "tc_ptx.cuh", "tril_inv.cuh", "common.cuh")],
 }
 
 
@@ -125,60 +124,55 @@ def ncu_traffic(kernel, workload_name):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples taken during the timed region."""
-    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle-reason samples taken during the timed region, from a
+    host thread polling NVML every few milliseconds (so short regions still
+    get samples)."""
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20), ("hw_thermal_slowdown", 0x40),
+               ("sw_power_cap", 0x4))
 
-    def __init__(self, device, enabled=True):
-        self.proc = None
+    def __init__(self, device, enabled=True, period_s=0.005):
+        import threading
         self.samples = []
+        self._stop = threading.Event()
+        self._thread = None
+        self.handle = None
         if not enabled:
             return
-        sel = []
         try:
-            uuid = torch.cuda.get_device_properties(device).uuid
-            sel = ["-i", "GPU-" + str(uuid)]
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.nvml = pynvml
         except Exception:
-            sel = []
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                                          "-lms", "100"] + sel, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                                         text=True)
-        except Exception:
-            self.proc = None
+            self.handle = None
+            return
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    sm = self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
+                    rs = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                    self.samples.append((sm, rs))
+                except Exception:
+                    pass
+                self._stop.wait(period_s)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except Exception:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        for line in out.splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 10:
-                continue
-            try:
-                self.samples.append(dict(sm=float(f[2]), smax=float(f[3]), power=float(f[4]),
-                                         hw=f[6], hwt=f[7], swt=f[8], pcap=f[9]))
-            except ValueError:
-                continue
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
 
     def summary(self):
         if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        reasons = set()
-        for s in self.samples:
-            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
-                              ("pcap", "sw_power_cap")):
-                if s[key].lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(s["sm"] for s in self.samples),
-                "sm_max_mhz": max(s["smax"] for s in self.samples), "reasons": sorted(reasons),
-                "samples": len(self.samples)}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "nvml"}
+        reasons = sorted({name for _, rs in self.samples for name, bit in self.REASONS if rs & bit})
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.smax,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
 
 def dist_setup(args):

@@ -17,6 +17,7 @@
 
 #include "chunk_ffma.cuh"
 #include "chunk_tc.cuh"
+#include "scan_tc.cuh"
 #include "scan_seq.cuh"
 #include "step.cuh"
 
@@ -125,20 +126,36 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 4-D bf16 tensor map over [B, T, H, width] (dims listed innermost first), box
-// {box0, 1, 64 tokens, 1}. The token dimension is its own dimension, so a box
+// {box0, 1, box_tokens, 1}. The token dimension is its own dimension, so a box
 // that runs past T reads zeros instead of the next sequence.
 int make_token_map(CUtensorMap* m, const void* base, int B, int T, int H, int width, int box0,
-                   CUtensorMapSwizzle swizzle) {
+                   CUtensorMapSwizzle swizzle, int box_tokens = 64) {
     auto enc = tensor_map_encoder();
     if (!enc) return fail(OSDN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const cuuint64_t dims[4] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)width * 2, (cuuint64_t)H * width * 2, (cuuint64_t)T * H * width * 2};
-    const cuuint32_t box[4] = {(cuuint32_t)box0, 1, 64, 1};
+    const cuuint32_t box[4] = {(cuuint32_t)box0, 1, (cuuint32_t)box_tokens, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(OSDN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return OSDN_OK;
+}
+
+// Phase 1 in chunk form on the tensor cores: bf16, dk = 128.
+int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bfloat16* beta,
+                   const __nv_bfloat16* r, const float* d0, float* final_d, __nv_bfloat16* kw, cudaStream_t st) {
+    CUtensorMap mk;
+    int rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128);
+    if (rc) return rc;
+    auto kern = osdn::scan_tc_kernel<0>;
+    const size_t smem = osdn::ScanSmem::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan kernel attribute");
+    kern<<<p->B * p->H, 128, smem, st>>>(mk, beta, r, d0, kw, final_d, p->B, p->T, p->H, p->eta,
+                                         g_wait_limit_ns.load());
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");
     return OSDN_OK;
 }
 
@@ -167,6 +184,9 @@ template <typename Tin>
 int launch_scan(const osdn_params* p, const Tin* k, const Tin* beta, const Tin* r, const float* d0, float* final_d,
                 Tin* kw, cudaStream_t st) {
     if (p->T == 0) return copy_initial_state(p, d0, nullptr, nullptr, final_d, false, true, st);
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
+        if (p->dk == 128) return launch_scan_tc(p, k, beta, r, d0, final_d, kw, st);
+    }
     const int units = p->B * p->H;
     const dim3 grid((units + 3) / 4);
     if (p->dk == 128)
