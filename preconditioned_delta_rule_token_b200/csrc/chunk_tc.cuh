@@ -36,7 +36,7 @@ namespace osdn {
 
 struct TcSmem {
     static constexpr uint32_t QK = 0;                 // [K;Q] K-halves of 16 KB: K rows (8 KB) then Q rows (8 KB)
-    static constexpr uint32_t KW = 32768;             // scaled keys, two K-halves of 8 KB
+    static constexpr uint32_t KW = 32768;             // scaled keys (even chunks), two K-halves of 8 KB
     static constexpr uint32_t V = 49152;              // V [64 t][128 v] bf16, unswizzled
     static constexpr uint32_t SB = 65536;             // S bf16 [128 v][128 i], two K-halves of 16 KB
     static constexpr uint32_t XU = 98304;             // Xh^T, then U^T: [128 v][64 t] bf16
@@ -45,7 +45,9 @@ struct TcSmem {
     static constexpr int LDF = tri::LD;               // fp32 row stride of A and T
     static constexpr uint32_t AF = 131072;            // A fp32 [64][LDF]
     static constexpr uint32_t TF = AF + 64 * LDF * 4;  // T fp32 [64][LDF]
-    static constexpr uint32_t BETA = TF + 64 * LDF * 4;
+    static constexpr uint32_t KW1 = 165888;           // second scaled-key buffer (odd chunks)
+    static constexpr uint32_t OS = KW1 + 16384;       // O [64 t][128 v] bf16 staging for the TMA store
+    static constexpr uint32_t BETA = OS + 16384;
     static constexpr uint32_t BAR = BETA + 256;       // tma_bar, mma_bar, tmem base address
     static constexpr uint32_t END = BAR + 64;
     static constexpr size_t kBytes = END + 1024;      // + slack to align the base to 1024
@@ -56,8 +58,8 @@ template <int kUnused = 0>
 __global__ void __launch_bounds__(128, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_v,
-                const __nv_bfloat16* __restrict__ beta, const float* __restrict__ S0,
-                __nv_bfloat16* __restrict__ out, float* __restrict__ S_final, int B, int T, int H,
+                const __grid_constant__ CUtensorMap tm_out, const __nv_bfloat16* __restrict__ beta,
+                const float* __restrict__ S0, float* __restrict__ S_final, int B, int T, int H,
                 unsigned long long wait_limit_ns)
 {
     constexpr int C = 64, DK = 128, DV = 128;
@@ -89,6 +91,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc::prefetch_tmap(&tm_k);
         tc::prefetch_tmap(&tm_kw);
         tc::prefetch_tmap(&tm_v);
+        tc::prefetch_tmap(&tm_out);
     }
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, NCOLS);
@@ -117,9 +120,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc::tmem_wait_st();
     }
 
+    // TMA of chunk ci: K, Q (two 64-column halves each) into the [K;Q] tile, its
+    // scaled keys into the buffer of its parity, V
+    auto issue_loads = [&](int ci) {
+        const int tt = ci * C;
+        const uint32_t kwb = (ci & 1) ? L::KW1 : L::KW;
+        tc::mbar_arrive_expect_tx(tma_bar, L::kTxBytes);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            tc::tma_load_4d(sm + L::QK + half * 16384, &tm_k, half * 64, h, tt, b, tma_bar);
+            tc::tma_load_4d(sm + L::QK + half * 16384 + 8192, &tm_q, half * 64, h, tt, b, tma_bar);
+            tc::tma_load_4d(sm + kwb + half * 8192, &tm_kw, half * 64, h, tt, b, tma_bar);
+        }
+        tc::tma_load_4d(sm + L::V, &tm_v, 0, h, tt, b, tma_bar);
+    };
     uint32_t tma_phase = 0, mma_phase = 0;
-    bool failed = false, tma_pending = false, mma_pending = false;
     const int nchunks = (T + C - 1) / C;
+    bool failed = false, tma_pending = nchunks > 0, mma_pending = false;
+    if (tid == 0 && nchunks > 0) issue_loads(0);
     for (int ci = 0; ci < nchunks; ++ci) {
         const int t0 = ci * C, Tc = min(C, T - t0);
 
@@ -148,18 +166,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc::tc_fence_before();
         __syncthreads();
 
-        // (1) TMA: K, Q, Kw (two 64-column halves each) and V for this chunk
-        if (tid == 0) {
-            tc::mbar_arrive_expect_tx(tma_bar, L::kTxBytes);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tc::tma_load_4d(sm + L::QK + half * 16384, &tm_k, half * 64, h, t0, b, tma_bar);
-                tc::tma_load_4d(sm + L::QK + half * 16384 + 8192, &tm_q, half * 64, h, t0, b, tma_bar);
-                tc::tma_load_4d(sm + L::KW + half * 8192, &tm_kw, half * 64, h, t0, b, tma_bar);
-            }
-            tc::tma_load_4d(sm + L::V, &tm_v, 0, h, t0, b, tma_bar);
-        }
-        tma_pending = true;
+        // (1) this chunk's tiles (issued in the prologue or after the previous chunk's MMA1/MMA2 epilogue)
+        const uint32_t KWc = (ci & 1) ? L::KW1 : L::KW;
         if (!tc::mbar_wait(tma_bar, tma_phase, wait_limit_ns)) failed = true;
         else { tma_phase ^= 1; tma_pending = false; }
         if (__syncthreads_or(failed)) break;
@@ -171,7 +179,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t half = ks >> 2, koff = (ks & 3) * 32;
                 tc::umma_bf16(tmem + COL_D1, tc::sdesc_sw128(sb + L::QK + half * 16384 + koff, 16, 1024),
-                              tc::sdesc_sw128(sb + L::KW + half * 8192 + koff, 16, 1024), ID_N64, ks > 0);
+                              tc::sdesc_sw128(sb + KWc + half * 8192 + koff, 16, 1024), ID_N64, ks > 0);
             }
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
@@ -240,6 +248,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         __syncthreads();
+        // Q, K and V of this chunk are consumed (MMA1, MMA2 done, V read): start the next chunk's loads
+        if (tid == 0 && ci + 1 < nchunks) issue_loads(ci + 1);
+        tma_pending = ci + 1 < nchunks;
 
         // (4) T = (I + A)^{-1}: blocked 16 x 16 inverse (fp32 diagonal blocks, tf32 block products)
         tri::tril_inv64(AF, TF, warp, tid & 31, [] { __syncthreads(); });
@@ -305,7 +316,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 tc::umma_bf16(tmem + COL_S, tc::sdesc_sw128(sb + L::XU + ks * 32, 16, 1024),
-                              tc::sdesc_sw128(sb + L::KW + ks * 2048, 8192, 1024), ID_N128_BMN, true);
+                              tc::sdesc_sw128(sb + KWc + ks * 2048, 8192, 1024), ID_N128_BMN, true);
             tc::umma_commit(mma_bar);
         }
         mma_pending = true;
@@ -314,23 +325,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (__syncthreads_or(failed)) break;
         tc::tc_fence_after();
 
-        // (8) O^T row v -> out[b, t0 + t, h, v]
+        // (8) O^T row v -> staging O[t][v] -> TMA store of the chunk (rows past T clipped)
+        if (tid == 0) tc::bulk_wait_read<0>();   // the previous chunk's store has left the staging tile
+        __syncthreads();
         {
+            __nv_bfloat16* Os = reinterpret_cast<__nv_bfloat16*>(sm + L::OS);
             uint32_t r[32];
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 tc::tmem_ld32(tl + COL_D2 + 64 + q * 32, r);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int t = q * 32 + e;
-                    if (t < Tc) out[(((size_t)b * T + t0 + t) * H + h) * DV + v] = __float2bfloat16_rn(__uint_as_float(r[e]));
-                }
+                for (int e = 0; e < 32; ++e) Os[(q * 32 + e) * DV + v] = __float2bfloat16_rn(__uint_as_float(r[e]));
             }
         }
+        tc::fence_proxy_async_smem();
         tc::tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc::tma_store_4d(&tm_out, sm + L::OS, 0, h, t0, b);
+            tc::bulk_commit();
+        }
     }
 
+    if (tid == 0) tc::bulk_wait<0>();
     if (!failed && S_final) {
         tc::tc_fence_after();
         float* srow = S_final + ((size_t)unit * DV + v) * DK;

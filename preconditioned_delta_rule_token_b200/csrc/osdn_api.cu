@@ -146,14 +146,16 @@ int make_token_map(CUtensorMap* m, const void* base, int B, int T, int H, int wi
 // Phase 1 in chunk form on the tensor cores: bf16, dk = 128.
 int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bfloat16* beta,
                    const __nv_bfloat16* r, const float* d0, float* final_d, __nv_bfloat16* kw, cudaStream_t st) {
-    CUtensorMap mk;
+    CUtensorMap mk, mkw;
     int rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128);
+    if (rc) return rc;
+    rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128);
     if (rc) return rc;
     auto kern = osdn::scan_tc_kernel<0>;
     const size_t smem = osdn::ScanSmem::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan kernel attribute");
-    kern<<<p->B * p->H, 128, smem, st>>>(mk, beta, r, d0, kw, final_d, p->B, p->T, p->H, p->eta,
+    kern<<<p->B * p->H, 128, smem, st>>>(mk, mkw, beta, r, d0, final_d, p->B, p->T, p->H, p->eta,
                                          g_wait_limit_ns.load());
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");
     return OSDN_OK;
@@ -163,17 +165,18 @@ int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bflo
 int launch_chunk_tc(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                     const __nv_bfloat16* beta, const float* S0, __nv_bfloat16* out, float* final_S,
                     const __nv_bfloat16* kw, cudaStream_t st) {
-    CUtensorMap mq, mk, mkw, mv;
+    CUtensorMap mq, mk, mkw, mv, mo;
     int rc;
     if ((rc = make_token_map(&mq, q, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
     if ((rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
     if ((rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
     if ((rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
+    if ((rc = make_token_map(&mo, out, p->B, p->T, p->H, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
     auto kern = osdn::chunk_tc_kernel<0>;
     const size_t smem = osdn::TcSmem::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk kernel attribute");
-    kern<<<p->B * p->H, 128, smem, st>>>(mq, mk, mkw, mv, beta, S0, out, final_S, p->B, p->T, p->H,
+    kern<<<p->B * p->H, 128, smem, st>>>(mq, mk, mkw, mv, mo, beta, S0, final_S, p->B, p->T, p->H,
                                          g_wait_limit_ns.load());
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core chunk launch");
     return OSDN_OK;

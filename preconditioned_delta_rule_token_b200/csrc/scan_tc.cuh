@@ -19,8 +19,10 @@
 //   thread t builds row t of M (decay products walked right to left);
 //   per sub-chunk: N = (I + M)^{-1} (blocked inverse), b_t = <d_c, a_t>,
 //   x = N c, then thread i runs feature i through the sub-chunk, writing
-//   kw_t[i] = d_t[i] k_t[i] and carrying d to the next sub-chunk.
-// Bounded mbarrier waits as in the chunk kernel.
+//   kw_t[i] = d_t[i] k_t[i] over k_t[i] and carrying d to the next sub-chunk.
+// K blocks are double-buffered (the next block loads while this one is
+// processed); the scaled keys overwrite K in shared memory and leave with one
+// TMA store per block. Bounded mbarrier waits as in the chunk kernel.
 #pragma once
 #include "tc_ptx.cuh"
 #include "tril_inv.cuh"
@@ -28,17 +30,18 @@
 namespace osdn {
 
 struct ScanSmem {
-    static constexpr uint32_t KS = 0;                     // K block [128 t][128 i] bf16, two 16 KB halves
-    static constexpr uint32_t AS = 32768;                 // a = k^2 (bf16), same layout
-    static constexpr uint32_t US = 65536;                 // u = a / ||k||^2 (bf16), same layout
+    static constexpr uint32_t KS = 0;                     // two K blocks [128 t][128 i] bf16 (two 16 KB halves
+                                                          // each); the scaled keys overwrite K in place
+    static constexpr uint32_t AS = 65536;                 // a = k^2 (bf16), same layout
+    static constexpr uint32_t US = 98304;                 // u = a / ||k||^2 (bf16), same layout
     static constexpr int LD = tri::LD;
-    static constexpr uint32_t MF = 98304;                 // M, two sub-chunks [64][LD] fp32
+    static constexpr uint32_t MF = 131072;                // M, two sub-chunks [64][LD] fp32
     static constexpr uint32_t NF = MF + 2 * 64 * LD * 4;  // N [64][LD] fp32
     static constexpr uint32_t VEC = NF + 64 * LD * 4;     // per-token / per-feature vectors
     // vector slots (floats), each 128 long
     static constexpr int V_BETA = 0, V_R = 128, V_G = 256, V_INVN = 384, V_R0 = 512, V_C = 640, V_X = 768,
                          V_D = 896, V_N = 1024;
-    static constexpr uint32_t BAR = VEC + V_N * 4;
+    static constexpr uint32_t BAR = VEC + V_N * 4;        // tma_bar[2], mma_bar, tmem base address
     static constexpr uint32_t END = BAR + 64;
     static constexpr size_t kBytes = END + 1024;
     static constexpr uint32_t kTxBytes = 2 * 16384;
@@ -46,9 +49,10 @@ struct ScanSmem {
 
 template <int kUnused = 0>
 __global__ void __launch_bounds__(128, 1)
-scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restrict__ beta,
-               const __nv_bfloat16* __restrict__ r, const float* __restrict__ d0, __nv_bfloat16* __restrict__ kw,
-               float* __restrict__ d_final, int B, int T, int H, float eta, unsigned long long wait_limit_ns)
+scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kw,
+               const __nv_bfloat16* __restrict__ beta, const __nv_bfloat16* __restrict__ r,
+               const float* __restrict__ d0, float* __restrict__ d_final, int B, int T, int H, float eta,
+               unsigned long long wait_limit_ns)
 {
     constexpr int DK = 128, BLK = 128, SUB = 64;
     constexpr uint32_t NCOLS = 128;
@@ -69,18 +73,25 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __
     float* s_c = vec + L::V_C;
     float* s_x = vec + L::V_X;
     float* s_d = vec + L::V_D;
-    uint64_t* tma_bar = reinterpret_cast<uint64_t*>(sm + L::BAR);
-    uint64_t* mma_bar = tma_bar + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tma_bar + 2);
+    uint64_t* tma_bar = reinterpret_cast<uint64_t*>(sm + L::BAR);   // one per K buffer
+    uint64_t* mma_bar = tma_bar + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tma_bar + 3);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int unit = blockIdx.x, b = unit / H, h = unit % H;
 
     if (tid == 0) {
         tc::mbar_init(tma_bar, 1);
+        tc::mbar_init(tma_bar + 1, 1);
         tc::mbar_init(mma_bar, 1);
         tc::fence_mbar_init();
         tc::prefetch_tmap(&tm_k);
+        tc::prefetch_tmap(&tm_kw);
+        if (T > 0) {   // first K block
+            tc::mbar_arrive_expect_tx(tma_bar, L::kTxBytes);
+            tc::tma_load_4d(sm + L::KS, &tm_k, 0, h, 0, b, tma_bar);
+            tc::tma_load_4d(sm + L::KS + 16384, &tm_k, 64, h, 0, b, tma_bar);
+        }
     }
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, NCOLS);
@@ -93,32 +104,30 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
 
-    // element i of K row t in the swizzled block
-    auto kelem = [&](int t, int i) -> float {
-        const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(
-            sm + L::KS + (i >> 6) * 16384 + tc::sw128_off(t, (i & 63) >> 3));
-        return __bfloat162float(p[i & 7]);
-    };
-
-    uint32_t tma_phase = 0, mma_phase = 0;
-    bool failed = false, tma_pending = false, mma_pending = false;
-    for (int t0 = 0; t0 < T; t0 += BLK) {
+    uint32_t tma_phase = 0, mma_phase = 0;     // tma_phase: bit per K buffer
+    bool failed = false, tma_pending = (T > 0), mma_pending = false;
+    for (int t0 = 0, blk = 0; t0 < T; t0 += BLK, ++blk) {
         const int Tb = min(BLK, T - t0);
-        // (1) TMA: K block; beta and r
-        if (tid == 0) {
-            tc::mbar_arrive_expect_tx(tma_bar, L::kTxBytes);
-            tc::tma_load_4d(sm + L::KS, &tm_k, 0, h, t0, b, tma_bar);
-            tc::tma_load_4d(sm + L::KS + 16384, &tm_k, 64, h, t0, b, tma_bar);
+        const int buf = blk & 1;
+        uint8_t* KS = sm + L::KS + buf * 32768;
+        // (1) prefetch the next K block into the other buffer once the store of
+        //     the block it held has finished reading it; beta and r of this block
+        if (tid == 0 && t0 + BLK < T) {
+            tc::bulk_wait_read<0>();
+            uint64_t* nb = tma_bar + (buf ^ 1);
+            uint8_t* nK = sm + L::KS + (buf ^ 1) * 32768;
+            tc::mbar_arrive_expect_tx(nb, L::kTxBytes);
+            tc::tma_load_4d(nK, &tm_k, 0, h, t0 + BLK, b, nb);
+            tc::tma_load_4d(nK + 16384, &tm_k, 64, h, t0 + BLK, b, nb);
         }
-        tma_pending = true;
         {
             const bool in = tid < Tb;
             const size_t tok = ((size_t)b * T + t0 + tid) * H + h;
             s_beta[tid] = in ? __bfloat162float(beta[tok]) : 0.f;
             s_r[tid] = (in && r) ? __bfloat162float(r[tok]) : 1.f;
         }
-        if (!tc::mbar_wait(tma_bar, tma_phase, wait_limit_ns)) failed = true;
-        else { tma_phase ^= 1; tma_pending = false; }
+        if (!tc::mbar_wait(tma_bar + buf, (tma_phase >> buf) & 1, wait_limit_ns)) failed = true;
+        else { tma_phase ^= 1u << buf; tma_pending = (t0 + BLK < T); }
         if (__syncthreads_or(failed)) break;
 
         // (2) thread t: a_t = k_t^2 and u_t = a_t / ||k_t||^2 as bf16 MMA operands
@@ -129,7 +138,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __
             for (int half = 0; half < 2; ++half)
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint4 raw = *reinterpret_cast<const uint4*>(sm + L::KS + half * 16384 + tc::sw128_off(t, c));
+                    const uint4 raw = *reinterpret_cast<const uint4*>(KS + half * 16384 + tc::sw128_off(t, c));
                     const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -146,7 +155,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const uint32_t off = half * 16384 + tc::sw128_off(t, c);
-                    const uint4 raw = *reinterpret_cast<const uint4*>(sm + L::KS + off);
+                    const uint4 raw = *reinterpret_cast<const uint4*>(KS + off);
                     const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
                     uint4 pa, pu;
                     uint32_t* wa = reinterpret_cast<uint32_t*>(&pa);
@@ -221,7 +230,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __
                 float acc = 0.f;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint4 raw = *reinterpret_cast<const uint4*>(sm + L::KS + half * 16384 + tc::sw128_off(t, c));
+                    const uint4 raw = *reinterpret_cast<const uint4*>(KS + half * 16384 + tc::sw128_off(t, c));
                     const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
                     const float* dd = s_d + half * 64 + c * 8;
 #pragma unroll
@@ -243,29 +252,52 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __
 #pragma unroll
                 for (int k2 = 0; k2 < 32; ++k2) acc = fmaf(Nrow[k2], cc[k2], acc);
                 acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                if (half == 0) s_x[s * SUB + tl_] = acc;
+                if (half == 0) s_x[s * SUB + tl_] = acc * s_invn[s * SUB + tl_];   // x_t / ||k_t||^2
             }
             __syncthreads();
-            {   // feature i through the sub-chunk: kw_t = d_t (.) k_t, d_{t+1} = r_t d_t + x_t u_t
+            {   // feature i through the sub-chunk: kw_t = d_t (.) k_t written over k_t in place,
+                // d_{t+1} = r_t d_t + (x_t / ||k_t||^2) k_t^2
                 const int i = tid;
+                uint8_t* colbase = KS + (i >> 6) * 16384 + 2 * (i & 7);
+                const int cidx = (i & 63) >> 3;
+                uint32_t roff[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) roff[j] = j * 128 + ((cidx ^ j) << 4);
                 float d = s_d[i];
                 const int n = min(SUB, Tb - s * SUB);
-                for (int tl_ = 0; tl_ < n; ++tl_) {
-                    const int t = s * SUB + tl_;
-                    const float kv = kelem(t, i);
-                    kw[(((size_t)b * T + t0 + t) * H + h) * DK + i] = __float2bfloat16_rn(d * kv);
-                    d = fmaf(s_r[t], d, s_x[t] * (kv * kv * s_invn[t]));
+                for (int g = 0; g < n; g += 8) {
+                    const int t8 = s * SUB + g;
+                    uint8_t* rowbase = colbase + (t8 >> 3) * 1024;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (g + j < n) {
+                            __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(rowbase + roff[j]);
+                            const float kv = __bfloat162float(*p);
+                            *p = __float2bfloat16_rn(d * kv);
+                            d = fmaf(s_r[t8 + j], d, s_x[t8 + j] * (kv * kv));
+                        }
+                    }
                 }
                 s_d[i] = d;
             }
             __syncthreads();
         }
+        // (6) the block now holds the scaled keys: one TMA store (rows past T are clipped)
+        tc::fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc::tma_store_4d(&tm_kw, KS, 0, h, t0, b);
+            tc::tma_store_4d(&tm_kw, KS + 16384, 64, h, t0, b);
+            tc::bulk_commit();
+        }
     }
+    if (tid == 0) tc::bulk_wait<0>();
     if (!failed && d_final) d_final[(size_t)unit * DK + tid] = s_d[tid];
     if (failed && tid == 0) {
         atomicOr(&g_osdn_status, kStatusTimeout);
         const unsigned long long drain_ns = wait_limit_ns > 1000000000ull ? wait_limit_ns : 1000000000ull;
-        if (tma_pending) tc::mbar_wait(tma_bar, tma_phase, drain_ns);
+        for (int q = 0; q < 2; ++q)   // any K block still in flight
+            if (tma_pending) tc::mbar_wait(tma_bar + q, (tma_phase >> q) & 1, drain_ns);
         if (mma_pending) tc::mbar_wait(mma_bar, mma_phase, drain_ns);
     }
     tc::tc_fence_before();
