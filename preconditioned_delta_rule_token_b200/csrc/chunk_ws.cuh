@@ -101,7 +101,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     using L = WsSmem;
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays a shared pointer
     const uint32_t sb = tc::smem_u32(sm);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::TSLOT);

@@ -16,7 +16,6 @@
 #include "osdn.h"
 
 #include "chunk_ffma.cuh"
-#include "chunk_tc.cuh"
 #include "chunk_ws.cuh"
 #include "scan_tc.cuh"
 #include "scan_seq.cuh"
@@ -182,26 +181,6 @@ int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bflo
     return OSDN_OK;
 }
 
-// Phase 2 on the tensor cores: bf16, dk = dv = 128.
-int launch_chunk_tc(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                    const __nv_bfloat16* beta, const float* S0, __nv_bfloat16* out, float* final_S,
-                    const __nv_bfloat16* kw, cudaStream_t st) {
-    CUtensorMap mq, mk, mkw, mv, mo;
-    int rc;
-    if ((rc = make_token_map(&mq, q, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-    if ((rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-    if ((rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-    if ((rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
-    if ((rc = make_token_map(&mo, out, p->B, p->T, p->H, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
-    auto kern = osdn::chunk_tc_kernel<0>;
-    const size_t smem = osdn::TcSmem::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk kernel attribute");
-    kern<<<p->B * p->H, 128, smem, st>>>(mq, mk, mkw, mv, mo, beta, S0, final_S, p->B, p->T, p->H,
-                                         g_wait_limit_ns.load());
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core chunk launch");
-    return OSDN_OK;
-}
 
 // Phase 1: preconditioner scan -> scaled write keys (workspace) and final d.
 template <typename Tin>

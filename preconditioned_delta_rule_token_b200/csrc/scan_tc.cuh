@@ -60,7 +60,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     using L = ScanSmem;
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);   // stays a shared pointer
     const uint32_t sb = tc::smem_u32(sm);
     float* MF = reinterpret_cast<float*>(sm + L::MF);
     float* NF = reinterpret_cast<float*>(sm + L::NF);
