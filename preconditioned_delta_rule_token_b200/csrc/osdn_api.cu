@@ -147,17 +147,18 @@ int make_token_map(CUtensorMap* m, const void* base, int B, int T, int H, int wi
 int launch_chunk_ws(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                     const __nv_bfloat16* beta, const float* S0, __nv_bfloat16* out, float* final_S,
                     const __nv_bfloat16* kw, cudaStream_t st) {
-    CUtensorMap mq, mk, mkw, mo;
+    CUtensorMap mq, mk, mkw, mv, mo;
     int rc;
     if ((rc = make_token_map(&mq, q, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
     if ((rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
     if ((rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    if ((rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
     if ((rc = make_token_map(&mo, out, p->B, p->T, p->H, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
     auto kern = osdn::chunk_ws_kernel<0>;
     const size_t smem = osdn::WsSmem::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "warp-specialized chunk kernel attribute");
-    kern<<<p->B * p->H, 384, smem, st>>>(mq, mk, mkw, mo, v, beta, S0, final_S, p->B, p->T, p->H,
+    kern<<<p->B * p->H, 256, smem, st>>>(mq, mk, mkw, mv, mo, beta, S0, final_S, p->B, p->T, p->H,
                                          g_wait_limit_ns.load());
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "warp-specialized chunk launch");
     return OSDN_OK;
