@@ -20,8 +20,8 @@
 //   per sub-chunk: N = (I + M)^{-1} (blocked inverse), b_t = <d_c, a_t>,
 //   x = N c, then thread i runs feature i through the sub-chunk, writing
 //   kw_t[i] = d_t[i] k_t[i] over k_t[i] and carrying d to the next sub-chunk.
-// K blocks are double-buffered (the next block loads while this one is
-// processed); the scaled keys overwrite K in shared memory and leave with one
+// K blocks are triple-buffered (the next block loads while this one is
+// processed and the previous one's store drains); the scaled keys overwrite K in shared memory and leave with one
 // TMA store per block. Bounded mbarrier waits as in the chunk kernel.
 #pragma once
 #include "tc_ptx.cuh"
@@ -30,18 +30,20 @@
 namespace osdn {
 
 struct ScanSmem {
-    static constexpr uint32_t KS = 0;                     // two K blocks [128 t][128 i] bf16 (two 16 KB halves
+    static constexpr int NBUF = 3;                        // K blocks in flight: load b+1 while b is processed
+                                                          // and the store of b-1 drains
+    static constexpr uint32_t KS = 0;                     // K blocks [128 t][128 i] bf16 (two 16 KB halves
                                                           // each); the scaled keys overwrite K in place
-    static constexpr uint32_t AS = 65536;                 // a = k^2 (bf16), same layout
-    static constexpr uint32_t US = 98304;                 // u = a / ||k||^2 (bf16), same layout
+    static constexpr uint32_t AS = NBUF * 32768;          // a = k^2 (bf16), same layout
+    static constexpr uint32_t US = AS + 32768;            // u = a / ||k||^2 (bf16), same layout
     static constexpr int LD = tri::LD;
-    static constexpr uint32_t MF = 131072;                // M, two sub-chunks [64][LD] fp32
+    static constexpr uint32_t MF = US + 32768;            // M, two sub-chunks [64][LD] fp32
     static constexpr uint32_t NF = MF + 2 * 64 * LD * 4;  // N [64][LD] fp32
     static constexpr uint32_t VEC = NF + 64 * LD * 4;     // per-token / per-feature vectors
     // vector slots (floats), each 128 long
     static constexpr int V_BETA = 0, V_R = 128, V_G = 256, V_INVN = 384, V_R0 = 512, V_C = 640, V_X = 768,
                          V_D = 896, V_N = 1024;
-    static constexpr uint32_t BAR = VEC + V_N * 4;        // tma_bar[2], mma_bar, tmem base address
+    static constexpr uint32_t BAR = VEC + V_N * 4;        // tma_bar[NBUF], mma_bar, tmem base address
     static constexpr uint32_t END = BAR + 64;
     static constexpr size_t kBytes = END + 1024;
     static constexpr uint32_t kTxBytes = 2 * 16384;
@@ -74,15 +76,14 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     float* s_x = vec + L::V_X;
     float* s_d = vec + L::V_D;
     uint64_t* tma_bar = reinterpret_cast<uint64_t*>(sm + L::BAR);   // one per K buffer
-    uint64_t* mma_bar = tma_bar + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tma_bar + 3);
+    uint64_t* mma_bar = tma_bar + L::NBUF;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tma_bar + L::NBUF + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int unit = blockIdx.x, b = unit / H, h = unit % H;
 
     if (tid == 0) {
-        tc::mbar_init(tma_bar, 1);
-        tc::mbar_init(tma_bar + 1, 1);
+        for (int q = 0; q < L::NBUF; ++q) tc::mbar_init(tma_bar + q, 1);
         tc::mbar_init(mma_bar, 1);
         tc::fence_mbar_init();
         tc::prefetch_tmap(&tm_k);
@@ -108,14 +109,15 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     bool failed = false, tma_pending = (T > 0), mma_pending = false;
     for (int t0 = 0, blk = 0; t0 < T; t0 += BLK, ++blk) {
         const int Tb = min(BLK, T - t0);
-        const int buf = blk & 1;
+        const int buf = blk % L::NBUF;
         uint8_t* KS = sm + L::KS + buf * 32768;
-        // (1) prefetch the next K block into the other buffer once the store of
-        //     the block it held has finished reading it; beta and r of this block
+        // (1) prefetch the next K block into the buffer of block blk - 2 once that block's
+        //     store has read it (the store of blk - 1 may still be in flight); beta and r
         if (tid == 0 && t0 + BLK < T) {
-            tc::bulk_wait_read<0>();
-            uint64_t* nb = tma_bar + (buf ^ 1);
-            uint8_t* nK = sm + L::KS + (buf ^ 1) * 32768;
+            tc::bulk_wait_read<1>();
+            const int nbuf = (blk + 1) % L::NBUF;
+            uint64_t* nb = tma_bar + nbuf;
+            uint8_t* nK = sm + L::KS + nbuf * 32768;
             tc::mbar_arrive_expect_tx(nb, L::kTxBytes);
             tc::tma_load_4d(nK, &tm_k, 0, h, t0 + BLK, b, nb);
             tc::tma_load_4d(nK + 16384, &tm_k, 64, h, t0 + BLK, b, nb);
@@ -130,46 +132,41 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         else { tma_phase ^= 1u << buf; tma_pending = (t0 + BLK < T); }
         if (__syncthreads_or(failed)) break;
 
-        // (2) thread t: a_t = k_t^2 and u_t = a_t / ||k_t||^2 as bf16 MMA operands
+        // (2) thread t: a_t = k_t^2 and u_t = a_t / ||k_t||^2 as bf16 MMA operands (one read of row t)
         {
             const int t = tid;
+            uint4 raw[16];
             float nrm = 0.f;
 #pragma unroll
-            for (int half = 0; half < 2; ++half)
+            for (int q = 0; q < 16; ++q) {
+                raw[q] = *reinterpret_cast<const uint4*>(KS + (q >> 3) * 16384 + tc::sw128_off(t, q & 7));
+                const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[q]);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 raw = *reinterpret_cast<const uint4*>(KS + half * 16384 + tc::sw128_off(t, c));
-                    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(p2[e]);
-                        nrm = fmaf(f.x, f.x, nrm);
-                        nrm = fmaf(f.y, f.y, nrm);
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(p2[e]);
+                    nrm = fmaf(f.x, f.x, fmaf(f.y, f.y, nrm));
                 }
+            }
             const float invn = nrm > 0.f ? 1.f / nrm : 0.f;
             s_invn[t] = invn;
             s_g[t] = nrm > 0.f ? eta * s_beta[t] : 0.f;
 #pragma unroll
-            for (int half = 0; half < 2; ++half)
+            for (int q = 0; q < 16; ++q) {
+                const uint32_t off = (q >> 3) * 16384 + tc::sw128_off(t, q & 7);
+                const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[q]);
+                uint4 pa, pu;
+                uint32_t* wa = reinterpret_cast<uint32_t*>(&pa);
+                uint32_t* wu = reinterpret_cast<uint32_t*>(&pu);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t off = half * 16384 + tc::sw128_off(t, c);
-                    const uint4 raw = *reinterpret_cast<const uint4*>(KS + off);
-                    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-                    uint4 pa, pu;
-                    uint32_t* wa = reinterpret_cast<uint32_t*>(&pa);
-                    uint32_t* wu = reinterpret_cast<uint32_t*>(&pu);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(p2[e]);
-                        const float ax = f.x * f.x, ay = f.y * f.y;
-                        wa[e] = tc::pack_bf16(ax, ay);
-                        wu[e] = tc::pack_bf16(ax * invn, ay * invn);
-                    }
-                    *reinterpret_cast<uint4*>(sm + L::AS + off) = pa;
-                    *reinterpret_cast<uint4*>(sm + L::US + off) = pu;
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(p2[e]);
+                    const float ax = f.x * f.x, ay = f.y * f.y;
+                    wa[e] = tc::pack_bf16(ax, ay);
+                    wu[e] = tc::pack_bf16(ax * invn, ay * invn);
                 }
+                *reinterpret_cast<uint4*>(sm + L::AS + off) = pa;
+                *reinterpret_cast<uint4*>(sm + L::US + off) = pu;
+            }
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
@@ -208,15 +205,18 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             const float* rr = s_r + s * SUB;
             float* Mrow = MF + s * 64 * L::LD + tl_ * L::LD;
             float R = 1.f;                       // R_{tl, j+1}, walked from j = tl - 1 down
+            float m[SUB];
 #pragma unroll
             for (int j = SUB - 1; j >= 0; --j) {
-                float m = 0.f;
+                m[j] = 0.f;
                 if (j < tl_) {
-                    m = coef * R * __uint_as_float(gr[j]);
+                    m[j] = coef * R * __uint_as_float(gr[j]);
                     R *= rr[j];
                 }
-                Mrow[j] = m;
             }
+#pragma unroll
+            for (int j = 0; j < SUB; j += 4)   // row stride 68 floats: conflict-free 16-byte stores
+                *reinterpret_cast<float4*>(Mrow + j) = make_float4(m[j], m[j + 1], m[j + 2], m[j + 3]);
             s_R0[t] = R;                         // R_{tl, 0}
         }
         tc::tc_fence_before();
@@ -255,28 +255,39 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                 if (half == 0) s_x[s * SUB + tl_] = acc * s_invn[s * SUB + tl_];   // x_t / ||k_t||^2
             }
             __syncthreads();
-            {   // feature i through the sub-chunk: kw_t = d_t (.) k_t written over k_t in place,
-                // d_{t+1} = r_t d_t + (x_t / ||k_t||^2) k_t^2
+            {   // feature i through the sub-chunk, 32 tokens at a time from registers:
+                // kw_t = d_t (.) k_t written over k_t in place, d_{t+1} = r_t d_t + (x_t / ||k_t||^2) k_t^2.
+                // Tokens past T have k = 0, r = 1, x = 0 and leave d unchanged (their rows are not stored).
                 const int i = tid;
                 uint8_t* colbase = KS + (i >> 6) * 16384 + 2 * (i & 7);
                 const int cidx = (i & 63) >> 3;
-                uint32_t roff[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) roff[j] = j * 128 + ((cidx ^ j) << 4);
                 float d = s_d[i];
-                const int n = min(SUB, Tb - s * SUB);
-                for (int g = 0; g < n; g += 8) {
-                    const int t8 = s * SUB + g;
-                    uint8_t* rowbase = colbase + (t8 >> 3) * 1024;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        if (g + j < n) {
-                            __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(rowbase + roff[j]);
-                            const float kv = __bfloat162float(*p);
-                            *p = __float2bfloat16_rn(d * kv);
-                            d = fmaf(s_r[t8 + j], d, s_x[t8 + j] * (kv * kv));
-                        }
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int tb = s * SUB + hh * 32;                    // multiple of 8
+                    uint8_t* rowbase = colbase + (tb >> 3) * 1024;
+                    float kk[32], rr[32], xx[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        kk[j] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                            rowbase + (j >> 3) * 1024 + (j & 7) * 128 + ((cidx ^ (j & 7)) << 4)));
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 r4 = *reinterpret_cast<const float4*>(s_r + tb + j);
+                        const float4 x4 = *reinterpret_cast<const float4*>(s_x + tb + j);
+                        rr[j] = r4.x; rr[j + 1] = r4.y; rr[j + 2] = r4.z; rr[j + 3] = r4.w;
+                        xx[j] = x4.x; xx[j + 1] = x4.y; xx[j + 2] = x4.z; xx[j + 3] = x4.w;
                     }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float kv = kk[j];
+                        kk[j] = d * kv;                                  // scaled key, with d before token j
+                        d = fmaf(rr[j], d, xx[j] * (kv * kv));
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        *reinterpret_cast<__nv_bfloat16*>(rowbase + (j >> 3) * 1024 + (j & 7) * 128 +
+                                                          ((cidx ^ (j & 7)) << 4)) = __float2bfloat16_rn(kk[j]);
                 }
                 s_d[i] = d;
             }
@@ -296,7 +307,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     if (failed && tid == 0) {
         atomicOr(&g_osdn_status, kStatusTimeout);
         const unsigned long long drain_ns = wait_limit_ns > 1000000000ull ? wait_limit_ns : 1000000000ull;
-        for (int q = 0; q < 2; ++q)   // any K block still in flight
+        for (int q = 0; q < L::NBUF; ++q)   // any K block still in flight
             if (tma_pending) tc::mbar_wait(tma_bar + q, (tma_phase >> q) & 1, drain_ns);
         if (mma_pending) tc::mbar_wait(mma_bar, mma_phase, drain_ns);
     }
