@@ -197,11 +197,33 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         };
 
-        int issued = 0, seen = 0;   // chunks whose loads were issued / waited on (elected thread)
-        if (gtid == 0) {
+        // gtid 0 issues the MMAs, gtid 32 (another warp) the TMA loads and stores, so
+        // neither waits behind the other
+        constexpr int kMmaThread = 0, kTmaThread = 32;
+        int issued = 0;   // chunks whose loads were issued (TMA thread)
+        if (gtid == kTmaThread) {
             if (nchunks > 0) issue_loads(issued++);
             if (nchunks > 1) issue_loads(issued++);
         }
+        // MMA2(c): S K^T (commit) then S Q^T; A = bf16 state in TMEM, B = chunk c's [K;Q] tile
+        auto mma2 = [&](int c) -> bool {
+            const int sc = c & 1;
+            if (!wait(L::B_FULL + sc, (c >> 1) & 1)) return false;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                tc::umma_bf16_ts(tmem + COL_D2, tmem + COL_SB + ks * 8, dQK[sc] + (off >> 4), ID_N64, ks > 0);
+            }
+            tc::umma_commit(bars + L::B_D2);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                tc::umma_bf16_ts(tmem + COL_D2 + 64, tmem + COL_SB + ks * 8, dQK[sc] + ((off + 8192) >> 4), ID_N64,
+                                 ks > 0);
+            }
+            return true;
+        };
         {   // initial state: TMEM fp32 and its bf16 copy
             const float* srow = S0 ? S0 + ((size_t)unit * DV + vrow) * DK : nullptr;
             uint32_t row[128];
@@ -223,30 +245,12 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         float bnext = nchunks > 0 ? load_beta(0) : 0.f;
         tc::tc_fence_before();
         named_sync(GRP_CHAIN, 128);
+        if (gtid == kMmaThread && nchunks > 0) mma2(0);
 
         bool fail = false;
-        for (int c = 0; c < nchunks; ++c) {
+        int c = 0;
+        for (; c < nchunks; ++c) {
             const int s = c & 1, t0 = c * C;
-            // MMA2(c): S K^T (commit) then S Q^T; A = bf16 state in TMEM, B = this chunk's [K;Q] tile
-            if (gtid == 0) {
-                if (wait(L::B_FULL + s, (c >> 1) & 1)) {
-                    seen = c + 1;
-                    tc::tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        tc::umma_bf16_ts(tmem + COL_D2, tmem + COL_SB + ks * 8, dQK[s] + (off >> 4), ID_N64, ks > 0);
-                    }
-                    tc::umma_commit(bars + L::B_D2);
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        tc::umma_bf16_ts(tmem + COL_D2 + 64, tmem + COL_SB + ks * 8, dQK[s] + ((off + 8192) >> 4),
-                                         ID_N64, ks > 0);
-                    }
-                }
-                tc::bulk_wait_read<0>();   // the previous O store has left the staging tile
-            }
             if (gtid < C) betac[gtid] = bnext;
             if (c + 1 < nchunks) bnext = load_beta(c + 1);
 
@@ -274,7 +278,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tc::tc_fence_before();
             named_sync(GRP_CHAIN, 128);
-            if (gtid == 0) {
+            if (gtid == kMmaThread) {
                 if (wait(L::B_TPREADY + s, (c >> 1) & 1)) {
                     tc::tc_fence_after();
 #pragma unroll
@@ -301,7 +305,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tc::tc_fence_before();
             named_sync(GRP_CHAIN, 128);
-            if (gtid == 0) {
+            if (gtid == kMmaThread) {
                 tc::tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
@@ -336,6 +340,10 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                                            __uint_as_float(row[i + 2]), __uint_as_float(row[i + 3]));
                 }
             }
+            if (gtid == kTmaThread) tc::bulk_wait_read<0>();   // the previous O store has left the staging tile
+            tc::tc_fence_before();
+            named_sync(GRP_CHAIN, 128);
+            if (gtid == kMmaThread && c + 1 < nchunks) mma2(c + 1);   // the next chunk starts on the tensor core now
             {   // O[t][v] into the staging tile; one TMA store
                 unsigned short* Os = reinterpret_cast<unsigned short*>(sm + L::OST);
 #pragma unroll
@@ -345,20 +353,20 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
             tc::fence_proxy_async_smem();
-            tc::tc_fence_before();
             named_sync(GRP_CHAIN, 128);
-            if (gtid == 0) {
+            if (gtid == kTmaThread) {
                 tc::tma_store_4d(&tm_out, sm + L::OST, 0, h, t0, b);
                 tc::bulk_commit();
                 if (c + 2 < nchunks) issue_loads(issued++);   // stage s is consumed
             }
         }
-        if (gtid == 0) {
-            tc::bulk_wait<0>();
-            // drain every MMA this thread issued, and any load still in flight, before TMEM is released
+        if (gtid == kMmaThread) {   // drain every MMA this thread issued before TMEM is released
             tc::umma_commit(bars + L::B_DRAIN);
             tc::mbar_wait(bars + L::B_DRAIN, 0, 1000000000ull);
-            for (int cc = seen; cc < issued; ++cc)
+        }
+        if (gtid == kTmaThread) {   // stores done; loads of chunks the loop did not reach have landed
+            tc::bulk_wait<0>();
+            for (int cc = c; cc < issued; ++cc)
                 tc::mbar_wait(bars + L::B_FULL + (cc & 1), (cc >> 1) & 1, 1000000000ull);
         }
         tc::tc_fence_before();
@@ -390,6 +398,9 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         if (gtid == 0 && nchunks > 0) mma1(0);
         float bnext = nchunks > 0 ? load_beta(0) : 0.f;
+        tri::tril_zero_upper(TF, gtid, 128);   // the inverse never writes those blocks
+        named_sync(GRP_PREP, 128);
+        int mma1_next = 1;                     // next chunk whose MMA1 is not issued yet
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
             if (gtid < C) betap[gtid] = bnext;
@@ -402,12 +413,16 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 uint32_t r[32];
                 tc::tmem_ld32(tl + COL_D1 + s * 64 + qh * 32, r);
                 tc::tmem_wait_ld();
-                if (row < C) {   // A[t][j] = beta_t <k_t, kw_j> for j < t
+                if (row < C) {   // A[t][j] = beta_t <k_t, kw_j> for j < t (row stride 68: conflict-free 16-byte stores)
                     const float bt = betap[row];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
+                    for (int e = 0; e < 32; e += 4) {
                         const int j = qh * 32 + e;
-                        AF[row * L::LDF + j] = (j < row) ? bt * __uint_as_float(r[e]) : 0.f;
+                        *reinterpret_cast<float4*>(AF + row * L::LDF + j) =
+                            make_float4((j < row) ? bt * __uint_as_float(r[e]) : 0.f,
+                                        (j + 1 < row) ? bt * __uint_as_float(r[e + 1]) : 0.f,
+                                        (j + 2 < row) ? bt * __uint_as_float(r[e + 2]) : 0.f,
+                                        (j + 3 < row) ? bt * __uint_as_float(r[e + 3]) : 0.f);
                     }
                 } else {         // P[t][j] = <q_t, kw_j> for j <= t  (MMA4 of chunk c - 2 has read P[s])
                     const int t = row - C;
@@ -428,23 +443,34 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tc::tc_fence_before();
             named_sync(GRP_PREP, 128);
+            // MMA1 of the next chunk now if its tiles have landed (D1[(c+1) % 2] was read in chunk c - 1),
+            // so it runs under the inverse; otherwise after it
+            if (gtid == 0 && mma1_next == c + 1 && c + 1 < nchunks &&
+                tc::mbar_test(bars + L::B_FULL + ((c + 1) & 1), ((c + 1) >> 1) & 1)) {
+                mma1(c + 1);
+                mma1_next = c + 2;
+            }
             tri::tril_inv64(AF, TF, gw, lane, [] { named_sync(2, 128); });
-            if (gtid < C) {   // T -> bf16 K-major swizzled (B operand of MMA3)
-                const int t = gtid;
+            {   // T -> bf16 K-major swizzled (B operand of MMA3): thread -> half a row
+                const int t = gtid & 63, hf = gtid >> 6;
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
+                for (int cc = 0; cc < 4; ++cc) {
+                    const float4 lo = *reinterpret_cast<const float4*>(TF + t * L::LDF + hf * 32 + cc * 8);
+                    const float4 hi = *reinterpret_cast<const float4*>(TF + t * L::LDF + hf * 32 + cc * 8 + 4);
                     uint4 pk;
-                    const float* rw = TF + t * L::LDF + cc * 8;
-                    pk.x = tc::pack_bf16(rw[0], rw[1]); pk.y = tc::pack_bf16(rw[2], rw[3]);
-                    pk.z = tc::pack_bf16(rw[4], rw[5]); pk.w = tc::pack_bf16(rw[6], rw[7]);
-                    *reinterpret_cast<uint4*>(sm + L::TB + s * 8192 + tc::sw128_off(t, cc)) = pk;
+                    pk.x = tc::pack_bf16(lo.x, lo.y); pk.y = tc::pack_bf16(lo.z, lo.w);
+                    pk.z = tc::pack_bf16(hi.x, hi.y); pk.w = tc::pack_bf16(hi.z, hi.w);
+                    *reinterpret_cast<uint4*>(sm + L::TB + s * 8192 + tc::sw128_off(t, hf * 4 + cc)) = pk;
                 }
             }
             tc::fence_proxy_async_smem();
             named_sync(GRP_PREP, 128);
             if (gtid == 0) {
                 mbar_arrive1(bars + L::B_TPREADY + s);
-                if (c + 1 < nchunks) mma1(c + 1);   // D1[(c+1) % 2] was read in chunk c - 1
+                if (mma1_next == c + 1 && c + 1 < nchunks) {
+                    mma1(c + 1);
+                    mma1_next = c + 2;
+                }
             }
         }
         if (gtid == 0) {   // drain this thread's MMAs

@@ -99,6 +99,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tc::tmem_relinquish();
     }
     s_d[tid] = d0 ? d0[(size_t)unit * DK + tid] : 1.f;
+    tri::tril_zero_upper(NF, tid, 128);   // the inverse never writes those blocks
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();

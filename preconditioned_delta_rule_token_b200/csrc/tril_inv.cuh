@@ -13,8 +13,10 @@
 // Executed by the 128 threads (4 warps) of one group; sync() must be a barrier
 // over exactly those threads. A and T are fp32 in shared memory with row
 // stride LD (68 keeps the fragment loads free of bank conflicts); T may not
-// alias A. On return T holds the full 64 x 64 inverse (zeros above the
-// diagonal) and every thread of the group has passed a final sync().
+// alias A. The blocks of T above the diagonal blocks are never written: the
+// caller zeroes them once (tril_zero_upper) before the first call. On return T
+// holds the full 64 x 64 inverse and every thread of the group has passed a
+// final sync().
 #pragma once
 #include "common.cuh"
 
@@ -77,12 +79,20 @@ __device__ __forceinline__ void blk_store(float* D, const float (&c)[2][4], floa
     }
 }
 
+// Zero the 16 x 16 blocks of T above its diagonal blocks (threads `tid` of `n`).
+__device__ __forceinline__ void tril_zero_upper(float* T, int tid, int n) {
+    for (int idx = tid; idx < 64 * 64; idx += n) {
+        const int r = idx >> 6, c = idx & 63;
+        if ((c >> 4) > (r >> 4)) T[r * LD + c] = 0.f;
+    }
+}
+
 template <class Sync>
 __device__ __forceinline__ void tril_inv64(const float* A, float* T, int warp, int lane, Sync sync) {
     auto blkA = [&](int i, int j) { return A + (i * 16) * LD + j * 16; };
     auto blkT = [&](int i, int j) { return T + (i * 16) * LD + j * 16; };
 
-    {   // level 0: diagonal block `warp`, lane j (< 16) owns column j; zero the rest of the block row
+    {   // level 0: diagonal block `warp`, lane j (< 16) owns column j
         const int j = lane & 15, o = warp * 16;
         float c[16];
 #pragma unroll
@@ -100,11 +110,6 @@ __device__ __forceinline__ void tril_inv64(const float* A, float* T, int warp, i
         if (lane < 16) {
 #pragma unroll
             for (int t = 0; t < 16; ++t) T[(o + t) * LD + o + j] = c[t];
-        }
-        // zeros above the diagonal blocks: row block `warp`, column blocks > warp
-        for (int idx = lane; idx < 16 * 48; idx += 32) {
-            const int r = idx / 48, cc = idx % 48;
-            if (o + 16 + cc < 64) T[(o + r) * LD + o + 16 + cc] = 0.f;
         }
     }
     sync();
