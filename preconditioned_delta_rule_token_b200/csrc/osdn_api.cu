@@ -16,7 +16,7 @@
 #include "osdn.h"
 
 #include "chunk_ffma.cuh"
-#include "chunk_ws.cuh"
+#include "chunk_wy.cuh"
 #include "scan_tc.cuh"
 #include "scan_seq.cuh"
 #include "step.cuh"
@@ -143,8 +143,8 @@ int make_token_map(CUtensorMap* m, const void* base, int B, int T, int H, int wi
     return OSDN_OK;
 }
 
-// Phase 2, warp-specialized tensor-core kernel: bf16, dk = dv = 128.
-int launch_chunk_ws(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+// Phase 2 on the tensor cores (WY form, state chain fed by prepared W and U0): bf16, dk = dv = 128.
+int launch_chunk_wy(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                     const __nv_bfloat16* beta, const float* S0, __nv_bfloat16* out, float* final_S,
                     const __nv_bfloat16* kw, cudaStream_t st) {
     CUtensorMap mq, mk, mkw, mv, mo;
@@ -152,15 +152,15 @@ int launch_chunk_ws(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfl
     if ((rc = make_token_map(&mq, q, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
     if ((rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
     if ((rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-    if ((rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
-    if ((rc = make_token_map(&mo, out, p->B, p->T, p->H, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
-    auto kern = osdn::chunk_ws_kernel<0>;
-    const size_t smem = osdn::WsSmem::kBytes;
+    if ((rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    if ((rc = make_token_map(&mo, out, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    auto kern = osdn::chunk_wy_kernel<0>;
+    const size_t smem = osdn::WyLayout::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "warp-specialized chunk kernel attribute");
-    kern<<<p->B * p->H, 256, smem, st>>>(mq, mk, mkw, mv, mo, beta, S0, final_S, p->B, p->T, p->H,
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk kernel attribute");
+    kern<<<p->B * p->H, 288, smem, st>>>(mq, mk, mkw, mv, mo, beta, S0, final_S, p->B, p->T, p->H,
                                          g_wait_limit_ns.load());
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "warp-specialized chunk launch");
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core chunk launch");
     return OSDN_OK;
 }
 
@@ -208,7 +208,7 @@ int launch_chunk(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v,
                  Tin* out, float* final_S, const Tin* kw, cudaStream_t st) {
     if (p->T == 0) return copy_initial_state(p, nullptr, S0, final_S, nullptr, true, false, st);
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
-        if (p->dk == 128 && p->dv == 128) return launch_chunk_ws(p, q, k, v, beta, S0, out, final_S, kw, st);
+        if (p->dk == 128 && p->dv == 128) return launch_chunk_wy(p, q, k, v, beta, S0, out, final_S, kw, st);
     }
     const int units = p->B * p->H;
     constexpr int DVT = 64;

@@ -154,5 +154,89 @@ __device__ __forceinline__ void tril_inv64(const float* A, float* T, int warp, i
     sync();
 }
 
+// Forward substitution for column j of (I + L)^{-1}, L the strictly lower
+// 16 x 16 block at Lb (row stride LD). Row t's entries 0..t-1 are read with
+// 16-byte loads: row starts are 16-byte aligned (LD * 4 and the block offsets
+// are multiples of 16 bytes, the matrix base is 16-byte aligned).
+__device__ __forceinline__ void diag16_inverse_column(const float* Lb, int j, float (&c)[16]) {
+#pragma unroll
+    for (int t = 0; t < 16; ++t) c[t] = (t == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int t = 1; t < 16; ++t) {
+        float l[16];
+#pragma unroll
+        for (int m4 = 0; m4 < t; m4 += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(Lb + t * LD + m4);
+            l[m4] = x.x; l[m4 + 1] = x.y; l[m4 + 2] = x.z; l[m4 + 3] = x.w;
+        }
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int m = 0; m < t; m += 2) {
+            s0 = fmaf(l[m], c[m], s0);
+            if (m + 1 < t) s1 = fmaf(l[m + 1], c[m + 1], s1);
+        }
+        if (t > j) c[t] = -(s0 + s1);
+    }
+}
+
+// In-place variant: on entry A holds the strictly lower 64 x 64 matrix (every
+// entry on and above the diagonal zero, the blocks above the diagonal blocks
+// included); on return it holds T = (I + A)^{-1}. Same blocking and arithmetic
+// as tril_inv64; each level computes its blocks into registers before any
+// warp overwrites an operand another warp still reads.
+template <class Sync>
+__device__ __forceinline__ void tril_inv64_inplace(float* A, int warp, int lane, Sync sync) {
+    auto blk = [&](int i, int j) { return A + (i * 16) * LD + j * 16; };
+    {   // level 0: diagonal block `warp`
+        const int j = lane & 15;
+        float c[16];
+        diag16_inverse_column(blk(warp, warp), j, c);
+        __syncwarp();
+        if (lane < 16) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) blk(warp, warp)[t * LD + j] = c[t];
+        }
+    }
+    sync();
+    if (warp < 2) {   // level 1: T_10 and T_32 (each warp owns its block)
+        const int i = warp * 2 + 1, j = warp * 2;
+        float c[2][4];
+        blk_zero(c);
+        blk_mma(c, blk(i, j), blk(j, j), lane);       // W = A_ij T_jj
+        __syncwarp();
+        blk_store(blk(i, j), c, 1.f, lane);
+        __syncwarp();
+        blk_zero(c);
+        blk_mma(c, blk(i, i), blk(i, j), lane);       // T_ii W
+        __syncwarp();
+        blk_store(blk(i, j), c, -1.f, lane);
+    }
+    sync();
+    {   // level 2: X_ab = sum_m A_am T_mb, a in {2,3}, b in {0,1}; stored over A_ab
+        const int a = 2 + (warp >> 1), bb = warp & 1;
+        float c[2][4];
+        blk_zero(c);
+        if (bb == 0) {
+            blk_mma(c, blk(a, 0), blk(0, 0), lane);
+            blk_mma(c, blk(a, 1), blk(1, 0), lane);
+        } else {
+            blk_mma(c, blk(a, 1), blk(1, 1), lane);
+        }
+        sync();
+        blk_store(blk(a, bb), c, 1.f, lane);
+    }
+    sync();
+    {   // level 3: T_ab = -(T_a2 X_2b + T_a3 X_3b), T_23 = 0
+        const int a = 2 + (warp >> 1), bb = warp & 1;
+        float c[2][4];
+        blk_zero(c);
+        blk_mma(c, blk(a, 2), blk(2, bb), lane);
+        if (a == 3) blk_mma(c, blk(3, 3), blk(3, bb), lane);
+        sync();
+        blk_store(blk(a, bb), c, -1.f, lane);
+    }
+    sync();
+}
+
 }  // namespace tri
 }  // namespace osdn
