@@ -103,7 +103,7 @@ def source_sha(files):
 _CSRC = "preconditioned_delta_rule_token_b200/csrc/"
 KERNEL_SOURCES = {   # the sources each timed kernel is built from (bf16, dk = dv = 128 path)
     "chunk": [_CSRC + f for f in ("chunk_wy.cuh", "tc_ptx.cuh", "tril_inv.cuh", "common.cuh")],
-    "scan": [_CSRC + f for f in ("scan_tc.cuh", "tc_ptx.cuh", "tril_inv.cuh", "common.cuh")],
+    "scan": [_CSRC + f for f in ("scan_ws.cuh", "tc_ptx.cuh", "tril_inv.cuh", "common.cuh")],
 }
 
 

@@ -77,30 +77,38 @@ struct WyLayout {
     static constexpr uint32_t kTxV = 2 * 8192;
 };
 
-__device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void named_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-// Named barrier with an OR over a predicate of the participating threads.
-__device__ __forceinline__ bool named_sync_or(int id, int n, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(n)
-        : "memory");
-    return r != 0;
-}
-
 __device__ __forceinline__ unsigned short bf16_bits(float x) {
     const __nv_bfloat16 h = __float2bfloat16_rn(x);
     return *reinterpret_cast<const unsigned short*>(&h);
 }
+
+// Transposing epilogue, one warp: TMEM lanes m0..m0+31 (matrix row index m)
+// x 64 columns (token t), fp32, become bf16 rows t of a 128-byte-swizzled
+// K-major tile: element (t, m) at tile + (m / 64) * half_stride, row t, 16-byte
+// chunk (m % 64) / 8. The load uses the 16x256b shape (two adjacent columns per
+// thread); the store writes 8 x 8 tiles transposed with stmatrix, 16 bytes per
+// row per tile.
+struct ColsToRows {
+    uint32_t lo[32], hi[32];
+    __device__ __forceinline__ void load(uint32_t taddr) {   // wait with tcgen05.wait::ld before store()
+        tc::tmem_ld16x256b_x8(taddr, lo);                   // lanes m0 + 0..15
+        tc::tmem_ld16x256b_x8(taddr + (16u << 16), hi);     // lanes m0 + 16..31
+    }
+    __device__ __forceinline__ void store(uint8_t* tile, uint32_t half_stride, int m0, float scale, int lane) const {
+        const int k = lane >> 3, c = lane & 7;              // this thread addresses row c of 8 x 8 tile k
+        const int mk = m0 + 8 * k;                          // first matrix row index of tile k
+        uint8_t* base = tile + (mk >> 6) * half_stride;
+        const int ch = (mk & 63) >> 3;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {                       // tokens 8j..8j+7
+            const uint32_t p0 = tc::pack_bf16(scale * __uint_as_float(lo[4 * j]), scale * __uint_as_float(lo[4 * j + 1]));
+            const uint32_t p1 = tc::pack_bf16(scale * __uint_as_float(lo[4 * j + 2]), scale * __uint_as_float(lo[4 * j + 3]));
+            const uint32_t p2 = tc::pack_bf16(scale * __uint_as_float(hi[4 * j]), scale * __uint_as_float(hi[4 * j + 1]));
+            const uint32_t p3 = tc::pack_bf16(scale * __uint_as_float(hi[4 * j + 2]), scale * __uint_as_float(hi[4 * j + 3]));
+            tc::stmatrix_x4_trans(tc::smem_u32(base + tc::sw128_off(8 * j + c, ch)), p0, p1, p2, p3);
+        }
+    }
+};
 
 template <int kUnused = 0>
 __global__ void __launch_bounds__(288, 1)
@@ -173,8 +181,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ================================================================ state group
         const int v = tid;                                   // TMEM lane: value row of S / key feature
         const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-        const int vch = (v & 63) >> 3, vby = (v & 7) * 2;    // 16-byte chunk and byte of column v in its half
-        constexpr int kTmaThread = 32;
+        constexpr int kTmaThread = 32, kPrefetchThread = 64;
         int issuedQ = 0, issuedV = 0;
         auto load_qk = [&](int c) {   // K, Q, Kw of chunk c into stage c % 3
             uint8_t* st = sm + (c % 3) * L::STAGE;
@@ -185,6 +192,15 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc::tma_load_4d(st + L::QK + half * 16384, &tm_k, half * 64, h, c * C, b, fb);
                 tc::tma_load_4d(st + L::QK + half * 16384 + 8192, &tm_q, half * 64, h, c * C, b, fb);
                 tc::tma_load_4d(st + L::KW + half * 8192, &tm_kw, half * 64, h, c * C, b, fb);
+            }
+        };
+        auto prefetch_l2 = [&](int c) {   // chunk c's tiles into L2, one ring slot ahead of its shared-memory load
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                tc::tma_prefetch_4d(&tm_k, half * 64, h, c * C, b);
+                tc::tma_prefetch_4d(&tm_q, half * 64, h, c * C, b);
+                tc::tma_prefetch_4d(&tm_kw, half * 64, h, c * C, b);
+                tc::tma_prefetch_4d(&tm_v, half * 64, h, c * C, b);
             }
         };
         auto load_v = [&](int c) {    // V of chunk c into V tile c % 2
@@ -198,6 +214,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             while (issuedQ < 3 && issuedQ < nchunks) load_qk(issuedQ++);
             while (issuedV < 2 && issuedV < nchunks) load_v(issuedV++);
         }
+        if (tid == kPrefetchThread && nchunks > 3) prefetch_l2(3);
         {   // initial state: fp32 S, its bf16 copy (A operand of GA), zeroed O^T columns
             const float* srow = S0 ? S0 + ((size_t)unit * DV + v) * DK : nullptr;
 #pragma unroll
@@ -224,25 +241,21 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc::tmem_wait_st();
         }
         tc::tc_fence_before();
-        named_sync(BAR_STATE, 128);
-        if (tid == 0 && nchunks > 0) mbar_arrive1(bars + L::ESB);
+        tc::named_sync(BAR_STATE, 128);
+        if (tid == 0 && nchunks > 0) tc::mbar_arrive1(bars + L::ESB);
 
         // -W of chunk c (from W^T in R1[c % 3], lane = key feature) into the K rows of its stage
         auto w_epilogue = [&](int c) -> bool {
-            if (named_sync_or(BAR_STATE, 128, !wait(L::BW, c & 1))) return false;
+            if (tc::named_sync_or(BAR_STATE, 128, !wait(L::BW, c & 1))) return false;
             tc::tc_fence_after();
-            uint32_t w[64];
-            tc::tmem_ld32(tl + COL_R1 + (c % 3) * 64, *reinterpret_cast<uint32_t(*)[32]>(w));
-            tc::tmem_ld32(tl + COL_R1 + (c % 3) * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(w + 32));
+            ColsToRows w;
+            w.load(tl + COL_R1 + (c % 3) * 64);
             tc::tmem_wait_ld();
-            uint8_t* kb = sm + (c % 3) * L::STAGE + L::QK + (v >> 6) * 16384 + vby;
-#pragma unroll
-            for (int t = 0; t < C; ++t)
-                *reinterpret_cast<unsigned short*>(kb + tc::sw128_off(t, vch)) = bf16_bits(-__uint_as_float(w[t]));
+            w.store(sm + (c % 3) * L::STAGE + L::QK, 16384, warp * 32, -1.f, lane);
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
-            named_sync(BAR_STATE, 128);
-            if (tid == 0) mbar_arrive1(bars + L::EWE);
+            tc::named_sync(BAR_STATE, 128);
+            if (tid == 0) tc::mbar_arrive1(bars + L::EWE);
             return true;
         };
 
@@ -251,7 +264,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (; ok && c < nchunks; ++c) {
             const int s2 = c & 1;
             // Vn^T = U0^T - S W^T (D columns 0-63) -> bf16 over columns 0-31 (A operand of GB)
-            if (named_sync_or(BAR_STATE, 128, !wait(L::BA, c & 1))) break;
+            if (tc::named_sync_or(BAR_STATE, 128, !wait(L::BA, c & 1))) break;
             tc::tc_fence_after();
             {
                 uint32_t x[64], w[32];
@@ -264,16 +277,15 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc::tmem_wait_st();
             }
             tc::tc_fence_before();
-            named_sync(BAR_STATE, 128);
-            if (tid == 0) mbar_arrive1(bars + L::EVN);
+            tc::named_sync(BAR_STATE, 128);
+            if (tid == 0) tc::mbar_arrive1(bars + L::EVN);
 
             // -W of the next chunk while GB runs
             if (c + 1 < nchunks && !w_epilogue(c + 1)) break;
 
             // S_{c+1} and O_c are complete; stage c % 3 is free
-            if (named_sync_or(BAR_STATE, 128, !wait(L::BS + s2, (c >> 1) & 1))) break;
+            if (tc::named_sync_or(BAR_STATE, 128, !wait(L::BS + s2, (c >> 1) & 1))) break;
             tc::tc_fence_after();
-            if (tid == kTmaThread && issuedQ < nchunks) load_qk(issuedQ++);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t x[64];
@@ -294,9 +306,8 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                                            __uint_as_float(x[i + 2]), __uint_as_float(x[i + 3]));
                 }
             }
-            uint32_t o[64];
-            tc::tmem_ld32(tl + COL_D + 64, *reinterpret_cast<uint32_t(*)[32]>(o));
-            tc::tmem_ld32(tl + COL_D + 96, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+            ColsToRows o;   // O^T columns, read before they are zeroed for the next chunk
+            o.load(tl + COL_D + 64);
             tc::tmem_wait_ld();
             if (c + 1 < nchunks) {
                 uint32_t z[32];
@@ -307,19 +318,18 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc::tmem_wait_st();
             }
             tc::tc_fence_before();
-            named_sync(BAR_STATE, 128);
-            if (tid == 0 && c + 1 < nchunks) mbar_arrive1(bars + L::ESB);
+            tc::named_sync(BAR_STATE, 128);
+            if (tid == 0 && c + 1 < nchunks) tc::mbar_arrive1(bars + L::ESB);
+            // stage c % 3 is free (GB(c) has completed): chunk c + 3's tiles, and chunk c + 4's into L2;
+            // issued after the hand-off so that their issue time stays off the state chain
+            if (tid == kTmaThread && issuedQ < nchunks) load_qk(issuedQ++);
+            if (tid == kPrefetchThread && c + 4 < nchunks) prefetch_l2(c + 4);
 
             // O_c -> the V tile of this chunk (free since GU(c) completed) -> TMA store
             uint8_t* ob = sm + L::VB + s2 * 16384;
-            {
-                uint8_t* col = ob + (v >> 6) * 8192 + vby;
-#pragma unroll
-                for (int t = 0; t < C; ++t)
-                    *reinterpret_cast<unsigned short*>(col + tc::sw128_off(t, vch)) = bf16_bits(__uint_as_float(o[t]));
-            }
+            o.store(ob, 8192, warp * 32, 1.f, lane);
             tc::fence_proxy_async_smem();
-            named_sync(BAR_STATE, 128);
+            tc::named_sync(BAR_STATE, 128);
             if (tid == kTmaThread) {
                 tc::tma_store_4d(&tm_out, ob, 0, h, c * C, b);
                 tc::tma_store_4d(&tm_out, ob + 8192, 64, h, c * C, b);
@@ -357,7 +367,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (c + 1 < nchunks) bnext = load_beta(c + 1);
             bool fail = !wait(L::D1 + c % 3, (c / 3) & 1);
             if (!fail && c >= 2) fail = !wait(L::BS + s2, ((c - 2) >> 1) & 1);   // GB(c-2) has read P tile s2
-            if (named_sync_or(BAR_PREP, 128, fail)) break;
+            if (tc::named_sync_or(BAR_PREP, 128, fail)) break;
             tc::tc_fence_after();
             if (gtid < C) betas[gtid] = bt;
 #pragma unroll
@@ -395,11 +405,11 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
-            named_sync(BAR_PREP, 128);
-            tri::tril_inv64_inplace(AF, gw, lane, [] { named_sync(BAR_PREP, 128); });
+            tc::named_sync(BAR_PREP, 128);
+            tri::tril_inv64_inplace(AF, gw, lane, [] { tc::named_sync(BAR_PREP, 128); });
             // T diag(beta) -> bf16 K-major (B operand of GW and GU), once GW(c-1) and GU(c-1) have read it
             fail = c >= 1 && !wait(L::BA, (c - 1) & 1);
-            if (named_sync_or(BAR_PREP, 128, fail)) break;
+            if (tc::named_sync_or(BAR_PREP, 128, fail)) break;
             {
                 const int t = gtid & 63, hf = gtid >> 6;
 #pragma unroll
@@ -416,8 +426,8 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
             tc::fence_proxy_async_smem();
-            named_sync(BAR_PREP, 128);
-            if (gtid == 0) mbar_arrive1(bars + L::ETB);
+            tc::named_sync(BAR_PREP, 128);
+            if (gtid == 0) tc::mbar_arrive1(bars + L::ETB);
         }
         tc::tc_fence_before();
     } else {
@@ -470,10 +480,10 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc::umma_commit(bars + L::BS + (c & 1));
             };
             // Static order per chunk c (each wait sleeps in hardware until its phase completes):
-            //   GA(c) | GW(c+1) if its operand is ready | GB(c) | GW(c+1) otherwise | G1(c+2) | GU(c+1)
-            // G1(c+2) reuses R1[(c+2)%3], whose W^T(c-1) was consumed before GA(c-1); GU(c+1) overwrites
-            // D[0,64) once GB(c) has read bf16 Vn from it. G1 and GU fill the tensor pipe while the state
-            // group turns S into bf16.
+            //   GA(c) | GW(c+1), G1(c+2) if their inputs are ready | GB(c) | the rest of GW(c+1), G1(c+2) | GU(c+1)
+            // GW and G1 fill the tensor pipe while the state group forms bf16 Vn after GA. G1(c+2) reuses
+            // R1[(c+2)%3], whose W^T(c-1) was consumed before GA(c-1); GU(c+1) overwrites D[0,64) once GB(c)
+            // has read bf16 Vn from it.
             auto issue_gu = [&](int c) -> bool {
                 if (c > 0 && !wait(L::BS + ((c - 1) & 1), ((c - 1) >> 1) & 1)) return false;
                 if (!wait(L::FULLV + (c & 1), (c >> 1) & 1)) return false;
@@ -499,17 +509,21 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (!ok) break;
                 tc::tc_fence_after();
                 GA(c);
-                bool gw_done = c + 1 >= nchunks;
+                bool gw_done = c + 1 >= nchunks, g1_done = c + 2 >= nchunks;
                 if (!gw_done && tc::mbar_test(bars + L::ETB, (c + 1) & 1)) {
                     tc::tc_fence_after();
                     GW(c + 1);
                     gw_done = true;
                 }
+                if (!g1_done && tc::mbar_test(bars + L::FULLQ + (c + 2) % 3, ((c + 2) / 3) & 1)) {
+                    G1(c + 2);
+                    g1_done = true;
+                }
                 if (!(ok = wait(L::EVN, c & 1))) break;
                 tc::tc_fence_after();
                 GB(c);
                 if (!gw_done && !(ok = issue_gw(c + 1))) break;
-                if (c + 2 < nchunks && !(ok = issue_g1(c + 2))) break;
+                if (!g1_done && !(ok = issue_g1(c + 2))) break;
                 if (c + 1 < nchunks && !(ok = issue_gu(c + 1))) break;
             }
             tc::umma_commit(bars + L::DRAIN);   // every MMA issued above has completed before TMEM is released

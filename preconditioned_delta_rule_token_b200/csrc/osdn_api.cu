@@ -17,7 +17,7 @@
 
 #include "chunk_ffma.cuh"
 #include "chunk_wy.cuh"
-#include "scan_tc.cuh"
+#include "scan_ws.cuh"
 #include "scan_seq.cuh"
 #include "step.cuh"
 
@@ -172,11 +172,11 @@ int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bflo
     if (rc) return rc;
     rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128);
     if (rc) return rc;
-    auto kern = osdn::scan_tc_kernel<0>;
-    const size_t smem = osdn::ScanSmem::kBytes;
+    auto kern = osdn::scan_ws_kernel<0>;
+    const size_t smem = osdn::ScanLayout::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan kernel attribute");
-    kern<<<p->B * p->H, 128, smem, st>>>(mk, mkw, beta, r, d0, final_d, p->B, p->T, p->H, p->eta,
+    kern<<<p->B * p->H, 384, smem, st>>>(mk, mkw, beta, r, d0, final_d, p->B, p->T, p->H, p->eta,
                                          g_wait_limit_ns.load());
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");
     return OSDN_OK;

@@ -60,6 +60,27 @@ __device__ __forceinline__ void blk_mma(float (&c)[2][4], const float* X, const 
     }
 }
 
+// Same product with the fp32 bit patterns passed as tf32 operands: the tensor
+// core reads the upper 19 bits (truncation instead of round-to-nearest, one
+// tf32 ulp at most), which saves the conversions.
+__device__ __forceinline__ void blk_mma_trunc(float (&c)[2][4], const float* X, const float* Y, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const int k0 = ks * 8;
+        const uint32_t a0 = __float_as_uint(X[g * LD + k0 + t]);
+        const uint32_t a1 = __float_as_uint(X[(g + 8) * LD + k0 + t]);
+        const uint32_t a2 = __float_as_uint(X[g * LD + k0 + t + 4]);
+        const uint32_t a3 = __float_as_uint(X[(g + 8) * LD + k0 + t + 4]);
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+            const uint32_t b0 = __float_as_uint(Y[(k0 + t) * LD + nh * 8 + g]);
+            const uint32_t b1 = __float_as_uint(Y[(k0 + t + 4) * LD + nh * 8 + g]);
+            mma_tf32(c[nh], a0, a1, a2, a3, b0, b1);
+        }
+    }
+}
+
 __device__ __forceinline__ void blk_zero(float (&c)[2][4]) {
 #pragma unroll
     for (int i = 0; i < 2; ++i)
@@ -169,21 +190,19 @@ __device__ __forceinline__ void diag16_inverse_column(const float* Lb, int j, fl
             const float4 x = *reinterpret_cast<const float4*>(Lb + t * LD + m4);
             l[m4] = x.x; l[m4 + 1] = x.y; l[m4 + 2] = x.z; l[m4 + 3] = x.w;
         }
-        float s0 = 0.f, s1 = 0.f;
+        float s[4] = {0.f, 0.f, 0.f, 0.f};   // four partial sums shorten the dependent FMA chain
 #pragma unroll
-        for (int m = 0; m < t; m += 2) {
-            s0 = fmaf(l[m], c[m], s0);
-            if (m + 1 < t) s1 = fmaf(l[m + 1], c[m + 1], s1);
-        }
-        if (t > j) c[t] = -(s0 + s1);
+        for (int m = 0; m < t; ++m) s[m & 3] = fmaf(l[m], c[m], s[m & 3]);
+        if (t > j) c[t] = -((s[0] + s[1]) + (s[2] + s[3]));
     }
 }
 
 // In-place variant: on entry A holds the strictly lower 64 x 64 matrix (every
 // entry on and above the diagonal zero, the blocks above the diagonal blocks
 // included); on return it holds T = (I + A)^{-1}. Same blocking and arithmetic
-// as tril_inv64; each level computes its blocks into registers before any
-// warp overwrites an operand another warp still reads.
+// as tril_inv64 except that the block products truncate their operands to
+// tf32 (blk_mma_trunc); each level computes its blocks into registers before
+// any warp overwrites an operand another warp still reads.
 template <class Sync>
 __device__ __forceinline__ void tril_inv64_inplace(float* A, int warp, int lane, Sync sync) {
     auto blk = [&](int i, int j) { return A + (i * 16) * LD + j * 16; };
@@ -202,12 +221,12 @@ __device__ __forceinline__ void tril_inv64_inplace(float* A, int warp, int lane,
         const int i = warp * 2 + 1, j = warp * 2;
         float c[2][4];
         blk_zero(c);
-        blk_mma(c, blk(i, j), blk(j, j), lane);       // W = A_ij T_jj
+        blk_mma_trunc(c, blk(i, j), blk(j, j), lane);       // W = A_ij T_jj
         __syncwarp();
         blk_store(blk(i, j), c, 1.f, lane);
         __syncwarp();
         blk_zero(c);
-        blk_mma(c, blk(i, i), blk(i, j), lane);       // T_ii W
+        blk_mma_trunc(c, blk(i, i), blk(i, j), lane);       // T_ii W
         __syncwarp();
         blk_store(blk(i, j), c, -1.f, lane);
     }
@@ -217,10 +236,10 @@ __device__ __forceinline__ void tril_inv64_inplace(float* A, int warp, int lane,
         float c[2][4];
         blk_zero(c);
         if (bb == 0) {
-            blk_mma(c, blk(a, 0), blk(0, 0), lane);
-            blk_mma(c, blk(a, 1), blk(1, 0), lane);
+            blk_mma_trunc(c, blk(a, 0), blk(0, 0), lane);
+            blk_mma_trunc(c, blk(a, 1), blk(1, 0), lane);
         } else {
-            blk_mma(c, blk(a, 1), blk(1, 1), lane);
+            blk_mma_trunc(c, blk(a, 1), blk(1, 1), lane);
         }
         sync();
         blk_store(blk(a, bb), c, 1.f, lane);
@@ -230,8 +249,8 @@ __device__ __forceinline__ void tril_inv64_inplace(float* A, int warp, int lane,
         const int a = 2 + (warp >> 1), bb = warp & 1;
         float c[2][4];
         blk_zero(c);
-        blk_mma(c, blk(a, 2), blk(2, bb), lane);
-        if (a == 3) blk_mma(c, blk(3, 3), blk(3, bb), lane);
+        blk_mma_trunc(c, blk(a, 2), blk(2, bb), lane);
+        if (a == 3) blk_mma_trunc(c, blk(3, 3), blk(3, bb), lane);
         sync();
         blk_store(blk(a, bb), c, -1.f, lane);
     }
