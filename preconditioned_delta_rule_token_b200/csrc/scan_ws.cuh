@@ -24,8 +24,8 @@
 //   chain group (warps 0-3): the carry. Per sub-chunk: b_t = <d_c, a_t> and
 //     c_t, x = N c, then thread i runs feature i through the sub-chunk, writing
 //     kw_t[i] = d_t[i] k_t[i] over k_t[i] and carrying d; then one TMA store of
-//     the block's scaled keys, after which its buffer takes the block three
-//     ahead.
+//     the block's scaled keys; its buffer takes the block three ahead once the
+//     store has read it (issued at the start of the next block).
 // K blocks are triple-buffered; N, the per-token vectors and the hand-offs are
 // double-buffered by block parity. Bounded mbarrier waits with a shared abort
 // flag, as in the chunk kernel.
@@ -155,7 +155,9 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                     for (int c = 0; c < 8; ++c) {
                         const uint4 raw = *reinterpret_cast<const uint4*>(KS + half * 16384 + tc::sw128_off(t, c));
                         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-                        const float* dd = s_d + half * 64 + c * 8;
+                        const float4 dlo = *reinterpret_cast<const float4*>(s_d + half * 64 + c * 8);
+                        const float4 dhi = *reinterpret_cast<const float4*>(s_d + half * 64 + c * 8 + 4);
+                        const float dd[8] = {dlo.x, dlo.y, dlo.z, dlo.w, dhi.x, dhi.y, dhi.z, dhi.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 f = __bfloat1622float2(p2[e]);
@@ -166,16 +168,25 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                     if (half == 0) s_c[tl_] = vb[L::V_G + t] * (1.f - vb[L::V_BETA + t] * vb[L::V_R0 + t] * acc);
                 }
+                if (s == 0 && tid == kTmaThread && blk > 0 && issued < nblk) {
+                    // the buffer of block blk - 1 takes block blk + 2 once its store has read it (issued
+                    // here, a step after that store, so that the wait is normally over already)
+                    tc::bulk_wait_read<0>();
+                    load_k(issued++);
+                }
                 tc::named_sync(BAR_CHAIN, 128);
                 {   // x = N c (two threads per row), kept as x_t / ||k_t||^2
                     const int tl_ = tid >> 1, half = tid & 1;
-                    const float* Nrow = Nm + tl_ * L::LD + half * 32;
-                    const float* cc = s_c + half * 32;
+                    // half h takes columns 16h + 32m + 4i (m < 2, i < 4): with the 68-float row stride the
+                    // eight threads of a quarter warp then read eight different 16-byte bank groups
+                    const float* Nrow = Nm + tl_ * L::LD + half * 16;
+                    const float* cc = s_c + half * 16;
                     float acc = 0.f;
 #pragma unroll
-                    for (int k4 = 0; k4 < 32; k4 += 4) {
-                        const float4 n4 = *reinterpret_cast<const float4*>(Nrow + k4);
-                        const float4 c4 = *reinterpret_cast<const float4*>(cc + k4);
+                    for (int m = 0; m < 8; ++m) {
+                        const int col = 32 * (m >> 2) + 4 * (m & 3);
+                        const float4 n4 = *reinterpret_cast<const float4*>(Nrow + col);
+                        const float4 c4 = *reinterpret_cast<const float4*>(cc + col);
                         acc = fmaf(n4.x, c4.x, fmaf(n4.y, c4.y, fmaf(n4.z, c4.z, fmaf(n4.w, c4.w, acc))));
                     }
                     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
@@ -223,14 +234,10 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             if (tid == 0) tc::mbar_arrive1(bars + L::MFREE + (blk & 1));   // N and vectors of this parity consumed
             tc::fence_proxy_async_smem();
             tc::named_sync(BAR_CHAIN, 128);
-            if (tid == kTmaThread) {   // the scaled keys leave; the buffer then takes the block three ahead
+            if (tid == kTmaThread) {   // the scaled keys leave
                 tc::tma_store_4d(&tm_kw, KS, 0, h, blk * BLK, b);
                 tc::tma_store_4d(&tm_kw, KS + 16384, 64, h, blk * BLK, b);
                 tc::bulk_commit();
-                if (issued < nblk) {
-                    tc::bulk_wait_read<0>();
-                    load_k(issued++);
-                }
             }
         }
         if (tid == kTmaThread) {   // stores complete; loads that were issued have landed
@@ -246,24 +253,24 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         const int row = tp & 127;              // token of the block and TMEM lane this thread serves
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         float* np = reinterpret_cast<float*>(sm + L::NP);
+        auto load_pv = [&](int blk) -> float {   // group 0: beta, group 1: r (1 past T or without APF)
+            const int tok = blk * BLK + row;
+            const size_t gi = ((size_t)b * T + tok) * H + h;
+            if (g == 0) return tok < T ? __bfloat162float(beta[gi]) : 0.f;
+            return (tok < T && r) ? __bfloat162float(r[gi]) : 1.f;
+        };
+        float pv = nblk > 0 ? load_pv(0) : 0.f;
         for (int blk = 0; blk < nblk; ++blk) {
-            const int t0 = blk * BLK;
             uint8_t* KS = kblock(blk);
             float* vb = vecs(blk);
             bool fail = !wait(L::FULL + blk % L::NKB, (blk / L::NKB) & 1);
             if (!fail && blk >= 2) fail = !wait(L::MFREE + (blk & 1), ((blk - 2) >> 1) & 1);
             if (tc::named_sync_or(BAR_PREP, 256, fail)) break;
-            // beta (group 0) or r (group 1) of token `row`
-            const int tok = t0 + row;
-            const bool in = tok < T;
-            const size_t gi = ((size_t)b * T + tok) * H + h;
-            float bt = 0.f;
-            if (g == 0) {
-                bt = in ? __bfloat162float(beta[gi]) : 0.f;
-                vb[L::V_BETA + row] = bt;
-            } else {
-                vb[L::V_R + row] = (in && r) ? __bfloat162float(r[gi]) : 1.f;
-            }
+            // beta (group 0) or r (group 1) of token `row`, loaded one block ahead
+            const float bt = pv;
+            if (g == 0) vb[L::V_BETA + row] = bt;
+            else vb[L::V_R + row] = bt;
+            if (blk + 1 < nblk) pv = load_pv(blk + 1);
             {   // a = k^2 (bf16 tile) over this group's half of the features; partial ||k||^2
                 float nrm = 0.f;
 #pragma unroll
@@ -313,17 +320,33 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                 const float coef = vb[L::V_G + row] * vb[L::V_BETA + row];
                 const float* rr = vb + L::V_R + s * SUB;
                 const float* iv = vb + L::V_INVN + s * SUB;
+                float rj[32], ivj[32];
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const float4 r4 = *reinterpret_cast<const float4*>(rr + jb + j4);
+                    const float4 i4 = *reinterpret_cast<const float4*>(iv + jb + j4);
+                    rj[j4] = r4.x; rj[j4 + 1] = r4.y; rj[j4 + 2] = r4.z; rj[j4 + 3] = r4.w;
+                    ivj[j4] = i4.x; ivj[j4 + 1] = i4.y; ivj[j4 + 2] = i4.z; ivj[j4 + 3] = i4.w;
+                }
                 float R = 1.f;   // R_{tl, jb + 32} when the walk enters this group's columns
-                if (g == 1)
-                    for (int m = 32; m < tl_; ++m) R *= rr[m];
+                if (g == 1) {    // product of r over columns 32..tl-1, from the other half
+#pragma unroll
+                    for (int j4 = 0; j4 < 32; j4 += 4) {
+                        const float4 r4 = *reinterpret_cast<const float4*>(rr + 32 + j4);
+                        if (32 + j4 < tl_) R *= r4.x;
+                        if (33 + j4 < tl_) R *= r4.y;
+                        if (34 + j4 < tl_) R *= r4.z;
+                        if (35 + j4 < tl_) R *= r4.w;
+                    }
+                }
                 float mrow[32];
 #pragma unroll
                 for (int jj = 31; jj >= 0; --jj) {
                     const int j = jb + jj;
                     mrow[jj] = 0.f;
                     if (j < tl_) {
-                        mrow[jj] = coef * R * __uint_as_float(gr[jj]) * iv[j];
-                        R *= rr[j];
+                        mrow[jj] = coef * R * __uint_as_float(gr[jj]) * ivj[jj];
+                        R *= rj[jj];
                     }
                 }
                 float* Mrow = reinterpret_cast<float*>(sm + L::MF + ((blk & 1) * 2 + s) * L::MAT) + tl_ * L::LD + jb;
