@@ -187,6 +187,31 @@ def dist_setup(args):
     return world, rank, local
 
 
+def rank_workload(w, rank):
+    """Rank r runs the same workload shape on its own inputs (seed + 1000 r): weak
+    scaling over independent sequences, no data shared between ranks."""
+    if rank == 0:
+        return w
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise max of per-rank timings (an all-reduce MAX over the process
+    group, device tensors under NCCL, host tensors under gloo)."""
+    if world <= 1:
+        return list(values)
+    t = torch.tensor(list(values), device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_tokens_per_s(w, world, ms):
+    """Whole-job throughput: every rank processes B*T tokens (of H heads each) in
+    the slowest rank's step time ms."""
+    return world * w.B * w.T / (ms / 1e3)
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -266,10 +291,7 @@ def run_ours(args, world, rank, local):
     import preconditioned_delta_rule_token_b200 as pk
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = WORKLOADS[args.workload]
-    if rank:
-        import dataclasses
-        w = dataclasses.replace(w, seed=w.seed + 1000 * rank)
+    w = rank_workload(WORKLOADS[args.workload], rank)
     inp = W.make_forward_inputs(w)
     g = {k: None if v is None else v.to(dev) for k, v in inp.items()}
     g["d0"] = None            # d0 = ones (the library's default), as in the workload
@@ -307,10 +329,7 @@ def run_ours(args, world, rank, local):
     scan_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     chunk_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     ms = total_ms / args.steps
-    if world > 1:
-        t = torch.tensor([ms, scan_ms, chunk_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, scan_ms, chunk_ms = t.tolist()
+    ms, scan_ms, chunk_ms = max_over_ranks([ms, scan_ms, chunk_ms], world, dev)
 
     # end-to-end through the public API with pinned host buffers
     e2e = None
@@ -345,12 +364,8 @@ def run_ours(args, world, rank, local):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = t.item()
-        e2e = {"value": world * w.B * w.T / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / n_e2e], world, dev)[0]
+        e2e = {"value": aggregate_tokens_per_s(w, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank != 0:
@@ -369,7 +384,7 @@ def run_ours(args, world, rank, local):
     achieved = kd["bytes"] / (kd["ms"] / 1e3) / 1e9
     traffic = ncu_traffic(dom, args.workload)
     line = {
-        "metric": "OSDN chunkwise fwd tokens/s", "value": world * w.B * w.T / (ms / 1e3), "unit": "tokens/s",
+        "metric": "OSDN chunkwise fwd tokens/s", "value": aggregate_tokens_per_s(w, world, ms), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == W.BF16
         else "f32", "data": "synthetic", "config": config_of(w, world),

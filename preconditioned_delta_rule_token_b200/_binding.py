@@ -91,6 +91,8 @@ def lib():
         L.osdn_step.restype = ctypes.c_int
         L.osdn_sync_status.argtypes = [vp]
         L.osdn_sync_status.restype = ctypes.c_int
+        L.osdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+        L.osdn_set_wait_limit_ns.restype = None
         L.osdn_get_last_error.argtypes = []
         L.osdn_get_last_error.restype = ctypes.c_char_p
         L.osdn_abi_version.argtypes = []
@@ -179,3 +181,8 @@ def osdn_step(params, q, k, v, beta, r, S, d, out, stream=None):
 
 def osdn_sync_status(stream=None) -> int:
     return lib().osdn_sync_status(_stream(stream))
+
+
+def osdn_set_wait_limit_ns(ns: int) -> None:
+    """Upper bound on any device-side wait of kernels launched afterwards (0 = the 4 s default)."""
+    lib().osdn_set_wait_limit_ns(int(ns))

@@ -165,10 +165,12 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // bounded wait that also stops when another role has aborted
     auto wait = [&](int bi, uint32_t parity) -> bool {
         uint64_t* bar = bars + bi;
-        if (tc::mbar_try_wait(bar, parity)) return true;
+        // the hardware suspend of one try is capped by the limit, so a short limit ends a wait promptly
+        const uint32_t hint = wait_limit_ns < 20000ull ? (uint32_t)wait_limit_ns : 20000u;
+        if (tc::mbar_try_wait(bar, parity, hint)) return true;
         const uint64_t t0 = tc::globaltimer_ns();
         while (true) {
-            if (tc::mbar_try_wait(bar, parity)) return true;
+            if (tc::mbar_try_wait(bar, parity, hint)) return true;
             if (*abort_flag) return false;
             if (tc::globaltimer_ns() - t0 > wait_limit_ns) {
                 give_up();

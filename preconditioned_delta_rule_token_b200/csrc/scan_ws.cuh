@@ -106,10 +106,12 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
     auto wait = [&](int bi, uint32_t parity) -> bool {   // bounded; stops when another role has aborted
         uint64_t* bar = bars + bi;
-        if (tc::mbar_try_wait(bar, parity)) return true;
+        // the hardware suspend of one try is capped by the limit, so a short limit ends a wait promptly
+        const uint32_t hint = wait_limit_ns < 20000ull ? (uint32_t)wait_limit_ns : 20000u;
+        if (tc::mbar_try_wait(bar, parity, hint)) return true;
         const uint64_t t0 = tc::globaltimer_ns();
         while (true) {
-            if (tc::mbar_try_wait(bar, parity)) return true;
+            if (tc::mbar_try_wait(bar, parity, hint)) return true;
             if (*abort_flag) return false;
             if (tc::globaltimer_ns() - t0 > wait_limit_ns) {
                 *abort_flag = 1;
