@@ -196,7 +196,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc::tma_load_4d(st + L::KW + half * 8192, &tm_kw, half * 64, h, c * C, b, fb);
             }
         };
-        auto prefetch_l2 = [&](int c) {   // chunk c's tiles into L2, one ring slot ahead of its shared-memory load
+        auto prefetch_l2 = [&](int c) {   // chunk c's tiles into L2, two ring slots ahead of their shared-memory load
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 tc::tma_prefetch_4d(&tm_k, half * 64, h, c * C, b);
@@ -216,7 +216,10 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             while (issuedQ < 3 && issuedQ < nchunks) load_qk(issuedQ++);
             while (issuedV < 2 && issuedV < nchunks) load_v(issuedV++);
         }
-        if (tid == kPrefetchThread && nchunks > 3) prefetch_l2(3);
+        if (tid == kPrefetchThread) {
+            if (nchunks > 3) prefetch_l2(3);
+            if (nchunks > 4) prefetch_l2(4);
+        }
         {   // initial state: fp32 S, its bf16 copy (A operand of GA), zeroed O^T columns
             const float* srow = S0 ? S0 + ((size_t)unit * DV + v) * DK : nullptr;
 #pragma unroll
@@ -322,10 +325,10 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc::tc_fence_before();
             tc::named_sync(BAR_STATE, 128);
             if (tid == 0 && c + 1 < nchunks) tc::mbar_arrive1(bars + L::ESB);
-            // stage c % 3 is free (GB(c) has completed): chunk c + 3's tiles, and chunk c + 4's into L2;
+            // stage c % 3 is free (GB(c) has completed): chunk c + 3's tiles, and chunk c + 5's into L2;
             // issued after the hand-off so that their issue time stays off the state chain
             if (tid == kTmaThread && issuedQ < nchunks) load_qk(issuedQ++);
-            if (tid == kPrefetchThread && c + 4 < nchunks) prefetch_l2(c + 4);
+            if (tid == kPrefetchThread && c + 5 < nchunks) prefetch_l2(c + 5);
 
             // O_c -> the V tile of this chunk (free since GU(c) completed) -> TMA store
             uint8_t* ob = sm + L::VB + s2 * 16384;

@@ -154,7 +154,10 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                     const int tl_ = tid >> 1, half = tid & 1, t = s * SUB + tl_;
                     float acc = 0.f;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
+                    for (int c0 = 0; c0 < 8; ++c0) {
+                        // the two halves walk their 16-byte chunks four apart, so the two threads of a
+                        // token never hit the same bank group
+                        const int c = (c0 + 4 * half) & 7;
                         const uint4 raw = *reinterpret_cast<const uint4*>(KS + half * 16384 + tc::sw128_off(t, c));
                         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
                         const float4 dlo = *reinterpret_cast<const float4*>(s_d + half * 64 + c * 8);
