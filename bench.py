@@ -51,6 +51,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the osdn_step (decode) measurement")
     return ap.parse_args()
 
 
@@ -279,6 +280,45 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def decode_bytes(w):
+    """HBM bytes of one decode call over all B*H heads: S read + written (fp32), d read +
+    written (fp32), q, k, v read and out written (storage dtype), beta and r."""
+    e = elem(w)
+    return w.B * w.H * (2 * w.dv * w.dk * 4 + 2 * w.dk * 4 + (2 * w.dk + w.dv) * e + w.dv * e + 2 * e)
+
+
+def run_decode(dev, stream, hbm, n_calls=200, warmup=5):
+    """osdn_step on the decode workload (B256 H16 d128 bf16): S, d and eight distinct
+    tokens resident in HBM (S alone is 268 MB > L2); per-call time by CUDA events."""
+    import preconditioned_delta_rule_token_b200 as pk
+    w = W.DECODE
+    st0 = W.make_decode_state(w)
+    S, d = st0["S0"].to(dev), st0["d0"].to(dev)
+    toks = [{k_: None if v_ is None else v_.to(dev) for k_, v_ in W.make_decode_token(w, i).items()}
+            for i in range(8)]
+    p = pk.make_params(w.B, 1, w.H, w.dk, w.dv, toks[0]["k"].dtype, w.eta)
+    out = torch.empty((w.B, w.H, w.dv), dtype=toks[0]["k"].dtype, device=dev)
+
+    def call(i):
+        t = toks[i % len(toks)]
+        pk.osdn_step(p, t["q"], t["k"], t["v"], t["beta"], t["r"], S, d, out, stream)
+
+    for i in range(warmup):
+        call(i)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n_calls):
+        call(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert pk.osdn_sync_status(stream) == 0
+    us = e0.elapsed_time(e1) * 1e3 / n_calls
+    gbs = decode_bytes(w) / (us * 1e-6) / 1e9
+    return {"workload": w.name, "calls": n_calls, "us_per_call": us, "tokens_per_s": w.B / (us * 1e-6),
+            "bytes_per_call": decode_bytes(w), "achieved_gbs": gbs, "peak_gbs": hbm, "frac": gbs / hbm,
+            "bound": "hbm"}
+
+
 def config_of(w, world):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
             "apf": w.apf, "eta": w.eta, "structure": w.structure, "global_batch": w.B * world, "seq_len": w.T,
@@ -402,6 +442,8 @@ def run_ours(args, world, rank, local):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if world == 1 and not args.no_decode:
+        line["decode"] = run_decode(dev, stream, hbm)
     if world == 1 and not args.no_cpu_baseline:
         v_, desc, cores = oracle_sample(w, seconds=12.0)
         line["cpu_baseline"] = {"value": v_, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
