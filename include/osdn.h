@@ -105,6 +105,24 @@ int osdn_fwd_scan(const osdn_params *p,
                   void *workspace, size_t workspace_bytes,
                   void *cuda_stream);
 
+/* osdn_fwd_scan plus a diagnostic of the preconditioner ("OSDN: Improving
+ * Delta Rule with Provable Online Preconditioning in Linear Attention",
+ * technical summary sections 4-5: the contraction factor of one write):
+ *   rho   [B, T, H] fp32, nullable: rho_t = (1 - beta_t <d_t, k_t^2>)^2, the
+ *         factor by which token t's write shrinks its own loss,
+ *         f_t(S_t) = rho_t f_t(S_{t-1}) with f_t(S) = 1/2 ||S k_t - v_t||^2;
+ *         1 when the token writes nothing (beta_t = 0 or k_t = 0).
+ *   q_geo [B, H] fp32, nullable: exp of the mean of log rho_t over the T tokens
+ *         of each (sequence, head); 1 when T = 0, 0 when some rho_t is 0.
+ * Both pointers 16-byte aligned, caller-owned. Every other argument, rule and
+ * error as osdn_fwd_scan; with rho == q_geo == NULL it is osdn_fwd_scan. */
+int osdn_fwd_scan_diag(const osdn_params *p,
+                       const void *k, const void *beta, const void *r,
+                       const float *d0, float *final_d,
+                       float *rho, float *q_geo,
+                       void *workspace, size_t workspace_bytes,
+                       void *cuda_stream);
+
 /* Phase 2 of osdn_fwd alone: the chunked delta rule with the scaled write
  * keys that a preceding osdn_fwd_scan with the same parameters left in the
  * workspace (ordered before this call on the stream). Writes out and

@@ -45,6 +45,8 @@ def _load():
         dp = ctypes.POINTER(ctypes.c_double)
         lib.osdn_oracle_fwd.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [dp] * 10 + [ctypes.c_int]
         lib.osdn_oracle_fwd.restype = ctypes.c_int
+        lib.osdn_oracle_fwd_rho.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [dp] * 11 + [ctypes.c_int]
+        lib.osdn_oracle_fwd_rho.restype = ctypes.c_int
         lib.osdn_oracle_step.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [dp] * 8
         lib.osdn_oracle_step.restype = ctypes.c_int
         _lib = lib
@@ -88,6 +90,31 @@ def fwd(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=None):
     if rc != 0:
         raise ValueError("oracle rejected the sizes")
     return out, S, d
+
+
+def residual_ratio(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=None):
+    """The forward of fwd() plus the per-token residual ratio
+    rho_t = (1 - beta_t <d_t, k_t^2>)^2 = f_t(S_t) / f_t(S_{t-1}) [B, T, H] and its
+    geometric mean over each sequence, q_geo = exp(mean_t log rho_t) [B, H]
+    (1 for an empty sequence). Returns (out, S_final, d_final, rho, q_geo)."""
+    q, k, v, beta, r, d0, S0 = map(_f64, (q, k, v, beta, r, d0, S0))
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    assert q.shape == k.shape and v.shape == (B, T, H, dv) and beta.shape == (B, T, H)
+    out = np.zeros((B, T, H, dv), np.float64)
+    S = np.zeros((B, H, dv, dk), np.float64)
+    d = np.zeros((B, H, dk), np.float64)
+    rho = np.zeros((B, T, H), np.float64)
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().osdn_oracle_fwd_rho(B, T, H, dk, dv, float(eta), _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(beta), _ptr(r), _ptr(d0), _ptr(S0),
+                                     _ptr(out), _ptr(S), _ptr(d), _ptr(rho), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the sizes")
+    with np.errstate(divide="ignore"):
+        q_geo = np.exp(np.log(rho).mean(axis=1)) if T > 0 else np.ones((B, H))
+    return out, S, d, rho, q_geo
 
 
 def step(q, k, v, beta, S, d, r=None, eta=1e-2):

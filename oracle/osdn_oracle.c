@@ -31,6 +31,12 @@
  *   - play-then-update: token t writes with d_t, and d_1 = d0;
  *   - r_t is an input per (token, head); r == NULL means APF off (r == 1);
  *   - ||k_t||^2 == 0 skips the gradient term (h is undefined there).
+ *
+ * Diagnostic (technical summary sections 4-5, the contraction factor of the
+ * gated Newton analysis): the residual ratio of token t,
+ *       rho_t = f_t(S_t) / f_t(S_{t-1}) = (1 - beta_t <d_t, k_t^2>)^2,
+ * from the same <d_t, k_t^2> the d step uses (pinned against the S
+ * trajectory in the tests).
  */
 #include <pthread.h>
 #include <stdint.h>
@@ -41,7 +47,7 @@ typedef struct {
     int B, T, H, dk, dv;
     double eta;
     const double *q, *k, *v, *beta, *r, *d0, *S0;
-    double *out, *S_final, *d_final;
+    double *out, *S_final, *d_final, *rho;
     int unit_begin, unit_end;
 } oracle_job;
 
@@ -50,7 +56,7 @@ typedef struct {
  * values. e and a are scratch of dv and dk entries. */
 static void oracle_token(int dk, int dv, double eta, double *S, double *d,
                          const double *q, const double *k, const double *v,
-                         double beta, double r, double *o, double *e, double *a)
+                         double beta, double r, double *o, double *e, double *a, double *rho)
 {
     double n = 0.0, s = 0.0;
     for (int i = 0; i < dk; ++i) {
@@ -58,6 +64,7 @@ static void oracle_token(int dk, int dv, double eta, double *S, double *d,
         n += a[i];                    /* ||k_t||^2 */
         s += d[i] * a[i];             /* <d_t, k_t^2> with the pre-update d */
     }
+    if (rho) *rho = (1.0 - beta * s) * (1.0 - beta * s);
     /* residual e = S_{t-1} k_t - v_t (gradient of f_t is e k_t^T) */
     for (int row = 0; row < dv; ++row) {
         double acc = 0.0;
@@ -103,7 +110,7 @@ static void *oracle_worker(void *arg)
             oracle_token(dk, dv, J->eta, S, d,
                          J->q + tok * dk, J->k + tok * dk, J->v + tok * dv,
                          J->beta[tok], J->r ? J->r[tok] : 1.0,
-                         J->out + tok * dv, e, a);
+                         J->out + tok * dv, e, a, J->rho ? J->rho + tok : NULL);
         }
         if (J->S_final) memcpy(J->S_final + (size_t)u * dv * dk, S, sizeof(double) * (size_t)dv * dk);
         if (J->d_final) memcpy(J->d_final + (size_t)u * dk, d, sizeof(double) * (size_t)dk);
@@ -115,15 +122,15 @@ static void *oracle_worker(void *arg)
 /* Forward over a whole sequence batch.
  * q, k: [B, T, H, dk]; v, out: [B, T, H, dv]; beta, r: [B, T, H] (r may be NULL);
  * d0: [B, H, dk] (NULL = ones); S0: [B, H, dv, dk] (NULL = zeros);
- * S_final: [B, H, dv, dk], d_final: [B, H, dk] (either may be NULL).
+ * S_final: [B, H, dv, dk], d_final: [B, H, dk], rho: [B, T, H] (any may be NULL).
  * The (b, h) units are independent; nthreads host threads share them.
  * Returns 0, or -1 on bad sizes. */
-int osdn_oracle_fwd(int B, int T, int H, int dk, int dv, double eta,
-                    const double *q, const double *k, const double *v,
-                    const double *beta, const double *r,
-                    const double *d0, const double *S0,
-                    double *out, double *S_final, double *d_final,
-                    int nthreads)
+int osdn_oracle_fwd_rho(int B, int T, int H, int dk, int dv, double eta,
+                        const double *q, const double *k, const double *v,
+                        const double *beta, const double *r,
+                        const double *d0, const double *S0,
+                        double *out, double *S_final, double *d_final, double *rho,
+                        int nthreads)
 {
     if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
     const int units = B * H;
@@ -134,7 +141,7 @@ int osdn_oracle_fwd(int B, int T, int H, int dk, int dv, double eta,
     pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
     for (int w = 0; w < nthreads; ++w) {
         oracle_job J = {B, T, H, dk, dv, eta, q, k, v, beta, r, d0, S0,
-                        out, S_final, d_final,
+                        out, S_final, d_final, rho,
                         (int)((long long)units * w / nthreads),
                         (int)((long long)units * (w + 1) / nthreads)};
         jobs[w] = J;
@@ -144,6 +151,17 @@ int osdn_oracle_fwd(int B, int T, int H, int dk, int dv, double eta,
     for (int w = 1; w < nthreads; ++w) pthread_join(th[w], NULL);
     free(jobs); free(th);
     return 0;
+}
+
+int osdn_oracle_fwd(int B, int T, int H, int dk, int dv, double eta,
+                    const double *q, const double *k, const double *v,
+                    const double *beta, const double *r,
+                    const double *d0, const double *S0,
+                    double *out, double *S_final, double *d_final,
+                    int nthreads)
+{
+    return osdn_oracle_fwd_rho(B, T, H, dk, dv, eta, q, k, v, beta, r, d0, S0, out, S_final, d_final, NULL,
+                               nthreads);
 }
 
 /* One decode token for every (b, h): q, k [B, H, dk]; v, out [B, H, dv];
@@ -160,7 +178,7 @@ int osdn_oracle_step(int B, int H, int dk, int dv, double eta,
     for (int u = 0; u < B * H; ++u) {
         oracle_token(dk, dv, eta, S + (size_t)u * dv * dk, d + (size_t)u * dk,
                      q + (size_t)u * dk, k + (size_t)u * dk, v + (size_t)u * dv,
-                     beta[u], r ? r[u] : 1.0, out + (size_t)u * dv, e, a);
+                     beta[u], r ? r[u] : 1.0, out + (size_t)u * dv, e, a, NULL);
     }
     free(e); free(a);
     return 0;

@@ -15,11 +15,11 @@ import torch
 
 from ._binding import (OSDN_BF16, OSDN_ERR_CUDA, OSDN_ERR_INVALID_ARG, OSDN_ERR_TIMEOUT, OSDN_ERR_UNSUPPORTED,
                        OSDN_FP32, OSDN_OK, LIB_PATH, OsdnError, build, get_last_error, make_params, osdn_fwd,
-                       osdn_fwd_chunk, osdn_fwd_scan,
+                       osdn_fwd_chunk, osdn_fwd_scan, osdn_fwd_scan_diag,
                        osdn_fwd_workspace_size, osdn_params, osdn_set_wait_limit_ns, osdn_step,
                        osdn_sync_status)
 
-__all__ = ["forward", "step", "osdn_fwd", "osdn_fwd_scan", "osdn_fwd_chunk", "osdn_step", "osdn_fwd_workspace_size", "osdn_sync_status",
+__all__ = ["forward", "step", "residual_ratio", "osdn_fwd_scan_diag", "osdn_fwd", "osdn_fwd_scan", "osdn_fwd_chunk", "osdn_step", "osdn_fwd_workspace_size", "osdn_sync_status",
            "osdn_set_wait_limit_ns",
            "osdn_params", "make_params", "get_last_error", "OsdnError", "build", "LIB_PATH",
            "OSDN_OK", "OSDN_ERR_INVALID_ARG", "OSDN_ERR_UNSUPPORTED", "OSDN_ERR_CUDA", "OSDN_ERR_TIMEOUT",
@@ -41,6 +41,21 @@ def forward(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, chunk=64, workspa
         workspace = torch.empty(osdn_fwd_workspace_size(p), dtype=torch.uint8, device=dev)
     osdn_fwd(p, q, k, v, beta, r, d0, S0, out, final_S, final_d, workspace, stream)
     return out, final_S, final_d
+
+
+def residual_ratio(k, beta, r=None, d0=None, eta=1e-2, stream=None):
+    """Preconditioner scan with its residual-ratio diagnostic: k [B,T,H,dk]; beta, r [B,T,H];
+    d0 [B,H,dk] fp32 (None = ones). Returns rho [B,T,H] fp32 (rho_t = (1 - beta_t <d_t, k_t^2>)^2,
+    the factor by which token t's write shrinks its own loss), q_geo [B,H] fp32 (exp of the mean
+    log rho over each sequence) and d after the last token [B,H,dk] fp32."""
+    B, T, H, dk = k.shape
+    p = make_params(B, T, H, dk, dk, k.dtype, eta)
+    rho = torch.empty((B, T, H), dtype=torch.float32, device=k.device)
+    q_geo = torch.empty((B, H), dtype=torch.float32, device=k.device)
+    d = torch.empty((B, H, dk), dtype=torch.float32, device=k.device)
+    ws = torch.empty(max(osdn_fwd_workspace_size(p), 256), dtype=torch.uint8, device=k.device)
+    osdn_fwd_scan_diag(p, k, beta, r, d0, d, rho, q_geo, ws, stream)
+    return rho, q_geo, d
 
 
 def step(q, k, v, beta, S, d, r=None, eta=1e-2, stream=None):

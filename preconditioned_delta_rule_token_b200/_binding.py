@@ -83,6 +83,8 @@ def lib():
         L.osdn_fwd.restype = ctypes.c_int
         L.osdn_fwd_scan.argtypes = [P] + [vp] * 5 + [vp, sz, vp]
         L.osdn_fwd_scan.restype = ctypes.c_int
+        L.osdn_fwd_scan_diag.argtypes = [P] + [vp] * 7 + [vp, sz, vp]
+        L.osdn_fwd_scan_diag.restype = ctypes.c_int
         L.osdn_fwd_chunk.argtypes = [P] + [vp] * 7 + [vp, sz, vp]
         L.osdn_fwd_chunk.restype = ctypes.c_int
         L.osdn_fwd_noalloc.argtypes = [P] + [vp] * 10 + [vp]
@@ -157,6 +159,13 @@ def osdn_fwd_scan(params, k, beta, r, d0, final_d, workspace, stream=None):
     """Raw C-ABI call of phase 1 (preconditioner scan into the workspace)."""
     _check(lib().osdn_fwd_scan(ctypes.byref(params), _ptr(k), _ptr(beta), _ptr(r), _ptr(d0), _ptr(final_d),
                                _ptr(workspace), ctypes.c_size_t(_ws_bytes(workspace)), _stream(stream)))
+
+
+def osdn_fwd_scan_diag(params, k, beta, r, d0, final_d, rho, q_geo, workspace, stream=None):
+    """Raw C-ABI call of phase 1 with the residual-ratio diagnostic (rho, q_geo nullable)."""
+    _check(lib().osdn_fwd_scan_diag(ctypes.byref(params), _ptr(k), _ptr(beta), _ptr(r), _ptr(d0), _ptr(final_d),
+                                    _ptr(rho), _ptr(q_geo), _ptr(workspace), ctypes.c_size_t(_ws_bytes(workspace)),
+                                    _stream(stream)))
 
 
 def osdn_fwd_chunk(params, q, k, v, beta, S0, out, final_S, workspace, stream=None):

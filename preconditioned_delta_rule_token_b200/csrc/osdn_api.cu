@@ -166,7 +166,8 @@ int launch_chunk_wy(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfl
 
 // Phase 1 in chunk form on the tensor cores: bf16, dk = 128.
 int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bfloat16* beta,
-                   const __nv_bfloat16* r, const float* d0, float* final_d, __nv_bfloat16* kw, cudaStream_t st) {
+                   const __nv_bfloat16* r, const float* d0, float* final_d, __nv_bfloat16* kw, float* rho,
+                   float* q_geo, cudaStream_t st) {
     CUtensorMap mk, mkw;
     int rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128);
     if (rc) return rc;
@@ -176,7 +177,7 @@ int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bflo
     const size_t smem = osdn::ScanLayout::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan kernel attribute");
-    kern<<<p->B * p->H, 384, smem, st>>>(mk, mkw, beta, r, d0, final_d, p->B, p->T, p->H, p->eta,
+    kern<<<p->B * p->H, 384, smem, st>>>(mk, mkw, beta, r, d0, final_d, rho, q_geo, p->B, p->T, p->H, p->eta,
                                          g_wait_limit_ns.load());
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");
     return OSDN_OK;
@@ -186,17 +187,27 @@ int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bflo
 // Phase 1: preconditioner scan -> scaled write keys (workspace) and final d.
 template <typename Tin>
 int launch_scan(const osdn_params* p, const Tin* k, const Tin* beta, const Tin* r, const float* d0, float* final_d,
-                Tin* kw, cudaStream_t st) {
-    if (p->T == 0) return copy_initial_state(p, d0, nullptr, nullptr, final_d, false, true, st);
+                Tin* kw, cudaStream_t st, float* rho = nullptr, float* q_geo = nullptr) {
+    if (p->T == 0) {
+        if (q_geo) {   // empty sequences: the geometric mean of no ratios is 1
+            const size_t n = (size_t)p->B * p->H, blocks = (n + 255) / 256;
+            fill_ones_kernel<<<(unsigned)(blocks > 1024 ? 1024 : blocks), 256, 0, st>>>(q_geo, n);
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return cuda_fail(e, "q_geo fill");
+        }
+        return copy_initial_state(p, d0, nullptr, nullptr, final_d, false, true, st);
+    }
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
-        if (p->dk == 128) return launch_scan_tc(p, k, beta, r, d0, final_d, kw, st);
+        if (p->dk == 128) return launch_scan_tc(p, k, beta, r, d0, final_d, kw, rho, q_geo, st);
     }
     const int units = p->B * p->H;
     const dim3 grid((units + 3) / 4);
     if (p->dk == 128)
-        osdn::scan_seq_kernel<128, Tin><<<grid, 128, 0, st>>>(k, beta, r, d0, kw, final_d, p->B, p->T, p->H, p->eta);
+        osdn::scan_seq_kernel<128, Tin><<<grid, 128, 0, st>>>(k, beta, r, d0, kw, final_d, rho, q_geo, p->B, p->T,
+                                                               p->H, p->eta);
     else
-        osdn::scan_seq_kernel<64, Tin><<<grid, 128, 0, st>>>(k, beta, r, d0, kw, final_d, p->B, p->T, p->H, p->eta);
+        osdn::scan_seq_kernel<64, Tin><<<grid, 128, 0, st>>>(k, beta, r, d0, kw, final_d, rho, q_geo, p->B, p->T,
+                                                              p->H, p->eta);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     return OSDN_OK;
@@ -346,6 +357,24 @@ int osdn_fwd_scan(const osdn_params* p, const void* k, const void* beta, const v
         return launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, (T*)ws, st);
     }
     return launch_scan<float>(p, (const float*)k, (const float*)beta, (const float*)r, d0, final_d, (float*)ws, st);
+}
+
+int osdn_fwd_scan_diag(const osdn_params* p, const void* k, const void* beta, const void* r, const float* d0,
+                       float* final_d, float* rho, float* q_geo, void* workspace, size_t workspace_bytes,
+                       void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    rc = check_fwd_args(p, {k, beta}, {k, beta, r, d0, final_d, rho, q_geo}, workspace, workspace_bytes);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    char* ws = reinterpret_cast<char*>(workspace) + layout_of(p).kw_off;
+    if (p->dtype == OSDN_BF16) {
+        using T = __nv_bfloat16;
+        return launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, (T*)ws, st, rho, q_geo);
+    }
+    return launch_scan<float>(p, (const float*)k, (const float*)beta, (const float*)r, d0, final_d, (float*)ws, st,
+                              rho, q_geo);
 }
 
 int osdn_fwd_chunk(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta,

@@ -10,6 +10,9 @@
 // per-token reductions (<d, k^2> and ||k||^2) are warp shuffles.  This form is
 // latency-bound (one warp reduction per token); it serves fp32 mode and short
 // sequences, and is the reference layout for the chunk-parallel scan.
+// Optional diagnostic (sections 4-5): the residual ratio of each write,
+// rho_t = (1 - beta_t <d_t, k_t^2>)^2 = f_t(S_t)/f_t(S_{t-1}) into rho [B, T, H],
+// and q_geo = exp(mean_t log rho_t) per (sequence, head) into q_geo [B, H].
 #pragma once
 #include "common.cuh"
 
@@ -19,7 +22,7 @@ template <int DK, typename Tin>
 __global__ void __launch_bounds__(128)
 scan_seq_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const Tin* __restrict__ r,
                 const float* __restrict__ d0, Tin* __restrict__ kw, float* __restrict__ d_final,
-                int B, int T, int H, float eta)
+                float* __restrict__ rho, float* __restrict__ q_geo, int B, int T, int H, float eta)
 {
     constexpr int PER = DK / 32;
     const int lane = threadIdx.x & 31;
@@ -39,6 +42,7 @@ scan_seq_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const T
     size_t tok = (size_t)b * T * H + h;              // token (b, 0, h)
     float kc[PER], kn[PER];
     float bc = 0.f, rc = 1.f, bn = 0.f, rn = 1.f;
+    float log_rho = 0.f;                             // sum over tokens of log rho_t
     if (T > 0) {
         VecIO<PER, Tin>::load(k + tok * DK + lane * PER, kc);
         bc = to_f32(beta[tok]);
@@ -64,6 +68,11 @@ scan_seq_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const T
         n = warp_sum(n);
         s = warp_sum(s);
         const float x = (n > 0.f) ? eta * bc * (1.f - bc * s) / n : 0.f;
+        if (rho || q_geo) {
+            const float rt = (1.f - bc * s) * (1.f - bc * s);
+            if (rho && lane == 0) rho[tok] = rt;
+            log_rho += logf(rt);
+        }
 #pragma unroll
         for (int i = 0; i < PER; ++i) d[i] = rc * d[i] + x * a[i];
         tok = nxt;
@@ -72,6 +81,7 @@ scan_seq_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const T
         bc = bn; rc = rn;
     }
     if (d_final) VecIO<PER, float>::store(d_final + (size_t)unit * DK + lane * PER, d);
+    if (q_geo && lane == 0) q_geo[unit] = T > 0 ? expf(log_rho / (float)T) : 1.f;
 }
 
 }  // namespace osdn

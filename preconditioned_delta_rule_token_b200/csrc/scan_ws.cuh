@@ -26,6 +26,13 @@
 //     kw_t[i] = d_t[i] k_t[i] over k_t[i] and carrying d; then one TMA store of
 //     the block's scaled keys; its buffer takes the block three ahead once the
 //     store has read it (issued at the start of the next block).
+// Optional diagnostic (sections 4-5): the residual ratio of each write,
+// rho_t = (1 - beta_t <d_t, k_t^2>)^2 = f_t(S_t)/f_t(S_{t-1}), into rho [B, T, H]
+// and q_geo = exp(mean_t log rho_t) per (sequence, head). Since
+// x_t = g_t (1 - beta_t <d_t, k_t^2>), 1 - beta_t <d_t, k_t^2> = x_t / g_t when
+// g_t != 0; with g_t = 0 and a write (eta = 0) the x are all zero, d_t = R_{t,0} d_c
+// and the factor is 1 - beta_t R_{t,0} b_t; with no write (beta_t = 0 or k_t = 0)
+// rho_t = 1.
 // K blocks are triple-buffered; N, the per-token vectors and the hand-offs are
 // double-buffered by block parity. Bounded mbarrier waits with a shared abort
 // flag, as in the chunk kernel.
@@ -47,7 +54,7 @@ struct ScanLayout {
     enum { V_BETA = 0, V_R = 128, V_G = 256, V_INVN = 384, V_R0 = 512, V_PAR = 640 };
     static constexpr uint32_t NP = VEC + 2 * V_PAR * 4;      // prep: ||k_t||^2 halves [2][128]
     static constexpr uint32_t CV = NP + 256 * 4;             // chain: c (64), x / ||k||^2 (64), d (128)
-    enum { C_C = 0, C_X = 64, C_D = 128, C_N = 256 };
+    enum { C_C = 0, C_X = 64, C_D = 128, C_B = 256, C_LR = 320, C_N = 324 };   // + b_t (64), log-rho sums (4)
     static constexpr uint32_t BAR = CV + C_N * 4;
     enum {
         FULL = 0,    // 3: K block landed
@@ -68,8 +75,8 @@ template <int kUnused = 0>
 __global__ void __launch_bounds__(384, 1)
 scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kw,
                const __nv_bfloat16* __restrict__ beta, const __nv_bfloat16* __restrict__ r,
-               const float* __restrict__ d0, float* __restrict__ d_final, int B, int T, int H, float eta,
-               unsigned long long wait_limit_ns)
+               const float* __restrict__ d0, float* __restrict__ d_final, float* __restrict__ rho,
+               float* __restrict__ q_geo, int B, int T, int H, float eta, unsigned long long wait_limit_ns)
 {
     constexpr int DK = 128, BLK = 128, SUB = 64;
     constexpr uint32_t NCOLS = 128;
@@ -129,6 +136,9 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         float* s_c = cv + L::C_C;
         float* s_x = cv + L::C_X;
         float* s_d = cv + L::C_D;
+        float* s_b = cv + L::C_B;
+        const bool diag = rho != nullptr || q_geo != nullptr;
+        float log_rho = 0.f;   // this thread's share of sum_t log rho_t
         constexpr int kTmaThread = 32;
         int issued = 0;   // K blocks whose load was issued
         auto load_k = [&](int blk) {
@@ -171,7 +181,10 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                         }
                     }
                     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                    if (half == 0) s_c[tl_] = vb[L::V_G + t] * (1.f - vb[L::V_BETA + t] * vb[L::V_R0 + t] * acc);
+                    if (half == 0) {
+                        s_c[tl_] = vb[L::V_G + t] * (1.f - vb[L::V_BETA + t] * vb[L::V_R0 + t] * acc);
+                        s_b[tl_] = acc;
+                    }
                 }
                 if (s == 0 && tid == kTmaThread && blk > 0 && issued < nblk) {
                     // the buffer of block blk - 1 takes block blk + 2 once its store has read it (issued
@@ -195,7 +208,17 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                         acc = fmaf(n4.x, c4.x, fmaf(n4.y, c4.y, fmaf(n4.z, c4.z, fmaf(n4.w, c4.w, acc))));
                     }
                     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                    if (half == 0) s_x[tl_] = acc * vb[L::V_INVN + s * SUB + tl_];
+                    const int t = s * SUB + tl_;
+                    if (half == 0) s_x[tl_] = acc * vb[L::V_INVN + t];
+                    if (diag && half == 0 && t < Tb) {   // residual ratio of token t (acc = x_t)
+                        const float gt = vb[L::V_G + t], bt = vb[L::V_BETA + t];
+                        float f = 1.f;
+                        if (gt != 0.f) f = acc / gt;
+                        else if (bt != 0.f && vb[L::V_INVN + t] > 0.f) f = 1.f - bt * vb[L::V_R0 + t] * s_b[tl_];
+                        const float rt = f * f;
+                        if (rho) rho[((size_t)b * T + blk * BLK + t) * H + h] = rt;
+                        log_rho += logf(rt);
+                    }
                 }
                 tc::named_sync(BAR_CHAIN, 128);
                 {   // feature i through the sub-chunk, 32 tokens at a time from registers:
@@ -251,6 +274,14 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                 tc::mbar_wait(bars + L::FULL + q % L::NKB, (q / L::NKB) & 1, 1000000000ull);
         }
         if (blk == nblk && !*abort_flag && d_final) d_final[(size_t)unit * DK + tid] = s_d[tid];
+        if (q_geo) {   // q_geo = exp(mean log rho): warp sums, then one thread
+            float* lr = cv + L::C_LR;
+            const float ws = warp_sum(log_rho);
+            if (lane == 0) lr[warp] = ws;
+            tc::named_sync(BAR_CHAIN, 128);
+            if (tid == 0 && blk == nblk && !*abort_flag)
+                q_geo[unit] = T > 0 ? expf((lr[0] + lr[1] + lr[2] + lr[3]) / (float)T) : 1.f;
+        }
     } else {
         // ================================================================ prep groups
         const int tp = tid - 128;              // 0..255

@@ -101,6 +101,18 @@ def test_full_size_workloads_on_sampled_units(w, units):
         assert max(errs) <= BF16_TOL, (b, h, errs)
 
 
+def test_more_units_than_sms_every_unit():
+    """320 (b, h) units (B5 H64) run the tensor-core scan and chunk kernels in more than
+    one wave of CTAs (one CTA per unit, 148 SMs); ragged T = 130 spans three 64-token
+    chunks and two 128-token scan blocks. Every unit is checked against the oracle."""
+    w = W.Workload("multi-wave B5 H64 T130 d128 bf16", 5, 64, 130, 128, 128, 64, W.BF16, True, "gaussian",
+                   d0="uniform", S0="normal", seed=21)
+    inp = W.make_forward_inputs(w)
+    gpu = _run_gpu(inp, w.eta)
+    errs = _errs(gpu, _oracle(inp, w.eta))
+    assert max(errs) <= BF16_TOL, errs
+
+
 def test_zero_tokens_returns_initial_state():
     import preconditioned_delta_rule_token_b200 as pk
     w = W.Workload("t0", 2, 2, 0, 128, 128, 64, W.BF16, True, d0="uniform", S0="normal", seed=5)
