@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define OSDN_ABI_VERSION 1
+#define OSDN_ABI_VERSION 2
 
 enum {
     OSDN_OK = 0,
@@ -66,7 +66,11 @@ typedef struct {
     int32_t chunk;          /* chunk length C of the chunkwise form; 64 */
     int32_t dtype;          /* osdn_dtype of q, k, v, beta, r, out */
     float eta;              /* hypergradient step size of the preconditioner */
+    int32_t apf_anchor;     /* 0: APF retention r d (toward 0); 1: anchored APF,
+                               r d + (1 - r) d_anchor, d_anchor = d0 in the forward */
 } osdn_params;
+/* Version 1 of this struct ended after eta (struct_size 36); such callers get
+ * apf_anchor = 0. */
 
 /* Bytes of device workspace osdn_fwd needs for these parameters (written to
  * *bytes). The workspace holds the scaled write keys d_t (.) k_t in the input
@@ -84,6 +88,8 @@ int osdn_fwd_workspace_size(const osdn_params *p, size_t *bytes);
  *   T = (I + A)^{-1}, U = T diag(beta) (V - K S^T),
  *   O = Q S^T + tril(Q Kw^T) U, S <- S + U^T Kw (Kw = scaled write keys).
  * r == NULL: APF off (r == 1). d0 == NULL: d0 = ones. S0 == NULL: S0 = 0.
+ * p->apf_anchor != 0: anchored APF, d_{t+1} = r_t d_t + (1 - r_t) d0 + (the same
+ * hypergradient step), i.e. the retention pulls d toward d0 instead of 0.
  * final_S, final_d may be NULL (not written). out may not be NULL when T > 0.
  * workspace must hold osdn_fwd_workspace_size() bytes (16-byte aligned).
  * Errors: OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED, OSDN_ERR_CUDA. */
@@ -144,6 +150,17 @@ int osdn_step(const osdn_params *p,
               const void *beta, const void *r,
               float *S, float *d, void *out,
               void *cuda_stream);
+
+/* osdn_step with anchored APF (p->apf_anchor != 0): the retention step becomes
+ * d <- r d + (1 - r) d_anchor + eta beta (1 - beta <d, k^2>) k^2 / ||k||^2,
+ * d_anchor [B, H, dk] fp32 (NULL: ones; the d0 of the forward). With
+ * p->apf_anchor == 0, d_anchor is ignored and this is osdn_step. */
+int osdn_step_ex(const osdn_params *p,
+                 const void *q, const void *k, const void *v,
+                 const void *beta, const void *r, const float *d_anchor,
+                 float *S, float *d, void *out,
+                 void *cuda_stream);
+
 
 /* Largest scratch osdn_fwd_noalloc can use: B * T * H * dk * element size
  * (2 bytes for bf16, 4 for fp32) must not exceed this. */

@@ -47,6 +47,11 @@ def _load():
         lib.osdn_oracle_fwd.restype = ctypes.c_int
         lib.osdn_oracle_fwd_rho.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [dp] * 11 + [ctypes.c_int]
         lib.osdn_oracle_fwd_rho.restype = ctypes.c_int
+        lib.osdn_oracle_fwd_ex.argtypes = ([ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int] + [dp] * 11 +
+                                           [ctypes.c_int])
+        lib.osdn_oracle_fwd_ex.restype = ctypes.c_int
+        lib.osdn_oracle_step_ex.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [dp] * 9
+        lib.osdn_oracle_step_ex.restype = ctypes.c_int
         lib.osdn_oracle_step.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [dp] * 8
         lib.osdn_oracle_step.restype = ctypes.c_int
         _lib = lib
@@ -65,8 +70,8 @@ def _f64(a):
     return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
 
 
-def fwd(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=None):
-    """Token-by-token OSDN forward in float64.
+def fwd(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=None, anchor=False):
+    """Token-by-token OSDN forward in float64 (anchor: anchored APF, retention toward d0).
 
     q, k: [B, T, H, dk]; v: [B, T, H, dv]; beta, r: [B, T, H] (r None = APF off);
     d0: [B, H, dk] (None = ones); S0: [B, H, dv, dk] (None = zeros).
@@ -84,15 +89,15 @@ def fwd(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=None):
     d = np.zeros((B, H, dk), np.float64)
     if nthreads is None:
         nthreads = os.cpu_count() or 1
-    rc = _load().osdn_oracle_fwd(B, T, H, dk, dv, float(eta), _ptr(q), _ptr(k), _ptr(v),
-                                 _ptr(beta), _ptr(r), _ptr(d0), _ptr(S0),
-                                 _ptr(out), _ptr(S), _ptr(d), int(nthreads))
+    rc = _load().osdn_oracle_fwd_ex(B, T, H, dk, dv, float(eta), int(bool(anchor)), _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(beta), _ptr(r), _ptr(d0), _ptr(S0),
+                                    _ptr(out), _ptr(S), _ptr(d), None, int(nthreads))
     if rc != 0:
         raise ValueError("oracle rejected the sizes")
     return out, S, d
 
 
-def residual_ratio(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=None):
+def residual_ratio(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=None, anchor=False):
     """The forward of fwd() plus the per-token residual ratio
     rho_t = (1 - beta_t <d_t, k_t^2>)^2 = f_t(S_t) / f_t(S_{t-1}) [B, T, H] and its
     geometric mean over each sequence, q_geo = exp(mean_t log rho_t) [B, H]
@@ -107,9 +112,9 @@ def residual_ratio(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=N
     rho = np.zeros((B, T, H), np.float64)
     if nthreads is None:
         nthreads = os.cpu_count() or 1
-    rc = _load().osdn_oracle_fwd_rho(B, T, H, dk, dv, float(eta), _ptr(q), _ptr(k), _ptr(v),
-                                     _ptr(beta), _ptr(r), _ptr(d0), _ptr(S0),
-                                     _ptr(out), _ptr(S), _ptr(d), _ptr(rho), int(nthreads))
+    rc = _load().osdn_oracle_fwd_ex(B, T, H, dk, dv, float(eta), int(bool(anchor)), _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(beta), _ptr(r), _ptr(d0), _ptr(S0),
+                                    _ptr(out), _ptr(S), _ptr(d), _ptr(rho), int(nthreads))
     if rc != 0:
         raise ValueError("oracle rejected the sizes")
     with np.errstate(divide="ignore"):
@@ -117,18 +122,19 @@ def residual_ratio(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=N
     return out, S, d, rho, q_geo
 
 
-def step(q, k, v, beta, S, d, r=None, eta=1e-2):
+def step(q, k, v, beta, S, d, r=None, eta=1e-2, d_anchor=None):
     """One decode token for every (b, h), float64, S [B,H,dv,dk] and d [B,H,dk]
-    updated in place (they must be contiguous float64 arrays). Returns out [B,H,dv]."""
-    q, k, v, beta, r = map(_f64, (q, k, v, beta, r))
+    updated in place (they must be contiguous float64 arrays); d_anchor [B,H,dk]
+    selects anchored APF toward it. Returns out [B,H,dv]."""
+    q, k, v, beta, r, d_anchor = map(_f64, (q, k, v, beta, r, d_anchor))
     assert S.dtype == np.float64 and S.flags.c_contiguous
     assert d.dtype == np.float64 and d.flags.c_contiguous
     B, H, dk = k.shape
     dv = v.shape[-1]
     assert S.shape == (B, H, dv, dk) and d.shape == (B, H, dk)
     out = np.zeros((B, H, dv), np.float64)
-    rc = _load().osdn_oracle_step(B, H, dk, dv, float(eta), _ptr(q), _ptr(k), _ptr(v),
-                                  _ptr(beta), _ptr(r), _ptr(S), _ptr(d), _ptr(out))
+    rc = _load().osdn_oracle_step_ex(B, H, dk, dv, float(eta), _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(beta), _ptr(r), _ptr(d_anchor), _ptr(S), _ptr(d), _ptr(out))
     if rc != 0:
         raise ValueError("oracle rejected the sizes")
     return out

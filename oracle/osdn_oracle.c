@@ -32,6 +32,10 @@
  *   - r_t is an input per (token, head); r == NULL means APF off (r == 1);
  *   - ||k_t||^2 == 0 skips the gradient term (h is undefined there).
  *
+ * Anchored APF (an option; the "refresh the calibration" reading of the APF
+ * section): the retention pulls d toward its initial value d0 instead of 0,
+ *       d_{t+1} = r_t d_t + (1 - r_t) d0 - eta grad_d h_t(d_t).
+ *
  * Diagnostic (technical summary sections 4-5, the contraction factor of the
  * gated Newton analysis): the residual ratio of token t,
  *       rho_t = f_t(S_t) / f_t(S_{t-1}) = (1 - beta_t <d_t, k_t^2>)^2,
@@ -48,6 +52,7 @@ typedef struct {
     double eta;
     const double *q, *k, *v, *beta, *r, *d0, *S0;
     double *out, *S_final, *d_final, *rho;
+    int anchor;                         /* anchored APF: retention toward d0 */
     int unit_begin, unit_end;
 } oracle_job;
 
@@ -56,7 +61,8 @@ typedef struct {
  * values. e and a are scratch of dv and dk entries. */
 static void oracle_token(int dk, int dv, double eta, double *S, double *d,
                          const double *q, const double *k, const double *v,
-                         double beta, double r, double *o, double *e, double *a, double *rho)
+                         double beta, double r, double *o, double *e, double *a, double *rho,
+                         const double *anchor)
 {
     double n = 0.0, s = 0.0;
     for (int i = 0; i < dk; ++i) {
@@ -85,10 +91,10 @@ static void oracle_token(int dk, int dv, double eta, double *S, double *d,
         for (int i = 0; i < dk; ++i) acc += Srow[i] * q[i];
         o[row] = acc;
     }
-    /* d_{t+1} = r d_t + eta beta (1 - beta s) k^2 / ||k||^2 */
+    /* d_{t+1} = r d_t (+ (1 - r) d0 when anchored) + eta beta (1 - beta s) k^2 / ||k||^2 */
     double x = 0.0;
     if (n > 0.0) x = eta * beta * (1.0 - beta * s) / n;
-    for (int i = 0; i < dk; ++i) d[i] = r * d[i] + x * a[i];
+    for (int i = 0; i < dk; ++i) d[i] = r * d[i] + (anchor ? (1.0 - r) * anchor[i] : 0.0) + x * a[i];
 }
 
 static void *oracle_worker(void *arg)
@@ -99,23 +105,26 @@ static void *oracle_worker(void *arg)
     double *d = (double *)malloc(sizeof(double) * (size_t)dk);
     double *e = (double *)malloc(sizeof(double) * (size_t)dv);
     double *a = (double *)malloc(sizeof(double) * (size_t)dk);
+    double *d_start = (double *)malloc(sizeof(double) * (size_t)dk);
     for (int u = J->unit_begin; u < J->unit_end; ++u) {
         const int b = u / H, h = u % H;
         if (J->S0) memcpy(S, J->S0 + (size_t)u * dv * dk, sizeof(double) * (size_t)dv * dk);
         else memset(S, 0, sizeof(double) * (size_t)dv * dk);
         if (J->d0) memcpy(d, J->d0 + (size_t)u * dk, sizeof(double) * (size_t)dk);
         else for (int i = 0; i < dk; ++i) d[i] = 1.0;
+        memcpy(d_start, d, sizeof(double) * (size_t)dk);
         for (int t = 0; t < T; ++t) {
             const size_t tok = ((size_t)b * T + t) * H + h;  /* [B, T, H] */
             oracle_token(dk, dv, J->eta, S, d,
                          J->q + tok * dk, J->k + tok * dk, J->v + tok * dv,
                          J->beta[tok], J->r ? J->r[tok] : 1.0,
-                         J->out + tok * dv, e, a, J->rho ? J->rho + tok : NULL);
+                         J->out + tok * dv, e, a, J->rho ? J->rho + tok : NULL,
+                         J->anchor ? d_start : NULL);
         }
         if (J->S_final) memcpy(J->S_final + (size_t)u * dv * dk, S, sizeof(double) * (size_t)dv * dk);
         if (J->d_final) memcpy(J->d_final + (size_t)u * dk, d, sizeof(double) * (size_t)dk);
     }
-    free(S); free(d); free(e); free(a);
+    free(S); free(d); free(e); free(a); free(d_start);
     return NULL;
 }
 
@@ -125,12 +134,12 @@ static void *oracle_worker(void *arg)
  * S_final: [B, H, dv, dk], d_final: [B, H, dk], rho: [B, T, H] (any may be NULL).
  * The (b, h) units are independent; nthreads host threads share them.
  * Returns 0, or -1 on bad sizes. */
-int osdn_oracle_fwd_rho(int B, int T, int H, int dk, int dv, double eta,
-                        const double *q, const double *k, const double *v,
-                        const double *beta, const double *r,
-                        const double *d0, const double *S0,
-                        double *out, double *S_final, double *d_final, double *rho,
-                        int nthreads)
+int osdn_oracle_fwd_ex(int B, int T, int H, int dk, int dv, double eta, int anchor,
+                       const double *q, const double *k, const double *v,
+                       const double *beta, const double *r,
+                       const double *d0, const double *S0,
+                       double *out, double *S_final, double *d_final, double *rho,
+                       int nthreads)
 {
     if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
     const int units = B * H;
@@ -141,7 +150,7 @@ int osdn_oracle_fwd_rho(int B, int T, int H, int dk, int dv, double eta,
     pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
     for (int w = 0; w < nthreads; ++w) {
         oracle_job J = {B, T, H, dk, dv, eta, q, k, v, beta, r, d0, S0,
-                        out, S_final, d_final, rho,
+                        out, S_final, d_final, rho, anchor,
                         (int)((long long)units * w / nthreads),
                         (int)((long long)units * (w + 1) / nthreads)};
         jobs[w] = J;
@@ -153,6 +162,17 @@ int osdn_oracle_fwd_rho(int B, int T, int H, int dk, int dv, double eta,
     return 0;
 }
 
+int osdn_oracle_fwd_rho(int B, int T, int H, int dk, int dv, double eta,
+                        const double *q, const double *k, const double *v,
+                        const double *beta, const double *r,
+                        const double *d0, const double *S0,
+                        double *out, double *S_final, double *d_final, double *rho,
+                        int nthreads)
+{
+    return osdn_oracle_fwd_ex(B, T, H, dk, dv, eta, 0, q, k, v, beta, r, d0, S0, out, S_final, d_final, rho,
+                              nthreads);
+}
+
 int osdn_oracle_fwd(int B, int T, int H, int dk, int dv, double eta,
                     const double *q, const double *k, const double *v,
                     const double *beta, const double *r,
@@ -160,17 +180,18 @@ int osdn_oracle_fwd(int B, int T, int H, int dk, int dv, double eta,
                     double *out, double *S_final, double *d_final,
                     int nthreads)
 {
-    return osdn_oracle_fwd_rho(B, T, H, dk, dv, eta, q, k, v, beta, r, d0, S0, out, S_final, d_final, NULL,
-                               nthreads);
+    return osdn_oracle_fwd_ex(B, T, H, dk, dv, eta, 0, q, k, v, beta, r, d0, S0, out, S_final, d_final, NULL,
+                              nthreads);
 }
 
 /* One decode token for every (b, h): q, k [B, H, dk]; v, out [B, H, dv];
  * beta, r [B, H] (r may be NULL); S [B, H, dv, dk] and d [B, H, dk] updated
- * in place. Same arithmetic as one step of osdn_oracle_fwd. */
-int osdn_oracle_step(int B, int H, int dk, int dv, double eta,
-                     const double *q, const double *k, const double *v,
-                     const double *beta, const double *r,
-                     double *S, double *d, double *out)
+ * in place; d_anchor [B, H, dk] (NULL: plain APF, non-NULL: anchored APF
+ * toward it). Same arithmetic as one step of osdn_oracle_fwd_ex. */
+int osdn_oracle_step_ex(int B, int H, int dk, int dv, double eta,
+                        const double *q, const double *k, const double *v,
+                        const double *beta, const double *r, const double *d_anchor,
+                        double *S, double *d, double *out)
 {
     if (B < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
     double *e = (double *)malloc(sizeof(double) * (size_t)dv);
@@ -178,8 +199,17 @@ int osdn_oracle_step(int B, int H, int dk, int dv, double eta,
     for (int u = 0; u < B * H; ++u) {
         oracle_token(dk, dv, eta, S + (size_t)u * dv * dk, d + (size_t)u * dk,
                      q + (size_t)u * dk, k + (size_t)u * dk, v + (size_t)u * dv,
-                     beta[u], r ? r[u] : 1.0, out + (size_t)u * dv, e, a, NULL);
+                     beta[u], r ? r[u] : 1.0, out + (size_t)u * dv, e, a, NULL,
+                     d_anchor ? d_anchor + (size_t)u * dk : NULL);
     }
     free(e); free(a);
     return 0;
+}
+
+int osdn_oracle_step(int B, int H, int dk, int dv, double eta,
+                     const double *q, const double *k, const double *v,
+                     const double *beta, const double *r,
+                     double *S, double *d, double *out)
+{
+    return osdn_oracle_step_ex(B, H, dk, dv, eta, q, k, v, beta, r, NULL, S, d, out);
 }

@@ -16,23 +16,25 @@ import torch
 from ._binding import (OSDN_BF16, OSDN_ERR_CUDA, OSDN_ERR_INVALID_ARG, OSDN_ERR_TIMEOUT, OSDN_ERR_UNSUPPORTED,
                        OSDN_FP32, OSDN_OK, LIB_PATH, OsdnError, build, get_last_error, make_params, osdn_fwd,
                        osdn_fwd_chunk, osdn_fwd_scan, osdn_fwd_scan_diag,
-                       osdn_fwd_workspace_size, osdn_params, osdn_set_wait_limit_ns, osdn_step,
+                       osdn_fwd_workspace_size, osdn_params, osdn_set_wait_limit_ns, osdn_step, osdn_step_ex,
                        osdn_sync_status)
 
 __all__ = ["forward", "step", "residual_ratio", "osdn_fwd_scan_diag", "osdn_fwd", "osdn_fwd_scan", "osdn_fwd_chunk", "osdn_step", "osdn_fwd_workspace_size", "osdn_sync_status",
-           "osdn_set_wait_limit_ns",
+           "osdn_set_wait_limit_ns", "osdn_step_ex",
            "osdn_params", "make_params", "get_last_error", "OsdnError", "build", "LIB_PATH",
            "OSDN_OK", "OSDN_ERR_INVALID_ARG", "OSDN_ERR_UNSUPPORTED", "OSDN_ERR_CUDA", "OSDN_ERR_TIMEOUT",
            "OSDN_BF16", "OSDN_FP32"]
 
 
-def forward(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, chunk=64, workspace=None, stream=None):
+def forward(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, chunk=64, workspace=None, stream=None,
+            apf_anchor=False):
     """OSDN forward. q, k [B,T,H,dk]; v [B,T,H,dv]; beta, r [B,T,H] (bf16 or fp32,
-    one dtype); d0 [B,H,dk] and S0 [B,H,dv,dk] fp32 or None.
+    one dtype); d0 [B,H,dk] and S0 [B,H,dv,dk] fp32 or None. apf_anchor: anchored
+    APF, the retention pulls d toward d0 instead of 0.
     Returns (out [B,T,H,dv], final_S [B,H,dv,dk] fp32, final_d [B,H,dk] fp32)."""
     B, T, H, dk = k.shape
     dv = v.shape[-1]
-    p = make_params(B, T, H, dk, dv, k.dtype, eta, chunk)
+    p = make_params(B, T, H, dk, dv, k.dtype, eta, chunk, apf_anchor)
     dev = k.device
     out = torch.empty((B, T, H, dv), dtype=k.dtype, device=dev)
     final_S = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
@@ -43,13 +45,13 @@ def forward(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, chunk=64, workspa
     return out, final_S, final_d
 
 
-def residual_ratio(k, beta, r=None, d0=None, eta=1e-2, stream=None):
+def residual_ratio(k, beta, r=None, d0=None, eta=1e-2, stream=None, apf_anchor=False):
     """Preconditioner scan with its residual-ratio diagnostic: k [B,T,H,dk]; beta, r [B,T,H];
     d0 [B,H,dk] fp32 (None = ones). Returns rho [B,T,H] fp32 (rho_t = (1 - beta_t <d_t, k_t^2>)^2,
     the factor by which token t's write shrinks its own loss), q_geo [B,H] fp32 (exp of the mean
     log rho over each sequence) and d after the last token [B,H,dk] fp32."""
     B, T, H, dk = k.shape
-    p = make_params(B, T, H, dk, dk, k.dtype, eta)
+    p = make_params(B, T, H, dk, dk, k.dtype, eta, apf_anchor=apf_anchor)
     rho = torch.empty((B, T, H), dtype=torch.float32, device=k.device)
     q_geo = torch.empty((B, H), dtype=torch.float32, device=k.device)
     d = torch.empty((B, H, dk), dtype=torch.float32, device=k.device)
@@ -58,12 +60,13 @@ def residual_ratio(k, beta, r=None, d0=None, eta=1e-2, stream=None):
     return rho, q_geo, d
 
 
-def step(q, k, v, beta, S, d, r=None, eta=1e-2, stream=None):
+def step(q, k, v, beta, S, d, r=None, eta=1e-2, stream=None, d_anchor=None, apf_anchor=False):
     """One decode token for every (b, h): q, k [B,H,dk]; v [B,H,dv]; beta, r [B,H];
-    S [B,H,dv,dk] and d [B,H,dk] fp32, updated in place. Returns out [B,H,dv]."""
+    S [B,H,dv,dk] and d [B,H,dk] fp32, updated in place. Anchored APF (apf_anchor, or a
+    d_anchor [B,H,dk] fp32 given) pulls d toward d_anchor (ones when None). Returns out [B,H,dv]."""
     B, H, dk = k.shape
     dv = v.shape[-1]
-    p = make_params(B, 1, H, dk, dv, k.dtype, eta)
+    p = make_params(B, 1, H, dk, dv, k.dtype, eta, apf_anchor=apf_anchor or d_anchor is not None)
     out = torch.empty((B, H, dv), dtype=k.dtype, device=k.device)
-    osdn_step(p, q, k, v, beta, r, S, d, out, stream)
+    osdn_step_ex(p, q, k, v, beta, r, d_anchor, S, d, out, stream)
     return out

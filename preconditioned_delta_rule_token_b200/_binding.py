@@ -30,7 +30,8 @@ NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", 
 class osdn_params(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("B", ctypes.c_int32), ("T", ctypes.c_int32),
                 ("H", ctypes.c_int32), ("dk", ctypes.c_int32), ("dv", ctypes.c_int32),
-                ("chunk", ctypes.c_int32), ("dtype", ctypes.c_int32), ("eta", ctypes.c_float)]
+                ("chunk", ctypes.c_int32), ("dtype", ctypes.c_int32), ("eta", ctypes.c_float),
+                ("apf_anchor", ctypes.c_int32)]
 
 
 class OsdnError(RuntimeError):
@@ -91,6 +92,8 @@ def lib():
         L.osdn_fwd_noalloc.restype = ctypes.c_int
         L.osdn_step.argtypes = [P] + [vp] * 8 + [vp]
         L.osdn_step.restype = ctypes.c_int
+        L.osdn_step_ex.argtypes = [P] + [vp] * 9 + [vp]
+        L.osdn_step_ex.restype = ctypes.c_int
         L.osdn_sync_status.argtypes = [vp]
         L.osdn_sync_status.restype = ctypes.c_int
         L.osdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
@@ -112,12 +115,13 @@ def _check(rc):
         raise OsdnError(rc, get_last_error())
 
 
-def make_params(B, T, H, dk, dv, dtype, eta, chunk=64) -> osdn_params:
+def make_params(B, T, H, dk, dv, dtype, eta, chunk=64, apf_anchor=False) -> osdn_params:
     p = osdn_params()
     p.struct_size = ctypes.sizeof(osdn_params)
     p.B, p.T, p.H, p.dk, p.dv, p.chunk = int(B), int(T), int(H), int(dk), int(dv), int(chunk)
     p.dtype = OSDN_BF16 if dtype == torch.bfloat16 else OSDN_FP32
     p.eta = float(eta)
+    p.apf_anchor = 1 if apf_anchor else 0
     return p
 
 
@@ -186,6 +190,12 @@ def osdn_step(params, q, k, v, beta, r, S, d, out, stream=None):
     """Raw C-ABI call: one decode token for every (b, h); S and d updated in place."""
     _check(lib().osdn_step(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(S), _ptr(d),
                            _ptr(out), _stream(stream)))
+
+
+def osdn_step_ex(params, q, k, v, beta, r, d_anchor, S, d, out, stream=None):
+    """Raw C-ABI call: osdn_step with anchored APF toward d_anchor when params.apf_anchor is set."""
+    _check(lib().osdn_step_ex(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(d_anchor),
+                              _ptr(S), _ptr(d), _ptr(out), _stream(stream)))
 
 
 def osdn_sync_status(stream=None) -> int:

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstddef>
 #include <cstdarg>
 #include <cstdio>
 #include <initializer_list>
@@ -46,11 +47,17 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 size_t elem_size(int dtype) { return dtype == OSDN_BF16 ? 2 : 4; }
 
 // Common checks of the parameter block. need_T: the forward (T used).
+// Version 1 of osdn_params ended after eta; its callers get the fields added since at their defaults.
+constexpr size_t kParamsV1Size = offsetof(osdn_params, apf_anchor);
+int anchor_of(const osdn_params* p) {
+    return p->struct_size >= offsetof(osdn_params, apf_anchor) + sizeof(int32_t) && p->apf_anchor ? 1 : 0;
+}
+
 int check_params(const osdn_params* p, bool need_T) {
     if (!p) return fail(OSDN_ERR_INVALID_ARG, "params is NULL");
-    if (p->struct_size != sizeof(osdn_params))
-        return fail(OSDN_ERR_INVALID_ARG, "params.struct_size is %u, expected %zu (ABI mismatch)",
-                    p->struct_size, sizeof(osdn_params));
+    if (p->struct_size != sizeof(osdn_params) && p->struct_size != kParamsV1Size)
+        return fail(OSDN_ERR_INVALID_ARG, "params.struct_size is %u, expected %zu (or %zu, version 1)",
+                    p->struct_size, sizeof(osdn_params), kParamsV1Size);
     if (p->B < 1 || p->H < 1) return fail(OSDN_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", p->B, p->H);
     if (need_T && p->T < 0) return fail(OSDN_ERR_INVALID_ARG, "T must be >= 0 (got %d)", p->T);
     if (p->dtype != OSDN_BF16 && p->dtype != OSDN_FP32)
@@ -177,7 +184,7 @@ int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bflo
     const size_t smem = osdn::ScanLayout::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan kernel attribute");
-    kern<<<p->B * p->H, 384, smem, st>>>(mk, mkw, beta, r, d0, final_d, rho, q_geo, p->B, p->T, p->H, p->eta,
+    kern<<<p->B * p->H, 384, smem, st>>>(mk, mkw, beta, r, d0, final_d, rho, q_geo, p->B, p->T, p->H, p->eta, anchor_of(p),
                                          g_wait_limit_ns.load());
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");
     return OSDN_OK;
@@ -204,10 +211,10 @@ int launch_scan(const osdn_params* p, const Tin* k, const Tin* beta, const Tin* 
     const dim3 grid((units + 3) / 4);
     if (p->dk == 128)
         osdn::scan_seq_kernel<128, Tin><<<grid, 128, 0, st>>>(k, beta, r, d0, kw, final_d, rho, q_geo, p->B, p->T,
-                                                               p->H, p->eta);
+                                                               p->H, p->eta, anchor_of(p));
     else
         osdn::scan_seq_kernel<64, Tin><<<grid, 128, 0, st>>>(k, beta, r, d0, kw, final_d, rho, q_geo, p->B, p->T,
-                                                              p->H, p->eta);
+                                                              p->H, p->eta, anchor_of(p));
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     return OSDN_OK;
@@ -261,12 +268,17 @@ int check_fwd_args(const osdn_params* p, std::initializer_list<const void*> requ
 
 template <typename Tin>
 int launch_step(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, const Tin* beta, const Tin* r,
-                float* S, float* d, Tin* out, cudaStream_t st) {
+                const float* d_anchor, float* S, float* d, Tin* out, cudaStream_t st) {
     const unsigned units = (unsigned)(p->B * p->H);
-    if (p->dk == 128 && p->dv == 128) osdn::step_kernel<128, 128, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta);
-    else if (p->dk == 128) osdn::step_kernel<128, 64, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta);
-    else if (p->dv == 128) osdn::step_kernel<64, 128, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta);
-    else osdn::step_kernel<64, 64, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta);
+    const int an = anchor_of(p);
+    if (p->dk == 128 && p->dv == 128)
+        osdn::step_kernel<128, 128, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor);
+    else if (p->dk == 128)
+        osdn::step_kernel<128, 64, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor);
+    else if (p->dv == 128)
+        osdn::step_kernel<64, 128, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor);
+    else
+        osdn::step_kernel<64, 64, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "step launch");
     return OSDN_OK;
@@ -429,23 +441,29 @@ int osdn_fwd_noalloc(const osdn_params* p, const void* q, const void* k, const v
                                (float*)out, final_S, kw, st);
 }
 
-int osdn_step(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
-              float* S, float* d, void* out, void* cuda_stream) {
+int osdn_step_ex(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
+                 const float* d_anchor, float* S, float* d, void* out, void* cuda_stream) {
     t_last_error.clear();
     int rc = check_params(p, false);
     if (rc) return rc;
     if (!q || !k || !v || !beta || !S || !d || !out)
         return fail(OSDN_ERR_INVALID_ARG, "q, k, v, beta, S, d and out must not be NULL");
-    const void* ptrs[] = {q, k, v, beta, r, S, d, out};
+    const void* ptrs[] = {q, k, v, beta, r, d_anchor, S, d, out};
     for (const void* x : ptrs)
         if (x && !aligned16(x)) return fail(OSDN_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
     if (p->dtype == OSDN_BF16) {
         using T = __nv_bfloat16;
-        return launch_step<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)r, S, d, (T*)out, st);
+        return launch_step<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)r, d_anchor, S, d,
+                              (T*)out, st);
     }
     return launch_step<float>(p, (const float*)q, (const float*)k, (const float*)v, (const float*)beta,
-                              (const float*)r, S, d, (float*)out, st);
+                              (const float*)r, d_anchor, S, d, (float*)out, st);
+}
+
+int osdn_step(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
+              float* S, float* d, void* out, void* cuda_stream) {
+    return osdn_step_ex(p, q, k, v, beta, r, nullptr, S, d, out, cuda_stream);
 }
 
 int osdn_sync_status(void* cuda_stream) {

@@ -5,7 +5,8 @@
 // light O(dk) scan over the key stream that yields the scaled write keys) and
 // section 2.3 (APF retention r_t on d only):
 //   k~_t = d_t (.) k_t,
-//   d_{t+1} = r_t d_t + eta beta_t (1 - beta_t <d_t, k_t^2>) k_t^2 / ||k_t||^2.
+//   d_{t+1} = r_t d_t + eta beta_t (1 - beta_t <d_t, k_t^2>) k_t^2 / ||k_t||^2,
+// or with anchored APF r_t d_t + (1 - r_t) d0 + (the same step).
 // Each lane holds DK/32 consecutive features of d in registers; the two
 // per-token reductions (<d, k^2> and ||k||^2) are warp shuffles.  This form is
 // latency-bound (one warp reduction per token); it serves fp32 mode and short
@@ -22,7 +23,7 @@ template <int DK, typename Tin>
 __global__ void __launch_bounds__(128)
 scan_seq_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const Tin* __restrict__ r,
                 const float* __restrict__ d0, Tin* __restrict__ kw, float* __restrict__ d_final,
-                float* __restrict__ rho, float* __restrict__ q_geo, int B, int T, int H, float eta)
+                float* __restrict__ rho, float* __restrict__ q_geo, int B, int T, int H, float eta, int anchor)
 {
     constexpr int PER = DK / 32;
     const int lane = threadIdx.x & 31;
@@ -38,6 +39,9 @@ scan_seq_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const T
         for (int i = 0; i < PER; ++i) d[i] = 1.f;
     }
 
+    float da[PER];                                   // retention target: d0 (anchored APF) or 0
+#pragma unroll
+    for (int i = 0; i < PER; ++i) da[i] = anchor ? d[i] : 0.f;
     const size_t tok_stride = (size_t)H;             // [B, T, H] index step per token
     size_t tok = (size_t)b * T * H + h;              // token (b, 0, h)
     float kc[PER], kn[PER];
@@ -74,7 +78,7 @@ scan_seq_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const T
             log_rho += logf(rt);
         }
 #pragma unroll
-        for (int i = 0; i < PER; ++i) d[i] = rc * d[i] + x * a[i];
+        for (int i = 0; i < PER; ++i) d[i] = rc * d[i] + (1.f - rc) * da[i] + x * a[i];
         tok = nxt;
 #pragma unroll
         for (int i = 0; i < PER; ++i) kc[i] = kn[i];

@@ -26,6 +26,10 @@
 //     kw_t[i] = d_t[i] k_t[i] over k_t[i] and carrying d; then one TMA store of
 //     the block's scaled keys; its buffer takes the block three ahead once the
 //     store has read it (issued at the start of the next block).
+// Anchored APF (retention toward d0): with e = d - d0 the recurrence is the
+// plain one, e_{t+1} = r_t e_t + x_t u_t, and <d_t, a_t> = <e_t, a_t> + <d0, a_t>;
+// the chain carries e and adds <d0, a_t> to the chunk-start term of c_t (the
+// plain case is d0 -> 0 in both).
 // Optional diagnostic (sections 4-5): the residual ratio of each write,
 // rho_t = (1 - beta_t <d_t, k_t^2>)^2 = f_t(S_t)/f_t(S_{t-1}), into rho [B, T, H]
 // and q_geo = exp(mean_t log rho_t) per (sequence, head). Since
@@ -54,7 +58,9 @@ struct ScanLayout {
     enum { V_BETA = 0, V_R = 128, V_G = 256, V_INVN = 384, V_R0 = 512, V_PAR = 640 };
     static constexpr uint32_t NP = VEC + 2 * V_PAR * 4;      // prep: ||k_t||^2 halves [2][128]
     static constexpr uint32_t CV = NP + 256 * 4;             // chain: c (64), x / ||k||^2 (64), d (128)
-    enum { C_C = 0, C_X = 64, C_D = 128, C_B = 256, C_LR = 320, C_N = 324 };   // + b_t (64), log-rho sums (4)
+    // c, x / ||k||^2, the carry e = d - d_anchor, the chunk-start part of <d_t, a_t>, log-rho sums (4),
+    // the retention target d_anchor (d0 under anchored APF, else 0)
+    enum { C_C = 0, C_X = 64, C_D = 128, C_B = 256, C_LR = 320, C_DA = 324, C_N = 452 };
     static constexpr uint32_t BAR = CV + C_N * 4;
     enum {
         FULL = 0,    // 3: K block landed
@@ -76,7 +82,8 @@ __global__ void __launch_bounds__(384, 1)
 scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kw,
                const __nv_bfloat16* __restrict__ beta, const __nv_bfloat16* __restrict__ r,
                const float* __restrict__ d0, float* __restrict__ d_final, float* __restrict__ rho,
-               float* __restrict__ q_geo, int B, int T, int H, float eta, unsigned long long wait_limit_ns)
+               float* __restrict__ q_geo, int B, int T, int H, float eta, int anchor,
+               unsigned long long wait_limit_ns)
 {
     constexpr int DK = 128, BLK = 128, SUB = 64;
     constexpr uint32_t NCOLS = 128;
@@ -137,6 +144,7 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         float* s_x = cv + L::C_X;
         float* s_d = cv + L::C_D;
         float* s_b = cv + L::C_B;
+        float* s_da = cv + L::C_DA;
         const bool diag = rho != nullptr || q_geo != nullptr;
         float log_rho = 0.f;   // this thread's share of sum_t log rho_t
         constexpr int kTmaThread = 32;
@@ -149,7 +157,11 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         };
         if (tid == kTmaThread)
             while (issued < L::NKB && issued < nblk) load_k(issued++);
-        s_d[tid] = d0 ? d0[(size_t)unit * DK + tid] : 1.f;
+        {
+            const float d_init = d0 ? d0[(size_t)unit * DK + tid] : 1.f;
+            s_da[tid] = anchor ? d_init : 0.f;
+            s_d[tid] = d_init - s_da[tid];   // the carry e = d - d_anchor
+        }
         tc::named_sync(BAR_CHAIN, 128);
 
         int blk = 0;
@@ -160,9 +172,9 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             if (tc::named_sync_or(BAR_CHAIN, 128, !wait(L::NRDY + (blk & 1), (blk >> 1) & 1))) break;
             for (int s = 0; s < 2 && s * SUB < Tb; ++s) {
                 const float* Nm = reinterpret_cast<const float*>(sm + L::MF + ((blk & 1) * 2 + s) * L::MAT);
-                {   // b_t = <d_c, a_t>; c_t = g_t (1 - beta_t R_{t,0} b_t); two threads per token
+                {   // b_t = <e_c, a_t>; c_t = g_t (1 - beta_t (R_{t,0} b_t + <d_anchor, a_t>)); two threads per token
                     const int tl_ = tid >> 1, half = tid & 1, t = s * SUB + tl_;
-                    float acc = 0.f;
+                    float acc = 0.f, acc_a = 0.f;
 #pragma unroll
                     for (int c0 = 0; c0 < 8; ++c0) {
                         // the two halves walk their 16-byte chunks four apart, so the two threads of a
@@ -179,11 +191,24 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                             acc = fmaf(f.x * f.x, dd[2 * e], acc);
                             acc = fmaf(f.y * f.y, dd[2 * e + 1], acc);
                         }
+                        if (anchor) {
+                            const float4 alo = *reinterpret_cast<const float4*>(s_da + half * 64 + c * 8);
+                            const float4 ahi = *reinterpret_cast<const float4*>(s_da + half * 64 + c * 8 + 4);
+                            const float da[8] = {alo.x, alo.y, alo.z, alo.w, ahi.x, ahi.y, ahi.z, ahi.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = __bfloat1622float2(p2[e]);
+                                acc_a = fmaf(f.x * f.x, da[2 * e], acc_a);
+                                acc_a = fmaf(f.y * f.y, da[2 * e + 1], acc_a);
+                            }
+                        }
                     }
                     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                    acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 1);
                     if (half == 0) {
-                        s_c[tl_] = vb[L::V_G + t] * (1.f - vb[L::V_BETA + t] * vb[L::V_R0 + t] * acc);
-                        s_b[tl_] = acc;
+                        const float known = vb[L::V_R0 + t] * acc + acc_a;   // <d_t, a_t> without the x terms
+                        s_c[tl_] = vb[L::V_G + t] * (1.f - vb[L::V_BETA + t] * known);
+                        s_b[tl_] = known;
                     }
                 }
                 if (s == 0 && tid == kTmaThread && blk > 0 && issued < nblk) {
@@ -214,7 +239,7 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                         const float gt = vb[L::V_G + t], bt = vb[L::V_BETA + t];
                         float f = 1.f;
                         if (gt != 0.f) f = acc / gt;
-                        else if (bt != 0.f && vb[L::V_INVN + t] > 0.f) f = 1.f - bt * vb[L::V_R0 + t] * s_b[tl_];
+                        else if (bt != 0.f && vb[L::V_INVN + t] > 0.f) f = 1.f - bt * s_b[tl_];
                         const float rt = f * f;
                         if (rho) rho[((size_t)b * T + blk * BLK + t) * H + h] = rt;
                         log_rho += logf(rt);
@@ -227,7 +252,8 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                     const int i = tid;
                     uint8_t* colbase = KS + (i >> 6) * 16384 + 2 * (i & 7);
                     const int cidx = (i & 63) >> 3;
-                    float d = s_d[i];
+                    const float da = s_da[i];
+                    float d = s_d[i];   // the carry e = d - d_anchor
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const int tb = s * SUB + hh * 32;   // multiple of 8
@@ -247,7 +273,7 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const float kv = kk[j];
-                            kk[j] = d * kv;                                  // scaled key, with d before token j
+                            kk[j] = (d + da) * kv;                           // scaled key, with d before token j
                             d = fmaf(rr[j], d, xx[j] * (kv * kv));
                         }
 #pragma unroll
@@ -273,7 +299,7 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             for (int q = issued > L::NKB ? issued - L::NKB : 0; q < issued; ++q)
                 tc::mbar_wait(bars + L::FULL + q % L::NKB, (q / L::NKB) & 1, 1000000000ull);
         }
-        if (blk == nblk && !*abort_flag && d_final) d_final[(size_t)unit * DK + tid] = s_d[tid];
+        if (blk == nblk && !*abort_flag && d_final) d_final[(size_t)unit * DK + tid] = s_d[tid] + s_da[tid];
         if (q_geo) {   // q_geo = exp(mean log rho): warp sums, then one thread
             float* lr = cv + L::C_LR;
             const float ws = warp_sum(log_rho);

@@ -6,7 +6,8 @@
 // 2.2-2.3 (preconditioner step), for one token:
 //   kw = d (.) k,  e = S k - v,  S' = S - beta e kw^T,
 //   o  = S' q = S q - beta e <kw, q>,
-//   d' = r d + eta beta (1 - beta <d, k^2>) k^2 / ||k||^2.
+//   d' = r d + eta beta (1 - beta <d, k^2>) k^2 / ||k||^2
+//   (anchored APF: r d + (1 - r) d_anchor + the same step).
 // Warp w owns rows w, w + 8, ... of S; lane l owns columns [l*PER, l*PER+PER).
 // The kernel is HBM-bound: 2 * dv * dk * 4 bytes of state per head and token.
 #pragma once
@@ -18,7 +19,8 @@ template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(256)
 step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
             const Tin* __restrict__ beta, const Tin* __restrict__ r,
-            float* __restrict__ S, float* __restrict__ d, Tin* __restrict__ out, float eta)
+            float* __restrict__ S, float* __restrict__ d, Tin* __restrict__ out, float eta,
+            int anchor, const float* __restrict__ d_anchor)
 {
     constexpr int PER = DK / 32;
     constexpr int NW = 8;
@@ -73,8 +75,15 @@ step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __r
     __syncthreads();   // every warp has read d before warp 0 overwrites it
     if (warp == 0) {
         const float x = (n > 0.f) ? eta * bt * (1.f - bt * s) / n : 0.f;
+        float da[PER];   // retention target: d_anchor (ones when NULL) under anchored APF, else 0
+        if (anchor && d_anchor) {
+            VecIO<PER, float>::load(d_anchor + unit * DK + lane * PER, da);
+        } else {
 #pragma unroll
-        for (int i = 0; i < PER; ++i) dd[i] = rt * dd[i] + x * (kk[i] * kk[i]);
+            for (int i = 0; i < PER; ++i) da[i] = anchor ? 1.f : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) dd[i] = rt * dd[i] + (1.f - rt) * da[i] + x * (kk[i] * kk[i]);
         VecIO<PER, float>::store(d + unit * DK + lane * PER, dd);
     }
 }

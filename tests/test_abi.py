@@ -30,7 +30,21 @@ def test_library_exports_every_declared_symbol(osdn_lib):
     lib = ctypes.CDLL(osdn_lib.LIB_PATH)
     for name in sorted(_declared_functions()):
         assert hasattr(lib, name), name
-    assert lib.osdn_abi_version() == 1
+    assert lib.osdn_abi_version() == 2
+
+
+def test_version_1_params_are_accepted(osdn_lib):
+    """osdn_params of ABI version 1 ended after eta (36 bytes); such callers are
+    accepted and get the plain APF retention (apf_anchor = 0)."""
+    L = osdn_lib.lib()
+    n = ctypes.c_size_t(0)
+    assert ctypes.sizeof(osdn_lib.osdn_params) == 40
+    p = _params(osdn_lib)
+    p.struct_size = 36
+    p.apf_anchor = 1            # beyond a version-1 struct: must be ignored
+    assert L.osdn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    p.struct_size = 44
+    assert L.osdn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == osdn_lib.OSDN_ERR_INVALID_ARG
 
 
 def _params(osdn_lib, **kw):
