@@ -47,10 +47,10 @@ def _load():
         lib.osdn_oracle_fwd.restype = ctypes.c_int
         lib.osdn_oracle_fwd_rho.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [dp] * 11 + [ctypes.c_int]
         lib.osdn_oracle_fwd_rho.restype = ctypes.c_int
-        lib.osdn_oracle_fwd_ex.argtypes = ([ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int] + [dp] * 11 +
+        lib.osdn_oracle_fwd_ex.argtypes = ([ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int] + [dp] * 12 +
                                            [ctypes.c_int])
         lib.osdn_oracle_fwd_ex.restype = ctypes.c_int
-        lib.osdn_oracle_step_ex.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [dp] * 9
+        lib.osdn_oracle_step_ex.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [dp] * 10
         lib.osdn_oracle_step_ex.restype = ctypes.c_int
         lib.osdn_oracle_step.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [dp] * 8
         lib.osdn_oracle_step.restype = ctypes.c_int
@@ -70,18 +70,20 @@ def _f64(a):
     return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
 
 
-def fwd(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=None, anchor=False):
-    """Token-by-token OSDN forward in float64 (anchor: anchored APF, retention toward d0).
+def fwd(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=None, anchor=False, alpha=None):
+    """Token-by-token OSDN forward in float64 (anchor: anchored APF, retention toward d0;
+    alpha [B, T, H]: gated OSDN, S_t = alpha_t S_{t-1} (I - beta k kw^T) + beta v kw^T).
 
     q, k: [B, T, H, dk]; v: [B, T, H, dv]; beta, r: [B, T, H] (r None = APF off);
     d0: [B, H, dk] (None = ones); S0: [B, H, dv, dk] (None = zeros).
     Returns (out [B, T, H, dv], S_final [B, H, dv, dk], d_final [B, H, dk]).
     """
-    q, k, v, beta, r, d0, S0 = map(_f64, (q, k, v, beta, r, d0, S0))
+    q, k, v, beta, r, d0, S0, alpha = map(_f64, (q, k, v, beta, r, d0, S0, alpha))
     B, T, H, dk = k.shape
     dv = v.shape[-1]
     assert q.shape == k.shape and v.shape == (B, T, H, dv) and beta.shape == (B, T, H)
     assert r is None or r.shape == (B, T, H)
+    assert alpha is None or alpha.shape == (B, T, H)
     assert d0 is None or d0.shape == (B, H, dk)
     assert S0 is None or S0.shape == (B, H, dv, dk)
     out = np.zeros((B, T, H, dv), np.float64)
@@ -90,7 +92,7 @@ def fwd(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=None, anchor
     if nthreads is None:
         nthreads = os.cpu_count() or 1
     rc = _load().osdn_oracle_fwd_ex(B, T, H, dk, dv, float(eta), int(bool(anchor)), _ptr(q), _ptr(k), _ptr(v),
-                                    _ptr(beta), _ptr(r), _ptr(d0), _ptr(S0),
+                                    _ptr(beta), _ptr(r), _ptr(alpha), _ptr(d0), _ptr(S0),
                                     _ptr(out), _ptr(S), _ptr(d), None, int(nthreads))
     if rc != 0:
         raise ValueError("oracle rejected the sizes")
@@ -113,7 +115,7 @@ def residual_ratio(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=N
     if nthreads is None:
         nthreads = os.cpu_count() or 1
     rc = _load().osdn_oracle_fwd_ex(B, T, H, dk, dv, float(eta), int(bool(anchor)), _ptr(q), _ptr(k), _ptr(v),
-                                    _ptr(beta), _ptr(r), _ptr(d0), _ptr(S0),
+                                    _ptr(beta), _ptr(r), None, _ptr(d0), _ptr(S0),
                                     _ptr(out), _ptr(S), _ptr(d), _ptr(rho), int(nthreads))
     if rc != 0:
         raise ValueError("oracle rejected the sizes")
@@ -122,11 +124,11 @@ def residual_ratio(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, nthreads=N
     return out, S, d, rho, q_geo
 
 
-def step(q, k, v, beta, S, d, r=None, eta=1e-2, d_anchor=None):
+def step(q, k, v, beta, S, d, r=None, eta=1e-2, d_anchor=None, alpha=None):
     """One decode token for every (b, h), float64, S [B,H,dv,dk] and d [B,H,dk]
     updated in place (they must be contiguous float64 arrays); d_anchor [B,H,dk]
     selects anchored APF toward it. Returns out [B,H,dv]."""
-    q, k, v, beta, r, d_anchor = map(_f64, (q, k, v, beta, r, d_anchor))
+    q, k, v, beta, r, d_anchor, alpha = map(_f64, (q, k, v, beta, r, d_anchor, alpha))
     assert S.dtype == np.float64 and S.flags.c_contiguous
     assert d.dtype == np.float64 and d.flags.c_contiguous
     B, H, dk = k.shape
@@ -134,7 +136,7 @@ def step(q, k, v, beta, S, d, r=None, eta=1e-2, d_anchor=None):
     assert S.shape == (B, H, dv, dk) and d.shape == (B, H, dk)
     out = np.zeros((B, H, dv), np.float64)
     rc = _load().osdn_oracle_step_ex(B, H, dk, dv, float(eta), _ptr(q), _ptr(k), _ptr(v),
-                                     _ptr(beta), _ptr(r), _ptr(d_anchor), _ptr(S), _ptr(d), _ptr(out))
+                                     _ptr(beta), _ptr(r), _ptr(alpha), _ptr(d_anchor), _ptr(S), _ptr(d), _ptr(out))
     if rc != 0:
         raise ValueError("oracle rejected the sizes")
     return out

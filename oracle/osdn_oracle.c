@@ -32,6 +32,10 @@
  *   - r_t is an input per (token, head); r == NULL means APF off (r == 1);
  *   - ||k_t||^2 == 0 skips the gradient term (h is undefined there).
  *
+ * Gated OSDN (an option; the gated delta rule backbone the pages run OSDN on):
+ *       S_t = alpha_t S_{t-1} (I - beta_t k_t (d_t (.) k_t)^T) + beta_t v_t (d_t (.) k_t)^T,
+ * i.e. the step above applied to the decayed state alpha_t S_{t-1}; d is unchanged.
+ *
  * Anchored APF (an option; the "refresh the calibration" reading of the APF
  * section): the retention pulls d toward its initial value d0 instead of 0,
  *       d_{t+1} = r_t d_t + (1 - r_t) d0 - eta grad_d h_t(d_t).
@@ -50,7 +54,7 @@
 typedef struct {
     int B, T, H, dk, dv;
     double eta;
-    const double *q, *k, *v, *beta, *r, *d0, *S0;
+    const double *q, *k, *v, *beta, *r, *d0, *S0, *alpha;
     double *out, *S_final, *d_final, *rho;
     int anchor;                         /* anchored APF: retention toward d0 */
     int unit_begin, unit_end;
@@ -62,8 +66,10 @@ typedef struct {
 static void oracle_token(int dk, int dv, double eta, double *S, double *d,
                          const double *q, const double *k, const double *v,
                          double beta, double r, double *o, double *e, double *a, double *rho,
-                         const double *anchor)
+                         const double *anchor, double alpha)
 {
+    if (alpha != 1.0)                                  /* gated: decay the state first */
+        for (size_t i = 0; i < (size_t)dv * dk; ++i) S[i] *= alpha;
     double n = 0.0, s = 0.0;
     for (int i = 0; i < dk; ++i) {
         a[i] = k[i] * k[i];           /* k_t^2, elementwise */
@@ -119,7 +125,7 @@ static void *oracle_worker(void *arg)
                          J->q + tok * dk, J->k + tok * dk, J->v + tok * dv,
                          J->beta[tok], J->r ? J->r[tok] : 1.0,
                          J->out + tok * dv, e, a, J->rho ? J->rho + tok : NULL,
-                         J->anchor ? d_start : NULL);
+                         J->anchor ? d_start : NULL, J->alpha ? J->alpha[tok] : 1.0);
         }
         if (J->S_final) memcpy(J->S_final + (size_t)u * dv * dk, S, sizeof(double) * (size_t)dv * dk);
         if (J->d_final) memcpy(J->d_final + (size_t)u * dk, d, sizeof(double) * (size_t)dk);
@@ -136,7 +142,7 @@ static void *oracle_worker(void *arg)
  * Returns 0, or -1 on bad sizes. */
 int osdn_oracle_fwd_ex(int B, int T, int H, int dk, int dv, double eta, int anchor,
                        const double *q, const double *k, const double *v,
-                       const double *beta, const double *r,
+                       const double *beta, const double *r, const double *alpha,
                        const double *d0, const double *S0,
                        double *out, double *S_final, double *d_final, double *rho,
                        int nthreads)
@@ -149,7 +155,7 @@ int osdn_oracle_fwd_ex(int B, int T, int H, int dk, int dv, double eta, int anch
     oracle_job *jobs = (oracle_job *)calloc((size_t)nthreads, sizeof(oracle_job));
     pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
     for (int w = 0; w < nthreads; ++w) {
-        oracle_job J = {B, T, H, dk, dv, eta, q, k, v, beta, r, d0, S0,
+        oracle_job J = {B, T, H, dk, dv, eta, q, k, v, beta, r, d0, S0, alpha,
                         out, S_final, d_final, rho, anchor,
                         (int)((long long)units * w / nthreads),
                         (int)((long long)units * (w + 1) / nthreads)};
@@ -169,7 +175,7 @@ int osdn_oracle_fwd_rho(int B, int T, int H, int dk, int dv, double eta,
                         double *out, double *S_final, double *d_final, double *rho,
                         int nthreads)
 {
-    return osdn_oracle_fwd_ex(B, T, H, dk, dv, eta, 0, q, k, v, beta, r, d0, S0, out, S_final, d_final, rho,
+    return osdn_oracle_fwd_ex(B, T, H, dk, dv, eta, 0, q, k, v, beta, r, NULL, d0, S0, out, S_final, d_final, rho,
                               nthreads);
 }
 
@@ -180,17 +186,17 @@ int osdn_oracle_fwd(int B, int T, int H, int dk, int dv, double eta,
                     double *out, double *S_final, double *d_final,
                     int nthreads)
 {
-    return osdn_oracle_fwd_ex(B, T, H, dk, dv, eta, 0, q, k, v, beta, r, d0, S0, out, S_final, d_final, NULL,
+    return osdn_oracle_fwd_ex(B, T, H, dk, dv, eta, 0, q, k, v, beta, r, NULL, d0, S0, out, S_final, d_final, NULL,
                               nthreads);
 }
 
 /* One decode token for every (b, h): q, k [B, H, dk]; v, out [B, H, dv];
- * beta, r [B, H] (r may be NULL); S [B, H, dv, dk] and d [B, H, dk] updated
- * in place; d_anchor [B, H, dk] (NULL: plain APF, non-NULL: anchored APF
- * toward it). Same arithmetic as one step of osdn_oracle_fwd_ex. */
+ * beta, r, alpha [B, H] (r, alpha may be NULL); S [B, H, dv, dk] and d
+ * [B, H, dk] updated in place; d_anchor [B, H, dk] (NULL: plain APF, non-NULL:
+ * anchored APF toward it). Same arithmetic as one step of osdn_oracle_fwd_ex. */
 int osdn_oracle_step_ex(int B, int H, int dk, int dv, double eta,
                         const double *q, const double *k, const double *v,
-                        const double *beta, const double *r, const double *d_anchor,
+                        const double *beta, const double *r, const double *alpha, const double *d_anchor,
                         double *S, double *d, double *out)
 {
     if (B < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
@@ -200,7 +206,7 @@ int osdn_oracle_step_ex(int B, int H, int dk, int dv, double eta,
         oracle_token(dk, dv, eta, S + (size_t)u * dv * dk, d + (size_t)u * dk,
                      q + (size_t)u * dk, k + (size_t)u * dk, v + (size_t)u * dv,
                      beta[u], r ? r[u] : 1.0, out + (size_t)u * dv, e, a, NULL,
-                     d_anchor ? d_anchor + (size_t)u * dk : NULL);
+                     d_anchor ? d_anchor + (size_t)u * dk : NULL, alpha ? alpha[u] : 1.0);
     }
     free(e); free(a);
     return 0;
@@ -211,5 +217,5 @@ int osdn_oracle_step(int B, int H, int dk, int dv, double eta,
                      const double *beta, const double *r,
                      double *S, double *d, double *out)
 {
-    return osdn_oracle_step_ex(B, H, dk, dv, eta, q, k, v, beta, r, NULL, S, d, out);
+    return osdn_oracle_step_ex(B, H, dk, dv, eta, q, k, v, beta, r, NULL, NULL, S, d, out);
 }

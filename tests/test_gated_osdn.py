@@ -1,0 +1,118 @@
+"""Gated OSDN: OSDN on the gated delta rule backbone,
+    S_t = alpha_t S_{t-1} (I - beta_t k_t kw_t^T) + beta_t v_t kw_t^T,  kw_t = d_t (.) k_t,
+with the preconditioner d unchanged ("OSDN: Improving Delta Rule with Provable
+Online Preconditioning in Linear Attention": the pages run OSDN on the gated
+DeltaNet backbone; the composition is the plainest one, the OSDN write key in the
+gated update). CPU tests pin the oracle option; GPU tests compare the kernels.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from preconditioned_delta_rule_token_b200 import workloads as W
+from tests._util import BF16_TOL, slice_rel_err
+from tests.test_chunk_algebra import chunked_scan
+
+
+def _case(seed, B=1, T=150, H=2, dk=16, dv=8, eta=0.5):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, T, H, dk))
+    k = rng.standard_normal((B, T, H, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    k[0, 5, 0] = 0.0
+    v = rng.standard_normal((B, T, H, dv))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((B, T, H))))
+    r = rng.uniform(0.8, 1.0, (B, T, H))
+    alpha = rng.uniform(0.85, 1.0, (B, T, H))
+    d0 = rng.uniform(0.5, 1.5, (B, H, dk))
+    S0 = 0.3 * rng.standard_normal((B, H, dv, dk))
+    return q, k, v, beta, r, alpha, d0, S0, eta
+
+
+def test_alpha_one_is_ungated():
+    q, k, v, beta, r, alpha, d0, S0, eta = _case(1)
+    g = oracle.fwd(q, k, v, beta, r, d0, S0, eta=eta, alpha=np.ones_like(alpha))
+    p = oracle.fwd(q, k, v, beta, r, d0, S0, eta=eta)
+    for x, y in zip(g, p):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_alpha_zero_restarts_the_state():
+    """alpha_t0 = 0 wipes S before token t0's write: the rest equals a fresh
+    forward from S = 0 with the d carried to t0 (d does not depend on S)."""
+    q, k, v, beta, r, alpha, d0, S0, eta = _case(2)
+    t0 = 60
+    alpha[:, t0] = 0.0
+    ro, rS, rd = oracle.fwd(q, k, v, beta, r, d0, S0, eta=eta, alpha=alpha)
+    _, _, d_mid = oracle.fwd(q[:, :t0], k[:, :t0], v[:, :t0], beta[:, :t0], r[:, :t0], d0, S0, eta=eta,
+                             alpha=alpha[:, :t0])
+    fo, fS, fd = oracle.fwd(q[:, t0:], k[:, t0:], v[:, t0:], beta[:, t0:], r[:, t0:], d_mid, None, eta=eta,
+                            alpha=alpha[:, t0:])
+    np.testing.assert_allclose(ro[:, t0:], fo, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(rS, fS, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(rd, fd, rtol=1e-12, atol=1e-12)
+
+
+def test_unit_preconditioner_is_textbook_gated_deltanet():
+    """eta = 0, d0 = 1, no APF: S_t = alpha S (I - beta k k^T) + beta v k^T, o = S q,
+    written out here from that definition."""
+    q, k, v, beta, _, alpha, _, S0, _ = _case(3, T=40)
+    ro, rS, _ = oracle.fwd(q, k, v, beta, None, None, S0, eta=0.0, alpha=alpha)
+    B, T, H, dk = k.shape
+    for b in range(B):
+        for h in range(H):
+            S = S0[b, h].copy()
+            for t in range(T):
+                kt = k[b, t, h]
+                S = alpha[b, t, h] * S @ (np.eye(dk) - beta[b, t, h] * np.outer(kt, kt)) + \
+                    beta[b, t, h] * np.outer(v[b, t, h], kt)
+                np.testing.assert_allclose(S @ q[b, t, h], ro[b, t, h], rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(S, rS[b, h], rtol=1e-12, atol=1e-12)
+
+
+def chunked_gated_delta(q, k, kw, v, beta, alpha, S0, C):
+    """Gated chunk form for one unit, as the tensor-core kernel computes it: gamma =
+    cumulative alpha within the chunk, A = strict_tril(diag(beta) (K Kw^T) (.) Gamma),
+    Gamma_tj = gamma_t / gamma_j, T = (I + A)^{-1}, W = T diag(beta gamma) K,
+    U0 = T diag(beta) V, Ut = diag(1/gamma) (U0 - W S^T),
+    O = diag(gamma) (Q S^T + tril(Q Kw^T) Ut), S <- gamma_C (S + Ut^T Kw)."""
+    T = k.shape[0]
+    S = S0.copy()
+    out = np.zeros((T, v.shape[1]))
+    for c0 in range(0, T, C):
+        Q, K, Kw, V = q[c0:c0 + C], k[c0:c0 + C], kw[c0:c0 + C], v[c0:c0 + C]
+        b, g = beta[c0:c0 + C], np.cumprod(alpha[c0:c0 + C])
+        n = len(K)
+        Gam = g[:, None] / g[None, :]
+        A = np.tril(b[:, None] * (K @ Kw.T) * Gam, -1)
+        Tm = np.linalg.inv(np.eye(n) + A)
+        Wm = Tm @ ((b * g)[:, None] * K)
+        U0 = Tm @ (b[:, None] * V)
+        Ut = (U0 - Wm @ S.T) / g[:, None]
+        out[c0:c0 + n] = g[:, None] * (Q @ S.T + np.tril(Q @ Kw.T) @ Ut)
+        S = g[-1] * (S + Ut.T @ Kw)
+    return out, S
+
+
+def test_gated_chunk_form_equals_the_recurrence():
+    q, k, v, beta, r, alpha, d0, S0, eta = _case(4)
+    ro, rS, rd = oracle.fwd(q, k, v, beta, r, d0, S0, eta=eta, alpha=alpha)
+    for h in range(k.shape[2]):
+        D, dT = chunked_scan(k[0, :, h], beta[0, :, h], r[0, :, h], d0[0, h], eta, 64)
+        np.testing.assert_allclose(dT, rd[0, h], rtol=1e-11, atol=1e-12)
+        out, S = chunked_gated_delta(q[0, :, h], k[0, :, h], D * k[0, :, h], v[0, :, h], beta[0, :, h],
+                                     alpha[0, :, h], S0[0, h], 64)
+        np.testing.assert_allclose(out, ro[0, :, h], rtol=1e-10, atol=1e-10)
+        np.testing.assert_allclose(S, rS[0, h], rtol=1e-10, atol=1e-10)
+
+
+def test_decode_steps_equal_the_forward():
+    q, k, v, beta, r, alpha, d0, S0, eta = _case(5, T=12)
+    ro, rS, rd = oracle.fwd(q, k, v, beta, r, d0, S0, eta=eta, alpha=alpha)
+    S, d = S0.copy(), d0.copy()
+    for t in range(q.shape[1]):
+        o = oracle.step(q[:, t], k[:, t], v[:, t], beta[:, t], S, d, r=r[:, t], eta=eta, alpha=alpha[:, t])
+        np.testing.assert_allclose(o, ro[:, t], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S, rS, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(d, rd, rtol=1e-12, atol=1e-12)
