@@ -52,6 +52,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the osdn_step (decode) measurement")
+    ap.add_argument("--no-gated", action="store_true", help="skip the gated-variant chunk measurement")
     return ap.parse_args()
 
 
@@ -319,6 +320,28 @@ def run_decode(dev, stream, hbm, n_calls=200, warmup=5):
             "bound": "hbm"}
 
 
+def run_gated(w, g, p, ws, out, Sf, stream, hbm, steps=20, warmup=3):
+    """Phase 2 of the gated variant (osdn_fwd_chunk_gated) on the same layer with
+    alpha ~ U(0.9, 1) (bf16, resident), after the scan has filled the workspace."""
+    import preconditioned_delta_rule_token_b200 as pk
+    alpha = (0.9 + 0.1 * torch.rand((w.B, w.T, w.H), generator=torch.Generator().manual_seed(w.seed + 5))).to(
+        g["k"].dtype).to(g["k"].device)
+    for _ in range(warmup):
+        pk.osdn_fwd_chunk_gated(p, g["q"], g["k"], g["v"], g["beta"], alpha, None, out, Sf, ws, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        pk.osdn_fwd_chunk_gated(p, g["q"], g["k"], g["v"], g["beta"], alpha, None, out, Sf, ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert pk.osdn_sync_status(stream) == 0
+    ms = e0.elapsed_time(e1) / steps
+    nbytes = chunk_bytes(w) + w.B * w.T * w.H * elem(w)            # + alpha
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": "osdn gated chunk kernel (phase 2)", "alpha": "U(0.9, 1)", "launch_ms": ms,
+            "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "peak_gbs": hbm, "frac": gbs / hbm, "bound": "hbm"}
+
+
 def config_of(w, world):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
             "apf": w.apf, "eta": w.eta, "structure": w.structure, "global_batch": w.B * world, "seq_len": w.T,
@@ -444,6 +467,9 @@ def run_ours(args, world, rank, local):
         line["e2e"] = e2e
     if world == 1 and not args.no_decode:
         line["decode"] = run_decode(dev, stream, hbm)
+    if world == 1 and not args.no_gated and w.dtype == W.BF16 and w.dk == 128 and w.dv == 128:
+        step()                                                      # the workspace holds this layer's scaled keys
+        line["gated"] = run_gated(w, g, p, ws, out, Sf, stream, hbm)
     if world == 1 and not args.no_cpu_baseline:
         v_, desc, cores = oracle_sample(w, seconds=12.0)
         line["cpu_baseline"] = {"value": v_, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}

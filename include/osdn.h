@@ -162,6 +162,39 @@ int osdn_step_ex(const osdn_params *p,
                  void *cuda_stream);
 
 
+/* Gated OSDN (the gated delta rule backbone the pages run OSDN on):
+ *   S_t = alpha_t S_{t-1} (I - beta_t k_t kw_t^T) + beta_t v_t kw_t^T,   kw_t = d_t (.) k_t,
+ * i.e. the OSDN write applied to the decayed state alpha_t S_{t-1}; the
+ * preconditioner d is unchanged. alpha [B, T, H] in the input dtype, in (0, 1].
+ * The chunk form divides by the decay accumulated inside a 64-token chunk, so
+ * the product of alpha over any 64 consecutive tokens of a sequence must stay
+ * above ~1e-30 (gates near 1, as in the gated DeltaNet layers).
+ * osdn_fwd_gated: as osdn_fwd plus alpha (not NULL when T > 0); bf16 inputs
+ * with dk = dv = 128 only (else OSDN_ERR_UNSUPPORTED).
+ * osdn_fwd_chunk_gated: phase 2 alone, after osdn_fwd_scan on the same stream.
+ * osdn_step_gated: osdn_step_ex with the decay (alpha [B, H], not NULL); every
+ * dtype and width osdn_step accepts. */
+int osdn_fwd_gated(const osdn_params *p,
+                   const void *q, const void *k, const void *v,
+                   const void *beta, const void *r, const void *alpha,
+                   const float *d0, const float *S0,
+                   void *out, float *final_S, float *final_d,
+                   void *workspace, size_t workspace_bytes,
+                   void *cuda_stream);
+
+int osdn_fwd_chunk_gated(const osdn_params *p,
+                         const void *q, const void *k, const void *v,
+                         const void *beta, const void *alpha,
+                         const float *S0, void *out, float *final_S,
+                         const void *workspace, size_t workspace_bytes,
+                         void *cuda_stream);
+
+int osdn_step_gated(const osdn_params *p,
+                    const void *q, const void *k, const void *v,
+                    const void *beta, const void *r, const void *alpha,
+                    const float *d_anchor, float *S, float *d, void *out,
+                    void *cuda_stream);
+
 /* Largest scratch osdn_fwd_noalloc can use: B * T * H * dk * element size
  * (2 bytes for bf16, 4 for fp32) must not exceed this. */
 #define OSDN_NOALLOC_SCRATCH_BYTES (32u << 20)

@@ -17,20 +17,23 @@ from ._binding import (OSDN_BF16, OSDN_ERR_CUDA, OSDN_ERR_INVALID_ARG, OSDN_ERR_
                        OSDN_FP32, OSDN_OK, LIB_PATH, OsdnError, build, get_last_error, make_params, osdn_fwd,
                        osdn_fwd_chunk, osdn_fwd_scan, osdn_fwd_scan_diag,
                        osdn_fwd_workspace_size, osdn_params, osdn_set_wait_limit_ns, osdn_step, osdn_step_ex,
+                       osdn_fwd_gated, osdn_fwd_chunk_gated, osdn_step_gated,
                        osdn_sync_status)
 
 __all__ = ["forward", "step", "residual_ratio", "osdn_fwd_scan_diag", "osdn_fwd", "osdn_fwd_scan", "osdn_fwd_chunk", "osdn_step", "osdn_fwd_workspace_size", "osdn_sync_status",
            "osdn_set_wait_limit_ns", "osdn_step_ex",
+           "osdn_fwd_gated", "osdn_fwd_chunk_gated", "osdn_step_gated",
            "osdn_params", "make_params", "get_last_error", "OsdnError", "build", "LIB_PATH",
            "OSDN_OK", "OSDN_ERR_INVALID_ARG", "OSDN_ERR_UNSUPPORTED", "OSDN_ERR_CUDA", "OSDN_ERR_TIMEOUT",
            "OSDN_BF16", "OSDN_FP32"]
 
 
 def forward(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, chunk=64, workspace=None, stream=None,
-            apf_anchor=False):
+            apf_anchor=False, alpha=None):
     """OSDN forward. q, k [B,T,H,dk]; v [B,T,H,dv]; beta, r [B,T,H] (bf16 or fp32,
     one dtype); d0 [B,H,dk] and S0 [B,H,dv,dk] fp32 or None. apf_anchor: anchored
-    APF, the retention pulls d toward d0 instead of 0.
+    APF, the retention pulls d toward d0 instead of 0. alpha [B,T,H] (same dtype): gated OSDN,
+    S_t = alpha_t S_{t-1} (I - beta k kw^T) + beta v kw^T (bf16, dk = dv = 128).
     Returns (out [B,T,H,dv], final_S [B,H,dv,dk] fp32, final_d [B,H,dk] fp32)."""
     B, T, H, dk = k.shape
     dv = v.shape[-1]
@@ -41,7 +44,10 @@ def forward(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, chunk=64, workspa
     final_d = torch.empty((B, H, dk), dtype=torch.float32, device=dev)
     if workspace is None:
         workspace = torch.empty(osdn_fwd_workspace_size(p), dtype=torch.uint8, device=dev)
-    osdn_fwd(p, q, k, v, beta, r, d0, S0, out, final_S, final_d, workspace, stream)
+    if alpha is None:
+        osdn_fwd(p, q, k, v, beta, r, d0, S0, out, final_S, final_d, workspace, stream)
+    else:
+        osdn_fwd_gated(p, q, k, v, beta, r, alpha, d0, S0, out, final_S, final_d, workspace, stream)
     return out, final_S, final_d
 
 
@@ -60,13 +66,17 @@ def residual_ratio(k, beta, r=None, d0=None, eta=1e-2, stream=None, apf_anchor=F
     return rho, q_geo, d
 
 
-def step(q, k, v, beta, S, d, r=None, eta=1e-2, stream=None, d_anchor=None, apf_anchor=False):
+def step(q, k, v, beta, S, d, r=None, eta=1e-2, stream=None, d_anchor=None, apf_anchor=False, alpha=None):
     """One decode token for every (b, h): q, k [B,H,dk]; v [B,H,dv]; beta, r [B,H];
     S [B,H,dv,dk] and d [B,H,dk] fp32, updated in place. Anchored APF (apf_anchor, or a
-    d_anchor [B,H,dk] fp32 given) pulls d toward d_anchor (ones when None). Returns out [B,H,dv]."""
+    d_anchor [B,H,dk] fp32 given) pulls d toward d_anchor (ones when None); alpha [B,H] decays S
+    first (gated OSDN). Returns out [B,H,dv]."""
     B, H, dk = k.shape
     dv = v.shape[-1]
     p = make_params(B, 1, H, dk, dv, k.dtype, eta, apf_anchor=apf_anchor or d_anchor is not None)
     out = torch.empty((B, H, dv), dtype=k.dtype, device=k.device)
-    osdn_step_ex(p, q, k, v, beta, r, d_anchor, S, d, out, stream)
+    if alpha is None:
+        osdn_step_ex(p, q, k, v, beta, r, d_anchor, S, d, out, stream)
+    else:
+        osdn_step_gated(p, q, k, v, beta, r, alpha, d_anchor, S, d, out, stream)
     return out

@@ -94,6 +94,12 @@ def lib():
         L.osdn_step.restype = ctypes.c_int
         L.osdn_step_ex.argtypes = [P] + [vp] * 9 + [vp]
         L.osdn_step_ex.restype = ctypes.c_int
+        L.osdn_step_gated.argtypes = [P] + [vp] * 10 + [vp]
+        L.osdn_step_gated.restype = ctypes.c_int
+        L.osdn_fwd_gated.argtypes = [P] + [vp] * 11 + [vp, sz, vp]
+        L.osdn_fwd_gated.restype = ctypes.c_int
+        L.osdn_fwd_chunk_gated.argtypes = [P] + [vp] * 8 + [vp, sz, vp]
+        L.osdn_fwd_chunk_gated.restype = ctypes.c_int
         L.osdn_sync_status.argtypes = [vp]
         L.osdn_sync_status.restype = ctypes.c_int
         L.osdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
@@ -196,6 +202,26 @@ def osdn_step_ex(params, q, k, v, beta, r, d_anchor, S, d, out, stream=None):
     """Raw C-ABI call: osdn_step with anchored APF toward d_anchor when params.apf_anchor is set."""
     _check(lib().osdn_step_ex(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(d_anchor),
                               _ptr(S), _ptr(d), _ptr(out), _stream(stream)))
+
+
+def osdn_fwd_gated(params, q, k, v, beta, r, alpha, d0, S0, out, final_S, final_d, workspace, stream=None):
+    """Raw C-ABI call of the gated forward (alpha decay of the state)."""
+    _check(lib().osdn_fwd_gated(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(alpha),
+                                _ptr(d0), _ptr(S0), _ptr(out), _ptr(final_S), _ptr(final_d), _ptr(workspace),
+                                ctypes.c_size_t(_ws_bytes(workspace)), _stream(stream)))
+
+
+def osdn_fwd_chunk_gated(params, q, k, v, beta, alpha, S0, out, final_S, workspace, stream=None):
+    """Raw C-ABI call of phase 2 of the gated forward."""
+    _check(lib().osdn_fwd_chunk_gated(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha),
+                                      _ptr(S0), _ptr(out), _ptr(final_S), _ptr(workspace),
+                                      ctypes.c_size_t(_ws_bytes(workspace)), _stream(stream)))
+
+
+def osdn_step_gated(params, q, k, v, beta, r, alpha, d_anchor, S, d, out, stream=None):
+    """Raw C-ABI call: one gated decode token for every (b, h)."""
+    _check(lib().osdn_step_gated(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(alpha),
+                                 _ptr(d_anchor), _ptr(S), _ptr(d), _ptr(out), _stream(stream)))
 
 
 def osdn_sync_status(stream=None) -> int:

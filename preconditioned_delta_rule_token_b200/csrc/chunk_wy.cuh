@@ -50,11 +50,14 @@ struct WyLayout {
     static constexpr uint32_t QK = 0, KW = 32768;
     static constexpr uint32_t VB = NSTAGE * STAGE;          // two V tiles [V0|V1], 16 KB each
     static constexpr uint32_t TB = VB + 2 * 16384;          // T diag(beta) bf16 [64 t][64 j]
-    static constexpr uint32_t PB = TB + 8192;               // two P tiles bf16 [64 t][64 j]
+    static constexpr uint32_t TB2 = TB + 8192;              // gated: T diag(beta / gamma) bf16 (B operand of GU)
+    static constexpr uint32_t PB = TB2 + 8192;              // two P tiles bf16 [64 t][64 j]
     static constexpr int LDF = tri::LD;
     static constexpr uint32_t AF = PB + 2 * 8192;           // A, then T, fp32 [64][LDF]
     static constexpr uint32_t BETA = AF + 64 * LDF * 4;     // prep group's beta of its chunk
-    static constexpr uint32_t BAR = BETA + 256;
+    static constexpr uint32_t BETAG = BETA + 256;           // gated: beta / gamma of the prep group's chunk
+    static constexpr uint32_t GSCR = BETAG + 256;           // gated: prep scratch (gamma_31)
+    static constexpr uint32_t BAR = GSCR + 16;
     enum {
         FULLQ = 0,   // 3: K, Q, Kw of a stage landed
         FULLV = 3,   // 2: V tile landed
@@ -94,29 +97,55 @@ struct ColsToRows {
         tc::tmem_ld16x256b_x8(taddr, lo);                   // lanes m0 + 0..15
         tc::tmem_ld16x256b_x8(taddr + (16u << 16), hi);     // lanes m0 + 16..31
     }
-    __device__ __forceinline__ void store(uint8_t* tile, uint32_t half_stride, int m0, float scale, int lane) const {
+    // Column (token) t = 8j + 2(lane % 4) + e of the thread's values is scaled by sc[2j + e].
+    __device__ __forceinline__ void store(uint8_t* tile, uint32_t half_stride, int m0, const float (&sc)[16],
+                                          int lane) const {
         const int k = lane >> 3, c = lane & 7;              // this thread addresses row c of 8 x 8 tile k
         const int mk = m0 + 8 * k;                          // first matrix row index of tile k
         uint8_t* base = tile + (mk >> 6) * half_stride;
         const int ch = (mk & 63) >> 3;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {                       // tokens 8j..8j+7
-            const uint32_t p0 = tc::pack_bf16(scale * __uint_as_float(lo[4 * j]), scale * __uint_as_float(lo[4 * j + 1]));
-            const uint32_t p1 = tc::pack_bf16(scale * __uint_as_float(lo[4 * j + 2]), scale * __uint_as_float(lo[4 * j + 3]));
-            const uint32_t p2 = tc::pack_bf16(scale * __uint_as_float(hi[4 * j]), scale * __uint_as_float(hi[4 * j + 1]));
-            const uint32_t p3 = tc::pack_bf16(scale * __uint_as_float(hi[4 * j + 2]), scale * __uint_as_float(hi[4 * j + 3]));
+            const float s0 = sc[2 * j], s1 = sc[2 * j + 1];
+            const uint32_t p0 = tc::pack_bf16(s0 * __uint_as_float(lo[4 * j]), s1 * __uint_as_float(lo[4 * j + 1]));
+            const uint32_t p1 = tc::pack_bf16(s0 * __uint_as_float(lo[4 * j + 2]), s1 * __uint_as_float(lo[4 * j + 3]));
+            const uint32_t p2 = tc::pack_bf16(s0 * __uint_as_float(hi[4 * j]), s1 * __uint_as_float(hi[4 * j + 1]));
+            const uint32_t p3 = tc::pack_bf16(s0 * __uint_as_float(hi[4 * j + 2]), s1 * __uint_as_float(hi[4 * j + 3]));
             tc::stmatrix_x4_trans(tc::smem_u32(base + tc::sw128_off(8 * j + c, ch)), p0, p1, p2, p3);
         }
     }
+    __device__ __forceinline__ void store(uint8_t* tile, uint32_t half_stride, int m0, float scale, int lane) const {
+        float sc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sc[i] = scale;
+        store(tile, half_stride, m0, sc, lane);
+    }
 };
 
-template <int kUnused = 0>
+// Inclusive prefix product over the 32 lanes of a warp.
+__device__ __forceinline__ float warp_prefix_product(float x, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x *= y;
+    }
+    return x;
+}
+
+// GATED: the gated delta rule backbone, S_t = alpha_t S_{t-1}(I - beta_t k_t kw_t^T) + beta_t v_t kw_t^T.
+// With gamma_t = prod_{m<=t} alpha_m inside the chunk and Th the inverse above (no decay in it), the
+// chunk is exactly
+//   Ut = Th diag(beta / gamma) V - W S^T,   O = diag(gamma) (Q S^T + P Ut),   S <- gamma_C (S + Ut^T Kw)
+// (T of the decayed Gram = diag(gamma) Th diag(1/gamma)), so only GU's B operand (T diag(beta / gamma)),
+// the O epilogue (x gamma_t) and the state carry (x gamma_C) change. It needs the decay within any
+// chunk to stay in the fp32 range (prod of 64 alphas above ~1e-30).
+template <bool GATED>
 __global__ void __launch_bounds__(288, 1)
 chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ CUtensorMap tm_out, const __nv_bfloat16* __restrict__ beta,
-                const float* __restrict__ S0, float* __restrict__ S_final, int B, int T, int H,
-                unsigned long long wait_limit_ns)
+                const __nv_bfloat16* __restrict__ alpha, const float* __restrict__ S0, float* __restrict__ S_final,
+                int B, int T, int H, unsigned long long wait_limit_ns)
 {
     constexpr int C = 64, DK = 128, DV = 128;
     // TMEM columns: state fp32 | bf16 state | D (U0^T -> Vn^T, bf16 Vn^T in its first 32 columns | O^T) | R1 x 3
@@ -264,10 +293,39 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             return true;
         };
 
+        // gated: alpha of tokens 2 lane, 2 lane + 1 of a chunk (1 past T), one chunk ahead
+        auto load_alpha = [&](int cc, float& a0, float& a1) {
+            const int t = cc * C + 2 * lane;
+            a0 = t < T ? __bfloat162float(alpha[((size_t)b * T + t) * H + h]) : 1.f;
+            a1 = t + 1 < T ? __bfloat162float(alpha[((size_t)b * T + t + 1) * H + h]) : 1.f;
+        };
+        float an0 = 1.f, an1 = 1.f;
+        if (GATED && nchunks > 0) load_alpha(0, an0, an1);
+
         bool ok = nchunks == 0 || w_epilogue(0);
         int c = 0;
         for (; ok && c < nchunks; ++c) {
             const int s2 = c & 1;
+            // gated: gamma_t = prod_{m<=t} alpha_m of this chunk (every warp computes all 64), the O scales
+            // for this thread's token columns, and gamma_C
+            float osc[16], gamma_c = 1.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) osc[i] = 1.f;
+            if (GATED) {
+                const float a0 = an0, a1 = an1;
+                if (c + 1 < nchunks) load_alpha(c + 1, an0, an1);
+                const float incl = warp_prefix_product(a0 * a1, lane);     // gamma_{2 lane + 1}
+                float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+                if (lane == 0) excl = 1.f;
+                const float g0 = excl * a0;                                  // gamma_{2 lane}
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int src = 4 * j + (lane & 3);                      // owner of tokens 8j + 2(lane % 4), +1
+                    osc[2 * j] = __shfl_sync(0xffffffffu, g0, src);
+                    osc[2 * j + 1] = __shfl_sync(0xffffffffu, incl, src);
+                }
+                gamma_c = __shfl_sync(0xffffffffu, incl, 31);
+            }
             // Vn^T = U0^T - S W^T (D columns 0-63) -> bf16 over columns 0-31 (A operand of GB)
             if (tc::named_sync_or(BAR_STATE, 128, !wait(L::BA, c & 1))) break;
             tc::tc_fence_after();
@@ -297,6 +355,14 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc::tmem_ld32(tl + COL_S + half * 64, *reinterpret_cast<uint32_t(*)[32]>(x));
                 tc::tmem_ld32(tl + COL_S + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
                 tc::tmem_wait_ld();
+                if (GATED) {   // S_{c+1} = gamma_C (S_c + Ut^T Kw): decay the fp32 state in place
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) x[i] = __float_as_uint(gamma_c * __uint_as_float(x[i]));
+                    if (c + 1 < nchunks) {
+                        tc::tmem_st32(tl + COL_S + half * 64, *reinterpret_cast<uint32_t(*)[32]>(x));
+                        tc::tmem_st32(tl + COL_S + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+                    }
+                }
                 if (c + 1 < nchunks) {
                     uint32_t w[32];
 #pragma unroll
@@ -332,7 +398,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
             // O_c -> the V tile of this chunk (free since GU(c) completed) -> TMA store
             uint8_t* ob = sm + L::VB + s2 * 16384;
-            o.store(ob, 8192, warp * 32, 1.f, lane);
+            o.store(ob, 8192, warp * 32, osc, lane);   // gated: O = diag(gamma) (...); else all ones
             tc::fence_proxy_async_smem();
             tc::named_sync(BAR_STATE, 128);
             if (tid == kTmaThread) {
@@ -366,10 +432,26 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             return (gtid < C && t < T) ? __bfloat162float(beta[((size_t)b * T + t) * H + h]) : 0.f;
         };
         float bnext = nchunks > 0 ? load_beta(0) : 0.f;
+        auto load_alpha_p = [&](int c) -> float {
+            const int t = c * C + gtid;
+            return (GATED && gtid < C && t < T) ? __bfloat162float(alpha[((size_t)b * T + t) * H + h]) : 1.f;
+        };
+        float anext = nchunks > 0 ? load_alpha_p(0) : 1.f;
+        float* betag = reinterpret_cast<float*>(sm + L::BETAG);
+        float* gscr = reinterpret_cast<float*>(sm + L::GSCR);
         for (int c = 0; c < nchunks; ++c) {
             const int s2 = c & 1;
             const float bt = bnext;
             if (c + 1 < nchunks) bnext = load_beta(c + 1);
+            float gam = 1.f;   // gated: gamma_t of token gtid (< 64), within its warp so far
+            if (GATED) {
+                const float at = anext;
+                if (c + 1 < nchunks) anext = load_alpha_p(c + 1);
+                if (gtid < C) {
+                    gam = warp_prefix_product(at, lane);
+                    if (gtid == 31) *gscr = gam;                  // gamma_31, for the second warp
+                }
+            }
             bool fail = !wait(L::D1 + c % 3, (c / 3) & 1);
             if (!fail && c >= 2) fail = !wait(L::BS + s2, ((c - 2) >> 1) & 1);   // GB(c-2) has read P tile s2
             if (tc::named_sync_or(BAR_PREP, 128, fail)) break;
@@ -411,6 +493,10 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
             tc::named_sync(BAR_PREP, 128);
+            if (GATED && gtid < C) {   // beta_t / gamma_t (read by the T diag(beta / gamma) write below)
+                if (gtid >= 32) gam *= *gscr;
+                betag[gtid] = bt / gam;
+            }
             tri::tril_inv64_inplace(AF, gw, lane, [] { tc::named_sync(BAR_PREP, 128); });
             // T diag(beta) -> bf16 K-major (B operand of GW and GU), once GW(c-1) and GU(c-1) have read it
             fail = c >= 1 && !wait(L::BA, (c - 1) & 1);
@@ -428,6 +514,14 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     pk.x = tc::pack_bf16(lo.x * blo.x, lo.y * blo.y); pk.y = tc::pack_bf16(lo.z * blo.z, lo.w * blo.w);
                     pk.z = tc::pack_bf16(hi.x * bhi.x, hi.y * bhi.y); pk.w = tc::pack_bf16(hi.z * bhi.z, hi.w * bhi.w);
                     *reinterpret_cast<uint4*>(sm + L::TB + tc::sw128_off(t, hf * 4 + cc)) = pk;
+                    if (GATED) {   // T diag(beta / gamma), the B operand of GU
+                        const float4 glo = *reinterpret_cast<const float4*>(betag + j);
+                        const float4 ghi = *reinterpret_cast<const float4*>(betag + j + 4);
+                        uint4 pg;
+                        pg.x = tc::pack_bf16(lo.x * glo.x, lo.y * glo.y); pg.y = tc::pack_bf16(lo.z * glo.z, lo.w * glo.w);
+                        pg.z = tc::pack_bf16(hi.x * ghi.x, hi.y * ghi.y); pg.w = tc::pack_bf16(hi.z * ghi.z, hi.w * ghi.w);
+                        *reinterpret_cast<uint4*>(sm + L::TB2 + tc::sw128_off(t, hf * 4 + cc)) = pg;
+                    }
                 }
             }
             tc::fence_proxy_async_smem();
@@ -439,6 +533,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ================================================================ issuer warp
         if (lane == 0) {
             const uint64_t dTB = tc::sdesc_sw128(sb + L::TB, 16, 1024);
+            const uint64_t dTBU = tc::sdesc_sw128(sb + (GATED ? L::TB2 : L::TB), 16, 1024);   // B of GU
             auto st = [&](int c) { return sb + (uint32_t)(c % 3) * L::STAGE; };
             auto G1 = [&](int c) {   // R1[c%3] = [K; Q] Kw^T
                 const uint64_t a = tc::sdesc_sw128(st(c) + L::QK, 16, 1024), bk = tc::sdesc_sw128(st(c) + L::KW, 16, 1024);
@@ -462,7 +557,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint64_t a = tc::sdesc_sw128(sb + L::VB + (c & 1) * 16384, 8192, 1024);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::umma_bf16(tmem + COL_D, a + ((ks * 2048) >> 4), dTB + ((ks * 32) >> 4), ID_N64_AMN, ks > 0);
+                    tc::umma_bf16(tmem + COL_D, a + ((ks * 2048) >> 4), dTBU + ((ks * 32) >> 4), ID_N64_AMN, ks > 0);
             };
             auto GA = [&](int c) {   // D += S_bf16 [-W; Q]^T
                 const uint64_t bq = tc::sdesc_sw128(st(c) + L::QK, 16, 1024);

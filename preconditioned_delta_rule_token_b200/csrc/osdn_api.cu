@@ -153,7 +153,7 @@ int make_token_map(CUtensorMap* m, const void* base, int B, int T, int H, int wi
 // Phase 2 on the tensor cores (WY form, state chain fed by prepared W and U0): bf16, dk = dv = 128.
 int launch_chunk_wy(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                     const __nv_bfloat16* beta, const float* S0, __nv_bfloat16* out, float* final_S,
-                    const __nv_bfloat16* kw, cudaStream_t st) {
+                    const __nv_bfloat16* kw, cudaStream_t st, const __nv_bfloat16* alpha = nullptr) {
     CUtensorMap mq, mk, mkw, mv, mo;
     int rc;
     if ((rc = make_token_map(&mq, q, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
@@ -161,11 +161,11 @@ int launch_chunk_wy(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfl
     if ((rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
     if ((rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
     if ((rc = make_token_map(&mo, out, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-    auto kern = osdn::chunk_wy_kernel<0>;
+    auto kern = alpha ? osdn::chunk_wy_kernel<true> : osdn::chunk_wy_kernel<false>;
     const size_t smem = osdn::WyLayout::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk kernel attribute");
-    kern<<<p->B * p->H, 288, smem, st>>>(mq, mk, mkw, mv, mo, beta, S0, final_S, p->B, p->T, p->H,
+    kern<<<p->B * p->H, 288, smem, st>>>(mq, mk, mkw, mv, mo, beta, alpha, S0, final_S, p->B, p->T, p->H,
                                          g_wait_limit_ns.load());
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core chunk launch");
     return OSDN_OK;
@@ -249,6 +249,17 @@ int launch_chunk(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v,
     return OSDN_OK;
 }
 
+// Phase 2 of the gated variant: the tensor-core kernel only (bf16, dk = dv = 128).
+int launch_chunk_gated(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta,
+                       const void* alpha, const float* S0, void* out, float* final_S, const void* kw, cudaStream_t st) {
+    if (p->dtype != OSDN_BF16 || p->dk != 128 || p->dv != 128)
+        return fail(OSDN_ERR_UNSUPPORTED, "the gated forward needs bf16 inputs with dk = dv = 128");
+    if (p->T == 0) return copy_initial_state(p, nullptr, S0, final_S, nullptr, true, false, st);
+    using T = __nv_bfloat16;
+    return launch_chunk_wy(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S,
+                           (const T*)kw, st, (const T*)alpha);
+}
+
 // Pointer and workspace checks shared by the forward entry points.
 int check_fwd_args(const osdn_params* p, std::initializer_list<const void*> required,
                    std::initializer_list<const void*> all, const void* workspace, size_t ws_bytes) {
@@ -268,17 +279,17 @@ int check_fwd_args(const osdn_params* p, std::initializer_list<const void*> requ
 
 template <typename Tin>
 int launch_step(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, const Tin* beta, const Tin* r,
-                const float* d_anchor, float* S, float* d, Tin* out, cudaStream_t st) {
+                const float* d_anchor, float* S, float* d, Tin* out, cudaStream_t st, const Tin* alpha = nullptr) {
     const unsigned units = (unsigned)(p->B * p->H);
     const int an = anchor_of(p);
     if (p->dk == 128 && p->dv == 128)
-        osdn::step_kernel<128, 128, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor);
+        osdn::step_kernel<128, 128, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor, alpha);
     else if (p->dk == 128)
-        osdn::step_kernel<128, 64, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor);
+        osdn::step_kernel<128, 64, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor, alpha);
     else if (p->dv == 128)
-        osdn::step_kernel<64, 128, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor);
+        osdn::step_kernel<64, 128, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor, alpha);
     else
-        osdn::step_kernel<64, 64, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor);
+        osdn::step_kernel<64, 64, Tin><<<units, 256, 0, st>>>(q, k, v, beta, r, S, d, out, p->eta, an, d_anchor, alpha);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "step launch");
     return OSDN_OK;
@@ -353,6 +364,40 @@ int osdn_fwd(const osdn_params* p, const void* q, const void* k, const void* v, 
     rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
     if (rc) return rc;
     return launch_chunk<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S, kw, st);
+}
+
+int osdn_fwd_gated(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
+                   const void* alpha, const float* d0, const float* S0, void* out, float* final_S, float* final_d,
+                   void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    if (p->T > 0 && !alpha) return fail(OSDN_ERR_INVALID_ARG, "alpha is NULL");
+    rc = check_fwd_args(p, {q, k, v, beta, out}, {q, k, v, beta, r, alpha, d0, S0, out, final_S, final_d}, workspace,
+                        workspace_bytes);
+    if (rc) return rc;
+    if (p->dtype != OSDN_BF16 || p->dk != 128 || p->dv != 128)
+        return fail(OSDN_ERR_UNSUPPORTED, "the gated forward needs bf16 inputs with dk = dv = 128");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    using T = __nv_bfloat16;
+    T* kw = (T*)(workspace ? reinterpret_cast<char*>(workspace) + layout_of(p).kw_off : nullptr);
+    rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
+    if (rc) return rc;
+    return launch_chunk_gated(p, q, k, v, beta, alpha, S0, out, final_S, kw, st);
+}
+
+int osdn_fwd_chunk_gated(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta,
+                         const void* alpha, const float* S0, void* out, float* final_S, const void* workspace,
+                         size_t workspace_bytes, void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    if (p->T > 0 && !alpha) return fail(OSDN_ERR_INVALID_ARG, "alpha is NULL");
+    rc = check_fwd_args(p, {q, k, v, beta, out}, {q, k, v, beta, alpha, S0, out, final_S}, workspace, workspace_bytes);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    const char* ws = reinterpret_cast<const char*>(workspace) + layout_of(p).kw_off;
+    return launch_chunk_gated(p, q, k, v, beta, alpha, S0, out, final_S, ws, st);
 }
 
 int osdn_fwd_scan(const osdn_params* p, const void* k, const void* beta, const void* r, const float* d0,
@@ -459,6 +504,27 @@ int osdn_step_ex(const osdn_params* p, const void* q, const void* k, const void*
     }
     return launch_step<float>(p, (const float*)q, (const float*)k, (const float*)v, (const float*)beta,
                               (const float*)r, d_anchor, S, d, (float*)out, st);
+}
+
+int osdn_step_gated(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta,
+                    const void* r, const void* alpha, const float* d_anchor, float* S, float* d, void* out,
+                    void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, false);
+    if (rc) return rc;
+    if (!q || !k || !v || !beta || !alpha || !S || !d || !out)
+        return fail(OSDN_ERR_INVALID_ARG, "q, k, v, beta, alpha, S, d and out must not be NULL");
+    const void* ptrs[] = {q, k, v, beta, r, alpha, d_anchor, S, d, out};
+    for (const void* x : ptrs)
+        if (x && !aligned16(x)) return fail(OSDN_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    if (p->dtype == OSDN_BF16) {
+        using T = __nv_bfloat16;
+        return launch_step<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)r, d_anchor, S, d,
+                              (T*)out, st, (const T*)alpha);
+    }
+    return launch_step<float>(p, (const float*)q, (const float*)k, (const float*)v, (const float*)beta,
+                              (const float*)r, d_anchor, S, d, (float*)out, st, (const float*)alpha);
 }
 
 int osdn_step(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,

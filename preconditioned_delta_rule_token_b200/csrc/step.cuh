@@ -7,7 +7,8 @@
 //   kw = d (.) k,  e = S k - v,  S' = S - beta e kw^T,
 //   o  = S' q = S q - beta e <kw, q>,
 //   d' = r d + eta beta (1 - beta <d, k^2>) k^2 / ||k||^2
-//   (anchored APF: r d + (1 - r) d_anchor + the same step).
+//   (anchored APF: r d + (1 - r) d_anchor + the same step);
+// gated (alpha non-NULL): S is first decayed, S <- alpha S, then the step above.
 // Warp w owns rows w, w + 8, ... of S; lane l owns columns [l*PER, l*PER+PER).
 // The kernel is HBM-bound: 2 * dv * dk * 4 bytes of state per head and token.
 #pragma once
@@ -20,7 +21,7 @@ __global__ void __launch_bounds__(256)
 step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
             const Tin* __restrict__ beta, const Tin* __restrict__ r,
             float* __restrict__ S, float* __restrict__ d, Tin* __restrict__ out, float eta,
-            int anchor, const float* __restrict__ d_anchor)
+            int anchor, const float* __restrict__ d_anchor, const Tin* __restrict__ alpha)
 {
     constexpr int PER = DK / 32;
     constexpr int NW = 8;
@@ -33,6 +34,14 @@ step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __r
 #pragma unroll
     for (int j = 0; j < ROWS; ++j)
         VecIO<PER, float>::load(Su + (size_t)(warp + NW * j) * DK + lane * PER, Sr[j]);
+
+    if (alpha) {   // gated: the write applies to the decayed state alpha S
+        const float a = to_f32(alpha[unit]);
+#pragma unroll
+        for (int j = 0; j < ROWS; ++j)
+#pragma unroll
+            for (int i = 0; i < PER; ++i) Sr[j][i] *= a;
+    }
 
     float kk[PER], qq[PER], dd[PER];
     VecIO<PER, Tin>::load(k + unit * DK + lane * PER, kk);

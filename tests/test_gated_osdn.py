@@ -95,14 +95,34 @@ def chunked_gated_delta(q, k, kw, v, beta, alpha, S0, C):
     return out, S
 
 
-def test_gated_chunk_form_equals_the_recurrence():
+def chunked_gated_delta_plain_inverse(q, k, kw, v, beta, alpha, S0, C):
+    """The same chunk form with the decay moved out of the triangular solve:
+    T = diag(gamma) Th diag(1/gamma) with Th = (I + strict_tril(diag(beta) K Kw^T))^{-1}
+    (no decay in it), so Ut = Th diag(beta/gamma) V - Th diag(beta) K S^T; O and the
+    state carry as above. This is the form the tensor-core kernel computes."""
+    T = k.shape[0]
+    S = S0.copy()
+    out = np.zeros((T, v.shape[1]))
+    for c0 in range(0, T, C):
+        Q, K, Kw, V = q[c0:c0 + C], k[c0:c0 + C], kw[c0:c0 + C], v[c0:c0 + C]
+        b, g = beta[c0:c0 + C], np.cumprod(alpha[c0:c0 + C])
+        n = len(K)
+        Th = np.linalg.inv(np.eye(n) + np.tril(b[:, None] * (K @ Kw.T), -1))
+        Ut = Th @ ((b / g)[:, None] * V) - (Th @ (b[:, None] * K)) @ S.T
+        out[c0:c0 + n] = g[:, None] * (Q @ S.T + np.tril(Q @ Kw.T) @ Ut)
+        S = g[-1] * (S + Ut.T @ Kw)
+    return out, S
+
+
+@pytest.mark.parametrize("form", [chunked_gated_delta, chunked_gated_delta_plain_inverse])
+def test_gated_chunk_form_equals_the_recurrence(form):
     q, k, v, beta, r, alpha, d0, S0, eta = _case(4)
     ro, rS, rd = oracle.fwd(q, k, v, beta, r, d0, S0, eta=eta, alpha=alpha)
     for h in range(k.shape[2]):
         D, dT = chunked_scan(k[0, :, h], beta[0, :, h], r[0, :, h], d0[0, h], eta, 64)
         np.testing.assert_allclose(dT, rd[0, h], rtol=1e-11, atol=1e-12)
-        out, S = chunked_gated_delta(q[0, :, h], k[0, :, h], D * k[0, :, h], v[0, :, h], beta[0, :, h],
-                                     alpha[0, :, h], S0[0, h], 64)
+        out, S = form(q[0, :, h], k[0, :, h], D * k[0, :, h], v[0, :, h], beta[0, :, h], alpha[0, :, h],
+                      S0[0, h], 64)
         np.testing.assert_allclose(out, ro[0, :, h], rtol=1e-10, atol=1e-10)
         np.testing.assert_allclose(S, rS[0, h], rtol=1e-10, atol=1e-10)
 
@@ -116,3 +136,113 @@ def test_decode_steps_equal_the_forward():
         np.testing.assert_allclose(o, ro[:, t], rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(S, rS, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(d, rd, rtol=1e-12, atol=1e-12)
+
+
+def _gated_inputs(dtype, B, H, T, dk, dv, eta, lo, seed):
+    w = W.Workload("gated", B, H, T, dk, dv, 64, dtype, True, "gaussian", d0="uniform", S0="normal", eta=eta,
+                   seed=seed)
+    inp = W.make_forward_inputs(w)
+    g = torch.Generator().manual_seed(seed + 7)
+    alpha = (lo + (1 - lo) * torch.rand((B, T, H), generator=g)).to(inp["k"].dtype)
+    return w, inp, alpha
+
+
+GATED_CASES = [
+    # B, H, T, eta, lowest alpha
+    (2, 3, 200, 1e-2, 0.9),
+    (1, 2, 130, 1.0, 0.5),
+    (2, 2, 64, 0.0, 0.8),
+    (1, 3, 1, 1e-2, 0.9),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", GATED_CASES, ids=lambda c: "B%dH%dT%d-eta%g-alpha%g" % c)
+def test_gpu_gated_forward_matches_oracle(case):
+    import preconditioned_delta_rule_token_b200 as pk
+    B, H, T, eta, lo = case
+    w, inp, alpha = _gated_inputs(W.BF16, B, H, T, 128, 128, eta, lo, seed=51)
+    dev = lambda x: None if x is None else x.cuda()
+    out, S, d = pk.forward(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["beta"]), dev(inp["r"]),
+                           dev(inp["d0"]), dev(inp["S0"]), eta=eta, alpha=dev(alpha))
+    assert pk.osdn_sync_status() == 0
+    f = W.to_f64
+    ro, rS, rd = oracle.fwd(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["beta"]), f(inp["r"]), f(inp["d0"]),
+                            f(inp["S0"]), eta=eta, alpha=f(alpha))
+    assert slice_rel_err(out.float().cpu().numpy(), ro, (0, 2)) <= BF16_TOL
+    assert slice_rel_err(S.cpu().numpy(), rS, (0, 1)) <= BF16_TOL
+    assert slice_rel_err(d.cpu().numpy(), rd, (0, 1)) <= BF16_TOL
+
+
+@pytest.mark.gpu
+def test_gpu_gated_with_unit_alpha_is_ungated():
+    import preconditioned_delta_rule_token_b200 as pk
+    w, inp, alpha = _gated_inputs(W.BF16, 2, 2, 150, 128, 128, 1e-2, 1.0, seed=52)
+    dev = lambda x: None if x is None else x.cuda()
+    args = (dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["beta"]), dev(inp["r"]), dev(inp["d0"]),
+            dev(inp["S0"]))
+    g = pk.forward(*args, eta=w.eta, alpha=dev(torch.ones_like(alpha)))
+    p = pk.forward(*args, eta=w.eta)
+    assert pk.osdn_sync_status() == 0
+    for x, y in zip(g, p):
+        torch.testing.assert_close(x.float(), y.float(), rtol=1e-6, atol=1e-6)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [W.FP32, W.BF16])
+def test_gpu_gated_decode_matches_oracle(dtype):
+    import preconditioned_delta_rule_token_b200 as pk
+    w, inp, alpha = _gated_inputs(dtype, 2, 3, 24, 128, 128, 0.5, 0.7, seed=53)
+    dev = lambda x: None if x is None else x.cuda()
+    S, d = dev(inp["S0"]).clone(), dev(inp["d0"]).clone()
+    outs = []
+    for t in range(w.T):
+        tok = {n: dev(inp[n][:, t].contiguous()) for n in ("q", "k", "v", "beta", "r")}
+        outs.append(pk.step(tok["q"], tok["k"], tok["v"], tok["beta"], S, d, r=tok["r"], eta=w.eta,
+                            alpha=dev(alpha[:, t].contiguous())))
+    assert pk.osdn_sync_status() == 0
+    f = W.to_f64
+    ro, rS, rd = oracle.fwd(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["beta"]), f(inp["r"]), f(inp["d0"]),
+                            f(inp["S0"]), eta=w.eta, alpha=f(alpha))
+    from tests._util import FP32_TOL
+    tol = BF16_TOL if dtype == W.BF16 else FP32_TOL
+    out = torch.stack(outs, 1).float().cpu().numpy()
+    assert slice_rel_err(out, ro, (0, 2)) <= tol
+    assert slice_rel_err(S.cpu().numpy(), rS, (0, 1)) <= tol
+    assert slice_rel_err(d.cpu().numpy(), rd, (0, 1)) <= tol
+
+
+@pytest.mark.gpu
+def test_gpu_gated_forward_unsupported_shapes_are_refused():
+    import preconditioned_delta_rule_token_b200 as pk
+    for dtype, dk in ((W.FP32, 128), (W.BF16, 64)):
+        w, inp, alpha = _gated_inputs(dtype, 1, 1, 70, dk, dk, 1e-2, 0.9, seed=54)
+        dev = lambda x: None if x is None else x.cuda()
+        with pytest.raises(pk.OsdnError) as e:
+            pk.forward(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["beta"]), dev(inp["r"]), None, None,
+                       eta=w.eta, alpha=dev(alpha))
+        assert e.value.code == pk.OSDN_ERR_UNSUPPORTED
+
+
+@pytest.mark.gpu
+def test_gpu_gated_full_size_layer_on_sampled_units():
+    """The 1.3B-shaped layer (B8 H16 T4096) with alpha ~ U(0.9, 1), three units re-run
+    by the oracle alone."""
+    import dataclasses
+    import preconditioned_delta_rule_token_b200 as pk
+    w = W.LAYER_1P3B
+    inp = W.make_forward_inputs(w)
+    alpha = (0.9 + 0.1 * torch.rand((w.B, w.T, w.H), generator=torch.Generator().manual_seed(55))).to(torch.bfloat16)
+    dev = lambda x: None if x is None else x.cuda()
+    out, S, d = pk.forward(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["beta"]), dev(inp["r"]), None, None,
+                           eta=w.eta, alpha=dev(alpha))
+    assert pk.osdn_sync_status() == 0
+    out, S, d = out.float().cpu().numpy(), S.cpu().numpy(), d.cpu().numpy()
+    f = W.to_f64
+    for (b, h) in [(0, 0), (5, 11), (7, 15)]:
+        sl = lambda x: f(x)[b:b + 1, :, h:h + 1]
+        ro, rS, rd = oracle.fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["beta"]), sl(inp["r"]), None, None,
+                                eta=w.eta, alpha=sl(alpha))
+        assert slice_rel_err(out[b:b + 1, :, h:h + 1], ro, (0, 2)) <= BF16_TOL, (b, h)
+        assert slice_rel_err(S[b:b + 1, h:h + 1], rS, (0, 1)) <= BF16_TOL, (b, h)
+        assert slice_rel_err(d[b:b + 1, h:h + 1], rd, (0, 1)) <= BF16_TOL, (b, h)
