@@ -1,4 +1,5 @@
-"""CPU oracle for the OSDN forward and decode step (test infrastructure only).
+"""CPU oracle for the OSDN forward, its backward and the decode step (test
+infrastructure only).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package. The product path (the CUDA library and
@@ -54,6 +55,9 @@ def _load():
         lib.osdn_oracle_step_ex.restype = ctypes.c_int
         lib.osdn_oracle_step.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [dp] * 8
         lib.osdn_oracle_step.restype = ctypes.c_int
+        lib.osdn_oracle_bwd_ex.argtypes = ([ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int] + [dp] * 19 +
+                                           [ctypes.c_int])
+        lib.osdn_oracle_bwd_ex.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -140,3 +144,42 @@ def step(q, k, v, beta, S, d, r=None, eta=1e-2, d_anchor=None, alpha=None):
     if rc != 0:
         raise ValueError("oracle rejected the sizes")
     return out
+
+
+def bwd(q, k, v, beta, dout, r=None, d0=None, S0=None, dS_final=None, dd_final=None, eta=1e-2,
+        nthreads=None, anchor=False, alpha=None):
+    """Reverse-mode gradients of fwd() in float64, token by token.
+
+    The loss is L = sum(dout * out) + sum(dS_final * S_final) + sum(dd_final * d_final)
+    (dS_final, dd_final None = 0). Returns a dict with dq, dk [B,T,H,dk], dv [B,T,H,dv],
+    dbeta [B,T,H], dr [B,T,H] (None without r), dalpha [B,T,H] (None without alpha),
+    dd0 [B,H,dk] and dS0 [B,H,dv,dk]. The adjoint formulas are written out at the top of
+    osdn_oracle.c.
+    """
+    q, k, v, beta, r, d0, S0, alpha, dout, dS_final, dd_final = map(
+        _f64, (q, k, v, beta, r, d0, S0, alpha, dout, dS_final, dd_final))
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    assert q.shape == k.shape and v.shape == (B, T, H, dv) and beta.shape == (B, T, H)
+    assert dout.shape == (B, T, H, dv)
+    assert r is None or r.shape == (B, T, H)
+    assert alpha is None or alpha.shape == (B, T, H)
+    assert d0 is None or d0.shape == (B, H, dk)
+    assert S0 is None or S0.shape == (B, H, dv, dk)
+    assert dS_final is None or dS_final.shape == (B, H, dv, dk)
+    assert dd_final is None or dd_final.shape == (B, H, dk)
+    g = {"dq": np.zeros((B, T, H, dk)), "dk": np.zeros((B, T, H, dk)), "dv": np.zeros((B, T, H, dv)),
+         "dbeta": np.zeros((B, T, H)), "dr": None if r is None else np.zeros((B, T, H)),
+         "dalpha": None if alpha is None else np.zeros((B, T, H)),
+         "dd0": np.zeros((B, H, dk)), "dS0": np.zeros((B, H, dv, dk))}
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    rc = _load().osdn_oracle_bwd_ex(B, T, H, dk, dv, float(eta), int(bool(anchor)), _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(beta), _ptr(r), _ptr(alpha), _ptr(d0), _ptr(S0),
+                                    _ptr(dout), _ptr(dS_final), _ptr(dd_final),
+                                    _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dbeta"]),
+                                    _ptr(g["dr"]), _ptr(g["dalpha"]), _ptr(g["dd0"]), _ptr(g["dS0"]),
+                                    int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the sizes")
+    return g
