@@ -195,6 +195,40 @@ int osdn_step_gated(const osdn_params *p,
                     const float *d_anchor, float *S, float *d, void *out,
                     void *cuda_stream);
 
+/* Backward (training). The pages give no backward pass; this is the exact
+ * reverse-mode derivative of osdn_fwd (plain or anchored APF, not gated) for
+ *     L = sum <dout, out> + <dS_final, final_S> + <dd_final, final_d>,
+ * through both phases: the chunked delta rule with the scaled write key
+ * (technical summary section 2.1) and the preconditioner recurrence of d
+ * (sections 2.2-2.3), including the dependence of the write keys d_t (.) k_t
+ * on k, beta, r and d0.
+ * Inputs: the osdn_fwd inputs (q, k, v, beta, r, d0, S0; same layouts, same
+ * NULL meanings) and the upstream gradients dout [B, T, H, dv] (input dtype),
+ * dS_final [B, H, dv, dk] fp32 (NULL = 0), dd_final [B, H, dk] fp32 (NULL = 0).
+ * Outputs (overwritten): dq, dk [B, T, H, dk]; dv [B, T, H, dv]; dbeta [B, T, H]
+ * in the input dtype (required when T > 0); dr [B, T, H] in the input dtype
+ * (written only when r and dr are both non-NULL); dd0 [B, H, dk] and
+ * dS0 [B, H, dv, dk] fp32 (nullable). Under anchored APF, dd0 includes the
+ * anchor's share (the anchor is d0).
+ * The forward is recomputed inside the call (nothing from osdn_fwd is reused).
+ * workspace: osdn_bwd_workspace_size() bytes, 16-byte aligned, no
+ * initialisation needed; it holds fp32 chunk intermediates (about
+ * (6 dk + 4 dv + 3 * 64) * 4 bytes per token and head, plus two fp32 states
+ * per 64-token chunk: 2 * dv * dk * 4 bytes per chunk and head).
+ * T = 0 copies dS_final to dS0 and dd_final to dd0 (zeros when NULL).
+ * Errors: OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED, OSDN_ERR_CUDA. */
+int osdn_bwd_workspace_size(const osdn_params *p, size_t *bytes);
+
+int osdn_bwd(const osdn_params *p,
+             const void *q, const void *k, const void *v,
+             const void *beta, const void *r,
+             const float *d0, const float *S0,
+             const void *dout, const float *dS_final, const float *dd_final,
+             void *dq, void *dk, void *dv, void *dbeta, void *dr,
+             float *dd0, float *dS0,
+             void *workspace, size_t workspace_bytes,
+             void *cuda_stream);
+
 /* Largest scratch osdn_fwd_noalloc can use: B * T * H * dk * element size
  * (2 bytes for bf16, 4 for fp32) must not exceed this. */
 #define OSDN_NOALLOC_SCRATCH_BYTES (32u << 20)

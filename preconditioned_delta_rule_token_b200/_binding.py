@@ -100,6 +100,10 @@ def lib():
         L.osdn_fwd_gated.restype = ctypes.c_int
         L.osdn_fwd_chunk_gated.argtypes = [P] + [vp] * 8 + [vp, sz, vp]
         L.osdn_fwd_chunk_gated.restype = ctypes.c_int
+        L.osdn_bwd_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+        L.osdn_bwd_workspace_size.restype = ctypes.c_int
+        L.osdn_bwd.argtypes = [P] + [vp] * 17 + [vp, sz, vp]
+        L.osdn_bwd.restype = ctypes.c_int
         L.osdn_sync_status.argtypes = [vp]
         L.osdn_sync_status.restype = ctypes.c_int
         L.osdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
@@ -222,6 +226,21 @@ def osdn_step_gated(params, q, k, v, beta, r, alpha, d_anchor, S, d, out, stream
     """Raw C-ABI call: one gated decode token for every (b, h)."""
     _check(lib().osdn_step_gated(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(alpha),
                                  _ptr(d_anchor), _ptr(S), _ptr(d), _ptr(out), _stream(stream)))
+
+
+def osdn_bwd_workspace_size(params: osdn_params) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().osdn_bwd_workspace_size(ctypes.byref(params), ctypes.byref(n)))
+    return n.value
+
+
+def osdn_bwd(params, q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta, dr, dd0, dS0, workspace,
+             stream=None):
+    """Raw C-ABI call of the backward: every tensor preallocated by the caller (device memory)."""
+    _check(lib().osdn_bwd(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(d0), _ptr(S0),
+                          _ptr(dout), _ptr(dS_final), _ptr(dd_final), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta),
+                          _ptr(dr), _ptr(dd0), _ptr(dS0), _ptr(workspace), ctypes.c_size_t(_ws_bytes(workspace)),
+                          _stream(stream)))
 
 
 def osdn_sync_status(stream=None) -> int:

@@ -16,6 +16,7 @@
 
 #include "osdn.h"
 
+#include "bwd.cuh"
 #include "chunk_ffma.cuh"
 #include "chunk_wy.cuh"
 #include "scan_ws.cuh"
@@ -295,6 +296,79 @@ int launch_step(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, 
     return OSDN_OK;
 }
 
+// Backward: seven launches on one stream (see bwd.cuh for what each computes).
+template <typename Tin, int DK, int DV>
+int launch_bwd_t(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, const Tin* beta, const Tin* r,
+                 const float* d0, const float* S0, const Tin* dout, const float* dS_final, const float* dd_final,
+                 Tin* dq, Tin* dk, Tin* dv, Tin* dbeta, Tin* dr, float* dd0, float* dS0, float* ws,
+                 cudaStream_t st) {
+    namespace B = osdn::bwd;
+    const B::Layout L = B::make_layout(p->B, p->T, p->H, DK, DV);
+    const int units = p->B * p->H, NC = (p->T + B::C - 1) / B::C, an = anchor_of(p);
+    const unsigned nchunks = (unsigned)((long long)units * NC), ntiles = (unsigned)(units * (DV / 32));
+    const unsigned warp_grid = (unsigned)((units + 3) / 4);
+    cudaError_t e;
+    auto attr = [](const void* kern, size_t smem) {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    };
+    B::bwd_dtraj_kernel<DK, Tin><<<warp_grid, 128, 0, st>>>(k, beta, r, d0, ws + L.d_all / sizeof(float), p->B,
+                                                             p->T, p->H, p->eta, an);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward d trajectory launch");
+
+    const size_t s_prep = B::PrepSmem<DK, DV>::kBytes;
+    if ((e = attr((const void*)B::bwd_prep_kernel<DK, DV, Tin>, s_prep)) != cudaSuccess)
+        return cuda_fail(e, "backward prep attribute");
+    B::bwd_prep_kernel<DK, DV, Tin><<<nchunks, B::NTHR, s_prep, st>>>(q, k, v, beta, ws, L, p->B, p->T, p->H, NC);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward prep launch");
+
+    const size_t s_sf = B::StateSmem<DK, 32>::kFwdBytes, s_sb = B::StateSmem<DK, 32>::kBwdBytes;
+    if ((e = attr((const void*)B::bwd_state_f_kernel<DK, DV, 32, Tin>, s_sf)) != cudaSuccess)
+        return cuda_fail(e, "backward state attribute");
+    B::bwd_state_f_kernel<DK, DV, 32, Tin><<<ntiles, B::NTHR, s_sf, st>>>(S0, ws, L, NC);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward state launch");
+    if ((e = attr((const void*)B::bwd_state_b_kernel<DK, DV, 32, Tin>, s_sb)) != cudaSuccess)
+        return cuda_fail(e, "backward adjoint state attribute");
+    B::bwd_state_b_kernel<DK, DV, 32, Tin><<<ntiles, B::NTHR, s_sb, st>>>(dout, q, dS_final, dS0, ws, L, p->B,
+                                                                          p->T, p->H, NC);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward adjoint state launch");
+
+    const size_t s_ga = B::GradSmem<DK>::kABytes, s_gb = B::GradSmem<DK>::kBBytes;
+    if ((e = attr((const void*)B::bwd_grads_a_kernel<DK, DV, Tin>, s_ga)) != cudaSuccess)
+        return cuda_fail(e, "backward gradient attribute");
+    B::bwd_grads_a_kernel<DK, DV, Tin><<<nchunks, B::NTHR, s_ga, st>>>(q, v, beta, dout, dq, dv, ws, L, p->B, p->T,
+                                                                       p->H, NC);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward gradient launch");
+    if ((e = attr((const void*)B::bwd_grads_b_kernel<DK, Tin>, s_gb)) != cudaSuccess)
+        return cuda_fail(e, "backward key gradient attribute");
+    B::bwd_grads_b_kernel<DK, Tin><<<nchunks, B::NTHR, s_gb, st>>>(k, beta, ws, L, p->B, p->T, p->H, NC);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward key gradient launch");
+
+    B::bwd_dchain_kernel<DK, Tin><<<warp_grid, 128, 0, st>>>(k, beta, r, d0, dd_final, dk, dbeta, dr, dd0, ws, L,
+                                                              p->B, p->T, p->H, NC, p->eta, an);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward d chain launch");
+    return OSDN_OK;
+}
+
+template <typename Tin>
+int launch_bwd(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
+               const float* d0, const float* S0, const void* dout, const float* dS_final, const float* dd_final,
+               void* dq, void* dk, void* dv, void* dbeta, void* dr, float* dd0, float* dS0, float* ws,
+               cudaStream_t st) {
+#define OSDN_BWD_ARGS                                                                                        \
+    p, (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)beta, (const Tin*)r, d0, S0, (const Tin*)dout, \
+        dS_final, dd_final, (Tin*)dq, (Tin*)dk, (Tin*)dv, (Tin*)dbeta, (Tin*)dr, dd0, dS0, ws, st
+    if (p->dk == 128 && p->dv == 128) return launch_bwd_t<Tin, 128, 128>(OSDN_BWD_ARGS);
+    if (p->dk == 128) return launch_bwd_t<Tin, 128, 64>(OSDN_BWD_ARGS);
+    if (p->dv == 128) return launch_bwd_t<Tin, 64, 128>(OSDN_BWD_ARGS);
+    return launch_bwd_t<Tin, 64, 64>(OSDN_BWD_ARGS);
+#undef OSDN_BWD_ARGS
+}
+
+size_t bwd_workspace_bytes(const osdn_params* p) {
+    const size_t n = osdn::bwd::make_layout(p->B, p->T, p->H, p->dk, p->dv).total;
+    return n ? n : 256;
+}
+
 // Scratch for osdn_fwd_noalloc: a fixed array in device memory, sized by
 // OSDN_NOALLOC_SCRATCH_BYTES. In host code the symbol is only a handle; its
 // device address is looked up once per device with cudaGetSymbolAddress.
@@ -530,6 +604,60 @@ int osdn_step_gated(const osdn_params* p, const void* q, const void* k, const vo
 int osdn_step(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
               float* S, float* d, void* out, void* cuda_stream) {
     return osdn_step_ex(p, q, k, v, beta, r, nullptr, S, d, out, cuda_stream);
+}
+
+int osdn_bwd_workspace_size(const osdn_params* p, size_t* bytes) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    if (!bytes) return fail(OSDN_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = bwd_workspace_bytes(p);
+    return OSDN_OK;
+}
+
+int osdn_bwd(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
+             const float* d0, const float* S0, const void* dout, const float* dS_final, const float* dd_final,
+             void* dq, void* dk, void* dv, void* dbeta, void* dr, float* dd0, float* dS0, void* workspace,
+             size_t workspace_bytes, void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    const void* ptrs[] = {q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta, dr, dd0, dS0,
+                          workspace};
+    for (const void* x : ptrs)
+        if (x && !aligned16(x)) return fail(OSDN_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    const size_t units = (size_t)p->B * p->H;
+    if (p->T == 0) {   // no tokens: the gradients of the initial state are those of the final state
+        cudaError_t e = cudaSuccess;
+        if (dS0) {
+            const size_t bytes = units * p->dv * p->dk * sizeof(float);
+            e = dS_final ? cudaMemcpyAsync(dS0, dS_final, bytes, cudaMemcpyDeviceToDevice, st)
+                         : cudaMemsetAsync(dS0, 0, bytes, st);
+            if (e != cudaSuccess) return cuda_fail(e, "initial state gradient copy");
+        }
+        if (dd0) {
+            const size_t bytes = units * p->dk * sizeof(float);
+            e = dd_final ? cudaMemcpyAsync(dd0, dd_final, bytes, cudaMemcpyDeviceToDevice, st)
+                         : cudaMemsetAsync(dd0, 0, bytes, st);
+            if (e != cudaSuccess) return cuda_fail(e, "initial preconditioner gradient copy");
+        }
+        return OSDN_OK;
+    }
+    if (!q || !k || !v || !beta || !dout || !dq || !dk || !dv || !dbeta)
+        return fail(OSDN_ERR_INVALID_ARG, "q, k, v, beta, dout, dq, dk, dv and dbeta must not be NULL");
+    if (!workspace) return fail(OSDN_ERR_INVALID_ARG, "workspace is NULL");
+    const size_t need = bwd_workspace_bytes(p);
+    if (workspace_bytes < need)
+        return fail(OSDN_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+    if ((double)units * (double)((p->T + 63) / 64) > 2147483647.0)
+        return fail(OSDN_ERR_INVALID_ARG, "B * H * ceil(T / 64) exceeds the grid limit");
+    float* ws = reinterpret_cast<float*>(workspace);
+    if (p->dtype == OSDN_BF16)
+        return launch_bwd<__nv_bfloat16>(p, q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta,
+                                         dr, dd0, dS0, ws, st);
+    return launch_bwd<float>(p, q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta, dr, dd0, dS0,
+                             ws, st);
 }
 
 int osdn_sync_status(void* cuda_stream) {

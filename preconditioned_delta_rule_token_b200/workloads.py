@@ -155,6 +155,21 @@ def make_forward_inputs(w: Workload) -> dict:
                 d0=d0.contiguous(), S0=None if S0 is None else S0.contiguous())
 
 
+def make_backward_cotangents(w: Workload, dS_final: bool = True, dd_final: bool = True) -> dict:
+    """Upstream gradients for a backward call on workload ``w``: dout [B, T, H, dv] in the
+    storage dtype, dS_final [B, H, dv, dk] and dd_final [B, H, dk] fp32 (None when not
+    requested), all N(0, 1), from a generator seeded apart from the forward inputs."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed) * 7919 + 17)
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    dout = torch.randn((B, T, H, dv), generator=g)
+    dS = torch.randn((B, H, dv, dk), generator=g)
+    dd = torch.randn((B, H, dk), generator=g)
+    return dict(dout=dout.to(_torch_dtype(w.dtype)).contiguous(),
+                dS_final=dS.contiguous() if dS_final else None,
+                dd_final=dd.contiguous() if dd_final else None)
+
+
 def make_decode_state(w: DecodeWorkload) -> dict:
     """Initial decode state: S0 ~ N(0, s0_std^2) fp32 [B, H, dv, dk], d0 = ones."""
     g = torch.Generator(device="cpu")

@@ -96,3 +96,23 @@ def test_binding_refuses_cpu_tensors(osdn_lib):
     x = torch.zeros((1, 4, 1, 64), dtype=torch.bfloat16)
     with pytest.raises(pk.OsdnError):
         pk.forward(x, x, x, torch.zeros((1, 4, 1), dtype=torch.bfloat16))
+
+
+def test_backward_workspace_and_argument_checks(osdn_lib):
+    L = osdn_lib.lib()
+    p = _params(osdn_lib)
+    n = ctypes.c_size_t(0)
+    assert L.osdn_bwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    # fp32 chunk intermediates: at least d_t, Kw, W, dD and dK per token and head (5 * dk floats)
+    assert n.value >= 5 * p.B * p.T * p.H * p.dk * 4 and n.value % 256 == 0
+    fake = ctypes.c_void_p(1 << 20)             # never dereferenced: checks fail first
+    args = [fake] * 4 + [None] * 3 + [fake, None, None] + [fake] * 4 + [None] * 3
+    rc = L.osdn_bwd(ctypes.byref(p), *args, fake, ctypes.c_size_t(n.value - 256), None)
+    assert rc == osdn_lib.OSDN_ERR_INVALID_ARG and "workspace" in osdn_lib.get_last_error()
+    rc = L.osdn_bwd(ctypes.byref(p), *args[:7], None, *args[8:], fake, n, None)     # dout NULL
+    assert rc == osdn_lib.OSDN_ERR_INVALID_ARG and "NULL" in osdn_lib.get_last_error()
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    rc = L.osdn_bwd(ctypes.byref(p), *args[:-4], odd, *args[-3:], fake, n, None)       # dbeta misaligned
+    assert rc == osdn_lib.OSDN_ERR_INVALID_ARG and "aligned" in osdn_lib.get_last_error()
+    bad = _params(osdn_lib, dk=96)
+    assert L.osdn_bwd_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == osdn_lib.OSDN_ERR_UNSUPPORTED
