@@ -48,21 +48,16 @@ namespace osdn {
 namespace bwd {
 
 constexpr int C = 64;         // chunk length
-constexpr int NTHR = 256;     // threads of the per-chunk and per-tile kernels (8 warps)
+constexpr int NTHR = 512;     // threads of the per-chunk and per-tile kernels (16 warps)
 constexpr int LDC = C + 4;    // row stride of C x C tiles (68 = 4 mod 32: conflict-free fragments)
 
-// X(i, j) = p[i * s0 + j * s1], fp32 in shared or global memory.
+// X(i, j) = p[i * S0 + j * S1], fp32 in shared memory; compile-time strides keep every
+// fragment load a single instruction with an immediate offset.
+template <int S0, int S1>
 struct Mat {
     const float* p;
-    int s0, s1;
-    __device__ __forceinline__ float operator()(int i, int j) const { return p[i * s0 + j * s1]; }
+    __device__ __forceinline__ float operator()(int i, int j) const { return p[i * S0 + j * S1]; }
 };
-
-__device__ __forceinline__ uint32_t tf32_rna(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
 
 __device__ __forceinline__ void mma8(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
     asm volatile(
@@ -72,22 +67,32 @@ __device__ __forceinline__ void mma8(float (&c)[4], const uint32_t (&a)[4], cons
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// c += a b for one m16n8k8 step; SPLIT: three tf32 products that recover fp32 accuracy.
+// c += a b for one m16n8k8 step. The fp32 bit patterns go to the tensor core as they
+// are: it reads the upper 19 bits (tf32 truncation, one tf32 ulp at most). SPLIT: a =
+// a_hi + a_lo with a_hi the truncated value and a_lo = a - a_hi (exact in fp32), and
+// c += a_lo b_hi + a_hi b_lo + a_hi b_hi, which recovers fp32 accuracy.
 template <bool SPLIT>
 __device__ __forceinline__ void mma_step(float (&c)[4], const float (&a)[4], const float (&b)[2]) {
     uint32_t ah[4], bh[2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) ah[i] = tf32_rna(a[i]);
-#pragma unroll
-    for (int i = 0; i < 2; ++i) bh[i] = tf32_rna(b[i]);
     if (SPLIT) {
         uint32_t al[4], bl[2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) al[i] = tf32_rna(a[i] - __uint_as_float(ah[i]));
+        for (int i = 0; i < 4; ++i) {
+            ah[i] = __float_as_uint(a[i]) & 0xffffe000u;
+            al[i] = __float_as_uint(a[i] - __uint_as_float(ah[i]));
+        }
 #pragma unroll
-        for (int i = 0; i < 2; ++i) bl[i] = tf32_rna(b[i] - __uint_as_float(bh[i]));
+        for (int i = 0; i < 2; ++i) {
+            bh[i] = __float_as_uint(b[i]) & 0xffffe000u;
+            bl[i] = __float_as_uint(b[i] - __uint_as_float(bh[i]));
+        }
         mma8(c, al, bh);
         mma8(c, ah, bl);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ah[i] = __float_as_uint(a[i]);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) bh[i] = __float_as_uint(b[i]);
     }
     mma8(c, ah, bh);
 }
@@ -95,10 +100,10 @@ __device__ __forceinline__ void mma_step(float (&c)[4], const float (&a)[4], con
 // One warp: acc[j] += sum_{k < K} A(m0 + ., k) B(k, n0 + 8 j + .) for a 16 x 8 NT tile.
 // Fragment element e of acc[j] sits at row m0 + g + 8 (e >> 1), column n0 + 8 j + 2 t + (e & 1),
 // with g = lane / 4, t = lane % 4.
-template <int NT, bool SPLIT>
-__device__ __forceinline__ void warp_mma(float (&acc)[NT][4], Mat A, Mat B, int m0, int n0, int K, int lane) {
+template <int NT, bool SPLIT, class MA, class MB>
+__device__ __forceinline__ void warp_mma(float (&acc)[NT][4], MA A, MB B, int m0, int n0, int K, int lane) {
     const int g = lane >> 2, t = lane & 3;
-#pragma unroll 2
+#pragma unroll 4
     for (int k0 = 0; k0 < K; k0 += 8) {
         const float a[4] = {A(m0 + g, k0 + t), A(m0 + g + 8, k0 + t), A(m0 + g, k0 + t + 4),
                             A(m0 + g + 8, k0 + t + 4)};
@@ -128,32 +133,40 @@ __device__ __forceinline__ void frag_each(float (&acc)[NT][4], int m0, int n0, i
 }
 
 // The CTA computes the M x N product sum_k A(m, k) B(k, n) (plus, for the two-term
-// form, a second product over K2) in 16 x 32 warp tiles taken round-robin, and calls
-// epi(m, n, value) once per output element on the thread that holds it.
-template <bool SPLIT, typename Epi>
-__device__ __forceinline__ void cta_gemm(int M, int N, int K, Mat A, Mat B, Epi epi) {
+// form, a second product over K2) in warp tiles of 16 x 8 NT taken round-robin, and
+// calls epi(m, n, value) once per output element on the thread that holds it.
+template <int NT, bool SPLIT, class MA1, class MB1, class MA2, class MB2, typename Epi>
+__device__ __forceinline__ void cta_gemm_nt(int M, int N, int K1, MA1 A1, MB1 B1, int K2, MA2 A2, MB2 B2, Epi epi) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const int tn = N / 32, tiles = (M / 16) * tn;
+    const int tn = N / (8 * NT), tiles = (M / 16) * tn;
     for (int tile = warp; tile < tiles; tile += nw) {
-        const int m0 = (tile / tn) * 16, n0 = (tile % tn) * 32;
-        float acc[4][4];
+        const int m0 = (tile / tn) * 16, n0 = (tile % tn) * 8 * NT;
+        float acc[NT][4];
         frag_zero(acc);
-        warp_mma<4, SPLIT>(acc, A, B, m0, n0, K, lane);
+        warp_mma<NT, SPLIT>(acc, A1, B1, m0, n0, K1, lane);
+        if (K2 > 0) warp_mma<NT, SPLIT>(acc, A2, B2, m0, n0, K2, lane);
         frag_each(acc, m0, n0, lane, epi);
     }
 }
 
-template <bool SPLIT, typename Epi>
-__device__ __forceinline__ void cta_gemm2(int M, int N, int K1, Mat A1, Mat B1, int K2, Mat A2, Mat B2, Epi epi) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const int tn = N / 32, tiles = (M / 16) * tn;
-    for (int tile = warp; tile < tiles; tile += nw) {
-        const int m0 = (tile / tn) * 16, n0 = (tile % tn) * 32;
-        float acc[4][4];
-        frag_zero(acc);
-        warp_mma<4, SPLIT>(acc, A1, B1, m0, n0, K1, lane);
-        warp_mma<4, SPLIT>(acc, A2, B2, m0, n0, K2, lane);
-        frag_each(acc, m0, n0, lane, epi);
+// 16 x 32 tiles when there are enough of them for every warp, else 16 x 16.
+template <bool SPLIT, class MA1, class MB1, class MA2, class MB2, typename Epi>
+__device__ __forceinline__ void cta_gemm2(int M, int N, int K1, MA1 A1, MB1 B1, int K2, MA2 A2, MB2 B2, Epi epi) {
+    if ((M / 16) * (N / 32) >= (int)(blockDim.x >> 5)) cta_gemm_nt<4, SPLIT>(M, N, K1, A1, B1, K2, A2, B2, epi);
+    else cta_gemm_nt<2, SPLIT>(M, N, K1, A1, B1, K2, A2, B2, epi);
+}
+
+template <bool SPLIT, class MA, class MB, typename Epi>
+__device__ __forceinline__ void cta_gemm(int M, int N, int K, MA A, MB B, Epi epi) {
+    cta_gemm2<SPLIT>(M, N, K, A, B, 0, A, B, epi);
+}
+
+// L2 prefetch hint for rows [0, rows) of row_bytes bytes each, stride_bytes apart from p.
+__device__ __forceinline__ void prefetch_rows(const void* p, size_t stride_bytes, int rows, int row_bytes) {
+    const int lines = (row_bytes + 127) / 128, n = rows * lines;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const char* a = static_cast<const char*>(p) + (size_t)(i / lines) * stride_bytes + (size_t)(i % lines) * 128;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
     }
 }
 
@@ -194,47 +207,174 @@ inline Layout make_layout(int B, int T, int H, int DK, int DV) {
 template <typename Tin>
 __device__ __forceinline__ float ld_or0(const Tin* p, size_t i, bool ok) { return ok ? to_f32(p[i]) : 0.f; }
 
+// 16-byte vector load of 4 fp32 or 8 bf16 values as fp32.
+__device__ __forceinline__ void load16(const float* p, float (&x)[4]) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+}
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&x)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+
+// The CTA copies a ROWS x COLS tile, dst[r * ldd + c] = src[r * lds + c] as fp32, with
+// rows r >= valid set to zero and every element scaled by scale[r] when scale is given.
+// COLS is a multiple of 16 / sizeof(Tsrc); src rows and dst rows are 16-byte aligned.
+// Every thread issues all of its loads before its first shared-memory store, so the
+// tile costs one memory round trip.
+template <int ROWS, int COLS, typename Tsrc>
+__device__ __forceinline__ void load_tile(float* dst, int ldd, const Tsrc* src, size_t lds, int valid,
+                                          const float* scale = nullptr) {
+    constexpr int V = 16 / sizeof(Tsrc), VPR = COLS / V, N = ROWS * VPR;
+    constexpr int PER = (N + NTHR - 1) / NTHR;
+    float x[PER][V];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int idx = threadIdx.x + u * NTHR, r = idx / VPR, c = (idx % VPR) * V;
+        if (idx < N && r < valid) {
+            load16(src + (size_t)r * lds + c, x[u]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < V; ++i) x[u][i] = 0.f;
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int idx = threadIdx.x + u * NTHR, r = idx / VPR, c = (idx % VPR) * V;
+        if (idx < N) {
+            const float sc = scale ? scale[r] : 1.f;
+#pragma unroll
+            for (int i = 0; i < V; i += 4)
+                *reinterpret_cast<float4*>(dst + r * ldd + c + i) =
+                    make_float4(sc * x[u][i], sc * x[u][i + 1], sc * x[u][i + 2], sc * x[u][i + 3]);
+        }
+    }
+}
+
+// Asynchronous copy (cp.async, 16 bytes per request) of a ROWS x COLS fp32 tile,
+// dst[r * ldd + c] = src[r * lds + c]; rows r >= valid are zero-filled (no global read).
+// Completes at cp_async_wait_all() followed by a CTA barrier.
+__device__ __forceinline__ void cp_async16(float* dst, const float* src, bool fill) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(fill ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <int ROWS, int COLS>
+__device__ __forceinline__ void async_tile(float* dst, int ldd, const float* src, size_t lds, int valid = ROWS) {
+    constexpr int VPR = COLS / 4, N = ROWS * VPR;
+    for (int idx = threadIdx.x; idx < N; idx += NTHR) {
+        const int r = idx / VPR, c = (idx % VPR) * 4;
+        const bool ok = r < valid;
+        cp_async16(dst + r * ldd + c, ok ? src + (size_t)r * lds + c : src, ok);
+    }
+}
+
+// dst[r * ldd + c] = src[r * COLS + c] for a dense fp32 ROWS x COLS block (the workspace layout).
+template <int ROWS, int COLS>
+__device__ __forceinline__ void async_block(float* dst, int ldd, const float* src) {
+    async_tile<ROWS, COLS>(dst, ldd, src, (size_t)COLS);
+}
+
 // ---------------------------------------------------------------------------
-// d_t (before the token's own update) for every token: one warp per unit.
+// The two token-serial kernels run one CTA of 128 threads per unit: warp 0
+// carries the recurrence, warps 1-3 stage the next slab of SLAB tokens into
+// shared memory meanwhile (double buffer), so no global load sits on the chain.
+constexpr int SLAB = 32;
+constexpr int SERIAL_THREADS = 128;
+
+// Warps 1-3 copy rows [0, n) of a slab, row t at src + t * stride (16-byte aligned,
+// width elements), into dst[t * width ..]; rows n .. SLAB - 1 become zero.
+template <typename T>
+__device__ __forceinline__ void stage_rows(T* dst, const T* src, size_t stride, int width, int n) {
+    constexpr int V = 16 / sizeof(T);
+    const int vpr = width / V;
+    for (int idx = threadIdx.x - 32; idx < SLAB * vpr; idx += SERIAL_THREADS - 32) {
+        const int t = idx / vpr, c = (idx % vpr) * V;
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (t < n) u = *reinterpret_cast<const uint4*>(src + (size_t)t * stride + c);
+        *reinterpret_cast<uint4*>(dst + (size_t)t * width + c) = u;
+    }
+}
+
 template <int DK, typename Tin>
-__global__ void __launch_bounds__(128)
+struct DtrajSmem {
+    static constexpr size_t kBytes = 2 * (SLAB * DK * sizeof(Tin) + 2 * SLAB * sizeof(float));
+};
+
+// d_t (before the token's own update) for every token.
+template <int DK, typename Tin>
+__global__ void __launch_bounds__(SERIAL_THREADS, 1)
 bwd_dtraj_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const Tin* __restrict__ r,
                  const float* __restrict__ d0, float* __restrict__ d_all, int B, int T, int H, float eta, int anchor)
 {
     constexpr int PER = DK / 32;
-    const int lane = threadIdx.x & 31;
-    const int unit = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (unit >= B * H) return;
-    const int b = unit / H, h = unit % H;
+    extern __shared__ __align__(16) unsigned char smraw[];
+    Tin* ks = reinterpret_cast<Tin*>(smraw);                                        // [2][SLAB][DK]
+    float* bs = reinterpret_cast<float*>(smraw + 2 * SLAB * DK * sizeof(Tin));      // [2][SLAB]
+    float* rs = bs + 2 * SLAB;                                                      // [2][SLAB]
+    const int unit = blockIdx.x, b = unit / H, h = unit % H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nslab = (T + SLAB - 1) / SLAB;
+    auto stage = [&](int sl, int buf) {
+        const int t0 = sl * SLAB, n = min(SLAB, T - t0);
+        const size_t tok0 = ((size_t)b * T + t0) * H + h;
+        stage_rows(ks + buf * SLAB * DK, k + tok0 * DK, (size_t)H * DK, DK, n);
+        for (int t = threadIdx.x - 32; t < SLAB; t += SERIAL_THREADS - 32) {
+            bs[buf * SLAB + t] = t < n ? to_f32(beta[tok0 + (size_t)t * H]) : 0.f;
+            rs[buf * SLAB + t] = (t < n && r) ? to_f32(r[tok0 + (size_t)t * H]) : 1.f;
+        }
+    };
     float d[PER], da[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) d[i] = d0 ? d0[(size_t)unit * DK + lane * PER + i] : 1.f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) da[i] = anchor ? d[i] : 0.f;
-    for (int t = 0; t < T; ++t) {
-        const size_t tok = ((size_t)b * T + t) * H + h;
-        float kk[PER], a[PER];
-        VecIO<PER, Tin>::load(k + tok * DK + lane * PER, kk);
-        VecIO<PER, float>::store(d_all + tok * DK + lane * PER, d);
-        const float bt = to_f32(beta[tok]), rt = r ? to_f32(r[tok]) : 1.f;
-        float n = 0.f, s = 0.f;
+    if (warp != 0 && nslab > 0) stage(0, 0);
+    __syncthreads();
+    for (int sl = 0; sl < nslab; ++sl) {
+        const int buf = sl & 1;
+        if (warp != 0) {
+            if (sl + 1 < nslab) stage(sl + 1, buf ^ 1);
+        } else {
+            const int t0 = sl * SLAB, n = min(SLAB, T - t0);
+            for (int t = 0; t < n; ++t) {
+                const size_t tok = ((size_t)b * T + t0 + t) * H + h;
+                float kk[PER], a[PER];
+                VecIO<PER, Tin>::load(ks + (buf * SLAB + t) * DK + lane * PER, kk);
+                const float bt = bs[buf * SLAB + t], rt = rs[buf * SLAB + t];
+                VecIO<PER, float>::store(d_all + tok * DK + lane * PER, d);
+                float n2 = 0.f, sd = 0.f;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            a[i] = kk[i] * kk[i];
-            n += a[i];
-            s += d[i] * a[i];
+                for (int i = 0; i < PER; ++i) {
+                    a[i] = kk[i] * kk[i];
+                    n2 += a[i];
+                    sd += d[i] * a[i];
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+                    sd += __shfl_xor_sync(0xffffffffu, sd, o);
+                }
+                const float x = (n2 > 0.f) ? eta * bt * (1.f - bt * sd) / n2 : 0.f;
+#pragma unroll
+                for (int i = 0; i < PER; ++i) d[i] = rt * d[i] + (1.f - rt) * da[i] + x * a[i];
+            }
         }
-        n = warp_sum(n);
-        s = warp_sum(s);
-        const float x = (n > 0.f) ? eta * bt * (1.f - bt * s) / n : 0.f;
-#pragma unroll
-        for (int i = 0; i < PER; ++i) d[i] = rt * d[i] + (1.f - rt) * da[i] + x * a[i];
+        __syncthreads();
     }
 }
 
 // ---------------------------------------------------------------------------
 // Per chunk: Kw = D (.) K, T = (I + strict_tril(Kb Kw^T))^{-1}, W = T Kb,
-// U0 = T diag(beta) V, P = tril(Q Kw^T).  One CTA per (unit, chunk).
+// U0 = T diag(beta) V, P = tril(Q Kw^T).  Persistent CTAs, one chunk at a time.
 template <int DK, int DV>
 struct PrepSmem {
     static constexpr int LDK = DK + 4, LDX = (DK > DV ? DK : DV) + 4;
@@ -258,62 +398,74 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     float* bs = Ts + C * LDC;        // [C] beta
 
     const int tid = threadIdx.x;
-    const size_t cid = blockIdx.x;                 // unit * NC + chunk
+    const size_t nchunks = (size_t)B * H * NC;
+    const float* d_all = ws + L.d_all / sizeof(float);
+    // persistent: chunk cid, then cid + gridDim.x, ...; the next chunk's inputs are
+    // prefetched into L2 while this one is computed
+    for (size_t cid = blockIdx.x; cid < nchunks; cid += gridDim.x) {
     const int unit = (int)(cid / NC), c = (int)(cid % NC), b = unit / H, h = unit % H;
     const int c0 = c * C, Tc = min(C, T - c0);
-    const float* d_all = ws + L.d_all / sizeof(float);
     float* kw_g = ws + L.kw / sizeof(float) + cid * C * DK;
     float* t_g = ws + L.tinv / sizeof(float) + cid * C * C;
     float* w_g = ws + L.w / sizeof(float) + cid * C * DK;
     float* u_g = ws + L.u0 / sizeof(float) + cid * C * DV;
     float* p_g = ws + L.p / sizeof(float) + cid * C * C;
 
-    if (tid < C) bs[tid] = ld_or0(beta, ((size_t)b * T + c0 + tid) * H + h, tid < Tc);
+    const size_t tok0 = ((size_t)b * T + c0) * H + h;     // token c0 of this (b, h)
+    const size_t tstride = (size_t)H;                     // token step in [B, T, H] order
+    __syncthreads();
+    if (cid + gridDim.x < nchunks) {
+        const size_t nx = cid + gridDim.x;
+        const int un = (int)(nx / NC), cn = (int)(nx % NC), bn = un / H, hn = un % H;
+        const int tcn = min(C, T - cn * C);
+        const size_t tokn = ((size_t)bn * T + cn * C) * H + hn;
+        prefetch_rows(k + tokn * DK, tstride * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
+        prefetch_rows(q + tokn * DK, tstride * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
+        prefetch_rows(v + tokn * DV, tstride * DV * sizeof(Tin), tcn, DV * sizeof(Tin));
+        prefetch_rows(d_all + tokn * DK, tstride * DK * sizeof(float), tcn, DK * sizeof(float));
+    }
+    if (tid < C) bs[tid] = ld_or0(beta, tok0 + tid * tstride, tid < Tc);
+    async_tile<C, DK>(Kw, LDK, d_all + tok0 * DK, tstride * DK, Tc);     // d_t for now
+    load_tile<C, DK>(Kb, LDK, k + tok0 * DK, tstride * DK, Tc);
+    cp_async_wait_all();
     __syncthreads();
     for (int idx = tid; idx < C * DK; idx += NTHR) {
         const int t = idx / DK, i = idx % DK;
-        const bool ok = t < Tc;
-        const size_t tok = ((size_t)b * T + c0 + t) * H + h;
-        const float kv = ld_or0(k, tok * DK + i, ok);
-        const float w = ok ? d_all[tok * DK + i] * kv : 0.f;
+        const float kv = Kb[t * LDK + i], w = Kw[t * LDK + i] * kv;
         Kb[t * LDK + i] = bs[t] * kv;
         Kw[t * LDK + i] = w;
         kw_g[idx] = w;
     }
-    for (int idx = tid; idx < C * DV; idx += NTHR) {
-        const int t = idx / DV, j = idx % DV;
-        X[t * LDX + j] = bs[t] * ld_or0(v, (((size_t)b * T + c0 + t) * H + h) * DV + j, t < Tc);
-    }
+    load_tile<C, DV>(X, LDX, v + tok0 * DV, tstride * DV, Tc, bs);
     __syncthreads();
-    cta_gemm<SPLIT>(C, C, DK, Mat{Kb, LDK, 1}, Mat{Kw, 1, LDK},
+    cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{Kb}, Mat<1, LDK>{Kw},
                     [&](int m, int n, float x) { As[m * LDC + n] = n < m ? x : 0.f; });
     __syncthreads();
-    {   // (I + A) T = I by forward substitution: column j on 4 threads that split the inner sum
-        const int j = tid >> 2, part = tid & 3;
+    {   // (I + A) T = I by forward substitution: column j on 8 threads that split the inner sum
+        const int j = tid >> 3, part = tid & 7;
         for (int i = 0; i < C; ++i) {
-            float s = 0.f;
-            for (int l = j + part; l < i; l += 4) s = fmaf(As[i * LDC + l], Ts[l * LDC + j], s);
-            s += __shfl_xor_sync(0xffffffffu, s, 1);
-            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            float sum = 0.f;
+            for (int l = j + part; l < i; l += 8) sum = fmaf(As[i * LDC + l], Ts[l * LDC + j], sum);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 4);
             __syncwarp();
-            if (part == 0) Ts[i * LDC + j] = (i < j) ? 0.f : (i == j ? 1.f : -s);
+            if (part == 0) Ts[i * LDC + j] = (i < j) ? 0.f : (i == j ? 1.f : -sum);
             __syncwarp();
         }
     }
     __syncthreads();
     for (int idx = tid; idx < C * C; idx += NTHR) t_g[idx] = Ts[(idx / C) * LDC + idx % C];
-    cta_gemm<SPLIT>(C, DK, C, Mat{Ts, LDC, 1}, Mat{Kb, LDK, 1},
+    cta_gemm<SPLIT>(C, DK, C, Mat<LDC, 1>{Ts}, Mat<LDK, 1>{Kb},
                     [&](int m, int n, float x) { w_g[m * DK + n] = x; });
-    cta_gemm<SPLIT>(C, DV, C, Mat{Ts, LDC, 1}, Mat{X, LDX, 1},
+    cta_gemm<SPLIT>(C, DV, C, Mat<LDC, 1>{Ts}, Mat<LDX, 1>{X},
                     [&](int m, int n, float x) { u_g[m * DV + n] = x; });
     __syncthreads();
-    for (int idx = tid; idx < C * DK; idx += NTHR) {
-        const int t = idx / DK, i = idx % DK;
-        X[t * LDX + i] = ld_or0(q, (((size_t)b * T + c0 + t) * H + h) * DK + i, t < Tc);
-    }
+    load_tile<C, DK>(X, LDX, q + tok0 * DK, tstride * DK, Tc);
     __syncthreads();
-    cta_gemm<SPLIT>(C, C, DK, Mat{X, LDX, 1}, Mat{Kw, 1, LDK},
+    cta_gemm<SPLIT>(C, C, DK, Mat<LDX, 1>{X}, Mat<1, LDK>{Kw},
                     [&](int m, int n, float x) { p_g[m * C + n] = n <= m ? x : 0.f; });
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -352,27 +504,27 @@ bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout 
         float* s_g = ws + L.ckS / sizeof(float) + cid * DV * DK;
         float* vn_g = ws + L.vn / sizeof(float) + cid * C * DV;
         __syncthreads();
+        if (c + 1 < NC) {   // L2 prefetch of the next chunk's blocks
+            prefetch_rows(w_g + C * DK, 0, 1, C * DK * 4);
+            prefetch_rows(kw_g + C * DK, 0, 1, C * DK * 4);
+            prefetch_rows(u_g + C * DV + v0, (size_t)DV * 4, C, DVT * 4);
+        }
         for (int idx = tid; idx < DVT * DK; idx += NTHR) {
             const int row = idx / DK, i = idx % DK;
             s_g[(size_t)(v0 + row) * DK + i] = Ss[row * LDK + i];
         }
-        for (int idx = tid; idx < C * DK; idx += NTHR) {
-            const int t = idx / DK, i = idx % DK;
-            Ws[t * LDK + i] = w_g[idx];
-            Kws[t * LDK + i] = kw_g[idx];
-        }
-        for (int idx = tid; idx < C * DVT; idx += NTHR) {
-            const int t = idx / DVT, j = idx % DVT;
-            Vs[t * LDT + j] = u_g[t * DV + v0 + j];
-        }
+        async_block<C, DK>(Ws, LDK, w_g);
+        async_block<C, DK>(Kws, LDK, kw_g);
+        async_tile<C, DVT>(Vs, LDT, u_g + v0, (size_t)DV);
+        cp_async_wait_all();
         __syncthreads();
-        cta_gemm<SPLIT>(C, DVT, DK, Mat{Ws, LDK, 1}, Mat{Ss, 1, LDK}, [&](int m, int n, float x) {
+        cta_gemm<SPLIT>(C, DVT, DK, Mat<LDK, 1>{Ws}, Mat<1, LDK>{Ss}, [&](int m, int n, float x) {
             const float vn = Vs[m * LDT + n] - x;
             Vs[m * LDT + n] = vn;
             vn_g[m * DV + v0 + n] = vn;
         });
         __syncthreads();
-        cta_gemm<SPLIT>(DVT, DK, C, Mat{Vs, 1, LDT}, Mat{Kws, LDK, 1},
+        cta_gemm<SPLIT>(DVT, DK, C, Mat<1, LDT>{Vs}, Mat<LDK, 1>{Kws},
                         [&](int m, int n, float x) { Ss[m * LDK + n] += x; });
     }
 }
@@ -409,32 +561,37 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
         float* ds_g = ws + L.ckdS / sizeof(float) + cid * DV * DK;
         float* dvn_g = ws + L.dvn / sizeof(float) + cid * C * DV;
         __syncthreads();
+        if (c > 0) {   // L2 prefetch of the previous chunk's blocks and rows (chunk c - 1 is full)
+            const size_t tokp = ((size_t)b * T + c0 - C) * H + h;
+            prefetch_rows(p_g - C * C, 0, 1, C * C * 4);
+            prefetch_rows(kw_g - C * DK, 0, 1, C * DK * 4);
+            prefetch_rows(w_g - C * DK, 0, 1, C * DK * 4);
+            prefetch_rows(dout + tokp * DV + v0, (size_t)H * DV * sizeof(Tin), C, DVT * sizeof(Tin));
+            prefetch_rows(q + tokp * DK, (size_t)H * DK * sizeof(Tin), C, DK * sizeof(Tin));
+        }
         for (int idx = tid; idx < DVT * DK; idx += NTHR) {
             const int row = idx / DK, i = idx % DK;
             ds_g[(size_t)(v0 + row) * DK + i] = dSs[row * LDK + i];
         }
-        for (int idx = tid; idx < C * C; idx += NTHR) Ps[(idx / C) * LDC + idx % C] = p_g[idx];
-        for (int idx = tid; idx < C * DVT; idx += NTHR) {
-            const int t = idx / DVT, j = idx % DVT;
-            dOs[t * LDT + j] = ld_or0(dout, (((size_t)b * T + c0 + t) * H + h) * DV + v0 + j, t < Tc);
-        }
-        for (int idx = tid; idx < C * DK; idx += NTHR) {
-            const int t = idx / DK, i = idx % DK;
-            B1[t * LDK + i] = kw_g[idx];
-            B2[t * LDK + i] = ld_or0(q, (((size_t)b * T + c0 + t) * H + h) * DK + i, t < Tc);
-        }
+        const size_t tok0 = ((size_t)b * T + c0) * H + h;
+        async_block<C, C>(Ps, LDC, p_g);
+        async_block<C, DK>(B1, LDK, kw_g);
+        load_tile<C, DVT>(dOs, LDT, dout + tok0 * DV + v0, (size_t)H * DV, Tc);
+        load_tile<C, DK>(B2, LDK, q + tok0 * DK, (size_t)H * DK, Tc);
+        cp_async_wait_all();
         __syncthreads();
         // dVn = P^T dO + Kw dS'^T
-        cta_gemm2<SPLIT>(C, DVT, C, Mat{Ps, 1, LDC}, Mat{dOs, LDT, 1}, DK, Mat{B1, LDK, 1}, Mat{dSs, 1, LDK},
+        cta_gemm2<SPLIT>(C, DVT, C, Mat<1, LDC>{Ps}, Mat<LDT, 1>{dOs}, DK, Mat<LDK, 1>{B1}, Mat<1, LDK>{dSs},
                          [&](int m, int n, float x) {
                              dVs[m * LDT + n] = -x;
                              dvn_g[m * DV + v0 + n] = x;
                          });
         __syncthreads();
-        for (int idx = tid; idx < C * DK; idx += NTHR) B1[(idx / DK) * LDK + idx % DK] = w_g[idx];
+        async_block<C, DK>(B1, LDK, w_g);
+        cp_async_wait_all();
         __syncthreads();
         // dS = dS' + dO^T Q + (-dVn)^T W
-        cta_gemm2<SPLIT>(DVT, DK, C, Mat{dOs, 1, LDT}, Mat{B2, LDK, 1}, C, Mat{dVs, 1, LDT}, Mat{B1, LDK, 1},
+        cta_gemm2<SPLIT>(DVT, DK, C, Mat<1, LDT>{dOs}, Mat<LDK, 1>{B2}, C, Mat<1, LDT>{dVs}, Mat<LDK, 1>{B1},
                          [&](int m, int n, float x) { dSs[m * LDK + n] += x; });
     }
     __syncthreads();
@@ -446,10 +603,11 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
 }
 
 // ---------------------------------------------------------------------------
-// Per chunk, over the dv tiles in turn: dP, dQ, dV, dW, dT (V part), the
-// dv-summed part of dKw (Vn dS' + dP^T Q) and of dbeta (rowdot(T^T dVn, V)).
-// dQ, dKw and dW stay in registers: warp w owns rows 16 (w % 4) .. + 15 and
-// columns (DK / 2) (w / 4) .. + DK / 2 - 1 of each.
+// Per chunk, over the dv tiles in turn: dP and dT (V part) summed over the
+// tiles, dV, and the tile terms of dQ (dO S), dKw (Vn dS') and dW (-dVn S);
+// then dQ += dP Kw and dKw += dP^T Q once, and the dv-summed part of dbeta
+// (rowdot(T^T dVn, V)). dQ, dKw and dW stay in registers: warp w (of 16) owns
+// rows 16 (w % 4) .. + 15 and columns (DK / 4) (w / 4) .. + DK / 4 - 1 of each.
 constexpr int J = 32;           // dv tile of the gradient kernel
 constexpr int LDJ = J + 4;
 
@@ -477,12 +635,12 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
                    float* __restrict__ ws, Layout L, int B, int T, int H, int NC)
 {
     constexpr bool SPLIT = std::is_same<Tin, float>::value;
-    constexpr int LDK = GradSmem<DK>::LDK, NT = DK / 16;
+    constexpr int LDK = GradSmem<DK>::LDK, NT = DK / 32;
     extern __shared__ float sm[];
     float* Qs = sm;                  // [C][LDK] Q
     float* Kws = Qs + C * LDK;       // [C][LDK] Kw
     float* Ts = Kws + C * LDK;       // [C][LDC] T
-    float* dPs = Ts + C * LDC;       // [C][LDC] dP of the current tile
+    float* dPs = Ts + C * LDC;       // [C][LDC] dP, summed over the tiles
     float* dTs = dPs + C * LDC;      // [C][LDC] dT (V part), summed over the tiles
     float* dOs = dTs + C * LDC;      // [C][LDJ] dO columns of the tile
     float* Vns = dOs + C * LDJ;      // [C][LDJ] Vn
@@ -494,7 +652,8 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
     float* dbs = bs + C;             // [C] dbeta (this kernel's part)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const size_t cid = blockIdx.x;
+    const size_t nchunks = (size_t)B * H * NC;
+    for (size_t cid = blockIdx.x; cid < nchunks; cid += gridDim.x) {   // persistent, as bwd_prep
     const int unit = (int)(cid / NC), c = (int)(cid % NC), b = unit / H, h = unit % H;
     const int c0 = c * C, Tc = min(C, T - c0);
     const float* kw_g = ws + L.kw / sizeof(float) + cid * C * DK;
@@ -509,58 +668,68 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
     float* dba_g = ws + L.dba / sizeof(float) + cid * C;
     auto tok = [&](int t) { return ((size_t)b * T + c0 + t) * H + h; };
 
-    for (int idx = tid; idx < C * DK; idx += NTHR) {
-        const int t = idx / DK, i = idx % DK;
-        Qs[t * LDK + i] = ld_or0(q, tok(t) * DK + i, t < Tc);
-        Kws[t * LDK + i] = kw_g[idx];
+    const size_t tok0 = tok(0);
+    __syncthreads();
+    if (cid + gridDim.x < nchunks) {   // L2 prefetch of the next chunk's inputs
+        const size_t nx = cid + gridDim.x;
+        const int un = (int)(nx / NC), cn = (int)(nx % NC), bn = un / H, hn = un % H;
+        const int tcn = min(C, T - cn * C);
+        const size_t tokn = ((size_t)bn * T + cn * C) * H + hn;
+        prefetch_rows(q + tokn * DK, (size_t)H * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
+        prefetch_rows(v + tokn * DV, (size_t)H * DV * sizeof(Tin), tcn, DV * sizeof(Tin));
+        prefetch_rows(dout + tokn * DV, (size_t)H * DV * sizeof(Tin), tcn, DV * sizeof(Tin));
+        prefetch_rows(ws + L.kw / sizeof(float) + nx * C * DK, 0, 1, C * DK * 4);
+        prefetch_rows(ws + L.tinv / sizeof(float) + nx * C * C, 0, 1, C * C * 4);
+        prefetch_rows(ws + L.vn / sizeof(float) + nx * C * DV, 0, 1, C * DV * 4);
+        prefetch_rows(ws + L.dvn / sizeof(float) + nx * C * DV, 0, 1, C * DV * 4);
+        prefetch_rows(ws + L.ckS / sizeof(float) + nx * DV * DK, 0, 1, DV * DK * 4);
+        prefetch_rows(ws + L.ckdS / sizeof(float) + nx * DV * DK, 0, 1, DV * DK * 4);
     }
+    async_block<C, DK>(Kws, LDK, kw_g);        // waited for with the first tile's copies
+    async_block<C, C>(Ts, LDC, t_g);
+    load_tile<C, DK>(Qs, LDK, q + tok0 * DK, (size_t)H * DK, Tc);
     for (int idx = tid; idx < C * C; idx += NTHR) {
-        Ts[(idx / C) * LDC + idx % C] = t_g[idx];
         dTs[(idx / C) * LDC + idx % C] = 0.f;
+        dPs[(idx / C) * LDC + idx % C] = 0.f;
     }
     if (tid < C) {
         bs[tid] = ld_or0(beta, tok(tid), tid < Tc);
         dbs[tid] = 0.f;
     }
 
-    const int m0 = 16 * (warp & 3), n0 = (DK / 2) * (warp >> 2);
+    const int m0 = 16 * (warp & 3), n0 = (DK / 4) * (warp >> 2);
     float aQ[NT][4], aKw[NT][4], aW[NT][4];
     frag_zero(aQ);
     frag_zero(aKw);
     frag_zero(aW);
     for (int v0 = 0; v0 < DV; v0 += J) {
         __syncthreads();
-        for (int idx = tid; idx < C * J; idx += NTHR) {
-            const int t = idx / J, j = idx % J;
-            dOs[t * LDJ + j] = ld_or0(dout, tok(t) * DV + v0 + j, t < Tc);
-            Vs[t * LDJ + j] = ld_or0(v, tok(t) * DV + v0 + j, t < Tc);
-            Vns[t * LDJ + j] = vn_g[t * DV + v0 + j];
-            dVns[t * LDJ + j] = dvn_g[t * DV + v0 + j];
-        }
-        for (int idx = tid; idx < J * DK; idx += NTHR) {
-            const int row = idx / DK, i = idx % DK;
-            SJ[row * LDK + i] = s_g[(size_t)(v0 + row) * DK + i];
-            dSJ[row * LDK + i] = ds_g[(size_t)(v0 + row) * DK + i];
-        }
+        async_tile<C, J>(Vns, LDJ, vn_g + v0, (size_t)DV);
+        async_tile<C, J>(dVns, LDJ, dvn_g + v0, (size_t)DV);
+        async_block<J, DK>(SJ, LDK, s_g + (size_t)v0 * DK);
+        async_block<J, DK>(dSJ, LDK, ds_g + (size_t)v0 * DK);
+        load_tile<C, J>(dOs, LDJ, dout + tok0 * DV + v0, (size_t)H * DV, Tc);
+        load_tile<C, J>(Vs, LDJ, v + tok0 * DV + v0, (size_t)H * DV, Tc);
+        cp_async_wait_all();
         __syncthreads();
-        // dP = tril(dO Vn^T) for this tile
-        cta_gemm<SPLIT>(C, C, J, Mat{dOs, LDJ, 1}, Mat{Vns, 1, LDJ},
-                        [&](int m, int n, float x) { dPs[m * LDC + n] = n <= m ? x : 0.f; });
+        // dP += tril(dO Vn^T) of this tile
+        cta_gemm<SPLIT>(C, C, J, Mat<LDJ, 1>{dOs}, Mat<1, LDJ>{Vns},
+                        [&](int m, int n, float x) { if (n <= m) dPs[m * LDC + n] += x; });
         // dT += (dVn V^T) diag(beta)
-        cta_gemm<SPLIT>(C, C, J, Mat{dVns, LDJ, 1}, Mat{Vs, 1, LDJ},
+        cta_gemm<SPLIT>(C, C, J, Mat<LDJ, 1>{dVns}, Mat<1, LDJ>{Vs},
                         [&](int m, int n, float x) { dTs[m * LDC + n] += bs[n] * x; });
         // dV = diag(beta) T^T dVn;  dbeta += rowdot(T^T dVn, V)
-        cta_gemm<SPLIT>(C, J, C, Mat{Ts, 1, LDC}, Mat{dVns, LDJ, 1}, [&](int m, int n, float x) {
+        cta_gemm<SPLIT>(C, J, C, Mat<1, LDC>{Ts}, Mat<LDJ, 1>{dVns}, [&](int m, int n, float x) {
             if (m < Tc) dv[tok(m) * DV + v0 + n] = from_f32<Tin>(bs[m] * x);
             atomicAdd(&dbs[m], x * Vs[m * LDJ + n]);
         });
-        __syncthreads();
-        warp_mma<NT, SPLIT>(aQ, Mat{dOs, LDJ, 1}, Mat{SJ, LDK, 1}, m0, n0, J, lane);     // dO S
-        warp_mma<NT, SPLIT>(aQ, Mat{dPs, LDC, 1}, Mat{Kws, LDK, 1}, m0, n0, C, lane);    // dP Kw
-        warp_mma<NT, SPLIT>(aKw, Mat{Vns, LDJ, 1}, Mat{dSJ, LDK, 1}, m0, n0, J, lane);   // Vn dS'
-        warp_mma<NT, SPLIT>(aKw, Mat{dPs, 1, LDC}, Mat{Qs, LDK, 1}, m0, n0, C, lane);    // dP^T Q
-        warp_mma<NT, SPLIT>(aW, Mat{dVns, LDJ, 1}, Mat{SJ, LDK, 1}, m0, n0, J, lane);    // dVn S
+        warp_mma<NT, SPLIT>(aQ, Mat<LDJ, 1>{dOs}, Mat<LDK, 1>{SJ}, m0, n0, J, lane);     // dO S
+        warp_mma<NT, SPLIT>(aKw, Mat<LDJ, 1>{Vns}, Mat<LDK, 1>{dSJ}, m0, n0, J, lane);   // Vn dS'
+        warp_mma<NT, SPLIT>(aW, Mat<LDJ, 1>{dVns}, Mat<LDK, 1>{SJ}, m0, n0, J, lane);    // dVn S
     }
+    __syncthreads();
+    warp_mma<NT, SPLIT>(aQ, Mat<LDC, 1>{dPs}, Mat<LDK, 1>{Kws}, m0, n0, C, lane);        // dP Kw
+    warp_mma<NT, SPLIT>(aKw, Mat<1, LDC>{dPs}, Mat<LDK, 1>{Qs}, m0, n0, C, lane);        // dP^T Q
     frag_each(aQ, m0, n0, lane, [&](int m, int n, float x) {
         if (m < Tc) dq[tok(m) * DK + n] = from_f32<Tin>(x);
     });
@@ -569,6 +738,7 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
     __syncthreads();
     for (int idx = tid; idx < C * C; idx += NTHR) dt_g[idx] = dTs[(idx / C) * LDC + idx % C];
     if (tid < C) dba_g[tid] = dbs[tid];
+    }
 }
 
 // Per chunk: dT += (dW K^T) diag(beta), dA = -strict_tril(T^T dT T^T), the
@@ -580,7 +750,7 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
                    int B, int T, int H, int NC)
 {
     constexpr bool SPLIT = std::is_same<Tin, float>::value;
-    constexpr int LDK = GradSmem<DK>::LDK, NT = DK / 16;
+    constexpr int LDK = GradSmem<DK>::LDK, NT = DK / 32;
     extern __shared__ float sm[];
     float* Ks = sm;                  // [C][LDK] K
     float* Kws = Ks + C * LDK;       // [C][LDK] Kw
@@ -593,10 +763,11 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
     float* dbs = bs + C;             // [C] dbeta (chunk part)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const size_t cid = blockIdx.x;
+    const size_t nchunks = (size_t)B * H * NC;
+    const float* d_all = ws + L.d_all / sizeof(float);
+    for (size_t cid = blockIdx.x; cid < nchunks; cid += gridDim.x) {   // persistent, as bwd_prep
     const int unit = (int)(cid / NC), c = (int)(cid % NC), b = unit / H, h = unit % H;
     const int c0 = c * C, Tc = min(C, T - c0);
-    const float* d_all = ws + L.d_all / sizeof(float);
     const float* kw_g = ws + L.kw / sizeof(float) + cid * C * DK;
     const float* t_g = ws + L.tinv / sizeof(float) + cid * C * C;
     const float* dkwa_g = ws + L.dkwa / sizeof(float) + cid * C * DK;
@@ -608,30 +779,40 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
     float* dbp_g = ws + L.dbp / sizeof(float) + cid * C;
     auto tok = [&](int t) { return ((size_t)b * T + c0 + t) * H + h; };
 
-    for (int idx = tid; idx < C * DK; idx += NTHR) {
-        const int t = idx / DK, i = idx % DK;
-        Ks[t * LDK + i] = ld_or0(k, tok(t) * DK + i, t < Tc);
-        Kws[t * LDK + i] = kw_g[idx];
-        dWs[t * LDK + i] = dw_g[idx];
+    __syncthreads();
+    if (cid + gridDim.x < nchunks) {   // L2 prefetch of the next chunk's inputs
+        const size_t nx = cid + gridDim.x;
+        const int un = (int)(nx / NC), cn = (int)(nx % NC), bn = un / H, hn = un % H;
+        const int tcn = min(C, T - cn * C);
+        const size_t tokn = ((size_t)bn * T + cn * C) * H + hn;
+        prefetch_rows(k + tokn * DK, (size_t)H * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
+        prefetch_rows(d_all + tokn * DK, (size_t)H * DK * sizeof(float), tcn, DK * sizeof(float));
+        prefetch_rows(ws + L.kw / sizeof(float) + nx * C * DK, 0, 1, C * DK * 4);
+        prefetch_rows(ws + L.dw / sizeof(float) + nx * C * DK, 0, 1, C * DK * 4);
+        prefetch_rows(ws + L.dkwa / sizeof(float) + nx * C * DK, 0, 1, C * DK * 4);
+        prefetch_rows(ws + L.tinv / sizeof(float) + nx * C * C, 0, 1, C * C * 4);
+        prefetch_rows(ws + L.dt / sizeof(float) + nx * C * C, 0, 1, C * C * 4);
     }
-    for (int idx = tid; idx < C * C; idx += NTHR) {
-        Ts[(idx / C) * LDC + idx % C] = t_g[idx];
-        dTs[(idx / C) * LDC + idx % C] = dt_g[idx];
-    }
+    async_block<C, DK>(Kws, LDK, kw_g);
+    async_block<C, DK>(dWs, LDK, dw_g);
+    async_block<C, C>(Ts, LDC, t_g);
+    async_block<C, C>(dTs, LDC, dt_g);
+    load_tile<C, DK>(Ks, LDK, k + tok(0) * DK, (size_t)H * DK, Tc);
     if (tid < C) {
         bs[tid] = ld_or0(beta, tok(tid), tid < Tc);
         dbs[tid] = dba_g[tid];
     }
+    cp_async_wait_all();
     __syncthreads();
-    cta_gemm<SPLIT>(C, C, DK, Mat{dWs, LDK, 1}, Mat{Ks, 1, LDK},
+    cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{dWs}, Mat<1, LDK>{Ks},
                     [&](int m, int n, float x) { dTs[m * LDC + n] += bs[n] * x; });
-    cta_gemm<SPLIT>(C, C, DK, Mat{Ks, LDK, 1}, Mat{Kws, 1, LDK},
+    cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{Ks}, Mat<1, LDK>{Kws},
                     [&](int m, int n, float x) { Gs[m * LDC + n] = x; });
     __syncthreads();
-    cta_gemm<SPLIT>(C, C, C, Mat{dTs, LDC, 1}, Mat{Ts, 1, LDC},
+    cta_gemm<SPLIT>(C, C, C, Mat<LDC, 1>{dTs}, Mat<1, LDC>{Ts},
                     [&](int m, int n, float x) { Xs[m * LDC + n] = x; });
     __syncthreads();
-    cta_gemm<SPLIT>(C, C, C, Mat{Ts, 1, LDC}, Mat{Xs, LDC, 1}, [&](int m, int n, float x) {
+    cta_gemm<SPLIT>(C, C, C, Mat<1, LDC>{Ts}, Mat<LDC, 1>{Xs}, [&](int m, int n, float x) {
         float ab = 0.f;
         if (n < m) {
             const float a = -x;                      // dA (strictly lower)
@@ -641,17 +822,17 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
         dTs[m * LDC + n] = ab;                       // diag(beta) dA
     });
     __syncthreads();
-    const int m0 = 16 * (warp & 3), n0 = (DK / 2) * (warp >> 2);
+    const int m0 = 16 * (warp & 3), n0 = (DK / 4) * (warp >> 2);
     float aK[NT][4], aKw[NT][4];
     frag_zero(aK);
-    warp_mma<NT, SPLIT>(aK, Mat{Ts, 1, LDC}, Mat{dWs, LDK, 1}, m0, n0, C, lane);        // T^T dW
+    warp_mma<NT, SPLIT>(aK, Mat<1, LDC>{Ts}, Mat<LDK, 1>{dWs}, m0, n0, C, lane);        // T^T dW
     frag_apply(aK, m0, n0, lane, [&](int m, int n, float& x) {
         atomicAdd(&dbs[m], x * Ks[m * LDK + n]);
         x *= bs[m];
     });
-    warp_mma<NT, SPLIT>(aK, Mat{dTs, LDC, 1}, Mat{Kws, LDK, 1}, m0, n0, C, lane);       // + dAb Kw
+    warp_mma<NT, SPLIT>(aK, Mat<LDC, 1>{dTs}, Mat<LDK, 1>{Kws}, m0, n0, C, lane);       // + dAb Kw
     frag_apply(aKw, m0, n0, lane, [&](int m, int n, float& x) { x = dkwa_g[m * DK + n]; });
-    warp_mma<NT, SPLIT>(aKw, Mat{dTs, 1, LDC}, Mat{Ks, LDK, 1}, m0, n0, C, lane);       // + dAb^T K
+    warp_mma<NT, SPLIT>(aKw, Mat<1, LDC>{dTs}, Mat<LDK, 1>{Ks}, m0, n0, C, lane);       // + dAb^T K
     #pragma unroll
     for (int jj = 0; jj < NT; ++jj)
         #pragma unroll
@@ -664,27 +845,57 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
         }
     __syncthreads();
     if (tid < C) dbp_g[tid] = dbs[tid];
+    }
 }
 
 // ---------------------------------------------------------------------------
-// Reverse of the d recurrence, token by token: one warp per unit, lane l owns
-// features l * DK / 32 ..; writes the final dk, dbeta, dr and dd0.
+// Reverse of the d recurrence, token by token, in slabs staged by warps 1-3;
+// lane l of warp 0 owns features l * DK / 32 ..; writes the final dk, dbeta, dr
+// and dd0.
 template <int DK, typename Tin>
-__global__ void __launch_bounds__(128)
+struct DchainSmem {
+    static constexpr size_t kBytes = 2 * (SLAB * DK * (sizeof(Tin) + 3 * sizeof(float)) + 3 * SLAB * sizeof(float));
+};
+
+template <int DK, typename Tin>
+__global__ void __launch_bounds__(SERIAL_THREADS, 1)
 bwd_dchain_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const Tin* __restrict__ r,
                   const float* __restrict__ d0, const float* __restrict__ dd_final,
                   Tin* __restrict__ dk, Tin* __restrict__ dbeta, Tin* __restrict__ dr, float* __restrict__ dd0,
                   const float* __restrict__ ws, Layout L, int B, int T, int H, int NC, float eta, int anchor)
 {
     constexpr int PER = DK / 32;
-    const int lane = threadIdx.x & 31;
-    const int unit = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (unit >= B * H) return;
-    const int b = unit / H, h = unit % H;
+    extern __shared__ __align__(16) unsigned char smraw[];
+    float* ds_ = reinterpret_cast<float*>(smraw);          // [2][SLAB][DK] d_t
+    float* dDs = ds_ + 2 * SLAB * DK;                      // [2][SLAB][DK] dL/dd_t through the write key
+    float* dks = dDs + 2 * SLAB * DK;                      // [2][SLAB][DK] chunk part of dk
+    float* bs = dks + 2 * SLAB * DK;                       // [2][SLAB] beta
+    float* rs = bs + 2 * SLAB;                             // [2][SLAB] r
+    float* dbs = rs + 2 * SLAB;                            // [2][SLAB] chunk part of dbeta
+    Tin* ks = reinterpret_cast<Tin*>(dbs + 2 * SLAB);      // [2][SLAB][DK] k
+    const int unit = blockIdx.x, b = unit / H, h = unit % H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nslab = (T + SLAB - 1) / SLAB;
     const float* d_all = ws + L.d_all / sizeof(float);
     const float* dd_g = ws + L.dd / sizeof(float);
     const float* dkp_g = ws + L.dkp / sizeof(float);
     const float* dbp_g = ws + L.dbp / sizeof(float);
+    // slab sl covers tokens [sl * SLAB, ...); SLAB divides the chunk length, so the
+    // slab's rows of the chunk-block arrays are contiguous
+    auto stage = [&](int sl, int buf) {
+        const int t0 = sl * SLAB, n = min(SLAB, T - t0);
+        const size_t tok0 = ((size_t)b * T + t0) * H + h;
+        const size_t crow0 = ((size_t)unit * NC + t0 / C) * C + t0 % C;
+        stage_rows(ks + buf * SLAB * DK, k + tok0 * DK, (size_t)H * DK, DK, n);
+        stage_rows(ds_ + buf * SLAB * DK, d_all + tok0 * DK, (size_t)H * DK, DK, n);
+        stage_rows(dDs + buf * SLAB * DK, dd_g + crow0 * DK, (size_t)DK, DK, n);
+        stage_rows(dks + buf * SLAB * DK, dkp_g + crow0 * DK, (size_t)DK, DK, n);
+        for (int t = threadIdx.x - 32; t < SLAB; t += SERIAL_THREADS - 32) {
+            bs[buf * SLAB + t] = t < n ? to_f32(beta[tok0 + (size_t)t * H]) : 0.f;
+            rs[buf * SLAB + t] = (t < n && r) ? to_f32(r[tok0 + (size_t)t * H]) : 1.f;
+            dbs[buf * SLAB + t] = t < n ? dbp_g[crow0 + t] : 0.f;
+        }
+    };
 
     float lam[PER], anc[PER], dda[PER];
 #pragma unroll
@@ -694,49 +905,63 @@ bwd_dchain_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const
         anc[i] = anchor ? (d0 ? d0[(size_t)unit * DK + f] : 1.f) : 0.f;
         dda[i] = 0.f;
     }
-    for (int t = T - 1; t >= 0; --t) {
-        const size_t tok = ((size_t)b * T + t) * H + h;
-        const size_t crow = ((size_t)unit * NC + t / C) * C + t % C;   // chunk-block row
-        float kk[PER], d[PER], dD[PER], dkp[PER], a[PER];
-        VecIO<PER, Tin>::load(k + tok * DK + lane * PER, kk);
-        VecIO<PER, float>::load(d_all + tok * DK + lane * PER, d);
-        VecIO<PER, float>::load(dd_g + crow * DK + lane * PER, dD);
-        VecIO<PER, float>::load(dkp_g + crow * DK + lane * PER, dkp);
-        const float bt = to_f32(beta[tok]), rt = r ? to_f32(r[tok]) : 1.f;
-        float n = 0.f, s = 0.f, dx = 0.f, drv = 0.f;
+    if (warp != 0 && nslab > 0) stage(nslab - 1, (nslab - 1) & 1);
+    __syncthreads();
+    for (int sl = nslab - 1; sl >= 0; --sl) {
+        const int buf = sl & 1;
+        if (warp != 0) {
+            if (sl > 0) stage(sl - 1, buf ^ 1);
+        } else {
+            const int t0 = sl * SLAB, n = min(SLAB, T - t0);
+            for (int t = n - 1; t >= 0; --t) {
+                const size_t tok = ((size_t)b * T + t0 + t) * H + h;
+                const int row = buf * SLAB + t;
+                float kk[PER], dc[PER], dD[PER], dkp[PER], a[PER];
+                VecIO<PER, Tin>::load(ks + row * DK + lane * PER, kk);
+                VecIO<PER, float>::load(ds_ + row * DK + lane * PER, dc);
+                VecIO<PER, float>::load(dDs + row * DK + lane * PER, dD);
+                VecIO<PER, float>::load(dks + row * DK + lane * PER, dkp);
+                const float bt = bs[row], rt = rs[row];
+                float n2 = 0.f, sd = 0.f, dx = 0.f, drv = 0.f;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            a[i] = kk[i] * kk[i];
-            n += a[i];
-            s += d[i] * a[i];
-            dx += a[i] * lam[i];
-            drv += (d[i] - anc[i]) * lam[i];
-        }
-        n = warp_sum(n);
-        s = warp_sum(s);
-        dx = warp_sum(dx);
-        drv = warp_sum(drv);
-        float db = dbp_g[crow], x = 0.f, ds = 0.f, dn = 0.f;
-        if (n > 0.f) {
-            x = eta * bt * (1.f - bt * s) / n;
-            db += dx * eta * (1.f - 2.f * bt * s) / n;
-            ds = -dx * eta * bt * bt / n;
-            dn = -dx * x / n;
-        }
-        float gk[PER];
+                for (int i = 0; i < PER; ++i) {
+                    a[i] = kk[i] * kk[i];
+                    n2 += a[i];
+                    sd += dc[i] * a[i];
+                    dx += a[i] * lam[i];
+                    drv += (dc[i] - anc[i]) * lam[i];
+                }
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            gk[i] = dkp[i] + 2.f * kk[i] * (x * lam[i] + ds * d[i] + dn);
-            if (anchor) dda[i] += (1.f - rt) * lam[i];
-            lam[i] = rt * lam[i] + dD[i] + ds * a[i];
+                for (int o = 16; o > 0; o >>= 1) {
+                    n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+                    sd += __shfl_xor_sync(0xffffffffu, sd, o);
+                    dx += __shfl_xor_sync(0xffffffffu, dx, o);
+                    drv += __shfl_xor_sync(0xffffffffu, drv, o);
+                }
+                float db = dbs[row], x = 0.f, dsv = 0.f, dnv = 0.f;
+                if (n2 > 0.f) {
+                    x = eta * bt * (1.f - bt * sd) / n2;
+                    db += dx * eta * (1.f - 2.f * bt * sd) / n2;
+                    dsv = -dx * eta * bt * bt / n2;
+                    dnv = -dx * x / n2;
+                }
+                float gk[PER];
+#pragma unroll
+                for (int i = 0; i < PER; ++i) {
+                    gk[i] = dkp[i] + 2.f * kk[i] * (x * lam[i] + dsv * dc[i] + dnv);
+                    if (anchor) dda[i] += (1.f - rt) * lam[i];
+                    lam[i] = rt * lam[i] + dD[i] + dsv * a[i];
+                }
+                VecIO<PER, Tin>::store(dk + tok * DK + lane * PER, gk);
+                if (lane == 0) {
+                    dbeta[tok] = from_f32<Tin>(db);
+                    if (r && dr) dr[tok] = from_f32<Tin>(drv);
+                }
+            }
         }
-        VecIO<PER, Tin>::store(dk + tok * DK + lane * PER, gk);
-        if (lane == 0) {
-            dbeta[tok] = from_f32<Tin>(db);
-            if (r && dr) dr[tok] = from_f32<Tin>(drv);
-        }
+        __syncthreads();
     }
-    if (dd0) {
+    if (warp == 0 && dd0) {
 #pragma unroll
         for (int i = 0; i < PER; ++i) dd0[(size_t)unit * DK + lane * PER + i] = lam[i] + dda[i];
     }

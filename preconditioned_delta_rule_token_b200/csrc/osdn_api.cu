@@ -296,6 +296,28 @@ int launch_step(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, 
     return OSDN_OK;
 }
 
+// Forward and reverse state passes of the backward with a dv tile of DVT rows.
+template <typename Tin, int DK, int DV, int DVT>
+int launch_state_passes(const osdn_params* p, const Tin* q, const Tin* dout, const float* S0, const float* dS_final,
+                        float* dS0, float* ws, const osdn::bwd::Layout& L, int NC, cudaStream_t st) {
+    namespace B = osdn::bwd;
+    const unsigned ntiles = (unsigned)(p->B * p->H * (DV / DVT));
+    const size_t s_sf = B::StateSmem<DK, DVT>::kFwdBytes, s_sb = B::StateSmem<DK, DVT>::kBwdBytes;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(B::bwd_state_f_kernel<DK, DV, DVT, Tin>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_sf)) != cudaSuccess)
+        return cuda_fail(e, "backward state attribute");
+    B::bwd_state_f_kernel<DK, DV, DVT, Tin><<<ntiles, B::NTHR, s_sf, st>>>(S0, ws, L, NC);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward state launch");
+    if ((e = cudaFuncSetAttribute(B::bwd_state_b_kernel<DK, DV, DVT, Tin>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_sb)) != cudaSuccess)
+        return cuda_fail(e, "backward adjoint state attribute");
+    B::bwd_state_b_kernel<DK, DV, DVT, Tin><<<ntiles, B::NTHR, s_sb, st>>>(dout, q, dS_final, dS0, ws, L, p->B,
+                                                                           p->T, p->H, NC);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward adjoint state launch");
+    return OSDN_OK;
+}
+
 // Backward: seven launches on one stream (see bwd.cuh for what each computes).
 template <typename Tin, int DK, int DV>
 int launch_bwd_t(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, const Tin* beta, const Tin* r,
@@ -305,46 +327,53 @@ int launch_bwd_t(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v,
     namespace B = osdn::bwd;
     const B::Layout L = B::make_layout(p->B, p->T, p->H, DK, DV);
     const int units = p->B * p->H, NC = (p->T + B::C - 1) / B::C, an = anchor_of(p);
-    const unsigned nchunks = (unsigned)((long long)units * NC), ntiles = (unsigned)(units * (DV / 32));
-    const unsigned warp_grid = (unsigned)((units + 3) / 4);
+    const long long nchunks = (long long)units * NC;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const unsigned pgrid = (unsigned)(nchunks < sms ? nchunks : sms);   // persistent per-chunk kernels
     cudaError_t e;
     auto attr = [](const void* kern, size_t smem) {
         return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     };
-    B::bwd_dtraj_kernel<DK, Tin><<<warp_grid, 128, 0, st>>>(k, beta, r, d0, ws + L.d_all / sizeof(float), p->B,
-                                                             p->T, p->H, p->eta, an);
+    const size_t s_dt = B::DtrajSmem<DK, Tin>::kBytes, s_dc = B::DchainSmem<DK, Tin>::kBytes;
+    if ((e = attr((const void*)B::bwd_dtraj_kernel<DK, Tin>, s_dt)) != cudaSuccess)
+        return cuda_fail(e, "backward d trajectory attribute");
+    B::bwd_dtraj_kernel<DK, Tin><<<(unsigned)units, B::SERIAL_THREADS, s_dt, st>>>(
+        k, beta, r, d0, ws + L.d_all / sizeof(float), p->B, p->T, p->H, p->eta, an);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward d trajectory launch");
 
     const size_t s_prep = B::PrepSmem<DK, DV>::kBytes;
     if ((e = attr((const void*)B::bwd_prep_kernel<DK, DV, Tin>, s_prep)) != cudaSuccess)
         return cuda_fail(e, "backward prep attribute");
-    B::bwd_prep_kernel<DK, DV, Tin><<<nchunks, B::NTHR, s_prep, st>>>(q, k, v, beta, ws, L, p->B, p->T, p->H, NC);
+    B::bwd_prep_kernel<DK, DV, Tin><<<pgrid, B::NTHR, s_prep, st>>>(q, k, v, beta, ws, L, p->B, p->T, p->H, NC);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward prep launch");
 
-    const size_t s_sf = B::StateSmem<DK, 32>::kFwdBytes, s_sb = B::StateSmem<DK, 32>::kBwdBytes;
-    if ((e = attr((const void*)B::bwd_state_f_kernel<DK, DV, 32, Tin>, s_sf)) != cudaSuccess)
-        return cuda_fail(e, "backward state attribute");
-    B::bwd_state_f_kernel<DK, DV, 32, Tin><<<ntiles, B::NTHR, s_sf, st>>>(S0, ws, L, NC);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward state launch");
-    if ((e = attr((const void*)B::bwd_state_b_kernel<DK, DV, 32, Tin>, s_sb)) != cudaSuccess)
-        return cuda_fail(e, "backward adjoint state attribute");
-    B::bwd_state_b_kernel<DK, DV, 32, Tin><<<ntiles, B::NTHR, s_sb, st>>>(dout, q, dS_final, dS0, ws, L, p->B,
-                                                                          p->T, p->H, NC);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward adjoint state launch");
+    // The two state passes are serial over the chunks; their dv tile is the widest of
+    // DV, DV / 2, ... (down to 32 rows) whose (unit, tile) CTAs still fit one wave, or
+    // the full DV when even that is more than one wave.
+    int dvt = DV;
+    while (dvt > 32 && (long long)units * (DV / dvt) * 2 <= sms) dvt /= 2;
+    int rcs;
+    if (dvt == 32) rcs = launch_state_passes<Tin, DK, DV, 32>(p, q, dout, S0, dS_final, dS0, ws, L, NC, st);
+    else if (dvt == 64) rcs = launch_state_passes<Tin, DK, DV, 64>(p, q, dout, S0, dS_final, dS0, ws, L, NC, st);
+    else rcs = launch_state_passes<Tin, DK, DV, DV>(p, q, dout, S0, dS_final, dS0, ws, L, NC, st);
+    if (rcs) return rcs;
 
     const size_t s_ga = B::GradSmem<DK>::kABytes, s_gb = B::GradSmem<DK>::kBBytes;
     if ((e = attr((const void*)B::bwd_grads_a_kernel<DK, DV, Tin>, s_ga)) != cudaSuccess)
         return cuda_fail(e, "backward gradient attribute");
-    B::bwd_grads_a_kernel<DK, DV, Tin><<<nchunks, B::NTHR, s_ga, st>>>(q, v, beta, dout, dq, dv, ws, L, p->B, p->T,
+    B::bwd_grads_a_kernel<DK, DV, Tin><<<pgrid, B::NTHR, s_ga, st>>>(q, v, beta, dout, dq, dv, ws, L, p->B, p->T,
                                                                        p->H, NC);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward gradient launch");
     if ((e = attr((const void*)B::bwd_grads_b_kernel<DK, Tin>, s_gb)) != cudaSuccess)
         return cuda_fail(e, "backward key gradient attribute");
-    B::bwd_grads_b_kernel<DK, Tin><<<nchunks, B::NTHR, s_gb, st>>>(k, beta, ws, L, p->B, p->T, p->H, NC);
+    B::bwd_grads_b_kernel<DK, Tin><<<pgrid, B::NTHR, s_gb, st>>>(k, beta, ws, L, p->B, p->T, p->H, NC);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward key gradient launch");
 
-    B::bwd_dchain_kernel<DK, Tin><<<warp_grid, 128, 0, st>>>(k, beta, r, d0, dd_final, dk, dbeta, dr, dd0, ws, L,
-                                                              p->B, p->T, p->H, NC, p->eta, an);
+    if ((e = attr((const void*)B::bwd_dchain_kernel<DK, Tin>, s_dc)) != cudaSuccess)
+        return cuda_fail(e, "backward d chain attribute");
+    B::bwd_dchain_kernel<DK, Tin><<<(unsigned)units, B::SERIAL_THREADS, s_dc, st>>>(
+        k, beta, r, d0, dd_final, dk, dbeta, dr, dd0, ws, L, p->B, p->T, p->H, NC, p->eta, an);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward d chain launch");
     return OSDN_OK;
 }

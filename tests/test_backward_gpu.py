@@ -124,3 +124,12 @@ def test_backward_full_size_sampled_units():
     w = W.LAYER_1P3B
     for got, ref in _run(w, units=[(0, 0), (w.B - 1, w.H - 1)]):
         _compare(got, ref, BF16_TOL, True)
+
+
+@pytest.mark.parametrize("B,H,dtype,tol", [(4, 10, W.BF16, BF16_TOL), (8, 10, W.FP32, FP32_TOL)])
+def test_backward_state_tile_widths(B, H, dtype, tol):
+    # 40 and 80 (b, h) units: on 148 SMs the state passes take dv tiles of 64 and 128 rows
+    # (the small cases above take 32), so every tile width runs against the oracle
+    w = _small("bwd tiles", B, H, 70, 128, 128, dtype, seed=13)
+    got, ref = _run(w)
+    _compare(got, ref, tol, True)
