@@ -53,6 +53,7 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the osdn_step (decode) measurement")
     ap.add_argument("--no-gated", action="store_true", help="skip the gated-variant chunk measurement")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward (osdn_bwd) measurement")
     return ap.parse_args()
 
 
@@ -342,6 +343,65 @@ def run_gated(w, g, p, ws, out, Sf, stream, hbm, steps=20, warmup=3):
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "peak_gbs": hbm, "frac": gbs / hbm, "bound": "hbm"}
 
 
+def backward_bytes(w):
+    """Algorithmic HBM bytes of one osdn_bwd call: reads q, k, v, dout, beta (and r),
+    writes dq, dk, dv, dbeta (and dr), all in the input dtype; per (b, h) reads dS_final,
+    dd_final and writes dS0, dd0 in fp32 (S0 and d0 are the defaults, not read)."""
+    e, apf = elem(w), 1 if w.apf else 0
+    per_tok = e * ((2 * w.dk + 2 * w.dv + 1 + apf) + (2 * w.dk + w.dv + 1 + apf))
+    per_unit = 4 * 2 * (w.dv * w.dk + w.dk)
+    return w.B * w.T * w.H * per_tok + w.B * w.H * per_unit
+
+
+def backward_flops(w):
+    """Algorithmic FLOPs of one osdn_bwd call: the chunk form's dense products (the
+    forward recomputed and the adjoint), triangular ones counted at half. Per chunk of C
+    tokens, multiply-adds = 8 C dk dv + C^2 (5.5 dk + 3 dv) + (7/6) C^3."""
+    C, nch = w.chunk, w.B * w.H * ((w.T + w.chunk - 1) // w.chunk)
+    mac = 8 * C * w.dk * w.dv + C * C * (5.5 * w.dk + 3 * w.dv) + (7.0 / 6.0) * C ** 3
+    return 2.0 * mac * nch
+
+
+def run_backward(w, g, stream, hbm, tf_peak, steps=5, warmup=2):
+    """osdn_bwd on the same layer with inputs and upstream gradients resident in HBM and
+    the workspace preallocated; CUDA events on the launching stream."""
+    import preconditioned_delta_rule_token_b200 as pk
+    dev = g["k"].device
+    cot = {k_: (None if v_ is None else v_.to(dev)) for k_, v_ in W.make_backward_cotangents(w).items()}
+    p = pk.make_params(w.B, w.T, w.H, w.dk, w.dv, g["k"].dtype, w.eta, w.chunk)
+    ws = torch.empty(pk.osdn_bwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    grads = {n: torch.empty_like(g[m]) for n, m in (("dq", "q"), ("dk", "k"), ("dv", "v"), ("dbeta", "beta"))}
+    grads["dr"] = None if g["r"] is None else torch.empty_like(g["r"])
+    dd0 = torch.empty((w.B, w.H, w.dk), dtype=torch.float32, device=dev)
+    dS0 = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+
+    def call():
+        pk.osdn_bwd(p, g["q"], g["k"], g["v"], g["beta"], g["r"], None, None, cot["dout"], cot["dS_final"],
+                    cot["dd_final"], grads["dq"], grads["dk"], grads["dv"], grads["dbeta"], grads["dr"], dd0, dS0,
+                    ws, stream)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert pk.osdn_sync_status(stream) == 0
+    ms = e0.elapsed_time(e1) / steps
+    nbytes, F = backward_bytes(w), backward_flops(w)
+    t_hbm, t_tc = nbytes / (hbm * 1e9), F / (tf_peak * 1e12)
+    t_roof = max(t_hbm, t_tc)
+    del ws
+    return {"call": "osdn_bwd (7 kernel launches)", "ms": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),
+            "algorithmic_bytes": nbytes, "flops": F, "t_roofline_us": t_roof * 1e6,
+            "bound": "tensor" if t_tc >= t_hbm else "hbm", "frac": t_roof / (ms / 1e3),
+            "tflops": F / (ms / 1e3) / 1e12, "gbs": nbytes / (ms / 1e3) / 1e9,
+            "dtype": "bf16 in and out; fp32 state and intermediates, tf32 tensor-core products"}
+
+
 def config_of(w, world):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
             "apf": w.apf, "eta": w.eta, "structure": w.structure, "global_batch": w.B * world, "seq_len": w.T,
@@ -470,6 +530,8 @@ def run_ours(args, world, rank, local):
     if world == 1 and not args.no_gated and w.dtype == W.BF16 and w.dk == 128 and w.dv == 128:
         step()                                                      # the workspace holds this layer's scaled keys
         line["gated"] = run_gated(w, g, p, ws, out, Sf, stream, hbm)
+    if world == 1 and not args.no_backward:
+        line["backward"] = run_backward(w, g, stream, hbm, tf_peak)
     if world == 1 and not args.no_cpu_baseline:
         v_, desc, cores = oracle_sample(w, seconds=12.0)
         line["cpu_baseline"] = {"value": v_, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}

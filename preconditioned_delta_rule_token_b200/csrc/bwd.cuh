@@ -290,26 +290,52 @@ __device__ __forceinline__ void async_block(float* dst, int ldd, const float* sr
 constexpr int SLAB = 32;
 constexpr int SERIAL_THREADS = 128;
 
-// Warps 1-3 copy rows [0, n) of a slab, row t at src + t * stride (16-byte aligned,
-// width elements), into dst[t * width ..]; rows n .. SLAB - 1 become zero.
+// Warp w of warps 1-3 takes rows w - 1, w + 2, ... of a slab; per row, lane l copies
+// the l-th 16-byte piece of each staged row and the warp reduces what the chain needs.
+constexpr int HELPERS = SERIAL_THREADS / 32 - 1;
+static_assert(SLAB <= SERIAL_THREADS - 32, "one helper thread per token of a slab");
+
+// Asynchronous copy of the lane-th 16-byte piece of a row (zero-filled when !ok); the
+// helpers issue every piece of a slab before waiting once.
 template <typename T>
-__device__ __forceinline__ void stage_rows(T* dst, const T* src, size_t stride, int width, int n) {
+__device__ __forceinline__ void stage_piece(T* dst, const T* src, int lane, int width, bool ok) {
     constexpr int V = 16 / sizeof(T);
-    const int vpr = width / V;
-    for (int idx = threadIdx.x - 32; idx < SLAB * vpr; idx += SERIAL_THREADS - 32) {
-        const int t = idx / vpr, c = (idx % vpr) * V;
-        uint4 u = make_uint4(0u, 0u, 0u, 0u);
-        if (t < n) u = *reinterpret_cast<const uint4*>(src + (size_t)t * stride + c);
-        *reinterpret_cast<uint4*>(dst + (size_t)t * width + c) = u;
+    if (lane * V < width) {
+        const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + lane * V);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(ok ? src + lane * V : src),
+                     "r"(ok ? 16 : 0)
+                     : "memory");
     }
+}
+
+// Barrier over the three helper warps only (named barrier 1).
+__device__ __forceinline__ void helpers_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(SERIAL_THREADS - 32) : "memory");
+}
+
+// sum over the row's features of f(k_i, d_i) for the piece this lane staged
+template <int DK, typename Tin>
+__device__ __forceinline__ float k2_piece(const Tin* krow, int lane) {
+    constexpr int V = 16 / sizeof(Tin);
+    float acc = 0.f;
+    if (lane * V < DK) {
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const float kv = to_f32(krow[lane * V + i]);
+            acc = fmaf(kv, kv, acc);
+        }
+    }
+    return acc;
 }
 
 template <int DK, typename Tin>
 struct DtrajSmem {
-    static constexpr size_t kBytes = 2 * (SLAB * DK * sizeof(Tin) + 2 * SLAB * sizeof(float));
+    static constexpr size_t kBytes = 2 * (SLAB * DK * sizeof(Tin) + 3 * SLAB * sizeof(float));
 };
 
-// d_t (before the token's own update) for every token.
+// d_t (before the token's own update) for every token. Per token the helpers stage
+// k and precompute c0 = eta beta / ||k||^2 and c1 = eta beta^2 / ||k||^2 (0 when k = 0),
+// so that x = c0 - c1 <d, k^2> and the chain carries one reduction per token.
 template <int DK, typename Tin>
 __global__ void __launch_bounds__(SERIAL_THREADS, 1)
 bwd_dtraj_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const Tin* __restrict__ r,
@@ -318,18 +344,35 @@ bwd_dtraj_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const 
     constexpr int PER = DK / 32;
     extern __shared__ __align__(16) unsigned char smraw[];
     Tin* ks = reinterpret_cast<Tin*>(smraw);                                        // [2][SLAB][DK]
-    float* bs = reinterpret_cast<float*>(smraw + 2 * SLAB * DK * sizeof(Tin));      // [2][SLAB]
-    float* rs = bs + 2 * SLAB;                                                      // [2][SLAB]
+    float* c0s = reinterpret_cast<float*>(smraw + 2 * SLAB * DK * sizeof(Tin));     // [2][SLAB]
+    float* c1s = c0s + 2 * SLAB;                                                    // [2][SLAB]
+    float* rs = c1s + 2 * SLAB;                                                     // [2][SLAB]
     const int unit = blockIdx.x, b = unit / H, h = unit % H;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nslab = (T + SLAB - 1) / SLAB;
-    auto stage = [&](int sl, int buf) {
+    auto stage = [&](int sl, int buf) {   // warps 1-3
         const int t0 = sl * SLAB, n = min(SLAB, T - t0);
-        const size_t tok0 = ((size_t)b * T + t0) * H + h;
-        stage_rows(ks + buf * SLAB * DK, k + tok0 * DK, (size_t)H * DK, DK, n);
-        for (int t = threadIdx.x - 32; t < SLAB; t += SERIAL_THREADS - 32) {
-            bs[buf * SLAB + t] = t < n ? to_f32(beta[tok0 + (size_t)t * H]) : 0.f;
-            rs[buf * SLAB + t] = (t < n && r) ? to_f32(r[tok0 + (size_t)t * H]) : 1.f;
+        for (int t = warp - 1; t < SLAB; t += HELPERS) {
+            const size_t tok = ((size_t)b * T + t0 + t) * H + h;
+            stage_piece(ks + (buf * SLAB + t) * DK, k + tok * DK, lane, DK, t < n);
+        }
+        const int ht = threadIdx.x - 32;                  // one helper thread per token: beta, r
+        if (ht < SLAB) {
+            const bool ok = ht < n;
+            const size_t tok = ((size_t)b * T + t0 + ht) * H + h;
+            c0s[buf * SLAB + ht] = ok ? to_f32(beta[tok]) : 0.f;      // beta for now
+            rs[buf * SLAB + ht] = (ok && r) ? to_f32(r[tok]) : 1.f;
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        helpers_sync();
+        for (int t = warp - 1; t < SLAB; t += HELPERS) {
+            const float n2 = warp_sum(k2_piece<DK>(ks + (buf * SLAB + t) * DK, lane));
+            if (lane == 0) {
+                const float bt = c0s[buf * SLAB + t];
+                const float inv = n2 > 0.f ? eta / n2 : 0.f;
+                c0s[buf * SLAB + t] = bt * inv;
+                c1s[buf * SLAB + t] = bt * bt * inv;
+            }
         }
     };
     float d[PER], da[PER];
@@ -345,25 +388,21 @@ bwd_dtraj_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const 
             if (sl + 1 < nslab) stage(sl + 1, buf ^ 1);
         } else {
             const int t0 = sl * SLAB, n = min(SLAB, T - t0);
+#pragma unroll 2
             for (int t = 0; t < n; ++t) {
                 const size_t tok = ((size_t)b * T + t0 + t) * H + h;
                 float kk[PER], a[PER];
                 VecIO<PER, Tin>::load(ks + (buf * SLAB + t) * DK + lane * PER, kk);
-                const float bt = bs[buf * SLAB + t], rt = rs[buf * SLAB + t];
+                const float c0 = c0s[buf * SLAB + t], c1 = c1s[buf * SLAB + t], rt = rs[buf * SLAB + t];
                 VecIO<PER, float>::store(d_all + tok * DK + lane * PER, d);
-                float n2 = 0.f, sd = 0.f;
+                float sd = 0.f;
 #pragma unroll
                 for (int i = 0; i < PER; ++i) {
                     a[i] = kk[i] * kk[i];
-                    n2 += a[i];
-                    sd += d[i] * a[i];
+                    sd = fmaf(d[i], a[i], sd);
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    n2 += __shfl_xor_sync(0xffffffffu, n2, o);
-                    sd += __shfl_xor_sync(0xffffffffu, sd, o);
-                }
-                const float x = (n2 > 0.f) ? eta * bt * (1.f - bt * sd) / n2 : 0.f;
+                sd = warp_sum(sd);
+                const float x = fmaf(-c1, sd, c0);
 #pragma unroll
                 for (int i = 0; i < PER; ++i) d[i] = rt * d[i] + (1.f - rt) * da[i] + x * a[i];
             }
@@ -854,9 +893,14 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
 // and dd0.
 template <int DK, typename Tin>
 struct DchainSmem {
-    static constexpr size_t kBytes = 2 * (SLAB * DK * (sizeof(Tin) + 3 * sizeof(float)) + 3 * SLAB * sizeof(float));
+    static constexpr size_t kBytes = 2 * (SLAB * DK * (sizeof(Tin) + 3 * sizeof(float)) + 6 * SLAB * sizeof(float));
 };
 
+// Per token the helpers stage k, d_t, dD_t and the chunk part of dk and precompute the
+// scalars of the step that do not depend on Ld: x, eta (1 - 2 beta s) / n,
+// -eta beta^2 / n and -x / n (all 0 when k = 0), with s = <d_t, k^2> and n = ||k||^2.
+// The chain then carries one reduction, <k^2, Ld>, per token (the <d - d0, Ld> of dr
+// is reduced alongside it but feeds nothing back).
 template <int DK, typename Tin>
 __global__ void __launch_bounds__(SERIAL_THREADS, 1)
 bwd_dchain_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const Tin* __restrict__ r,
@@ -869,10 +913,8 @@ bwd_dchain_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const
     float* ds_ = reinterpret_cast<float*>(smraw);          // [2][SLAB][DK] d_t
     float* dDs = ds_ + 2 * SLAB * DK;                      // [2][SLAB][DK] dL/dd_t through the write key
     float* dks = dDs + 2 * SLAB * DK;                      // [2][SLAB][DK] chunk part of dk
-    float* bs = dks + 2 * SLAB * DK;                       // [2][SLAB] beta
-    float* rs = bs + 2 * SLAB;                             // [2][SLAB] r
-    float* dbs = rs + 2 * SLAB;                            // [2][SLAB] chunk part of dbeta
-    Tin* ks = reinterpret_cast<Tin*>(dbs + 2 * SLAB);      // [2][SLAB][DK] k
+    float* sc = dks + 2 * SLAB * DK;                       // [2][SLAB][6] x, c1, c2, c3, r, chunk dbeta
+    Tin* ks = reinterpret_cast<Tin*>(sc + 2 * SLAB * 6);   // [2][SLAB][DK] k
     const int unit = blockIdx.x, b = unit / H, h = unit % H;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nslab = (T + SLAB - 1) / SLAB;
@@ -880,20 +922,57 @@ bwd_dchain_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const
     const float* dd_g = ws + L.dd / sizeof(float);
     const float* dkp_g = ws + L.dkp / sizeof(float);
     const float* dbp_g = ws + L.dbp / sizeof(float);
-    // slab sl covers tokens [sl * SLAB, ...); SLAB divides the chunk length, so the
-    // slab's rows of the chunk-block arrays are contiguous
-    auto stage = [&](int sl, int buf) {
+    // slab sl covers tokens [sl * SLAB, ...); SLAB divides the chunk length, so a token's
+    // rows of the chunk-block arrays are at crow0 + t
+    auto stage = [&](int sl, int buf) {   // warps 1-3
         const int t0 = sl * SLAB, n = min(SLAB, T - t0);
-        const size_t tok0 = ((size_t)b * T + t0) * H + h;
         const size_t crow0 = ((size_t)unit * NC + t0 / C) * C + t0 % C;
-        stage_rows(ks + buf * SLAB * DK, k + tok0 * DK, (size_t)H * DK, DK, n);
-        stage_rows(ds_ + buf * SLAB * DK, d_all + tok0 * DK, (size_t)H * DK, DK, n);
-        stage_rows(dDs + buf * SLAB * DK, dd_g + crow0 * DK, (size_t)DK, DK, n);
-        stage_rows(dks + buf * SLAB * DK, dkp_g + crow0 * DK, (size_t)DK, DK, n);
-        for (int t = threadIdx.x - 32; t < SLAB; t += SERIAL_THREADS - 32) {
-            bs[buf * SLAB + t] = t < n ? to_f32(beta[tok0 + (size_t)t * H]) : 0.f;
-            rs[buf * SLAB + t] = (t < n && r) ? to_f32(r[tok0 + (size_t)t * H]) : 1.f;
-            dbs[buf * SLAB + t] = t < n ? dbp_g[crow0 + t] : 0.f;
+        for (int t = warp - 1; t < SLAB; t += HELPERS) {
+            const bool ok = t < n;
+            const size_t tok = ((size_t)b * T + t0 + t) * H + h;
+            const int row = buf * SLAB + t;
+            stage_piece(ks + row * DK, k + tok * DK, lane, DK, ok);
+            stage_piece(ds_ + row * DK, d_all + tok * DK, lane, DK, ok);
+            stage_piece(dDs + row * DK, dd_g + (crow0 + t) * DK, lane, DK, ok);
+            stage_piece(dks + row * DK, dkp_g + (crow0 + t) * DK, lane, DK, ok);
+        }
+        const int ht = threadIdx.x - 32;                  // one helper thread per token: beta, r, dbeta
+        if (ht < SLAB) {
+            const bool ok = ht < n;
+            const size_t tok = ((size_t)b * T + t0 + ht) * H + h;
+            float* q6 = sc + (buf * SLAB + ht) * 6;
+            q6[0] = ok ? to_f32(beta[tok]) : 0.f;          // beta for now
+            q6[4] = (ok && r) ? to_f32(r[tok]) : 1.f;
+            q6[5] = ok ? dbp_g[crow0 + ht] : 0.f;
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        helpers_sync();
+        for (int t = warp - 1; t < SLAB; t += HELPERS) {
+            const int row = buf * SLAB + t;
+            float n2 = 0.f, sd = 0.f;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const float kv = to_f32(ks[row * DK + lane * PER + i]);
+                n2 = fmaf(kv, kv, n2);
+                sd = fmaf(ds_[row * DK + lane * PER + i], kv * kv, sd);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+                sd += __shfl_xor_sync(0xffffffffu, sd, o);
+            }
+            if (lane == 0) {
+                float* q6 = sc + row * 6;
+                const float bt = q6[0];
+                float x = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+                if (n2 > 0.f) {
+                    x = eta * bt * (1.f - bt * sd) / n2;
+                    c1 = eta * (1.f - 2.f * bt * sd) / n2;
+                    c2 = -eta * bt * bt / n2;
+                    c3 = -x / n2;
+                }
+                q6[0] = x; q6[1] = c1; q6[2] = c2; q6[3] = c3;
+            }
         }
     };
 
@@ -913,6 +992,7 @@ bwd_dchain_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const
             if (sl > 0) stage(sl - 1, buf ^ 1);
         } else {
             const int t0 = sl * SLAB, n = min(SLAB, T - t0);
+#pragma unroll 2
             for (int t = n - 1; t >= 0; --t) {
                 const size_t tok = ((size_t)b * T + t0 + t) * H + h;
                 const int row = buf * SLAB + t;
@@ -921,30 +1001,21 @@ bwd_dchain_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const
                 VecIO<PER, float>::load(ds_ + row * DK + lane * PER, dc);
                 VecIO<PER, float>::load(dDs + row * DK + lane * PER, dD);
                 VecIO<PER, float>::load(dks + row * DK + lane * PER, dkp);
-                const float bt = bs[row], rt = rs[row];
-                float n2 = 0.f, sd = 0.f, dx = 0.f, drv = 0.f;
+                const float* q6 = sc + row * 6;
+                const float x = q6[0], c1 = q6[1], c2 = q6[2], c3 = q6[3], rt = q6[4], dbc = q6[5];
+                float dx = 0.f, drv = 0.f;
 #pragma unroll
                 for (int i = 0; i < PER; ++i) {
                     a[i] = kk[i] * kk[i];
-                    n2 += a[i];
-                    sd += dc[i] * a[i];
-                    dx += a[i] * lam[i];
-                    drv += (dc[i] - anc[i]) * lam[i];
+                    dx = fmaf(a[i], lam[i], dx);
+                    drv = fmaf(dc[i] - anc[i], lam[i], drv);
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
-                    n2 += __shfl_xor_sync(0xffffffffu, n2, o);
-                    sd += __shfl_xor_sync(0xffffffffu, sd, o);
                     dx += __shfl_xor_sync(0xffffffffu, dx, o);
                     drv += __shfl_xor_sync(0xffffffffu, drv, o);
                 }
-                float db = dbs[row], x = 0.f, dsv = 0.f, dnv = 0.f;
-                if (n2 > 0.f) {
-                    x = eta * bt * (1.f - bt * sd) / n2;
-                    db += dx * eta * (1.f - 2.f * bt * sd) / n2;
-                    dsv = -dx * eta * bt * bt / n2;
-                    dnv = -dx * x / n2;
-                }
+                const float dsv = c2 * dx, dnv = c3 * dx;
                 float gk[PER];
 #pragma unroll
                 for (int i = 0; i < PER; ++i) {
@@ -954,7 +1025,7 @@ bwd_dchain_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const
                 }
                 VecIO<PER, Tin>::store(dk + tok * DK + lane * PER, gk);
                 if (lane == 0) {
-                    dbeta[tok] = from_f32<Tin>(db);
+                    dbeta[tok] = from_f32<Tin>(fmaf(c1, dx, dbc));
                     if (r && dr) dr[tok] = from_f32<Tin>(drv);
                 }
             }
