@@ -43,6 +43,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "tril_inv.cuh"
 
 namespace osdn {
 namespace bwd {
@@ -480,7 +481,12 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{Kb}, Mat<1, LDK>{Kw},
                     [&](int m, int n, float x) { As[m * LDC + n] = n < m ? x : 0.f; });
     __syncthreads();
-    {   // (I + A) T = I by forward substitution: column j on 8 threads that split the inner sum
+    // T = (I + A)^{-1}. fp32 mode: exact forward substitution into Ts, column j on 8
+    // threads that split the inner sum. bf16 inputs: the blocked inverse in place over A
+    // on warps 0-3 (16 x 16 diagonal blocks by substitution, the rest on tf32 mma.sync),
+    // the same routine as the forward chunk kernel's.
+    const float* Tm = SPLIT ? Ts : As;
+    if (SPLIT) {
         const int j = tid >> 3, part = tid & 7;
         for (int i = 0; i < C; ++i) {
             float sum = 0.f;
@@ -492,12 +498,15 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
             if (part == 0) Ts[i * LDC + j] = (i < j) ? 0.f : (i == j ? 1.f : -sum);
             __syncwarp();
         }
+    } else if (tid < 128) {
+        static_assert(LDC == tri::LD, "the blocked inverse takes the 68-float row stride");
+        tri::tril_inv64_inplace(As, tid >> 5, tid & 31, [] { asm volatile("bar.sync 1, 128;" ::: "memory"); });
     }
     __syncthreads();
-    for (int idx = tid; idx < C * C; idx += NTHR) t_g[idx] = Ts[(idx / C) * LDC + idx % C];
-    cta_gemm<SPLIT>(C, DK, C, Mat<LDC, 1>{Ts}, Mat<LDK, 1>{Kb},
+    for (int idx = tid; idx < C * C; idx += NTHR) t_g[idx] = Tm[(idx / C) * LDC + idx % C];
+    cta_gemm<SPLIT>(C, DK, C, Mat<LDC, 1>{Tm}, Mat<LDK, 1>{Kb},
                     [&](int m, int n, float x) { w_g[m * DK + n] = x; });
-    cta_gemm<SPLIT>(C, DV, C, Mat<LDC, 1>{Ts}, Mat<LDX, 1>{X},
+    cta_gemm<SPLIT>(C, DV, C, Mat<LDC, 1>{Tm}, Mat<LDX, 1>{X},
                     [&](int m, int n, float x) { u_g[m * DV + n] = x; });
     __syncthreads();
     load_tile<C, DK>(X, LDX, q + tok0 * DK, tstride * DK, Tc);
