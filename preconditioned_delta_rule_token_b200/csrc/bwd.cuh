@@ -124,13 +124,30 @@ __device__ __forceinline__ void frag_zero(float (&acc)[NT][4]) {
         for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 }
 
+// Calls f(m, n, value) for every element a thread holds, or f(m, n, v_n, v_{n+1}) once per
+// pair of adjacent columns (n even) when f takes two values, so that a store can be 8 bytes.
 template <int NT, typename F>
 __device__ __forceinline__ void frag_each(float (&acc)[NT][4], int m0, int n0, int lane, F f) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) f(m0 + g + 8 * (e >> 1), n0 + 8 * j + 2 * t + (e & 1), acc[j][e]);
+        for (int hh = 0; hh < 2; ++hh) {
+            const int m = m0 + g + 8 * hh, n = n0 + 8 * j + 2 * t;
+            if constexpr (std::is_invocable_v<F, int, int, float, float>) {
+                f(m, n, acc[j][2 * hh], acc[j][2 * hh + 1]);
+            } else {
+                f(m, n, acc[j][2 * hh]);
+                f(m, n + 1, acc[j][2 * hh + 1]);
+            }
+        }
+}
+
+__device__ __forceinline__ void store2(float* p, float a, float b) {
+    *reinterpret_cast<float2*>(p) = make_float2(a, b);
+}
+__device__ __forceinline__ void store2(__nv_bfloat16* p, float a, float b) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
 
 // The CTA computes the M x N product sum_k A(m, k) B(k, n) (plus, for the two-term
@@ -150,11 +167,13 @@ __device__ __forceinline__ void cta_gemm_nt(int M, int N, int K1, MA1 A1, MB1 B1
     }
 }
 
-// 16 x 32 tiles when there are enough of them for every warp, else 16 x 16.
+// The widest of 16 x 32, 16 x 16 and 16 x 8 tiles that still gives every warp one.
 template <bool SPLIT, class MA1, class MB1, class MA2, class MB2, typename Epi>
 __device__ __forceinline__ void cta_gemm2(int M, int N, int K1, MA1 A1, MB1 B1, int K2, MA2 A2, MB2 B2, Epi epi) {
-    if ((M / 16) * (N / 32) >= (int)(blockDim.x >> 5)) cta_gemm_nt<4, SPLIT>(M, N, K1, A1, B1, K2, A2, B2, epi);
-    else cta_gemm_nt<2, SPLIT>(M, N, K1, A1, B1, K2, A2, B2, epi);
+    const int nw = (int)(blockDim.x >> 5);
+    if ((M / 16) * (N / 32) >= nw) cta_gemm_nt<4, SPLIT>(M, N, K1, A1, B1, K2, A2, B2, epi);
+    else if ((M / 16) * (N / 16) >= nw) cta_gemm_nt<2, SPLIT>(M, N, K1, A1, B1, K2, A2, B2, epi);
+    else cta_gemm_nt<1, SPLIT>(M, N, K1, A1, B1, K2, A2, B2, epi);
 }
 
 template <bool SPLIT, class MA, class MB, typename Epi>
@@ -505,14 +524,16 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     __syncthreads();
     for (int idx = tid; idx < C * C; idx += NTHR) t_g[idx] = Tm[(idx / C) * LDC + idx % C];
     cta_gemm<SPLIT>(C, DK, C, Mat<LDC, 1>{Tm}, Mat<LDK, 1>{Kb},
-                    [&](int m, int n, float x) { w_g[m * DK + n] = x; });
+                    [&](int m, int n, float x0, float x1) { store2(w_g + m * DK + n, x0, x1); });
     cta_gemm<SPLIT>(C, DV, C, Mat<LDC, 1>{Tm}, Mat<LDX, 1>{X},
-                    [&](int m, int n, float x) { u_g[m * DV + n] = x; });
+                    [&](int m, int n, float x0, float x1) { store2(u_g + m * DV + n, x0, x1); });
     __syncthreads();
     load_tile<C, DK>(X, LDX, q + tok0 * DK, tstride * DK, Tc);
     __syncthreads();
     cta_gemm<SPLIT>(C, C, DK, Mat<LDX, 1>{X}, Mat<1, LDK>{Kw},
-                    [&](int m, int n, float x) { p_g[m * C + n] = n <= m ? x : 0.f; });
+                    [&](int m, int n, float x0, float x1) {
+                        store2(p_g + m * C + n, n <= m ? x0 : 0.f, n + 1 <= m ? x1 : 0.f);
+                    });
     }
 }
 
@@ -566,10 +587,11 @@ bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout 
         async_tile<C, DVT>(Vs, LDT, u_g + v0, (size_t)DV);
         cp_async_wait_all();
         __syncthreads();
-        cta_gemm<SPLIT>(C, DVT, DK, Mat<LDK, 1>{Ws}, Mat<1, LDK>{Ss}, [&](int m, int n, float x) {
-            const float vn = Vs[m * LDT + n] - x;
-            Vs[m * LDT + n] = vn;
-            vn_g[m * DV + v0 + n] = vn;
+        cta_gemm<SPLIT>(C, DVT, DK, Mat<LDK, 1>{Ws}, Mat<1, LDK>{Ss}, [&](int m, int n, float x0, float x1) {
+            const float vn0 = Vs[m * LDT + n] - x0, vn1 = Vs[m * LDT + n + 1] - x1;
+            Vs[m * LDT + n] = vn0;
+            Vs[m * LDT + n + 1] = vn1;
+            store2(vn_g + m * DV + v0 + n, vn0, vn1);
         });
         __syncthreads();
         cta_gemm<SPLIT>(DVT, DK, C, Mat<1, LDT>{Vs}, Mat<LDK, 1>{Kws},
@@ -630,9 +652,10 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
         __syncthreads();
         // dVn = P^T dO + Kw dS'^T
         cta_gemm2<SPLIT>(C, DVT, C, Mat<1, LDC>{Ps}, Mat<LDT, 1>{dOs}, DK, Mat<LDK, 1>{B1}, Mat<1, LDK>{dSs},
-                         [&](int m, int n, float x) {
-                             dVs[m * LDT + n] = -x;
-                             dvn_g[m * DV + v0 + n] = x;
+                         [&](int m, int n, float x0, float x1) {
+                             dVs[m * LDT + n] = -x0;
+                             dVs[m * LDT + n + 1] = -x1;
+                             store2(dvn_g + m * DV + v0 + n, x0, x1);
                          });
         __syncthreads();
         async_block<C, DK>(B1, LDK, w_g);
@@ -767,9 +790,9 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
         cta_gemm<SPLIT>(C, C, J, Mat<LDJ, 1>{dVns}, Mat<1, LDJ>{Vs},
                         [&](int m, int n, float x) { dTs[m * LDC + n] += bs[n] * x; });
         // dV = diag(beta) T^T dVn;  dbeta += rowdot(T^T dVn, V)
-        cta_gemm<SPLIT>(C, J, C, Mat<1, LDC>{Ts}, Mat<LDJ, 1>{dVns}, [&](int m, int n, float x) {
-            if (m < Tc) dv[tok(m) * DV + v0 + n] = from_f32<Tin>(bs[m] * x);
-            atomicAdd(&dbs[m], x * Vs[m * LDJ + n]);
+        cta_gemm<SPLIT>(C, J, C, Mat<1, LDC>{Ts}, Mat<LDJ, 1>{dVns}, [&](int m, int n, float x0, float x1) {
+            if (m < Tc) store2(dv + tok(m) * DV + v0 + n, bs[m] * x0, bs[m] * x1);
+            atomicAdd(&dbs[m], x0 * Vs[m * LDJ + n] + x1 * Vs[m * LDJ + n + 1]);
         });
         warp_mma<NT, SPLIT>(aQ, Mat<LDJ, 1>{dOs}, Mat<LDK, 1>{SJ}, m0, n0, J, lane);     // dO S
         warp_mma<NT, SPLIT>(aKw, Mat<LDJ, 1>{Vns}, Mat<LDK, 1>{dSJ}, m0, n0, J, lane);   // Vn dS'
@@ -778,11 +801,11 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
     __syncthreads();
     warp_mma<NT, SPLIT>(aQ, Mat<LDC, 1>{dPs}, Mat<LDK, 1>{Kws}, m0, n0, C, lane);        // dP Kw
     warp_mma<NT, SPLIT>(aKw, Mat<1, LDC>{dPs}, Mat<LDK, 1>{Qs}, m0, n0, C, lane);        // dP^T Q
-    frag_each(aQ, m0, n0, lane, [&](int m, int n, float x) {
-        if (m < Tc) dq[tok(m) * DK + n] = from_f32<Tin>(x);
+    frag_each(aQ, m0, n0, lane, [&](int m, int n, float x0, float x1) {
+        if (m < Tc) store2(dq + tok(m) * DK + n, x0, x1);
     });
-    frag_each(aKw, m0, n0, lane, [&](int m, int n, float x) { dkwa_g[m * DK + n] = x; });
-    frag_each(aW, m0, n0, lane, [&](int m, int n, float x) { dw_g[m * DK + n] = -x; });
+    frag_each(aKw, m0, n0, lane, [&](int m, int n, float x0, float x1) { store2(dkwa_g + m * DK + n, x0, x1); });
+    frag_each(aW, m0, n0, lane, [&](int m, int n, float x0, float x1) { store2(dw_g + m * DK + n, -x0, -x1); });
     __syncthreads();
     for (int idx = tid; idx < C * C; idx += NTHR) dt_g[idx] = dTs[(idx / C) * LDC + idx % C];
     if (tid < C) dba_g[tid] = dbs[tid];
@@ -881,15 +904,16 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
     warp_mma<NT, SPLIT>(aK, Mat<LDC, 1>{dTs}, Mat<LDK, 1>{Kws}, m0, n0, C, lane);       // + dAb Kw
     frag_apply(aKw, m0, n0, lane, [&](int m, int n, float& x) { x = dkwa_g[m * DK + n]; });
     warp_mma<NT, SPLIT>(aKw, Mat<1, LDC>{dTs}, Mat<LDK, 1>{Ks}, m0, n0, C, lane);       // + dAb^T K
-    #pragma unroll
+#pragma unroll
     for (int jj = 0; jj < NT; ++jj)
-        #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int m = m0 + (lane >> 2) + 8 * (e >> 1), n = n0 + 8 * jj + 2 * (lane & 3) + (e & 1);
-            const float dkw = aKw[jj][e];
-            const float dval = m < Tc ? d_all[tok(m) * DK + n] : 0.f;
-            dd_g[m * DK + n] = dkw * Ks[m * LDK + n];
-            dkp_g[m * DK + n] = aK[jj][e] + dkw * dval;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {   // columns n, n + 1 of row m
+            const int m = m0 + (lane >> 2) + 8 * hh, n = n0 + 8 * jj + 2 * (lane & 3);
+            const float w0 = aKw[jj][2 * hh], w1 = aKw[jj][2 * hh + 1];
+            float2 dval = make_float2(0.f, 0.f);
+            if (m < Tc) dval = *reinterpret_cast<const float2*>(d_all + tok(m) * DK + n);
+            store2(dd_g + m * DK + n, w0 * Ks[m * LDK + n], w1 * Ks[m * LDK + n + 1]);
+            store2(dkp_g + m * DK + n, aK[jj][2 * hh] + w0 * dval.x, aK[jj][2 * hh + 1] + w1 * dval.y);
         }
     __syncthreads();
     if (tid < C) dbp_g[tid] = dbs[tid];
