@@ -297,6 +297,17 @@ __device__ __forceinline__ void async_tile(float* dst, int ldd, const float* src
     }
 }
 
+// 16-byte stores of a ROWS x COLS fp32 tile from shared memory (row stride lds, rows
+// 16-byte aligned) to global memory (row stride ldd).
+template <int ROWS, int COLS>
+__device__ __forceinline__ void store_rows(float* dst, size_t ldd, const float* src, int lds) {
+    constexpr int VPR = COLS / 4, N = ROWS * VPR;
+    for (int idx = threadIdx.x; idx < N; idx += NTHR) {
+        const int r = idx / VPR, c = (idx % VPR) * 4;
+        *reinterpret_cast<float4*>(dst + (size_t)r * ldd + c) = *reinterpret_cast<const float4*>(src + r * lds + c);
+    }
+}
+
 // dst[r * ldd + c] = src[r * COLS + c] for a dense fp32 ROWS x COLS block (the workspace layout).
 template <int ROWS, int COLS>
 __device__ __forceinline__ void async_block(float* dst, int ldd, const float* src) {
@@ -493,10 +504,10 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
         const float kv = Kb[t * LDK + i], w = Kw[t * LDK + i] * kv;
         Kb[t * LDK + i] = bs[t] * kv;
         Kw[t * LDK + i] = w;
-        kw_g[idx] = w;
     }
     load_tile<C, DV>(X, LDX, v + tok0 * DV, tstride * DV, Tc, bs);
     __syncthreads();
+    store_rows<C, DK>(kw_g, DK, Kw, LDK);
     cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{Kb}, Mat<1, LDK>{Kw},
                     [&](int m, int n, float x) { As[m * LDC + n] = n < m ? x : 0.f; });
     __syncthreads();
@@ -522,7 +533,7 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
         tri::tril_inv64_inplace(As, tid >> 5, tid & 31, [] { asm volatile("bar.sync 1, 128;" ::: "memory"); });
     }
     __syncthreads();
-    for (int idx = tid; idx < C * C; idx += NTHR) t_g[idx] = Tm[(idx / C) * LDC + idx % C];
+    store_rows<C, C>(t_g, C, Tm, LDC);
     cta_gemm<SPLIT>(C, DK, C, Mat<LDC, 1>{Tm}, Mat<LDK, 1>{Kb},
                     [&](int m, int n, float x0, float x1) { store2(w_g + m * DK + n, x0, x1); });
     cta_gemm<SPLIT>(C, DV, C, Mat<LDC, 1>{Tm}, Mat<LDX, 1>{X},
@@ -578,10 +589,7 @@ bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout 
             prefetch_rows(kw_g + C * DK, 0, 1, C * DK * 4);
             prefetch_rows(u_g + C * DV + v0, (size_t)DV * 4, C, DVT * 4);
         }
-        for (int idx = tid; idx < DVT * DK; idx += NTHR) {
-            const int row = idx / DK, i = idx % DK;
-            s_g[(size_t)(v0 + row) * DK + i] = Ss[row * LDK + i];
-        }
+        store_rows<DVT, DK>(s_g + (size_t)v0 * DK, DK, Ss, LDK);
         async_block<C, DK>(Ws, LDK, w_g);
         async_block<C, DK>(Kws, LDK, kw_g);
         async_tile<C, DVT>(Vs, LDT, u_g + v0, (size_t)DV);
@@ -639,10 +647,7 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
             prefetch_rows(dout + tokp * DV + v0, (size_t)H * DV * sizeof(Tin), C, DVT * sizeof(Tin));
             prefetch_rows(q + tokp * DK, (size_t)H * DK * sizeof(Tin), C, DK * sizeof(Tin));
         }
-        for (int idx = tid; idx < DVT * DK; idx += NTHR) {
-            const int row = idx / DK, i = idx % DK;
-            ds_g[(size_t)(v0 + row) * DK + i] = dSs[row * LDK + i];
-        }
+        store_rows<DVT, DK>(ds_g + (size_t)v0 * DK, DK, dSs, LDK);
         const size_t tok0 = ((size_t)b * T + c0) * H + h;
         async_block<C, C>(Ps, LDC, p_g);
         async_block<C, DK>(B1, LDK, kw_g);
@@ -666,11 +671,7 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
                          [&](int m, int n, float x) { dSs[m * LDK + n] += x; });
     }
     __syncthreads();
-    if (dS0)
-        for (int idx = tid; idx < DVT * DK; idx += NTHR) {
-            const int row = idx / DK, i = idx % DK;
-            dS0[((size_t)unit * DV + v0 + row) * DK + i] = dSs[row * LDK + i];
-        }
+    if (dS0) store_rows<DVT, DK>(dS0 + ((size_t)unit * DV + v0) * DK, DK, dSs, LDK);
 }
 
 // ---------------------------------------------------------------------------
@@ -789,11 +790,24 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
         // dT += (dVn V^T) diag(beta)
         cta_gemm<SPLIT>(C, C, J, Mat<LDJ, 1>{dVns}, Mat<1, LDJ>{Vs},
                         [&](int m, int n, float x) { dTs[m * LDC + n] += bs[n] * x; });
-        // dV = diag(beta) T^T dVn;  dbeta += rowdot(T^T dVn, V)
-        cta_gemm<SPLIT>(C, J, C, Mat<1, LDC>{Ts}, Mat<LDJ, 1>{dVns}, [&](int m, int n, float x0, float x1) {
-            if (m < Tc) store2(dv + tok(m) * DV + v0 + n, bs[m] * x0, bs[m] * x1);
-            atomicAdd(&dbs[m], x0 * Vs[m * LDJ + n] + x1 * Vs[m * LDJ + n + 1]);
-        });
+        {   // dV = diag(beta) T^T dVn, one 16 x 8 tile per warp; dbeta += rowdot(T^T dVn, V), the
+            // 4 lanes that share a row reducing before one atomic
+            static_assert(NTHR == 512 && J == 32, "16 warps cover the 64 x 32 tile as 4 x 4 tiles of 16 x 8");
+            const int mv = 16 * (warp & 3), nv = 8 * (warp >> 2), t4 = lane & 3;
+            float acc[1][4];
+            frag_zero(acc);
+            warp_mma<1, SPLIT>(acc, Mat<1, LDC>{Ts}, Mat<LDJ, 1>{dVns}, mv, nv, C, lane);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int m = mv + (lane >> 2) + 8 * hh, n = nv + 2 * t4;
+                const float x0 = acc[0][2 * hh], x1 = acc[0][2 * hh + 1];
+                if (m < Tc) store2(dv + tok(m) * DV + v0 + n, bs[m] * x0, bs[m] * x1);
+                float part = x0 * Vs[m * LDJ + n] + x1 * Vs[m * LDJ + n + 1];
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                part += __shfl_xor_sync(0xffffffffu, part, 2);
+                if (t4 == 0) atomicAdd(&dbs[m], part);
+            }
+        }
         warp_mma<NT, SPLIT>(aQ, Mat<LDJ, 1>{dOs}, Mat<LDK, 1>{SJ}, m0, n0, J, lane);     // dO S
         warp_mma<NT, SPLIT>(aKw, Mat<LDJ, 1>{Vns}, Mat<LDK, 1>{dSJ}, m0, n0, J, lane);   // Vn dS'
         warp_mma<NT, SPLIT>(aW, Mat<LDJ, 1>{dVns}, Mat<LDK, 1>{SJ}, m0, n0, J, lane);    // dVn S
@@ -807,7 +821,7 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
     frag_each(aKw, m0, n0, lane, [&](int m, int n, float x0, float x1) { store2(dkwa_g + m * DK + n, x0, x1); });
     frag_each(aW, m0, n0, lane, [&](int m, int n, float x0, float x1) { store2(dw_g + m * DK + n, -x0, -x1); });
     __syncthreads();
-    for (int idx = tid; idx < C * C; idx += NTHR) dt_g[idx] = dTs[(idx / C) * LDC + idx % C];
+    store_rows<C, C>(dt_g, C, dTs, LDC);
     if (tid < C) dba_g[tid] = dbs[tid];
     }
 }
@@ -883,24 +897,36 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
     cta_gemm<SPLIT>(C, C, C, Mat<LDC, 1>{dTs}, Mat<1, LDC>{Ts},
                     [&](int m, int n, float x) { Xs[m * LDC + n] = x; });
     __syncthreads();
-    cta_gemm<SPLIT>(C, C, C, Mat<1, LDC>{Ts}, Mat<LDC, 1>{Xs}, [&](int m, int n, float x) {
-        float ab = 0.f;
-        if (n < m) {
-            const float a = -x;                      // dA (strictly lower)
-            atomicAdd(&dbs[m], a * Gs[m * LDC + n]);
-            ab = bs[m] * a;
-        }
-        dTs[m * LDC + n] = ab;                       // diag(beta) dA
+    cta_gemm<SPLIT>(C, C, C, Mat<1, LDC>{Ts}, Mat<LDC, 1>{Xs}, [&](int m, int n, float x0, float x1) {
+        const float a0 = n < m ? -x0 : 0.f, a1 = n + 1 < m ? -x1 : 0.f;   // dA (strictly lower)
+        if (n < m) atomicAdd(&dbs[m], a0 * Gs[m * LDC + n] + a1 * Gs[m * LDC + n + 1]);
+        dTs[m * LDC + n] = bs[m] * a0;                                    // diag(beta) dA
+        dTs[m * LDC + n + 1] = bs[m] * a1;
     });
     __syncthreads();
     const int m0 = 16 * (warp & 3), n0 = (DK / 4) * (warp >> 2);
     float aK[NT][4], aKw[NT][4];
     frag_zero(aK);
     warp_mma<NT, SPLIT>(aK, Mat<1, LDC>{Ts}, Mat<LDK, 1>{dWs}, m0, n0, C, lane);        // T^T dW
-    frag_apply(aK, m0, n0, lane, [&](int m, int n, float& x) {
-        atomicAdd(&dbs[m], x * Ks[m * LDK + n]);
-        x *= bs[m];
-    });
+    {   // dbeta += rowdot(T^T dW, K): the 4 lanes that share a row reduce before one atomic
+        const int t4 = lane & 3;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int m = m0 + (lane >> 2) + 8 * hh;
+            float part = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < NT; ++jj) {
+                const int n = n0 + 8 * jj + 2 * t4;
+                part = fmaf(aK[jj][2 * hh], Ks[m * LDK + n], part);
+                part = fmaf(aK[jj][2 * hh + 1], Ks[m * LDK + n + 1], part);
+                aK[jj][2 * hh] *= bs[m];
+                aK[jj][2 * hh + 1] *= bs[m];
+            }
+            part += __shfl_xor_sync(0xffffffffu, part, 1);
+            part += __shfl_xor_sync(0xffffffffu, part, 2);
+            if (t4 == 0) atomicAdd(&dbs[m], part);
+        }
+    }
     warp_mma<NT, SPLIT>(aK, Mat<LDC, 1>{dTs}, Mat<LDK, 1>{Kws}, m0, n0, C, lane);       // + dAb Kw
     frag_apply(aKw, m0, n0, lane, [&](int m, int n, float& x) { x = dkwa_g[m * DK + n]; });
     warp_mma<NT, SPLIT>(aKw, Mat<1, LDC>{dTs}, Mat<LDK, 1>{Ks}, m0, n0, C, lane);       // + dAb^T K
