@@ -149,6 +149,12 @@ __device__ __forceinline__ void store2(float* p, float a, float b) {
 __device__ __forceinline__ void store2(__nv_bfloat16* p, float a, float b) {
     *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
+__device__ __forceinline__ void add2(float* p, float a, float b) {
+    float2 v = *reinterpret_cast<float2*>(p);
+    v.x += a;
+    v.y += b;
+    *reinterpret_cast<float2*>(p) = v;
+}
 
 // The CTA computes the M x N product sum_k A(m, k) B(k, n) (plus, for the two-term
 // form, a second product over K2) in warp tiles of 16 x 8 NT taken round-robin, and
@@ -509,7 +515,9 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     __syncthreads();
     store_rows<C, DK>(kw_g, DK, Kw, LDK);
     cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{Kb}, Mat<1, LDK>{Kw},
-                    [&](int m, int n, float x) { As[m * LDC + n] = n < m ? x : 0.f; });
+                    [&](int m, int n, float x0, float x1) {
+                        store2(As + m * LDC + n, n < m ? x0 : 0.f, n + 1 < m ? x1 : 0.f);
+                    });
     __syncthreads();
     // T = (I + A)^{-1}. fp32 mode: exact forward substitution into Ts, column j on 8
     // threads that split the inner sum. bf16 inputs: the blocked inverse in place over A
@@ -603,7 +611,7 @@ bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout 
         });
         __syncthreads();
         cta_gemm<SPLIT>(DVT, DK, C, Mat<1, LDT>{Vs}, Mat<LDK, 1>{Kws},
-                        [&](int m, int n, float x) { Ss[m * LDK + n] += x; });
+                        [&](int m, int n, float x0, float x1) { add2(Ss + m * LDK + n, x0, x1); });
     }
 }
 
@@ -668,7 +676,7 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
         __syncthreads();
         // dS = dS' + dO^T Q + (-dVn)^T W
         cta_gemm2<SPLIT>(DVT, DK, C, Mat<1, LDT>{dOs}, Mat<LDK, 1>{B2}, C, Mat<1, LDT>{dVs}, Mat<LDK, 1>{B1},
-                         [&](int m, int n, float x) { dSs[m * LDK + n] += x; });
+                         [&](int m, int n, float x0, float x1) { add2(dSs + m * LDK + n, x0, x1); });
     }
     __syncthreads();
     if (dS0) store_rows<DVT, DK>(dS0 + ((size_t)unit * DV + v0) * DK, DK, dSs, LDK);
@@ -786,10 +794,12 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
         __syncthreads();
         // dP += tril(dO Vn^T) of this tile
         cta_gemm<SPLIT>(C, C, J, Mat<LDJ, 1>{dOs}, Mat<1, LDJ>{Vns},
-                        [&](int m, int n, float x) { if (n <= m) dPs[m * LDC + n] += x; });
+                        [&](int m, int n, float x0, float x1) {
+                            if (n <= m) add2(dPs + m * LDC + n, x0, n + 1 <= m ? x1 : 0.f);
+                        });
         // dT += (dVn V^T) diag(beta)
         cta_gemm<SPLIT>(C, C, J, Mat<LDJ, 1>{dVns}, Mat<1, LDJ>{Vs},
-                        [&](int m, int n, float x) { dTs[m * LDC + n] += bs[n] * x; });
+                        [&](int m, int n, float x0, float x1) { add2(dTs + m * LDC + n, bs[n] * x0, bs[n + 1] * x1); });
         {   // dV = diag(beta) T^T dVn, one 16 x 8 tile per warp; dbeta += rowdot(T^T dVn, V), the
             // 4 lanes that share a row reducing before one atomic
             static_assert(NTHR == 512 && J == 32, "16 warps cover the 64 x 32 tile as 4 x 4 tiles of 16 x 8");
@@ -890,12 +900,12 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
     cp_async_wait_all();
     __syncthreads();
     cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{dWs}, Mat<1, LDK>{Ks},
-                    [&](int m, int n, float x) { dTs[m * LDC + n] += bs[n] * x; });
+                    [&](int m, int n, float x0, float x1) { add2(dTs + m * LDC + n, bs[n] * x0, bs[n + 1] * x1); });
     cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{Ks}, Mat<1, LDK>{Kws},
-                    [&](int m, int n, float x) { Gs[m * LDC + n] = x; });
+                    [&](int m, int n, float x0, float x1) { store2(Gs + m * LDC + n, x0, x1); });
     __syncthreads();
     cta_gemm<SPLIT>(C, C, C, Mat<LDC, 1>{dTs}, Mat<1, LDC>{Ts},
-                    [&](int m, int n, float x) { Xs[m * LDC + n] = x; });
+                    [&](int m, int n, float x0, float x1) { store2(Xs + m * LDC + n, x0, x1); });
     __syncthreads();
     cta_gemm<SPLIT>(C, C, C, Mat<1, LDC>{Ts}, Mat<LDC, 1>{Xs}, [&](int m, int n, float x0, float x1) {
         const float a0 = n < m ? -x0 : 0.f, a1 = n + 1 < m ? -x1 : 0.f;   // dA (strictly lower)
