@@ -395,7 +395,7 @@ def run_backward(w, g, stream, hbm, tf_peak, steps=5, warmup=2):
     t_hbm, t_tc = nbytes / (hbm * 1e9), F / (tf_peak * 1e12)
     t_roof = max(t_hbm, t_tc)
     del ws
-    return {"call": "osdn_bwd (7 kernel launches)", "ms": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),
+    return {"call": "osdn_bwd (6 kernel launches)", "ms": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),
             "algorithmic_bytes": nbytes, "flops": F, "t_roofline_us": t_roof * 1e6,
             "bound": "tensor" if t_tc >= t_hbm else "hbm", "frac": t_roof / (ms / 1e3),
             "tflops": F / (ms / 1e3) / 1e12, "gbs": nbytes / (ms / 1e3) / 1e9,

@@ -214,9 +214,9 @@ int osdn_step_gated(const osdn_params *p,
  * workspace: osdn_bwd_workspace_size() bytes, 16-byte aligned, no
  * initialisation needed; it holds fp32 intermediates: d_t for every token
  * (dk values) and, per 64-token chunk and head (the last chunk padded),
- * 64 * (6 dk + 3 dv + 3 * 64 + 2) values plus two states (2 dv dk values),
- * i.e. about (7 dk + 3 dv + 194) * 4 bytes per token and head plus
- * 8 dv dk bytes per chunk and head (4.2 GB at B8 T4096 H16 dk = dv = 128).
+ * 64 * (4 dk + 3 dv + 2 * 64 + 1) values plus two states (2 dv dk values),
+ * i.e. about (5 dk + 3 dv + 129) * 4 bytes per token and head plus
+ * 8 dv dk bytes per chunk and head (3.5 GB at B8 T4096 H16 dk = dv = 128).
  * T = 0 copies dS_final to dS0 and dd_final to dd0 (zeros when NULL).
  * Errors: OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED, OSDN_ERR_CUDA. */
 int osdn_bwd_workspace_size(const osdn_params *p, size_t *bytes);

@@ -31,8 +31,8 @@
 //   bwd_prep    per chunk: Kw, T, W, U0, P;
 //   bwd_state_f per (unit, dv tile): S at every chunk start, Vn;
 //   bwd_state_b per (unit, dv tile), chunks in reverse: dS' at every chunk end, dVn, dS0;
-//   bwd_grads_a per chunk, dv tiles in turn: dQ, dV, dW, dT, the dv-summed part of dKw and dbeta;
-//   bwd_grads_b per chunk: dA, dK, dKw, dD and the rest of dbeta;
+//   bwd_grads   per chunk: dQ, dV (dv tiles in turn), then dA, dK, dKw, dD and the
+//               chunk part of dbeta;
 //   bwd_dchain  token-serial reverse of the d recurrence: dk, dbeta, dr, dd0.
 // Rows of S are independent given the chunk matrices, so the two state passes
 // split dv into tiles with no exchange.  The contractions run on mma.sync
@@ -198,7 +198,7 @@ __device__ __forceinline__ void prefetch_rows(const void* p, size_t stride_bytes
 
 // Workspace layout of one backward call (fp32 regions, 256-byte aligned).
 struct Layout {
-    size_t d_all, kw, tinv, w, u0, p, ckS, ckdS, vn, dvn, dkwa, dw, dt, dba, dd, dkp, dbp, total;
+    size_t d_all, kw, tinv, w, u0, p, ckS, ckdS, vn, dvn, dd, dkp, dbp, total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -219,10 +219,6 @@ inline Layout make_layout(int B, int T, int H, int DK, int DV) {
     L.ckdS = take(f * ch * DV * DK);
     L.vn = take(f * ch * C * DV);
     L.dvn = take(f * ch * C * DV);
-    L.dkwa = take(f * ch * C * DK);
-    L.dw = take(f * ch * C * DK);
-    L.dt = take(f * ch * C * C);
-    L.dba = take(f * ch * C);
     L.dd = take(f * ch * C * DK);
     L.dkp = take(f * ch * C * DK);
     L.dbp = take(f * ch * C);
@@ -683,36 +679,27 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
 }
 
 // ---------------------------------------------------------------------------
-// Per chunk, over the dv tiles in turn: dP and dT (V part) summed over the
-// tiles, dV, and the tile terms of dQ (dO S), dKw (Vn dS') and dW (-dVn S);
-// then dQ += dP Kw and dKw += dP^T Q once, and the dv-summed part of dbeta
-// (rowdot(T^T dVn, V)). dQ, dKw and dW stay in registers: warp w (of 16) owns
-// rows 16 (w % 4) .. + 15 and columns (DK / 4) (w / 4) .. + DK / 4 - 1 of each.
+// Every gradient of one chunk. Value side, over the dv tiles in turn: dP and dT
+// (V part) summed over the tiles, dV, the tile terms of dQ (dO S), dKw (Vn dS')
+// and dW (-dVn S), the dbeta term rowdot(T^T dVn, V); then dQ += dP Kw and
+// dKw += dP^T Q once. Key side, as written below. dQ, dKw, dW and dK stay in
+// registers: warp w (of 16) owns rows 16 (w % 4) .. + 15 and columns
+// (DK / 4) (w / 4) .. + DK / 4 - 1 of each.
 constexpr int J = 32;           // dv tile of the gradient kernel
 constexpr int LDJ = J + 4;
 
 template <int DK>
 struct GradSmem {
     static constexpr int LDK = DK + 4;
-    static constexpr size_t kABytes =
+    static constexpr size_t kBytes =
         sizeof(float) * (size_t)(2 * C * LDK + 3 * C * LDC + 4 * C * LDJ + 2 * J * LDK + 2 * C);
-    static constexpr size_t kBBytes = sizeof(float) * (size_t)(3 * C * LDK + 4 * C * LDC + 2 * C);
 };
-
-template <int NT, typename F>
-__device__ __forceinline__ void frag_apply(float (&acc)[NT][4], int m0, int n0, int lane, F f) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int j = 0; j < NT; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) f(m0 + g + 8 * (e >> 1), n0 + 8 * j + 2 * t + (e & 1), acc[j][e]);
-}
 
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(NTHR, 1)
-bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const Tin* __restrict__ beta,
-                   const Tin* __restrict__ dout, Tin* __restrict__ dq, Tin* __restrict__ dv,
-                   float* __restrict__ ws, Layout L, int B, int T, int H, int NC)
+bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                 const Tin* __restrict__ beta, const Tin* __restrict__ dout, Tin* __restrict__ dq,
+                 Tin* __restrict__ dv, float* __restrict__ ws, Layout L, int B, int T, int H, int NC)
 {
     constexpr bool SPLIT = std::is_same<Tin, float>::value;
     constexpr int LDK = GradSmem<DK>::LDK, NT = DK / 32;
@@ -729,10 +716,11 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
     float* SJ = Vs + C * LDJ;        // [J][LDK] rows of S (chunk start)
     float* dSJ = SJ + J * LDK;       // [J][LDK] rows of dS' (chunk end)
     float* bs = dSJ + J * LDK;       // [C] beta
-    float* dbs = bs + C;             // [C] dbeta (this kernel's part)
+    float* dbs = bs + C;             // [C] dbeta (the chunk part)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t nchunks = (size_t)B * H * NC;
+    const float* d_all = ws + L.d_all / sizeof(float);
     for (size_t cid = blockIdx.x; cid < nchunks; cid += gridDim.x) {   // persistent, as bwd_prep
     const int unit = (int)(cid / NC), c = (int)(cid % NC), b = unit / H, h = unit % H;
     const int c0 = c * C, Tc = min(C, T - c0);
@@ -742,10 +730,9 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
     const float* dvn_g = ws + L.dvn / sizeof(float) + cid * C * DV;
     const float* s_g = ws + L.ckS / sizeof(float) + cid * DV * DK;
     const float* ds_g = ws + L.ckdS / sizeof(float) + cid * DV * DK;
-    float* dkwa_g = ws + L.dkwa / sizeof(float) + cid * C * DK;
-    float* dw_g = ws + L.dw / sizeof(float) + cid * C * DK;
-    float* dt_g = ws + L.dt / sizeof(float) + cid * C * C;
-    float* dba_g = ws + L.dba / sizeof(float) + cid * C;
+    float* dd_g = ws + L.dd / sizeof(float) + cid * C * DK;
+    float* dkp_g = ws + L.dkp / sizeof(float) + cid * C * DK;
+    float* dbp_g = ws + L.dbp / sizeof(float) + cid * C;
     auto tok = [&](int t) { return ((size_t)b * T + c0 + t) * H + h; };
 
     const size_t tok0 = tok(0);
@@ -756,6 +743,8 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
         const int tcn = min(C, T - cn * C);
         const size_t tokn = ((size_t)bn * T + cn * C) * H + hn;
         prefetch_rows(q + tokn * DK, (size_t)H * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
+        prefetch_rows(k + tokn * DK, (size_t)H * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
+        prefetch_rows(d_all + tokn * DK, (size_t)H * DK * sizeof(float), tcn, DK * sizeof(float));
         prefetch_rows(v + tokn * DV, (size_t)H * DV * sizeof(Tin), tcn, DV * sizeof(Tin));
         prefetch_rows(dout + tokn * DV, (size_t)H * DV * sizeof(Tin), tcn, DV * sizeof(Tin));
         prefetch_rows(ws + L.kw / sizeof(float) + nx * C * DK, 0, 1, C * DK * 4);
@@ -828,76 +817,18 @@ bwd_grads_a_kernel(const Tin* __restrict__ q, const Tin* __restrict__ v, const T
     frag_each(aQ, m0, n0, lane, [&](int m, int n, float x0, float x1) {
         if (m < Tc) store2(dq + tok(m) * DK + n, x0, x1);
     });
-    frag_each(aKw, m0, n0, lane, [&](int m, int n, float x0, float x1) { store2(dkwa_g + m * DK + n, x0, x1); });
-    frag_each(aW, m0, n0, lane, [&](int m, int n, float x0, float x1) { store2(dw_g + m * DK + n, -x0, -x1); });
-    __syncthreads();
-    store_rows<C, C>(dt_g, C, dTs, LDC);
-    if (tid < C) dba_g[tid] = dbs[tid];
-    }
-}
 
-// Per chunk: dT += (dW K^T) diag(beta), dA = -strict_tril(T^T dT T^T), the
-// dbeta terms of T^T dW and of dA, dK, the rest of dKw, then dD = dKw (.) K and
-// the chunk part of dk, dK + dKw (.) D.
-template <int DK, typename Tin>
-__global__ void __launch_bounds__(NTHR, 1)
-bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, float* __restrict__ ws, Layout L,
-                   int B, int T, int H, int NC)
-{
-    constexpr bool SPLIT = std::is_same<Tin, float>::value;
-    constexpr int LDK = GradSmem<DK>::LDK, NT = DK / 32;
-    extern __shared__ float sm[];
-    float* Ks = sm;                  // [C][LDK] K
-    float* Kws = Ks + C * LDK;       // [C][LDK] Kw
-    float* dWs = Kws + C * LDK;      // [C][LDK] dW
-    float* Ts = dWs + C * LDK;       // [C][LDC] T
-    float* dTs = Ts + C * LDC;       // [C][LDC] dT, then diag(beta) dA
-    float* Xs = dTs + C * LDC;       // [C][LDC] dT T^T
-    float* Gs = Xs + C * LDC;        // [C][LDC] K Kw^T
-    float* bs = Gs + C * LDC;        // [C] beta
-    float* dbs = bs + C;             // [C] dbeta (chunk part)
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const size_t nchunks = (size_t)B * H * NC;
-    const float* d_all = ws + L.d_all / sizeof(float);
-    for (size_t cid = blockIdx.x; cid < nchunks; cid += gridDim.x) {   // persistent, as bwd_prep
-    const int unit = (int)(cid / NC), c = (int)(cid % NC), b = unit / H, h = unit % H;
-    const int c0 = c * C, Tc = min(C, T - c0);
-    const float* kw_g = ws + L.kw / sizeof(float) + cid * C * DK;
-    const float* t_g = ws + L.tinv / sizeof(float) + cid * C * C;
-    const float* dkwa_g = ws + L.dkwa / sizeof(float) + cid * C * DK;
-    const float* dw_g = ws + L.dw / sizeof(float) + cid * C * DK;
-    const float* dt_g = ws + L.dt / sizeof(float) + cid * C * C;
-    const float* dba_g = ws + L.dba / sizeof(float) + cid * C;
-    float* dd_g = ws + L.dd / sizeof(float) + cid * C * DK;
-    float* dkp_g = ws + L.dkp / sizeof(float) + cid * C * DK;
-    float* dbp_g = ws + L.dbp / sizeof(float) + cid * C;
-    auto tok = [&](int t) { return ((size_t)b * T + c0 + t) * H + h; };
-
-    __syncthreads();
-    if (cid + gridDim.x < nchunks) {   // L2 prefetch of the next chunk's inputs
-        const size_t nx = cid + gridDim.x;
-        const int un = (int)(nx / NC), cn = (int)(nx % NC), bn = un / H, hn = un % H;
-        const int tcn = min(C, T - cn * C);
-        const size_t tokn = ((size_t)bn * T + cn * C) * H + hn;
-        prefetch_rows(k + tokn * DK, (size_t)H * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
-        prefetch_rows(d_all + tokn * DK, (size_t)H * DK * sizeof(float), tcn, DK * sizeof(float));
-        prefetch_rows(ws + L.kw / sizeof(float) + nx * C * DK, 0, 1, C * DK * 4);
-        prefetch_rows(ws + L.dw / sizeof(float) + nx * C * DK, 0, 1, C * DK * 4);
-        prefetch_rows(ws + L.dkwa / sizeof(float) + nx * C * DK, 0, 1, C * DK * 4);
-        prefetch_rows(ws + L.tinv / sizeof(float) + nx * C * C, 0, 1, C * C * 4);
-        prefetch_rows(ws + L.dt / sizeof(float) + nx * C * C, 0, 1, C * C * 4);
-    }
-    async_block<C, DK>(Kws, LDK, kw_g);
-    async_block<C, DK>(dWs, LDK, dw_g);
-    async_block<C, C>(Ts, LDC, t_g);
-    async_block<C, C>(dTs, LDC, dt_g);
-    load_tile<C, DK>(Ks, LDK, k + tok(0) * DK, (size_t)H * DK, Tc);
-    if (tid < C) {
-        bs[tid] = ld_or0(beta, tok(tid), tid < Tc);
-        dbs[tid] = dba_g[tid];
-    }
-    cp_async_wait_all();
+    // Key side: dT += (dW K^T) diag(beta), dA = -strict_tril(T^T dT T^T), the dbeta terms
+    // of T^T dW and of dA, dK and the rest of dKw (still in registers), then dD = dKw (.) K
+    // and the chunk part of dk, dK + dKw (.) D. Q's buffer and the dv-tile buffers are reused.
+    float* Ks = Qs;                  // [C][LDK] K
+    float* dWs = dOs;                // [C][LDK] dW, over the four dv-tile buffers
+    float* Xs = dPs;                 // [C][LDC] dT T^T
+    float* Gs = SJ;                  // [C][LDC] K Kw^T, over the rows of S and dS'
+    static_assert(C * LDK <= 4 * C * LDJ && C * LDC <= 2 * J * LDK, "key-side buffers fit the reused ones");
+    __syncthreads();                 // every warp is done with Q, dP and the dv tiles
+    frag_each(aW, m0, n0, lane, [&](int m, int n, float x0, float x1) { store2(dWs + m * LDK + n, -x0, -x1); });
+    load_tile<C, DK>(Ks, LDK, k + tok0 * DK, (size_t)H * DK, Tc);
     __syncthreads();
     cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{dWs}, Mat<1, LDK>{Ks},
                     [&](int m, int n, float x0, float x1) { add2(dTs + m * LDC + n, bs[n] * x0, bs[n + 1] * x1); });
@@ -914,8 +845,7 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
         dTs[m * LDC + n + 1] = bs[m] * a1;
     });
     __syncthreads();
-    const int m0 = 16 * (warp & 3), n0 = (DK / 4) * (warp >> 2);
-    float aK[NT][4], aKw[NT][4];
+    float aK[NT][4];
     frag_zero(aK);
     warp_mma<NT, SPLIT>(aK, Mat<1, LDC>{Ts}, Mat<LDK, 1>{dWs}, m0, n0, C, lane);        // T^T dW
     {   // dbeta += rowdot(T^T dW, K): the 4 lanes that share a row reduce before one atomic
@@ -938,7 +868,6 @@ bwd_grads_b_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, floa
         }
     }
     warp_mma<NT, SPLIT>(aK, Mat<LDC, 1>{dTs}, Mat<LDK, 1>{Kws}, m0, n0, C, lane);       // + dAb Kw
-    frag_apply(aKw, m0, n0, lane, [&](int m, int n, float& x) { x = dkwa_g[m * DK + n]; });
     warp_mma<NT, SPLIT>(aKw, Mat<1, LDC>{dTs}, Mat<LDK, 1>{Ks}, m0, n0, C, lane);       // + dAb^T K
 #pragma unroll
     for (int jj = 0; jj < NT; ++jj)

@@ -318,7 +318,7 @@ int launch_state_passes(const osdn_params* p, const Tin* q, const Tin* dout, con
     return OSDN_OK;
 }
 
-// Backward: seven launches on one stream (see bwd.cuh for what each computes).
+// Backward: six launches on one stream (see bwd.cuh for what each computes).
 template <typename Tin, int DK, int DV>
 int launch_bwd_t(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, const Tin* beta, const Tin* r,
                  const float* d0, const float* S0, const Tin* dout, const float* dS_final, const float* dd_final,
@@ -359,16 +359,12 @@ int launch_bwd_t(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v,
     else rcs = launch_state_passes<Tin, DK, DV, DV>(p, q, dout, S0, dS_final, dS0, ws, L, NC, st);
     if (rcs) return rcs;
 
-    const size_t s_ga = B::GradSmem<DK>::kABytes, s_gb = B::GradSmem<DK>::kBBytes;
-    if ((e = attr((const void*)B::bwd_grads_a_kernel<DK, DV, Tin>, s_ga)) != cudaSuccess)
+    const size_t s_g = B::GradSmem<DK>::kBytes;
+    if ((e = attr((const void*)B::bwd_grads_kernel<DK, DV, Tin>, s_g)) != cudaSuccess)
         return cuda_fail(e, "backward gradient attribute");
-    B::bwd_grads_a_kernel<DK, DV, Tin><<<pgrid, B::NTHR, s_ga, st>>>(q, v, beta, dout, dq, dv, ws, L, p->B, p->T,
-                                                                       p->H, NC);
+    B::bwd_grads_kernel<DK, DV, Tin><<<pgrid, B::NTHR, s_g, st>>>(q, k, v, beta, dout, dq, dv, ws, L, p->B, p->T,
+                                                                   p->H, NC);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward gradient launch");
-    if ((e = attr((const void*)B::bwd_grads_b_kernel<DK, Tin>, s_gb)) != cudaSuccess)
-        return cuda_fail(e, "backward key gradient attribute");
-    B::bwd_grads_b_kernel<DK, Tin><<<pgrid, B::NTHR, s_gb, st>>>(k, beta, ws, L, p->B, p->T, p->H, NC);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward key gradient launch");
 
     if ((e = attr((const void*)B::bwd_dchain_kernel<DK, Tin>, s_dc)) != cudaSuccess)
         return cuda_fail(e, "backward d chain attribute");
