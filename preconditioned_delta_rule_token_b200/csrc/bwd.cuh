@@ -737,23 +737,6 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
 
     const size_t tok0 = tok(0);
     __syncthreads();
-    if (cid + gridDim.x < nchunks) {   // L2 prefetch of the next chunk's inputs
-        const size_t nx = cid + gridDim.x;
-        const int un = (int)(nx / NC), cn = (int)(nx % NC), bn = un / H, hn = un % H;
-        const int tcn = min(C, T - cn * C);
-        const size_t tokn = ((size_t)bn * T + cn * C) * H + hn;
-        prefetch_rows(q + tokn * DK, (size_t)H * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
-        prefetch_rows(k + tokn * DK, (size_t)H * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
-        prefetch_rows(d_all + tokn * DK, (size_t)H * DK * sizeof(float), tcn, DK * sizeof(float));
-        prefetch_rows(v + tokn * DV, (size_t)H * DV * sizeof(Tin), tcn, DV * sizeof(Tin));
-        prefetch_rows(dout + tokn * DV, (size_t)H * DV * sizeof(Tin), tcn, DV * sizeof(Tin));
-        prefetch_rows(ws + L.kw / sizeof(float) + nx * C * DK, 0, 1, C * DK * 4);
-        prefetch_rows(ws + L.tinv / sizeof(float) + nx * C * C, 0, 1, C * C * 4);
-        prefetch_rows(ws + L.vn / sizeof(float) + nx * C * DV, 0, 1, C * DV * 4);
-        prefetch_rows(ws + L.dvn / sizeof(float) + nx * C * DV, 0, 1, C * DV * 4);
-        prefetch_rows(ws + L.ckS / sizeof(float) + nx * DV * DK, 0, 1, DV * DK * 4);
-        prefetch_rows(ws + L.ckdS / sizeof(float) + nx * DV * DK, 0, 1, DV * DK * 4);
-    }
     async_block<C, DK>(Kws, LDK, kw_g);        // waited for with the first tile's copies
     async_block<C, C>(Ts, LDC, t_g);
     load_tile<C, DK>(Qs, LDK, q + tok0 * DK, (size_t)H * DK, Tc);
@@ -817,6 +800,24 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     frag_each(aQ, m0, n0, lane, [&](int m, int n, float x0, float x1) {
         if (m < Tc) store2(dq + tok(m) * DK + n, x0, x1);
     });
+    if (cid + gridDim.x < nchunks) {   // L2 prefetch of the next chunk's inputs, issued here rather than
+        // at the chunk start: it keeps about one chunk per CTA in flight instead of two
+        const size_t nx = cid + gridDim.x;
+        const int un = (int)(nx / NC), cn = (int)(nx % NC), bn = un / H, hn = un % H;
+        const int tcn = min(C, T - cn * C);
+        const size_t tokn = ((size_t)bn * T + cn * C) * H + hn;
+        prefetch_rows(q + tokn * DK, (size_t)H * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
+        prefetch_rows(k + tokn * DK, (size_t)H * DK * sizeof(Tin), tcn, DK * sizeof(Tin));
+        prefetch_rows(d_all + tokn * DK, (size_t)H * DK * sizeof(float), tcn, DK * sizeof(float));
+        prefetch_rows(v + tokn * DV, (size_t)H * DV * sizeof(Tin), tcn, DV * sizeof(Tin));
+        prefetch_rows(dout + tokn * DV, (size_t)H * DV * sizeof(Tin), tcn, DV * sizeof(Tin));
+        prefetch_rows(ws + L.kw / sizeof(float) + nx * C * DK, 0, 1, C * DK * 4);
+        prefetch_rows(ws + L.tinv / sizeof(float) + nx * C * C, 0, 1, C * C * 4);
+        prefetch_rows(ws + L.vn / sizeof(float) + nx * C * DV, 0, 1, C * DV * 4);
+        prefetch_rows(ws + L.dvn / sizeof(float) + nx * C * DV, 0, 1, C * DV * 4);
+        prefetch_rows(ws + L.ckS / sizeof(float) + nx * DV * DK, 0, 1, DV * DK * 4);
+        prefetch_rows(ws + L.ckdS / sizeof(float) + nx * DV * DK, 0, 1, DV * DK * 4);
+    }
 
     // Key side: dT += (dW K^T) diag(beta), dA = -strict_tril(T^T dT T^T), the dbeta terms
     // of T^T dW and of dA, dK and the rest of dKw (still in registers), then dD = dKw (.) K
