@@ -58,6 +58,16 @@ template <int S0, int S1>
 struct Mat {
     const float* p;
     __device__ __forceinline__ float operator()(int i, int j) const { return p[i * S0 + j * S1]; }
+    // X(i, j) and X(i, j + 1), one 8-byte load when the second index is contiguous (j even)
+    __device__ __forceinline__ float2 pair_j(int i, int j) const {
+        if constexpr (S1 == 1) return *reinterpret_cast<const float2*>(p + i * S0 + j);
+        else return make_float2(p[i * S0 + j * S1], p[i * S0 + (j + 1) * S1]);
+    }
+    // X(i, j) and X(i + 1, j), one 8-byte load when the first index is contiguous (i even)
+    __device__ __forceinline__ float2 pair_i(int i, int j) const {
+        if constexpr (S0 == 1) return *reinterpret_cast<const float2*>(p + i + j * S1);
+        else return make_float2(p[i * S0 + j * S1], p[(i + 1) * S0 + j * S1]);
+    }
 };
 
 __device__ __forceinline__ void mma8(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
@@ -100,17 +110,20 @@ __device__ __forceinline__ void mma_step(float (&c)[4], const float (&a)[4], con
 
 // One warp: acc[j] += sum_{k < K} A(m0 + ., k) B(k, n0 + 8 j + .) for a 16 x 8 NT tile.
 // Fragment element e of acc[j] sits at row m0 + g + 8 (e >> 1), column n0 + 8 j + 2 t + (e & 1),
-// with g = lane / 4, t = lane % 4.
+// with g = lane / 4, t = lane % 4. Within each step of 8, the instruction's k slots t and t + 4
+// carry k0 + 2t and k0 + 2t + 1 in both operands (a permutation of the summation index), so a
+// lane's two k values are adjacent and load as one pair where the layout allows.
 template <int NT, bool SPLIT, class MA, class MB>
 __device__ __forceinline__ void warp_mma(float (&acc)[NT][4], MA A, MB B, int m0, int n0, int K, int lane) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll 4
     for (int k0 = 0; k0 < K; k0 += 8) {
-        const float a[4] = {A(m0 + g, k0 + t), A(m0 + g + 8, k0 + t), A(m0 + g, k0 + t + 4),
-                            A(m0 + g + 8, k0 + t + 4)};
+        const float2 lo = A.pair_j(m0 + g, k0 + 2 * t), hi = A.pair_j(m0 + g + 8, k0 + 2 * t);
+        const float a[4] = {lo.x, hi.x, lo.y, hi.y};
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-            const float b[2] = {B(k0 + t, n0 + 8 * j + g), B(k0 + t + 4, n0 + 8 * j + g)};
+            const float2 bb = B.pair_i(k0 + 2 * t, n0 + 8 * j + g);
+            const float b[2] = {bb.x, bb.y};
             mma_step<SPLIT>(acc[j], a, b);
         }
     }
