@@ -27,13 +27,15 @@
 //
 // Kernels, in launch order (every chunk quantity lives in the workspace in a
 // chunk-block layout [unit][chunk][row][col], fp32):
-//   bwd_dtraj   d_t for every token (token-serial, one warp per unit);
+//   bwd_dtraj   d_t for every token (token-serial: one CTA per unit, a chain warp
+//               and three warps that stage the next slab of tokens);
 //   bwd_prep    per chunk: Kw, T, W, U0, P;
 //   bwd_state_f per (unit, dv tile): S at every chunk start, Vn;
 //   bwd_state_b per (unit, dv tile), chunks in reverse: dS' at every chunk end, dVn, dS0;
 //   bwd_grads   per chunk: dQ, dV (dv tiles in turn), then dA, dK, dKw, dD and the
 //               chunk part of dbeta;
-//   bwd_dchain  token-serial reverse of the d recurrence: dk, dbeta, dr, dd0.
+//   bwd_dchain  token-serial reverse of the d recurrence, staged as bwd_dtraj:
+//               dk, dbeta, dr, dd0.
 // Rows of S are independent given the chunk matrices, so the two state passes
 // split dv into tiles with no exchange.  The contractions run on mma.sync
 // m16n8k8 tf32 with fp32 accumulation; for fp32 inputs every product uses the
