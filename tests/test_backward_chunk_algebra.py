@@ -1,0 +1,140 @@
+"""Design check (CPU, float64): the chunk form of the adjoint that the backward
+kernels compute equals the oracle's token-by-token gradients.
+
+The forward per chunk of C tokens with chunk-start state S ("OSDN: Improving Delta
+Rule with Provable Online Preconditioning in Linear Attention", technical summary
+section 2.1, the DeltaNet chunk pipeline with the scaled write key Kw = D (.) K):
+    Kb = diag(beta) K,  A = strict_tril(Kb Kw^T),  T = (I + A)^{-1},  W = T Kb,
+    U0 = T diag(beta) V,  Vn = U0 - W S^T,  P = tril(Q Kw^T),
+    O = Q S^T + P Vn,  S' = S + Vn^T Kw.
+Its reverse, chunk by chunk from the last with dS' = dL/dS':
+    dVn = P^T dO + Kw dS'^T,        dS = dS' + dO^T Q - dVn^T W,
+    dP = tril(dO Vn^T),             dQ = dO S + dP Kw,
+    dW = -dVn S,                    dT = (dW K^T + dVn V^T) diag(beta),
+    dA = -strict_tril(T^T dT T^T),  dAb = diag(beta) dA,
+    dKw = Vn dS' + dP^T Q + dAb^T K,
+    dV = diag(beta) T^T dVn,        dK = diag(beta) T^T dW + dAb Kw + dKw (.) D,
+    dbeta = rowdot(T^T dW, K) + rowdot(T^T dVn, V) + rowsum(dA (.) K Kw^T),
+    dD = dKw (.) K,
+followed by the reverse of the APF recurrence token by token (section 2.3). This is
+the algebra written at the top of csrc/bwd.cuh; here it is restated in numpy and
+compared with oracle.bwd (itself pinned by finite differences).
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def _case(seed, T, dk=8, dv=6, apf=True):
+    rng = np.random.default_rng(seed)
+    c = dict(q=rng.standard_normal((1, T, 1, dk)), k=rng.standard_normal((1, T, 1, dk)),
+             v=rng.standard_normal((1, T, 1, dv)), beta=rng.uniform(0.1, 0.9, (1, T, 1)),
+             r=rng.uniform(0.8, 1.0, (1, T, 1)) if apf else None,
+             d0=rng.uniform(0.5, 1.5, (1, 1, dk)), S0=0.3 * rng.standard_normal((1, 1, dv, dk)))
+    c["k"] /= np.linalg.norm(c["k"], axis=-1, keepdims=True)
+    if T > 5:
+        c["k"][0, 5, 0] = 0.0                            # a zero key: the d step is skipped
+    cot = dict(dout=rng.standard_normal((1, T, 1, dv)), dS_final=rng.standard_normal((1, 1, dv, dk)),
+               dd_final=rng.standard_normal((1, 1, dk)))
+    return c, cot
+
+
+def _d_trajectory(k, beta, r, d0, eta, anchor):
+    """d_t before each token's own update (the forward recurrence, written out)."""
+    T, dk = k.shape
+    D = np.zeros((T, dk))
+    d = d0.copy()
+    for t in range(T):
+        D[t] = d
+        a = k[t] ** 2
+        n = a.sum()
+        x = eta * beta[t] * (1 - beta[t] * (d @ a)) / n if n > 0 else 0.0
+        d = r[t] * d + ((1 - r[t]) * d0 if anchor else 0.0) + x * a
+    return D, d
+
+
+def chunk_backward(q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, eta, anchor, C):
+    """Gradients of one (b, h) unit by the chunk-form adjoint. q, k: [T, dk]; v, dout: [T, dv]."""
+    T, dk = k.shape
+    dv = v.shape[1]
+    r = np.ones(T) if r is None else r
+    D, _ = _d_trajectory(k, beta, r, d0, eta, anchor)
+    Kw_all = D * k
+    starts = list(range(0, T, C))
+    # forward over the chunks: the state at every chunk start and the chunk matrices
+    S = S0.copy()
+    saved = []
+    for c0 in starts:
+        sl = slice(c0, min(T, c0 + C))
+        K, Kw, Q, V, be = k[sl], Kw_all[sl], q[sl], v[sl], beta[sl]
+        n = len(K)
+        Kb = be[:, None] * K
+        A = np.tril(Kb @ Kw.T, -1)
+        Tm = np.linalg.inv(np.eye(n) + A)
+        W = Tm @ Kb
+        U0 = Tm @ (be[:, None] * V)
+        Vn = U0 - W @ S.T
+        P = np.tril(Q @ Kw.T)
+        saved.append((sl, S.copy(), Tm, W, Vn, P))
+        S = S + Vn.T @ Kw
+    # reverse over the chunks
+    dS = dS_final.copy()
+    dq, dk_, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dbeta, dD = np.zeros(T), np.zeros((T, dk))
+    for sl, Sc, Tm, W, Vn, P in reversed(saved):
+        K, Kw, Q, V, be, dO, Dc = k[sl], Kw_all[sl], q[sl], v[sl], beta[sl], dout[sl], D[sl]
+        dVn = P.T @ dO + Kw @ dS.T
+        dS_prev = dS + dO.T @ Q - dVn.T @ W
+        dP = np.tril(dO @ Vn.T)
+        dq[sl] = dO @ Sc + dP @ Kw
+        dW = -dVn @ Sc
+        dT = (dW @ K.T + dVn @ V.T) * be[None, :]
+        dA = -np.tril(Tm.T @ dT @ Tm.T, -1)
+        dAb = be[:, None] * dA
+        dKw = Vn @ dS + dP.T @ Q + dAb.T @ K
+        TdW, TdVn = Tm.T @ dW, Tm.T @ dVn
+        dvv[sl] = be[:, None] * TdVn
+        dk_[sl] = be[:, None] * TdW + dAb @ Kw + dKw * Dc
+        dbeta[sl] = (TdW * K).sum(1) + (TdVn * V).sum(1) + (dA * (K @ Kw.T)).sum(1)
+        dD[sl] = dKw * K
+        dS = dS_prev
+    # reverse of the preconditioner recurrence
+    Ld = dd_final.copy()
+    dr = np.zeros(T)
+    dd_anchor = np.zeros(dk)
+    anc = d0 if anchor else np.zeros(dk)
+    for t in range(T - 1, -1, -1):
+        a, d = k[t] ** 2, D[t]
+        n, s = a.sum(), D[t] @ a
+        dr[t] = (d - anc) @ Ld
+        if anchor:
+            dd_anchor += (1 - r[t]) * Ld
+        ds = 0.0
+        if n > 0:
+            x = eta * beta[t] * (1 - beta[t] * s) / n
+            dx = a @ Ld
+            dbeta[t] += dx * eta * (1 - 2 * beta[t] * s) / n
+            ds = -dx * eta * beta[t] ** 2 / n
+            dk_[t] += 2 * k[t] * (x * Ld + ds * d - dx * x / n)
+        Ld = r[t] * Ld + dD[t] + ds * a
+    return dict(dq=dq, dk=dk_, dv=dvv, dbeta=dbeta, dr=dr, dd0=Ld + dd_anchor, dS0=dS)
+
+
+@pytest.mark.parametrize("T,C,anchor,apf", [(150, 64, False, True), (150, 64, True, True), (64, 64, False, True),
+                                             (97, 16, True, True), (130, 32, False, False)])
+def test_chunk_adjoint_matches_the_token_gradients(T, C, anchor, apf):
+    c, cot = _case(T + C, T, apf=apf)
+    eta = 0.3
+    ref = oracle.bwd(c["q"], c["k"], c["v"], c["beta"], cot["dout"], c["r"], c["d0"], c["S0"], cot["dS_final"],
+                     cot["dd_final"], eta=eta, anchor=anchor)
+    u = lambda x: None if x is None else x[0, :, 0]
+    got = chunk_backward(u(c["q"]), u(c["k"]), u(c["v"]), u(c["beta"]), u(c["r"]), c["d0"][0, 0], c["S0"][0, 0],
+                         u(cot["dout"]), cot["dS_final"][0, 0], cot["dd_final"][0, 0], eta, anchor, C)
+    pairs = [("dq", u(ref["dq"])), ("dk", u(ref["dk"])), ("dv", u(ref["dv"])), ("dbeta", u(ref["dbeta"])),
+             ("dd0", ref["dd0"][0, 0]), ("dS0", ref["dS0"][0, 0])]
+    if apf:
+        pairs.append(("dr", u(ref["dr"])))
+    for name, want in pairs:
+        np.testing.assert_allclose(got[name], want, rtol=1e-9, atol=1e-10 * max(1.0, np.abs(want).max()),
+                                   err_msg=name)
