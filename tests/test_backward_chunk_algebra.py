@@ -19,6 +19,17 @@ Its reverse, chunk by chunk from the last with dS' = dL/dS':
 followed by the reverse of the APF recurrence token by token (section 2.3). This is
 the algebra written at the top of csrc/bwd.cuh; here it is restated in numpy and
 compared with oracle.bwd (itself pinned by finite differences).
+
+The reverse of the APF recurrence also has a chunk form, the transposed counterpart
+of the forward scan's: with Ld_j = dL/dd of token j of a block of L tokens,
+Ld_L the adjoint entering from the next block, rho(i, j) = prod_{m=i}^{j-1} r_m,
+a_j = k_j^2 and c2_j = -eta beta_j^2 / ||k_j||^2 (0 for a zero key), the unknowns
+y_j = <a_j, Ld_{j+1}> solve the upper-triangular system
+    y_j - sum_{i>j} rho(j+1, i) c2_i <a_j, a_i> y_i
+        = rho(j+1, L) <a_j, Ld_L> + sum_{i>j} rho(j+1, i) <a_j, dD_i>,
+after which Ld_{j} = rho(j, L) Ld_L + sum_{i>=j} rho(j, i) (dD_i + c2_i y_i a_i) for every j
+(Ld_0 leaves the block). Only <a_j, Ld_L> and the last sum depend on the carried
+Ld_L; the system's matrix and its inverse do not.
 """
 import numpy as np
 import pytest
@@ -138,3 +149,58 @@ def test_chunk_adjoint_matches_the_token_gradients(T, C, anchor, apf):
     for name, want in pairs:
         np.testing.assert_allclose(got[name], want, rtol=1e-9, atol=1e-10 * max(1.0, np.abs(want).max()),
                                    err_msg=name)
+
+
+def chunk_dchain(k, beta, r, dD, dd_final, eta, L):
+    """Ld_{t+1} for every token (the adjoint of d entering token t from later tokens)
+    and Ld_0, by the chunk form above. k, dD: [T, dk]."""
+    T, dk = k.shape
+    a_all = k * k
+    nrm = a_all.sum(1)
+    c2 = np.where(nrm > 0, -eta * beta ** 2 / np.where(nrm > 0, nrm, 1.0), 0.0)
+    Ld = dd_final.copy()
+    L_next = np.zeros((T, dk))                     # Ld_{t+1} for token t
+    for c0 in reversed(range(0, T, L)):
+        n = min(L, T - c0)
+        a, rr, cc, dDc = a_all[c0:c0 + n], r[c0:c0 + n], c2[c0:c0 + n], dD[c0:c0 + n]
+        rho = np.ones((n + 1, n + 1))              # rho[i, j] = prod_{m=i}^{j-1} r_m (i <= j)
+        for i in range(n + 1):
+            for j in range(i + 1, n + 1):
+                rho[i, j] = rho[i, j - 1] * rr[j - 1]
+        G, E = a @ a.T, a @ dDc.T                  # <a_j, a_i>, <a_j, dD_i>
+        U = np.zeros((n, n))
+        bvec = np.zeros(n)
+        for j in range(n):
+            bvec[j] = rho[j + 1, n] * (a[j] @ Ld)
+            for i in range(j + 1, n):
+                U[j, i] = rho[j + 1, i] * cc[i] * G[j, i]
+                bvec[j] += rho[j + 1, i] * E[j, i]
+        y = np.linalg.solve(np.eye(n) - U, bvec)
+        w = dDc + (cc * y)[:, None] * a            # dD_i + c2_i y_i a_i
+        for j in range(n):                         # Ld_{j+1} for every token of the block
+            L_next[c0 + j] = rho[j + 1, n] * Ld + sum(rho[j + 1, i] * w[i] for i in range(j + 1, n))
+        Ld = rho[0, n] * Ld + sum(rho[0, i] * w[i] for i in range(n))
+    return L_next, Ld
+
+
+@pytest.mark.parametrize("T,L", [(150, 64), (97, 16), (64, 64), (5, 8)])
+def test_chunk_form_of_the_reverse_preconditioner_recurrence(T, L):
+    # the token-serial reverse, written out, against the chunk form above
+    rng = np.random.default_rng(T * 7 + L)
+    dk = 8
+    k = rng.standard_normal((T, dk))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    if T > 3:
+        k[3] = 0.0
+    beta, r = rng.uniform(0.1, 0.9, T), rng.uniform(0.8, 1.0, T)
+    dD, dd_final, eta = rng.standard_normal((T, dk)), rng.standard_normal(dk), 0.3
+    Ld = dd_final.copy()
+    want = np.zeros((T, dk))
+    for t in range(T - 1, -1, -1):
+        want[t] = Ld
+        a, n = k[t] ** 2, (k[t] ** 2).sum()
+        ds = -(a @ Ld) * eta * beta[t] ** 2 / n if n > 0 else 0.0
+        Ld = r[t] * Ld + dD[t] + ds * a
+    got, got0 = chunk_dchain(k, beta, r, dD, dd_final, eta, L)
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(got0, Ld, rtol=1e-10, atol=1e-12)
