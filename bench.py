@@ -274,7 +274,9 @@ def run_reference(args, world, rank):
     value = statistics.median(toks)
     line = {"impl": "reference", "metric": "OSDN chunkwise fwd tokens/s", "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": w.B * w.T / value * 1e3,
+            "ms_per_step_note": "one step over the whole workload at the sample's rate (extrapolated)",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
             "config": config_of(w, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
