@@ -153,3 +153,11 @@ def test_backward_default_initial_state_and_preconditioner():
     for n in g_def:   # dbeta sums shared-memory atomic adds, whose order may differ between calls
         a_, b_ = g_def[n].cpu().numpy(), g_exp[n].cpu().numpy()
         np.testing.assert_allclose(a_, b_, rtol=1e-5, atol=1e-6 * np.abs(b_).max(), err_msg=n)
+
+
+@pytest.mark.parametrize("dv,anchor", [(64, False), (128, True)])
+def test_backward_bf16_narrow_keys(dv, anchor):
+    # bf16 inputs with dk = 64 (the tensor-core tile paths at the narrow key width)
+    w = _small("bwd bf16 dk64", 2, 2, 130, 64, dv, W.BF16, seed=31)
+    got, ref = _run(w, anchor=anchor)
+    _compare(got, ref, BF16_TOL, True)
