@@ -1,6 +1,7 @@
 /*
- * osdn.h - C ABI of libosdn.so: the Online Scaled DeltaNet (OSDN) forward and
- * single-token decode on NVIDIA B200 (sm_100a).
+ * osdn.h - C ABI of libosdn.so: the Online Scaled DeltaNet (OSDN) forward, its
+ * backward (gradients for training) and single-token decode on NVIDIA B200
+ * (sm_100a).
  *
  * Method: "OSDN: Improving Delta Rule with Provable Online Preconditioning in
  * Linear Attention" (gist.science technical summary).
