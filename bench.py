@@ -508,6 +508,11 @@ def run_ours(args, world, rank, local):
     kd = kernels[dom]
     achieved = kd["bytes"] / (kd["ms"] / 1e3) / 1e9
     traffic = ncu_traffic(dom, args.workload)
+    # the method's own bytes (q, k, v, beta, r, out + state: 1,028 B per token-head) over the
+    # dominant kernel's time, and the DRAM traffic of the whole step over those bytes
+    method_gbs = path_bytes(w) / (kd["ms"] / 1e3) / 1e9
+    step_traffic = [ncu_traffic(k_, args.workload) for k_ in kernels]
+    step_traffic = None if any(t_ is None for t_ in step_traffic) else sum(step_traffic)
     line = {
         "metric": "OSDN chunkwise fwd tokens/s", "value": aggregate_tokens_per_s(w, world, ms), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -519,7 +524,10 @@ def run_ours(args, world, rank, local):
                           "bytes": path_bytes(w), "flops": F, "peak_kind": peak_kind},
         "roofline": {"kernel": kd["name"], "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "algorithmic_bytes": kd["bytes"],
-                     "launch_ms": kd["ms"], "peak_kind": peak_kind + " hbm_gbs"},
+                     "launch_ms": kd["ms"], "peak_kind": peak_kind + " hbm_gbs",
+                     "method_bytes": path_bytes(w), "frac_method_bytes": method_gbs / hbm,
+                     "step_traffic": step_traffic,
+                     "step_traffic_over_method_bytes": None if step_traffic is None else step_traffic / path_bytes(w)},
         "kernels_ms": {k_: v_["ms"] for k_, v_ in kernels.items()},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks.summary(),

@@ -246,9 +246,12 @@ int osdn_bwd(const osdn_params *p,
  * The scaled write keys go to one fixed scratch array inside the library
  * (OSDN_NOALLOC_SCRATCH_BYTES of device memory that every GPU which loads the
  * library keeps until the process exits). The library calls no cudaMalloc or
- * cudaFree for it. The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture. Every call uses the same array, and the
+ * cudaFree for it. Each call made outside stream capture looks up the array's
+ * device address (cudaGetSymbolAddress) with the calling device current, so a
+ * device reset between calls is harmless; a call made while cuda_stream is
+ * capturing reuses the address of that device's last uncaptured call, so make
+ * the first call on a device before any stream capture (a captured first call
+ * returns OSDN_ERR_INVALID_ARG). Every call uses the same array, and the
  * scan overwrites every scratch entry the chunk phase reads, so stale contents
  * from an earlier call are never used. Two calls that overlap on the GPU (for
  * example on two streams) race on the array: order them on one stream.

@@ -396,25 +396,32 @@ size_t bwd_workspace_bytes(const osdn_params* p) {
 
 // Scratch for osdn_fwd_noalloc: a fixed array in device memory, sized by
 // OSDN_NOALLOC_SCRATCH_BYTES. In host code the symbol is only a handle; its
-// device address is looked up once per device with cudaGetSymbolAddress.
+// device address comes from cudaGetSymbolAddress with the device current.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[OSDN_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (set up on first use).
-int noalloc_scratch(void** out) {
+// Device address of the scratch array on the current device. Outside stream capture the
+// address is looked up again on every call (a device reset can move the array); during a
+// capture, where the lookup may not run, the address of this device's last lookup is used.
+int noalloc_scratch(cudaStream_t st, void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return fail(OSDN_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if ((e = cudaStreamIsCapturing(st, &cs)) != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    if (cs == cudaStreamCaptureStatusNone) {
         void* ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the scratch array");
         g_noalloc_ptr[dev] = ptr;
+    } else if (!g_noalloc_ptr[dev]) {
+        return fail(OSDN_ERR_INVALID_ARG,
+                    "osdn_fwd_noalloc: the first call on a device must come before any stream capture");
     }
     *out = g_noalloc_ptr[dev];
     return OSDN_OK;
@@ -564,7 +571,7 @@ int osdn_fwd_noalloc(const osdn_params* p, const void* q, const void* k, const v
                     need, (size_t)OSDN_NOALLOC_SCRATCH_BYTES);
     void* scratch = nullptr;
     if (p->T > 0) {
-        rc = noalloc_scratch(&scratch);
+        rc = noalloc_scratch(reinterpret_cast<cudaStream_t>(cuda_stream), &scratch);
         if (rc) return rc;
     }
     rc = check_fwd_args(p, {q, k, v, beta, out}, {q, k, v, beta, r, d0, S0, out, final_S, final_d}, scratch,

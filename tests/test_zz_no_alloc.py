@@ -16,7 +16,6 @@ import pytest
 import torch
 
 from preconditioned_delta_rule_token_b200 import workloads as W
-from tests._util import BF16_TOL, FP32_TOL, slice_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -38,17 +37,18 @@ def _both(w):
 
 
 def test_noalloc_matches_workspace_forward_on_two_calls_in_a_row():
+    # The two entry points launch the same kernels on the same inputs, so their results are
+    # bit-identical. The second (smaller) case runs after a larger one, so the shared array
+    # still holds stale data beyond its range: equality shows none of it is read.
     cases = [
         W.Workload("na1", 2, 3, 200, 128, 128, 64, W.BF16, True, d0="uniform", S0="normal", eta=0.1, seed=31),
         W.Workload("na2", 1, 2, 130, 64, 128, 64, W.FP32, False, S0="normal", eta=1e-2, seed=32),
+        W.Workload("na3", 1, 2, 70, 128, 128, 64, W.BF16, True, d0="uniform", S0="normal", eta=0.1, seed=33),
     ]
     for w in cases:
         ref, got = _both(w)
-        tol = FP32_TOL if w.dtype == W.FP32 else BF16_TOL
-        axes = ((0, 2), (0, 1), (0, 1))
-        for a, b, ax in zip(got, ref, axes):
-            err = slice_rel_err(a.float().cpu().numpy(), b.float().cpu().numpy(), ax)
-            assert err <= tol, (w.name, err)
+        for name, a, b in zip(("out", "final_S", "final_d"), got, ref):
+            assert torch.equal(a, b), (w.name, name)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
