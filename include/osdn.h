@@ -166,10 +166,10 @@ int osdn_step_ex(const osdn_params *p,
 /* Gated OSDN (the gated delta rule backbone the pages run OSDN on):
  *   S_t = alpha_t S_{t-1} (I - beta_t k_t kw_t^T) + beta_t v_t kw_t^T,   kw_t = d_t (.) k_t,
  * i.e. the OSDN write applied to the decayed state alpha_t S_{t-1}; the
- * preconditioner d is unchanged. alpha [B, T, H] in the input dtype, in (0, 1].
- * The chunk form divides by the decay accumulated inside a 64-token chunk, so
- * the product of alpha over any 64 consecutive tokens of a sequence must stay
- * above ~1e-30 (gates near 1, as in the gated DeltaNet layers).
+ * preconditioner d is unchanged. alpha [B, T, H] in the input dtype, in [0, 1]
+ * (alpha_t = 0 restarts the state before token t's write). The chunk form uses
+ * the decay only as ratios gamma_t / gamma_j <= 1 of the cumulative gate within
+ * a 64-token chunk, so every gate value in [0, 1] stays in range.
  * osdn_fwd_gated: as osdn_fwd plus alpha (not NULL when T > 0); bf16 inputs
  * with dk = dv = 128 only (else OSDN_ERR_UNSUPPORTED).
  * osdn_fwd_chunk_gated: phase 2 alone, after osdn_fwd_scan on the same stream.

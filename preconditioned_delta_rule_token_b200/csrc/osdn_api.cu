@@ -166,7 +166,8 @@ int launch_chunk_wy(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfl
     const size_t smem = osdn::WyLayout::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk kernel attribute");
-    kern<<<p->B * p->H, 288, smem, st>>>(mq, mk, mkw, mv, mo, beta, alpha, S0, final_S, p->B, p->T, p->H,
+    kern<<<p->B * p->H, osdn::WyLayout::kThreads, smem, st>>>(mq, mk, mkw, mv, mo, beta, alpha, S0, final_S, p->B,
+                                                             p->T, p->H,
                                          g_wait_limit_ns.load());
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core chunk launch");
     return OSDN_OK;

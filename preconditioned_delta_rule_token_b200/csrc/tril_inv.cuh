@@ -257,5 +257,134 @@ __device__ __forceinline__ void tril_inv64_inplace(float* A, int warp, int lane,
     sync();
 }
 
+// Byte offset of element (row r, column j) in a 128-byte-swizzled K-major bf16 tile whose
+// 8-row groups are 1024 bytes apart (64 columns of 2 bytes per row).
+__device__ __forceinline__ uint32_t sw128_elem(int r, int j) {
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((((j >> 3) ^ (r & 7))) << 4) + (j & 7) * 2);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// bf16 of sgn * c * sc[column] into block (a, b) of a swizzled 64 x 64 tile, from the m16n8
+// accumulator layout of blk_mma (4-byte stores; the 8 rows of a store hit 8 distinct 16-byte
+// bank groups).
+__device__ __forceinline__ void blk_store_bf16(uint8_t* tile, const float (&c)[2][4], float sgn, const float* sc,
+                                               int a, int b, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        const int col = 16 * b + 8 * nh + 2 * t;
+        const float s0 = sgn * sc[col], s1 = sgn * sc[col + 1];
+        *reinterpret_cast<uint32_t*>(tile + sw128_elem(16 * a + g, col)) = pack_bf16x2(s0 * c[nh][0], s1 * c[nh][1]);
+        *reinterpret_cast<uint32_t*>(tile + sw128_elem(16 * a + g + 8, col)) = pack_bf16x2(s0 * c[nh][2], s1 * c[nh][3]);
+    }
+}
+
+// bf16 of the fp32 block (a, b) of T (stride LD) times sc[column], into the swizzled tile; one warp,
+// lane L takes row L / 2 and columns 8 (L % 2) .. + 7 of the block (one 16-byte store).
+__device__ __forceinline__ void blk_convert_bf16(uint8_t* tile, const float* T, const float* sc, int a, int b,
+                                                 int lane) {
+    const int r = lane >> 1, j0 = 16 * b + 8 * (lane & 1);
+    const float* src = T + (16 * a + r) * LD + j0;
+    const float4 x0 = *reinterpret_cast<const float4*>(src), x1 = *reinterpret_cast<const float4*>(src + 4);
+    const float4 s0 = *reinterpret_cast<const float4*>(sc + j0), s1 = *reinterpret_cast<const float4*>(sc + j0 + 4);
+    uint4 pk;
+    pk.x = pack_bf16x2(x0.x * s0.x, x0.y * s0.y);
+    pk.y = pack_bf16x2(x0.z * s0.z, x0.w * s0.w);
+    pk.z = pack_bf16x2(x1.x * s1.x, x1.y * s1.y);
+    pk.w = pack_bf16x2(x1.z * s1.z, x1.w * s1.w);
+    *reinterpret_cast<uint4*>(tile + sw128_elem(16 * a + r, j0)) = pk;
+}
+
+// T = (I + A)^{-1} for a strictly lower 64 x 64 A (fp32, stride LD, 16-byte aligned rows), written
+// only as bf16 tiles: tb = T diag(sc) and, when tb2 is not null, tb2 = T diag(sc2) (128-byte-swizzled
+// K-major, row t, column j; 16 x 16 blocks above the diagonal blocks are not written and must hold
+// zeros). A's lower blocks are overwritten by intermediates. The same blocking as tril_inv64 in three
+// barrier-separated phases after the diagonal blocks:
+//   phase 0: T_ii = (I + A_ii)^{-1}, right-looking forward substitution, one warp per block;
+//   phase 1: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22) (warps 0, 1);
+//            Y_a0 = A_a0 T_00, X_a1 = A_a1 T_11 for a = 2, 3 (warp a, kept in registers);
+//   phase 2: X_a0 = Y_a0 + A_a1 T_10 (warp a; X_a0, X_a1 stored over A_a0, A_a1), while warps 0
+//            and 1 convert the finished blocks T_00, T_10, T_11 / T_22, T_32, T_33;
+//   phase 3: T_2b = -T_22 X_2b, T_3b = -(T_32 X_2b + T_33 X_3b) (one block per warp), straight to bf16.
+// Executed by the 4 warps of one group; sync() is a barrier over exactly those threads.
+// tiles_free() is called by every thread after phase 1, before the first tile write; it must act
+// as a barrier of the group and return true on every thread when the group is to stop (the
+// function then returns false right away). Returns true after a final sync().
+template <class Sync, class TilesFree>
+__device__ __forceinline__ bool tril_inv64_to_bf16(float* A, uint8_t* tb, const float* sc, uint8_t* tb2,
+                                                   const float* sc2, int warp, int lane, Sync sync,
+                                                   TilesFree tiles_free) {
+    auto blk = [&](int i, int j) { return A + (i * 16) * LD + j * 16; };
+    {   // phase 0: column j of T_ww by right-looking substitution (lanes 16-31 repeat lanes 0-15)
+        const int j = lane & 15;
+        const float* Ab = blk(warp, warp);
+        float c[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) c[t] = (t == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int m = 0; m < 15; ++m) {
+#pragma unroll
+            for (int t = m + 1; t < 16; ++t) c[t] = fmaf(-Ab[t * LD + m], c[m], c[t]);
+        }
+        __syncwarp();
+        if (lane < 16) {
+            float* Tb = blk(warp, warp);
+#pragma unroll
+            for (int t = 0; t < 16; ++t) Tb[t * LD + j] = c[t];
+        }
+    }
+    sync();
+    float y[2][4], x1[2][4];
+    blk_zero(y);
+    blk_zero(x1);
+    if (warp < 2) {   // phase 1: T_10 (warp 0), T_32 (warp 1)
+        const int i = 2 * warp + 1, j = 2 * warp;
+        blk_mma_trunc(y, blk(i, j), blk(j, j), lane);       // W = A_ij T_jj
+        __syncwarp();
+        blk_store(blk(i, j), y, 1.f, lane);
+        __syncwarp();
+        blk_zero(y);
+        blk_mma_trunc(y, blk(i, i), blk(i, j), lane);       // T_ii W
+        __syncwarp();
+        blk_store(blk(i, j), y, -1.f, lane);
+    } else {          // Y_a0 = A_a0 T_00, X_a1 = A_a1 T_11
+        blk_mma_trunc(y, blk(warp, 0), blk(0, 0), lane);
+        blk_mma_trunc(x1, blk(warp, 1), blk(1, 1), lane);
+    }
+    if (tiles_free()) return false;
+    if (warp >= 2) {  // phase 2: X_a0 = Y_a0 + A_a1 T_10
+        blk_mma_trunc(y, blk(warp, 1), blk(1, 0), lane);
+        __syncwarp();
+        blk_store(blk(warp, 0), y, 1.f, lane);
+        blk_store(blk(warp, 1), x1, 1.f, lane);
+    } else {          // finished blocks of T to bf16
+        const int o = 2 * warp;
+        blk_convert_bf16(tb, A, sc, o, o, lane);
+        blk_convert_bf16(tb, A, sc, o + 1, o, lane);
+        blk_convert_bf16(tb, A, sc, o + 1, o + 1, lane);
+        if (tb2) {
+            blk_convert_bf16(tb2, A, sc2, o, o, lane);
+            blk_convert_bf16(tb2, A, sc2, o + 1, o, lane);
+            blk_convert_bf16(tb2, A, sc2, o + 1, o + 1, lane);
+        }
+    }
+    sync();
+    {                 // phase 3: block (a, b) of T, a = 2 + warp / 2, b = warp % 2
+        const int a = 2 + (warp >> 1), bb = warp & 1;
+        float c[2][4];
+        blk_zero(c);
+        blk_mma_trunc(c, blk(a, 2), blk(2, bb), lane);
+        if (a == 3) blk_mma_trunc(c, blk(3, 3), blk(3, bb), lane);
+        blk_store_bf16(tb, c, -1.f, sc, a, bb, lane);
+        if (tb2) blk_store_bf16(tb2, c, -1.f, sc2, a, bb, lane);
+    }
+    sync();
+    return true;
+}
+
 }  // namespace tri
 }  // namespace osdn
