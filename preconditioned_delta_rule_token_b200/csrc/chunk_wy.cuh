@@ -56,9 +56,9 @@
 // The ratios are exp2 of differences of the in-chunk cumulative log2(alpha) (each log2 clamped at
 // -120, so alpha = 0 restarts the state to within 2^-120), which keeps every gate value in [0, 1]
 // in range. The kernel applies them in the prep (A_g, P_g and the second operand T diag(beta gamma)
-// of GW) and in the state group: with the -W rows, the chunk's Q rows x gamma_t and its Kw rows
-// x gamma_C / gamma_t (GBS then adds U^T diag(gamma_C / gamma) Kw), and the fp32 state x gamma_C
-// of the next chunk when it is converted to bf16.
+// of GW), in the epilogue group (the chunk's Q rows x gamma_t and its Kw rows x gamma_C / gamma_t, so
+// that GBS adds U^T diag(gamma_C / gamma) Kw; done two chunks ahead, once G1 has read both tiles), and
+// in the state group (the fp32 state x gamma_C of the next chunk when it is converted to bf16).
 #pragma once
 #include "tc_ptx.cuh"
 #include "tril_inv.cuh"
@@ -93,8 +93,10 @@ struct WyLayout {
         EVN = 16,    // state: bf16 Vn written
         EOR = 17,    // epilogue: O^T columns read and zeroed
         BAP = 18,    // 2: GA done (by chunk parity; the prep reuses T diag(beta) tile c % 2)
-        DRAIN = 20,
-        NBAR = 21
+        ESC = 20,    // 2, gated, epilogue: Q and Kw of a chunk scaled by its gates (by chunk parity: the
+                     // epilogue may finish chunk c + 2 before the issuer has consumed chunk c + 1)
+        DRAIN = 22,
+        NBAR = 23
     };
     static constexpr uint32_t TSLOT = BAR + NBAR * 8;       // TMEM base address
     static constexpr uint32_t ABORT = TSLOT + 4;
@@ -315,30 +317,11 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc::named_sync(BAR_STATE, 128);
         if (tid == 0 && nchunks > 0) tc::mbar_arrive1(bars + L::ESB);
 
-        // -W of chunk c (from W^T in R1[c % 3], lane = key feature) into the K rows of its stage;
-        // gated: the Q rows of the stage x gamma_t and its Kw rows x gamma_C / gamma_t (gates g of chunk c;
-        // G1(c), the other reader of Q and Kw, has completed)
-        auto w_epilogue = [&](int c, const ChunkGates& g) -> bool {
+        // -W of chunk c (from W^T in R1[c % 3], lane = key feature) into the K rows of its stage
+        auto w_epilogue = [&](int c) -> bool {
             if (tc::named_sync_or(BAR_STATE, 128, !wait(L::BW, c & 1))) return false;
             tc::tc_fence_after();
             uint8_t* st = sm + (c % 3) * L::STAGE + L::QK;
-            if (GATED) {   // thread (tid % 8) takes 16-byte chunk tid % 8 of rows t = tid / 8 + 16 i of each tile
-                const int ch = tid & 7;
-                const float gl = g.last();
-                uint8_t* kw = sm + (c % 3) * L::STAGE + L::KW;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int t = (tid >> 3) + 16 * i;
-                    const float gt = g.at(t);
-                    const float sq = sfu_exp2(gt), sk = sfu_exp2(gl - gt);
-                    const uint32_t row = (t >> 3) * 1024 + (t & 7) * 128 + ch * 16;
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        scale_bf16x8(st + half * 16384 + 8192 + row, sq);   // Q
-                        scale_bf16x8(kw + half * 8192 + row, sk);           // Kw
-                    }
-                }
-            }
             ColsToRows w;
             w.copy64(tl + COL_R1 + (c % 3) * 64, st, 16384, warp * 32, -1.f, lane);
             tc::fence_proxy_async_smem();
@@ -355,7 +338,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (nchunks > 1) gates_of(1, nxt);
                 if (nchunks > 2) load_la(2);
             }
-            ok = w_epilogue(0, cur);
+            ok = w_epilogue(0);
         }
         int c = 0;
         for (; ok && c < nchunks; ++c) {
@@ -377,7 +360,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (tid == 0) tc::mbar_arrive1(bars + L::EVN);
 
             // -W of the next chunk while GBS runs
-            if (c + 1 < nchunks && !w_epilogue(c + 1, nxt)) break;
+            if (c + 1 < nchunks && !w_epilogue(c + 1)) break;
 
             // S_{c+1} is complete: its bf16 copy for GA(c + 1) (gated: the fp32 state x gamma_C of chunk c + 1)
             if (tc::named_sync_or(BAR_STATE, 128, !wait(L::BS, c & 1))) break;
@@ -561,9 +544,43 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (nchunks > 3) prefetch_l2(3);
             if (nchunks > 4) prefetch_l2(4);
         }
-        for (int c = 0; c < nchunks; ++c) {
+        // gated: chunk c's Q rows x gamma_t and Kw rows x gamma_C / gamma_t (GBS then adds U^T diag(gamma_C /
+        // gamma) Kw), once G1(c), their other reader, has completed; the issuer waits for it before GA(c)
+        auto gate_scale = [&](int c) -> bool {
+            if (tc::named_sync_or(BAR_EPI, 128, !wait(L::D1 + c % 3, (c / 3) & 1))) return false;
+            ChunkGates g;
+            const int t0 = c * C + 2 * lane;
+            g.scan(ChunkGates::log2_alpha(alpha, alpha_idx(t0), t0 < T),
+                   ChunkGates::log2_alpha(alpha, alpha_idx(t0 + 1), t0 + 1 < T), lane);
+            uint8_t* st = sm + (c % 3) * L::STAGE + L::QK;
+            {   // thread (et % 8) takes 16-byte chunk et % 8 of rows t = et / 8 + 16 i of each tile
+                const int ch = et & 7;
+                const float gl = g.last();
+                uint8_t* kw = sm + (c % 3) * L::STAGE + L::KW;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int t = (et >> 3) + 16 * i;
+                    const float gt = g.at(t);
+                    const float sq = sfu_exp2(gt), sk = sfu_exp2(gl - gt);
+                    const uint32_t row = (t >> 3) * 1024 + (t & 7) * 128 + ch * 16;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        scale_bf16x8(st + half * 16384 + 8192 + row, sq);   // Q
+                        scale_bf16x8(kw + half * 8192 + row, sk);           // Kw
+                    }
+                }
+            }
+            tc::fence_proxy_async_smem();
+            tc::named_sync(BAR_EPI, 128);
+            if (et == 0) tc::mbar_arrive1(bars + L::ESC + (c & 1));
+            return true;
+        };
+        bool ok = true;
+        if (GATED)
+            for (int c = 0; ok && c < 2 && c < nchunks; ++c) ok = gate_scale(c);
+        for (int c = 0; ok && c < nchunks; ++c) {
             // O_c = (Q S^T + P Vn)^T complete: read it out and zero the columns for GA(c + 1)
-            if (tc::named_sync_or(BAR_EPI, 128, !wait(L::BO + (c & 1), (c >> 1) & 1))) break;
+            if (tc::named_sync_or(BAR_EPI, 128, !wait(L::BO + (c & 1), (c >> 1) & 1))) { ok = false; break; }
             tc::tc_fence_after();
             ColsToRows o0, o1;
             o0.load(tl + COL_D + 64);
@@ -596,6 +613,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     load_v(issuedV++);
                 }
             }
+            if (GATED && c + 2 < nchunks && !(ok = gate_scale(c + 2))) break;
         }
         if (et == kTmaThread) {   // stores complete; loads that were issued have landed
             tc::bulk_wait<0>();
@@ -683,7 +701,8 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                       (issue_g1(0) && (nchunks < 2 || issue_g1(1)) && issue_gw(0) && issue_gu(0));
             for (int c = 0; ok && c < nchunks; ++c) {
                 // GA(c) needs bf16 S_c, -W(c) and (c > 0) the O^T columns read out and zeroed
-                ok = wait(L::ESB, c & 1) && wait(L::EWE, c & 1) && (c == 0 || wait(L::EOR, (c - 1) & 1));
+                ok = wait(L::ESB, c & 1) && wait(L::EWE, c & 1) && (c == 0 || wait(L::EOR, (c - 1) & 1)) &&
+                     (!GATED || wait(L::ESC + (c & 1), (c >> 1) & 1));
                 if (!ok) break;
                 tc::tc_fence_after();
                 GA(c);
