@@ -19,7 +19,8 @@
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller. The library
  *     never allocates device memory and never frees anything.
- *   - Layouts are dense row-major (last dimension contiguous):
+ *   - Layouts are row-major (last dimension contiguous), dense unless the
+ *     strides of osdn_params say otherwise (forward only):
  *       q, k   [B, T, H, dk]     v, out [B, T, H, dv]
  *       beta, r [B, T, H]
  *       d (d0, final_d) [B, H, dk] fp32     S (S0, final_S) [B, H, dv, dk] fp32
@@ -45,7 +46,7 @@
 extern "C" {
 #endif
 
-#define OSDN_ABI_VERSION 2
+#define OSDN_ABI_VERSION 3
 
 enum {
     OSDN_OK = 0,
@@ -69,9 +70,23 @@ typedef struct {
     float eta;              /* hypergradient step size of the preconditioner */
     int32_t apf_anchor;     /* 0: APF retention r d (toward 0); 1: anchored APF,
                                r d + (1 - r) d_anchor, d_anchor = d0 in the forward */
+    /* Element strides of q, k, v and out over their (b, t, h) dimensions (the
+     * last dimension is always contiguous). All three zero: the dense layout
+     * [B, T, H, width]. Otherwise each stride must be a non-negative multiple of
+     * 8 elements (16-byte rows for the tensor-memory-accelerator loads), for
+     * example q, k, v read in place as column slices of one fused projection
+     * [B, T, H, 2 dk + dv]. Honoured by the forward entry points (osdn_fwd and
+     * its phases, the gated and no-allocation forwards); osdn_step* and osdn_bwd
+     * take dense tensors only and return OSDN_ERR_UNSUPPORTED otherwise.
+     * beta, r and alpha are always dense [B, T, H]. */
+    int64_t stride_q[3];
+    int64_t stride_k[3];
+    int64_t stride_v[3];
+    int64_t stride_o[3];
 } osdn_params;
-/* Version 1 of this struct ended after eta (struct_size 36); such callers get
- * apf_anchor = 0. */
+/* Earlier versions of this struct are accepted by struct_size: version 1
+ * ended after eta (36 bytes; apf_anchor = 0), version 2 after apf_anchor
+ * (40 bytes); both get the dense layout. */
 
 /* Bytes of device workspace osdn_fwd needs for these parameters (written to
  * *bytes). The workspace holds the scaled write keys d_t (.) k_t in the input

@@ -31,7 +31,8 @@ class osdn_params(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("B", ctypes.c_int32), ("T", ctypes.c_int32),
                 ("H", ctypes.c_int32), ("dk", ctypes.c_int32), ("dv", ctypes.c_int32),
                 ("chunk", ctypes.c_int32), ("dtype", ctypes.c_int32), ("eta", ctypes.c_float),
-                ("apf_anchor", ctypes.c_int32)]
+                ("apf_anchor", ctypes.c_int32), ("stride_q", ctypes.c_int64 * 3), ("stride_k", ctypes.c_int64 * 3),
+                ("stride_v", ctypes.c_int64 * 3), ("stride_o", ctypes.c_int64 * 3)]
 
 
 class OsdnError(RuntimeError):
@@ -145,6 +146,26 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _ptr_tok(t):
+    """Pointer of a token tensor [B, T, H, width] that may be a strided view (last dimension contiguous);
+    its other strides go into the parameter block (_set_strides)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise OsdnError(OSDN_ERR_INVALID_ARG, "tensor is not on a CUDA device (the library has no CPU path)")
+    if t.dim() != 4 or (t.numel() > 0 and t.stride(-1) != 1):
+        raise OsdnError(OSDN_ERR_INVALID_ARG, "token tensors are [B, T, H, width] with the last dimension contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _set_strides(params, q=None, k=None, v=None, out=None):
+    """Copy the (b, t, h) element strides of q, k, v, out into params (zeros: dense)."""
+    for name, t in (("stride_q", q), ("stride_k", k), ("stride_v", v), ("stride_o", out)):
+        dense = t is None or t.is_contiguous()
+        getattr(params, name)[:] = (0, 0, 0) if dense else (t.stride(0), t.stride(1), t.stride(2))
+    return params
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -160,8 +181,9 @@ def osdn_fwd_workspace_size(params: osdn_params) -> int:
 def osdn_fwd(params, q, k, v, beta, r, d0, S0, out, final_S, final_d, workspace, stream=None):
     """Raw C-ABI call: every tensor preallocated by the caller (device memory)."""
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().osdn_fwd(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(d0), _ptr(S0),
-                          _ptr(out), _ptr(final_S), _ptr(final_d), _ptr(workspace), ctypes.c_size_t(ws_bytes),
+    _set_strides(params, q, k, v, out)
+    _check(lib().osdn_fwd(ctypes.byref(params), _ptr_tok(q), _ptr_tok(k), _ptr_tok(v), _ptr(beta), _ptr(r), _ptr(d0),
+                          _ptr(S0), _ptr_tok(out), _ptr(final_S), _ptr(final_d), _ptr(workspace), ctypes.c_size_t(ws_bytes),
                           _stream(stream)))
 
 
@@ -171,20 +193,24 @@ def _ws_bytes(workspace):
 
 def osdn_fwd_scan(params, k, beta, r, d0, final_d, workspace, stream=None):
     """Raw C-ABI call of phase 1 (preconditioner scan into the workspace)."""
-    _check(lib().osdn_fwd_scan(ctypes.byref(params), _ptr(k), _ptr(beta), _ptr(r), _ptr(d0), _ptr(final_d),
+    _set_strides(params, k=k)
+    _check(lib().osdn_fwd_scan(ctypes.byref(params), _ptr_tok(k), _ptr(beta), _ptr(r), _ptr(d0), _ptr(final_d),
                                _ptr(workspace), ctypes.c_size_t(_ws_bytes(workspace)), _stream(stream)))
 
 
 def osdn_fwd_scan_diag(params, k, beta, r, d0, final_d, rho, q_geo, workspace, stream=None):
     """Raw C-ABI call of phase 1 with the residual-ratio diagnostic (rho, q_geo nullable)."""
-    _check(lib().osdn_fwd_scan_diag(ctypes.byref(params), _ptr(k), _ptr(beta), _ptr(r), _ptr(d0), _ptr(final_d),
+    _set_strides(params, k=k)
+    _check(lib().osdn_fwd_scan_diag(ctypes.byref(params), _ptr_tok(k), _ptr(beta), _ptr(r), _ptr(d0), _ptr(final_d),
                                     _ptr(rho), _ptr(q_geo), _ptr(workspace), ctypes.c_size_t(_ws_bytes(workspace)),
                                     _stream(stream)))
 
 
 def osdn_fwd_chunk(params, q, k, v, beta, S0, out, final_S, workspace, stream=None):
     """Raw C-ABI call of phase 2 (chunked delta rule reading the workspace)."""
-    _check(lib().osdn_fwd_chunk(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(out),
+    _set_strides(params, q, k, v, out)
+    _check(lib().osdn_fwd_chunk(ctypes.byref(params), _ptr_tok(q), _ptr_tok(k), _ptr_tok(v), _ptr(beta), _ptr(S0),
+                                _ptr_tok(out),
                                 _ptr(final_S), _ptr(workspace), ctypes.c_size_t(_ws_bytes(workspace)),
                                 _stream(stream)))
 
@@ -192,8 +218,9 @@ def osdn_fwd_chunk(params, q, k, v, beta, S0, out, final_S, workspace, stream=No
 def osdn_fwd_noalloc(params, q, k, v, beta, r, d0, S0, out, final_S, final_d, stream=None):
     """Raw C-ABI call of the forward that takes no workspace: the library uses
     its own fixed scratch array (see OSDN_NOALLOC_SCRATCH_BYTES in osdn.h)."""
-    _check(lib().osdn_fwd_noalloc(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(d0),
-                                  _ptr(S0), _ptr(out), _ptr(final_S), _ptr(final_d), _stream(stream)))
+    _set_strides(params, q, k, v, out)
+    _check(lib().osdn_fwd_noalloc(ctypes.byref(params), _ptr_tok(q), _ptr_tok(k), _ptr_tok(v), _ptr(beta), _ptr(r),
+                                  _ptr(d0), _ptr(S0), _ptr_tok(out), _ptr(final_S), _ptr(final_d), _stream(stream)))
 
 
 def osdn_step(params, q, k, v, beta, r, S, d, out, stream=None):
@@ -210,15 +237,18 @@ def osdn_step_ex(params, q, k, v, beta, r, d_anchor, S, d, out, stream=None):
 
 def osdn_fwd_gated(params, q, k, v, beta, r, alpha, d0, S0, out, final_S, final_d, workspace, stream=None):
     """Raw C-ABI call of the gated forward (alpha decay of the state)."""
-    _check(lib().osdn_fwd_gated(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(alpha),
-                                _ptr(d0), _ptr(S0), _ptr(out), _ptr(final_S), _ptr(final_d), _ptr(workspace),
+    _set_strides(params, q, k, v, out)
+    _check(lib().osdn_fwd_gated(ctypes.byref(params), _ptr_tok(q), _ptr_tok(k), _ptr_tok(v), _ptr(beta), _ptr(r),
+                                _ptr(alpha), _ptr(d0), _ptr(S0), _ptr_tok(out), _ptr(final_S), _ptr(final_d),
+                                _ptr(workspace),
                                 ctypes.c_size_t(_ws_bytes(workspace)), _stream(stream)))
 
 
 def osdn_fwd_chunk_gated(params, q, k, v, beta, alpha, S0, out, final_S, workspace, stream=None):
     """Raw C-ABI call of phase 2 of the gated forward."""
-    _check(lib().osdn_fwd_chunk_gated(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha),
-                                      _ptr(S0), _ptr(out), _ptr(final_S), _ptr(workspace),
+    _set_strides(params, q, k, v, out)
+    _check(lib().osdn_fwd_chunk_gated(ctypes.byref(params), _ptr_tok(q), _ptr_tok(k), _ptr_tok(v), _ptr(beta),
+                                      _ptr(alpha), _ptr(S0), _ptr_tok(out), _ptr(final_S), _ptr(workspace),
                                       ctypes.c_size_t(_ws_bytes(workspace)), _stream(stream)))
 
 

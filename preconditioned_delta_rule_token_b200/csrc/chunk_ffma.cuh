@@ -53,11 +53,16 @@ struct FfmaSmem {
     static constexpr size_t kBytes = sizeof(float) * (size_t)kFloats;
 };
 
+// Element strides of q, k, v and out over (b, t, h) (the scaled keys in the workspace are dense).
+struct FfmaStrides {
+    Tok3 q, k, v, o;
+};
+
 template <int DK, int DVT, typename Tin>
 __global__ void __launch_bounds__(256, 1)
 chunk_ffma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ kw,
                   const Tin* __restrict__ v, const Tin* __restrict__ beta, const float* __restrict__ S0,
-                  Tin* __restrict__ out, float* __restrict__ S_final, int B, int T, int H, int DV)
+                  Tin* __restrict__ out, float* __restrict__ S_final, int B, int T, int H, int DV, FfmaStrides st)
 {
     using L = FfmaSmem<DK, DVT>;
     constexpr int C = L::C, LDK = L::LDK, LDV = L::LDV, LDC = L::LDC;
@@ -88,9 +93,9 @@ chunk_ffma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
             const int t = idx / DK, i = idx % DK;
             float qv = 0.f, kv = 0.f, wv = 0.f;
             if (t < Tc) {
-                const size_t tok = ((size_t)b * T + c0 + t) * H + h;
-                qv = to_f32(q[tok * DK + i]);
-                kv = to_f32(k[tok * DK + i]);
+                const size_t tok = ((size_t)b * T + c0 + t) * H + h;   // the scaled keys are dense
+                qv = to_f32(q[st.q.at(b, c0 + t, h) + i]);
+                kv = to_f32(k[st.k.at(b, c0 + t, h) + i]);
                 wv = to_f32(kw[tok * DK + i]);
             }
             Qs[t * LDK + i] = qv; Ks[t * LDK + i] = kv; Ws[t * LDK + i] = wv;
@@ -98,7 +103,7 @@ chunk_ffma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
         for (int idx = tid; idx < C * DVT; idx += NT) {
             const int t = idx / DVT, j = idx % DVT;
             float vv = 0.f;
-            if (t < Tc) vv = to_f32(v[(((size_t)b * T + c0 + t) * H + h) * DV + v0 + j]);
+            if (t < Tc) vv = to_f32(v[st.v.at(b, c0 + t, h) + v0 + j]);
             Xs[t * LDV + j] = vv;
         }
         if (tid < C) bs[tid] = (tid < Tc) ? to_f32(beta[((size_t)b * T + c0 + tid) * H + h]) : 0.f;
@@ -162,10 +167,10 @@ chunk_ffma_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
             for (int i = 0; i < 4; ++i) {
                 const int t = ty + 16 * i;
                 if (t < Tc) {
-                    const size_t tok = ((size_t)b * T + c0 + t) * H + h;
+                    const int64_t o = st.o.at(b, c0 + t, h);
 #pragma unroll
                     for (int j = 0; j < DVT / 16; ++j)
-                        out[tok * DV + v0 + tx + 16 * j] = from_f32<Tin>(acc[i][j]);
+                        out[o + v0 + tx + 16 * j] = from_f32<Tin>(acc[i][j]);
                 }
             }
         }

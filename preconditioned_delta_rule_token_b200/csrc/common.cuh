@@ -66,6 +66,14 @@ template <> struct VecIO<2, __nv_bfloat16> {
     }
 };
 
+// Element strides of a token tensor [B, T, H, width] over (b, t, h); the last dimension is contiguous.
+struct Tok3 {
+    int64_t b, t, h;
+    __host__ __device__ __forceinline__ int64_t at(int64_t bb, int64_t tt, int64_t hh) const {
+        return bb * b + tt * t + hh * h;
+    }
+};
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

@@ -48,17 +48,43 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 size_t elem_size(int dtype) { return dtype == OSDN_BF16 ? 2 : 4; }
 
 // Common checks of the parameter block. need_T: the forward (T used).
-// Version 1 of osdn_params ended after eta; its callers get the fields added since at their defaults.
+// Versions 1 and 2 of osdn_params ended after eta and after apf_anchor; their callers get the fields
+// added since at their defaults.
 constexpr size_t kParamsV1Size = offsetof(osdn_params, apf_anchor);
+constexpr size_t kParamsV2Size = offsetof(osdn_params, stride_q);
 int anchor_of(const osdn_params* p) {
     return p->struct_size >= offsetof(osdn_params, apf_anchor) + sizeof(int32_t) && p->apf_anchor ? 1 : 0;
 }
 
+// Element strides of a token tensor [B, T, H, width] over (b, t, h), the caller's or the dense ones.
+int64_t all_zero(const int64_t (&s)[3]) { return !(s[0] | s[1] | s[2]); }
+osdn::Tok3 dense_tok3(const osdn_params* p, int width) {
+    return {(int64_t)p->T * p->H * width, (int64_t)p->H * width, (int64_t)width};
+}
+osdn::Tok3 tok3_of(const osdn_params* p, const int64_t (&s)[3], int width) {
+    if (p->struct_size < sizeof(osdn_params) || all_zero(s)) return dense_tok3(p, width);
+    return {s[0], s[1], s[2]};
+}
+struct TokStrides {
+    osdn::Tok3 q, k, v, o;
+};
+TokStrides strides_of(const osdn_params* p) {
+    return {tok3_of(p, p->stride_q, p->dk), tok3_of(p, p->stride_k, p->dk), tok3_of(p, p->stride_v, p->dv),
+            tok3_of(p, p->stride_o, p->dv)};
+}
+// True when every stride the caller gave is the dense one (or none was given).
+bool dense_layout(const osdn_params* p) {
+    const TokStrides s = strides_of(p);
+    auto same = [](const osdn::Tok3& a, const osdn::Tok3& b) { return a.b == b.b && a.t == b.t && a.h == b.h; };
+    return same(s.q, dense_tok3(p, p->dk)) && same(s.k, dense_tok3(p, p->dk)) && same(s.v, dense_tok3(p, p->dv)) &&
+           same(s.o, dense_tok3(p, p->dv));
+}
+
 int check_params(const osdn_params* p, bool need_T) {
     if (!p) return fail(OSDN_ERR_INVALID_ARG, "params is NULL");
-    if (p->struct_size != sizeof(osdn_params) && p->struct_size != kParamsV1Size)
-        return fail(OSDN_ERR_INVALID_ARG, "params.struct_size is %u, expected %zu (or %zu, version 1)",
-                    p->struct_size, sizeof(osdn_params), kParamsV1Size);
+    if (p->struct_size != sizeof(osdn_params) && p->struct_size != kParamsV2Size && p->struct_size != kParamsV1Size)
+        return fail(OSDN_ERR_INVALID_ARG, "params.struct_size is %u, expected %zu (or %zu, %zu: versions 2, 1)",
+                    p->struct_size, sizeof(osdn_params), kParamsV2Size, kParamsV1Size);
     if (p->B < 1 || p->H < 1) return fail(OSDN_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", p->B, p->H);
     if (need_T && p->T < 0) return fail(OSDN_ERR_INVALID_ARG, "T must be >= 0 (got %d)", p->T);
     if (p->dtype != OSDN_BF16 && p->dtype != OSDN_FP32)
@@ -72,6 +98,15 @@ int check_params(const osdn_params* p, bool need_T) {
     if (tokens * (double)(p->dk > p->dv ? p->dk : p->dv) > 9.0e18)
         return fail(OSDN_ERR_INVALID_ARG, "tensor sizes overflow 64-bit indexing");
     if ((double)p->B * p->H > 2147483647.0) return fail(OSDN_ERR_INVALID_ARG, "B * H exceeds the grid limit");
+    if (p->struct_size >= sizeof(osdn_params)) {
+        const int64_t* all[4] = {p->stride_q, p->stride_k, p->stride_v, p->stride_o};
+        for (const int64_t* st : all)
+            for (int i = 0; i < 3; ++i)
+                if (st[i] < 0 || (st[i] & 7) || st[i] > ((int64_t)1 << 38))
+                    return fail(OSDN_ERR_INVALID_ARG,
+                                "strides must be non-negative multiples of 8 elements below 2^38 (got %lld)",
+                                (long long)st[i]);
+    }
     return OSDN_OK;
 }
 
@@ -133,15 +168,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 4-D bf16 tensor map over [B, T, H, width] (dims listed innermost first), box
-// {box0, 1, box_tokens, 1}. The token dimension is its own dimension, so a box
+// 4-D bf16 tensor map over [B, T, H, width] (dims listed innermost first) with element strides s
+// over (b, t, h), box {box0, 1, box_tokens, 1}. The token dimension is its own dimension, so a box
 // that runs past T reads zeros instead of the next sequence.
 int make_token_map(CUtensorMap* m, const void* base, int B, int T, int H, int width, int box0,
-                   CUtensorMapSwizzle swizzle, int box_tokens = 64) {
+                   CUtensorMapSwizzle swizzle, int box_tokens, osdn::Tok3 s) {
     auto enc = tensor_map_encoder();
     if (!enc) return fail(OSDN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const cuuint64_t dims[4] = {(cuuint64_t)width, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)width * 2, (cuuint64_t)H * width * 2, (cuuint64_t)T * H * width * 2};
+    const cuuint64_t strides[3] = {(cuuint64_t)s.h * 2, (cuuint64_t)s.t * 2, (cuuint64_t)s.b * 2};
     const cuuint32_t box[4] = {(cuuint32_t)box0, 1, (cuuint32_t)box_tokens, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
@@ -156,12 +191,14 @@ int launch_chunk_wy(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfl
                     const __nv_bfloat16* beta, const float* S0, __nv_bfloat16* out, float* final_S,
                     const __nv_bfloat16* kw, cudaStream_t st, const __nv_bfloat16* alpha = nullptr) {
     CUtensorMap mq, mk, mkw, mv, mo;
+    const TokStrides s = strides_of(p);
+    const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
     int rc;
-    if ((rc = make_token_map(&mq, q, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-    if ((rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-    if ((rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-    if ((rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-    if ((rc = make_token_map(&mo, out, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    if ((rc = make_token_map(&mq, q, p->B, p->T, p->H, 128, 64, sw, 64, s.q))) return rc;
+    if ((rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, sw, 64, s.k))) return rc;
+    if ((rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, sw, 64, dense_tok3(p, 128)))) return rc;
+    if ((rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 64, sw, 64, s.v))) return rc;
+    if ((rc = make_token_map(&mo, out, p->B, p->T, p->H, 128, 64, sw, 64, s.o))) return rc;
     auto kern = alpha ? osdn::chunk_wy_kernel<true> : osdn::chunk_wy_kernel<false>;
     const size_t smem = osdn::WyLayout::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -178,9 +215,9 @@ int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bflo
                    const __nv_bfloat16* r, const float* d0, float* final_d, __nv_bfloat16* kw, float* rho,
                    float* q_geo, cudaStream_t st) {
     CUtensorMap mk, mkw;
-    int rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128);
+    int rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128, strides_of(p).k);
     if (rc) return rc;
-    rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128);
+    rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128, dense_tok3(p, 128));
     if (rc) return rc;
     auto kern = osdn::scan_ws_kernel<0>;
     const size_t smem = osdn::ScanLayout::kBytes;
@@ -211,11 +248,12 @@ int launch_scan(const osdn_params* p, const Tin* k, const Tin* beta, const Tin* 
     }
     const int units = p->B * p->H;
     const dim3 grid((units + 3) / 4);
+    const osdn::Tok3 sk = strides_of(p).k;
     if (p->dk == 128)
-        osdn::scan_seq_kernel<128, Tin><<<grid, 128, 0, st>>>(k, beta, r, d0, kw, final_d, rho, q_geo, p->B, p->T,
+        osdn::scan_seq_kernel<128, Tin><<<grid, 128, 0, st>>>(k, sk, beta, r, d0, kw, final_d, rho, q_geo, p->B, p->T,
                                                                p->H, p->eta, anchor_of(p));
     else
-        osdn::scan_seq_kernel<64, Tin><<<grid, 128, 0, st>>>(k, beta, r, d0, kw, final_d, rho, q_geo, p->B, p->T,
+        osdn::scan_seq_kernel<64, Tin><<<grid, 128, 0, st>>>(k, sk, beta, r, d0, kw, final_d, rho, q_geo, p->B, p->T,
                                                               p->H, p->eta, anchor_of(p));
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
@@ -233,19 +271,21 @@ int launch_chunk(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v,
     const int units = p->B * p->H;
     constexpr int DVT = 64;
     const dim3 grid(units, p->dv / DVT);
+    const TokStrides ts = strides_of(p);
+    const osdn::FfmaStrides s{ts.q, ts.k, ts.v, ts.o};
     cudaError_t e;
     if (p->dk == 128) {
         auto kern = osdn::chunk_ffma_kernel<128, DVT, Tin>;
         const size_t smem = osdn::FfmaSmem<128, DVT>::kBytes;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
             return cuda_fail(e, "chunk kernel attribute");
-        kern<<<grid, 256, smem, st>>>(q, k, kw, v, beta, S0, out, final_S, p->B, p->T, p->H, p->dv);
+        kern<<<grid, 256, smem, st>>>(q, k, kw, v, beta, S0, out, final_S, p->B, p->T, p->H, p->dv, s);
     } else {
         auto kern = osdn::chunk_ffma_kernel<64, DVT, Tin>;
         const size_t smem = osdn::FfmaSmem<64, DVT>::kBytes;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
             return cuda_fail(e, "chunk kernel attribute");
-        kern<<<grid, 256, smem, st>>>(q, k, kw, v, beta, S0, out, final_S, p->B, p->T, p->H, p->dv);
+        kern<<<grid, 256, smem, st>>>(q, k, kw, v, beta, S0, out, final_S, p->B, p->T, p->H, p->dv, s);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "chunk launch");
     return OSDN_OK;
@@ -598,6 +638,9 @@ int osdn_step_ex(const osdn_params* p, const void* q, const void* k, const void*
     t_last_error.clear();
     int rc = check_params(p, false);
     if (rc) return rc;
+    if (p->struct_size >= sizeof(osdn_params) &&
+        !(all_zero(p->stride_q) && all_zero(p->stride_k) && all_zero(p->stride_v) && all_zero(p->stride_o)))
+        return fail(OSDN_ERR_UNSUPPORTED, "the decode step takes dense tensors only (strides must be zero)");
     if (!q || !k || !v || !beta || !S || !d || !out)
         return fail(OSDN_ERR_INVALID_ARG, "q, k, v, beta, S, d and out must not be NULL");
     const void* ptrs[] = {q, k, v, beta, r, d_anchor, S, d, out};
@@ -619,6 +662,9 @@ int osdn_step_gated(const osdn_params* p, const void* q, const void* k, const vo
     t_last_error.clear();
     int rc = check_params(p, false);
     if (rc) return rc;
+    if (p->struct_size >= sizeof(osdn_params) &&
+        !(all_zero(p->stride_q) && all_zero(p->stride_k) && all_zero(p->stride_v) && all_zero(p->stride_o)))
+        return fail(OSDN_ERR_UNSUPPORTED, "the decode step takes dense tensors only (strides must be zero)");
     if (!q || !k || !v || !beta || !alpha || !S || !d || !out)
         return fail(OSDN_ERR_INVALID_ARG, "q, k, v, beta, alpha, S, d and out must not be NULL");
     const void* ptrs[] = {q, k, v, beta, r, alpha, d_anchor, S, d, out};
@@ -655,6 +701,7 @@ int osdn_bwd(const osdn_params* p, const void* q, const void* k, const void* v, 
     t_last_error.clear();
     int rc = check_params(p, true);
     if (rc) return rc;
+    if (!dense_layout(p)) return fail(OSDN_ERR_UNSUPPORTED, "the backward takes dense tensors only");
     const void* ptrs[] = {q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta, dr, dd0, dS0,
                           workspace};
     for (const void* x : ptrs)

@@ -21,7 +21,7 @@ namespace osdn {
 
 template <int DK, typename Tin>
 __global__ void __launch_bounds__(128)
-scan_seq_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const Tin* __restrict__ r,
+scan_seq_kernel(const Tin* __restrict__ k, Tok3 sk, const Tin* __restrict__ beta, const Tin* __restrict__ r,
                 const float* __restrict__ d0, Tin* __restrict__ kw, float* __restrict__ d_final,
                 float* __restrict__ rho, float* __restrict__ q_geo, int B, int T, int H, float eta, int anchor)
 {
@@ -48,14 +48,14 @@ scan_seq_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const T
     float bc = 0.f, rc = 1.f, bn = 0.f, rn = 1.f;
     float log_rho = 0.f;                             // sum over tokens of log rho_t
     if (T > 0) {
-        VecIO<PER, Tin>::load(k + tok * DK + lane * PER, kc);
+        VecIO<PER, Tin>::load(k + sk.at(b, 0, h) + lane * PER, kc);
         bc = to_f32(beta[tok]);
         if (r) rc = to_f32(r[tok]);
     }
     for (int t = 0; t < T; ++t) {
         const size_t nxt = tok + tok_stride;
         if (t + 1 < T) {                               // prefetch the next token
-            VecIO<PER, Tin>::load(k + nxt * DK + lane * PER, kn);
+            VecIO<PER, Tin>::load(k + sk.at(b, t + 1, h) + lane * PER, kn);
             bn = to_f32(beta[nxt]);
             if (r) rn = to_f32(r[nxt]);
         }

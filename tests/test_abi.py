@@ -30,21 +30,45 @@ def test_library_exports_every_declared_symbol(osdn_lib):
     lib = ctypes.CDLL(osdn_lib.LIB_PATH)
     for name in sorted(_declared_functions()):
         assert hasattr(lib, name), name
-    assert lib.osdn_abi_version() == 2
+    assert lib.osdn_abi_version() == 3
 
 
-def test_version_1_params_are_accepted(osdn_lib):
-    """osdn_params of ABI version 1 ended after eta (36 bytes); such callers are
-    accepted and get the plain APF retention (apf_anchor = 0)."""
+def test_earlier_params_versions_are_accepted(osdn_lib):
+    """osdn_params of ABI version 1 ended after eta (36 bytes) and version 2 after
+    apf_anchor (40 bytes); such callers are accepted (plain APF for version 1, the
+    dense layout for both). Version 3 appends the (b, t, h) element strides of q,
+    k, v and out (136 bytes); any other size is refused."""
     L = osdn_lib.lib()
     n = ctypes.c_size_t(0)
-    assert ctypes.sizeof(osdn_lib.osdn_params) == 40
+    assert ctypes.sizeof(osdn_lib.osdn_params) == 136
+    assert osdn_lib.osdn_params.stride_q.offset == 40
     p = _params(osdn_lib)
-    p.struct_size = 36
-    p.apf_anchor = 1            # beyond a version-1 struct: must be ignored
-    assert L.osdn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    for size in (36, 40, 136):
+        p.struct_size = size
+        p.apf_anchor = 1
+        assert L.osdn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0, size
     p.struct_size = 44
     assert L.osdn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == osdn_lib.OSDN_ERR_INVALID_ARG
+
+
+def test_strides_are_checked_on_the_host(osdn_lib):
+    """Strides are non-negative multiples of 8 elements; the decode step and the
+    backward take dense tensors only."""
+    L = osdn_lib.lib()
+    n = ctypes.c_size_t(0)
+    fake = ctypes.c_void_p(1 << 20)             # never dereferenced: checks fail first
+    for bad in ((4, 0, 0), (-8, 0, 0), (0, 0, 1 << 40)):
+        p = _params(osdn_lib)
+        p.stride_k[:] = bad
+        assert L.osdn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == osdn_lib.OSDN_ERR_INVALID_ARG, bad
+        assert "stride" in osdn_lib.get_last_error()
+    p = _params(osdn_lib)
+    p.stride_q[:] = (100 * 3 * 384, 3 * 384, 384)   # q as a column slice of a fused [B, T, H, 384] projection
+    assert L.osdn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    assert L.osdn_step(ctypes.byref(p), fake, fake, fake, fake, None, fake, fake, fake, None) == \
+        osdn_lib.OSDN_ERR_UNSUPPORTED
+    assert L.osdn_bwd(ctypes.byref(p), *([fake] * 4), None, None, None, fake, None, None, *([fake] * 4), None, None,
+                      None, fake, ctypes.c_size_t(1 << 40), None) == osdn_lib.OSDN_ERR_UNSUPPORTED
 
 
 def _params(osdn_lib, **kw):
@@ -96,6 +120,17 @@ def test_binding_refuses_cpu_tensors(osdn_lib):
     x = torch.zeros((1, 4, 1, 64), dtype=torch.bfloat16)
     with pytest.raises(pk.OsdnError):
         pk.forward(x, x, x, torch.zeros((1, 4, 1), dtype=torch.bfloat16))
+
+
+def test_binding_copies_the_strides_of_views(osdn_lib):
+    """A column slice of a fused projection passes its (b, t, h) strides in the
+    parameter block; a contiguous tensor passes zeros (dense)."""
+    import torch
+    fused = torch.zeros((2, 5, 3, 3 * 64))
+    q, k = fused[..., :64], fused[..., 64:128]
+    p = _params(osdn_lib, T=5, dk=64, dv=64)
+    osdn_lib._set_strides(p, q=q, k=k.contiguous())
+    assert tuple(p.stride_q) == (5 * 3 * 192, 3 * 192, 192) and tuple(p.stride_k) == (0, 0, 0)
 
 
 def test_backward_workspace_and_argument_checks(osdn_lib):

@@ -132,6 +132,37 @@ def test_more_units_than_sms_every_unit():
     assert max(errs) <= BF16_TOL, errs
 
 
+@pytest.mark.parametrize("dtype,dk,dv", [(W.BF16, 128, 128), (W.FP32, 128, 128), (W.BF16, 64, 128)])
+def test_qkv_read_in_place_from_a_fused_projection(dtype, dk, dv):
+    """q, k and v as column slices of one fused projection [B, T, H, 2 dk + dv]
+    (strided views, last dimension contiguous), and out written into a column
+    slice of a wider buffer: the library reads and writes them in place through
+    the strides of osdn_params, with the result of dense inputs and the oracle."""
+    import preconditioned_delta_rule_token_b200 as pk
+    w = W.Workload("fused qkv", 2, 3, 150, dk, dv, 64, dtype, True, "gaussian", eta=0.1, seed=61, d0="uniform",
+                   S0="normal")
+    inp = W.make_forward_inputs(w)
+    g = {k_: _dev(v_) for k_, v_ in inp.items()}
+    fused = torch.cat([g["q"], g["k"], g["v"]], dim=-1)                    # [B, T, H, 2 dk + dv]
+    q, k, v = fused[..., :dk], fused[..., dk:2 * dk], fused[..., 2 * dk:]
+    assert not q.is_contiguous() and q.stride(-1) == 1
+    wide = torch.full((w.B, w.T, w.H, dv + 64), 7.0, dtype=g["q"].dtype, device=q.device)
+    out = wide[..., 32:32 + dv]
+    p = pk.make_params(w.B, w.T, w.H, dk, dv, g["k"].dtype, w.eta, w.chunk)
+    S = torch.empty((w.B, w.H, dv, dk), dtype=torch.float32, device=q.device)
+    d = torch.empty((w.B, w.H, dk), dtype=torch.float32, device=q.device)
+    ws = torch.empty(pk.osdn_fwd_workspace_size(p), dtype=torch.uint8, device=q.device)
+    pk.osdn_fwd(p, q, k, v, g["beta"], g["r"], g["d0"], g["S0"], out, S, d, ws)
+    assert pk.osdn_sync_status() == 0
+    dense = pk.forward(g["q"], g["k"], g["v"], g["beta"], g["r"], g["d0"], g["S0"], eta=w.eta)
+    torch.cuda.synchronize()
+    assert torch.equal(out, dense[0]) and torch.equal(S, dense[1]) and torch.equal(d, dense[2])
+    assert torch.all(wide[..., :32] == 7.0) and torch.all(wide[..., 32 + dv:] == 7.0)   # nothing outside out
+    got = (out.float().cpu().numpy(), S.cpu().numpy(), d.cpu().numpy())
+    tol = FP32_TOL if dtype == W.FP32 else BF16_TOL
+    assert max(_errs(got, _oracle(inp, w.eta))) <= tol
+
+
 def test_zero_tokens_returns_initial_state():
     import preconditioned_delta_rule_token_b200 as pk
     w = W.Workload("t0", 2, 2, 0, 128, 128, 64, W.BF16, True, d0="uniform", S0="normal", seed=5)
