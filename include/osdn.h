@@ -212,7 +212,7 @@ int osdn_step_gated(const osdn_params *p,
                     void *cuda_stream);
 
 /* Backward (training). The pages give no backward pass; this is the exact
- * reverse-mode derivative of osdn_fwd (plain or anchored APF, not gated) for
+ * reverse-mode derivative of osdn_fwd (plain or anchored APF) for
  *     L = sum <dout, out> + <dS_final, final_S> + <dd_final, final_d>,
  * through both phases: the chunked delta rule with the scaled write key
  * (technical summary section 2.1) and the preconditioner recurrence of d
@@ -230,8 +230,8 @@ int osdn_step_gated(const osdn_params *p,
  * workspace: osdn_bwd_workspace_size() bytes, 16-byte aligned, no
  * initialisation needed; it holds fp32 intermediates: d_t for every token
  * (dk values) and, per 64-token chunk and head (the last chunk padded),
- * 64 * (4 dk + 3 dv + 2 * 64 + 1) values plus two states (2 dv dk values),
- * i.e. about (5 dk + 3 dv + 129) * 4 bytes per token and head plus
+ * 64 * (4 dk + 3 dv + 2 * 64 + 2) values plus two states (2 dv dk values),
+ * i.e. about (5 dk + 3 dv + 130) * 4 bytes per token and head plus
  * 8 dv dk bytes per chunk and head (3.5 GB at B8 T4096 H16 dk = dv = 128).
  * T = 0 copies dS_final to dS0 and dd_final to dd0 (zeros when NULL).
  * Errors: OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED, OSDN_ERR_CUDA. */
@@ -246,6 +246,31 @@ int osdn_bwd(const osdn_params *p,
              float *dd0, float *dS0,
              void *workspace, size_t workspace_bytes,
              void *cuda_stream);
+
+/* osdn_bwd_gated: the reverse-mode derivative of gated OSDN, the forward that
+ * osdn_fwd_gated computes (the recurrence stated above: the OSDN write
+ * applied to the decayed state alpha_t S_{t-1}), for the same L as osdn_bwd.
+ * Arguments as osdn_bwd,
+ * plus alpha [B, T, H] (input dtype, every value in [0, 1]; not NULL when
+ * T > 0) and dalpha [B, T, H] (input dtype, overwritten; not NULL when T > 0).
+ * Unlike osdn_fwd_gated it takes every dtype and width osdn_bwd takes, plain
+ * or anchored APF (the gate does not enter the preconditioner recurrence).
+ * Inside a 64-token chunk the gate products run as powers of two of sums of
+ * log2 alpha, each term clamped at -120, as in the forward: dalpha is the
+ * derivative with respect to alpha_eff = max(alpha, 2^-120), and it stays
+ * finite (and accurate) for alpha = 0. The workspace is osdn_bwd's, of
+ * osdn_bwd_workspace_size() bytes.
+ * Errors: those of osdn_bwd; OSDN_ERR_INVALID_ARG when alpha or dalpha is
+ * NULL with T > 0. */
+int osdn_bwd_gated(const osdn_params *p,
+                   const void *q, const void *k, const void *v,
+                   const void *beta, const void *r, const void *alpha,
+                   const float *d0, const float *S0,
+                   const void *dout, const float *dS_final, const float *dd_final,
+                   void *dq, void *dk, void *dv, void *dbeta, void *dr,
+                   void *dalpha, float *dd0, float *dS0,
+                   void *workspace, size_t workspace_bytes,
+                   void *cuda_stream);
 
 /* Largest scratch osdn_fwd_noalloc can use: B * T * H * dk * element size
  * (2 bytes for bf16, 4 for fp32) must not exceed this. */

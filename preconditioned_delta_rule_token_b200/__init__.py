@@ -19,9 +19,9 @@ from ._binding import (OSDN_BF16, OSDN_ERR_CUDA, OSDN_ERR_INVALID_ARG, OSDN_ERR_
                        osdn_fwd_chunk, osdn_fwd_scan, osdn_fwd_scan_diag,
                        osdn_fwd_workspace_size, osdn_params, osdn_set_wait_limit_ns, osdn_step, osdn_step_ex,
                        osdn_fwd_gated, osdn_fwd_chunk_gated, osdn_step_gated,
-                       osdn_bwd, osdn_bwd_workspace_size, osdn_sync_status)
+                       osdn_bwd, osdn_bwd_gated, osdn_bwd_workspace_size, osdn_sync_status)
 
-__all__ = ["forward", "backward", "step", "osdn_bwd", "osdn_bwd_workspace_size", "residual_ratio", "osdn_fwd_scan_diag", "osdn_fwd", "osdn_fwd_scan", "osdn_fwd_chunk", "osdn_step", "osdn_fwd_workspace_size", "osdn_sync_status",
+__all__ = ["forward", "backward", "step", "osdn_bwd", "osdn_bwd_gated", "osdn_bwd_workspace_size", "residual_ratio", "osdn_fwd_scan_diag", "osdn_fwd", "osdn_fwd_scan", "osdn_fwd_chunk", "osdn_step", "osdn_fwd_workspace_size", "osdn_sync_status",
            "osdn_set_wait_limit_ns", "osdn_step_ex",
            "osdn_fwd_gated", "osdn_fwd_chunk_gated", "osdn_step_gated",
            "osdn_params", "make_params", "get_last_error", "OsdnError", "build", "LIB_PATH",
@@ -53,11 +53,12 @@ def forward(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, chunk=64, workspa
 
 
 def backward(q, k, v, beta, dout, r=None, d0=None, S0=None, dS_final=None, dd_final=None, eta=1e-2, chunk=64,
-             workspace=None, stream=None, apf_anchor=False):
+             workspace=None, stream=None, apf_anchor=False, alpha=None):
     """Gradients of L = sum(dout * out) + sum(dS_final * final_S) + sum(dd_final * final_d) for the
-    forward() with the same inputs (plain or anchored APF). dout [B,T,H,dv] in the input dtype;
-    dS_final [B,H,dv,dk], dd_final [B,H,dk] fp32 or None (= 0). Returns a dict with dq, dk, dv,
-    dbeta, dr (None without r) in the input dtype and dd0 [B,H,dk], dS0 [B,H,dv,dk] fp32."""
+    forward() with the same inputs (plain or anchored APF; gated OSDN when alpha [B,T,H] is given).
+    dout [B,T,H,dv] in the input dtype; dS_final [B,H,dv,dk], dd_final [B,H,dk] fp32 or None (= 0).
+    Returns a dict with dq, dk, dv, dbeta, dr (None without r), dalpha (None without alpha) in the
+    input dtype and dd0 [B,H,dk], dS0 [B,H,dv,dk] fp32."""
     B, T, H, dk = k.shape
     dv = v.shape[-1]
     p = make_params(B, T, H, dk, dv, k.dtype, eta, chunk, apf_anchor)
@@ -68,8 +69,14 @@ def backward(q, k, v, beta, dout, r=None, d0=None, S0=None, dS_final=None, dd_fi
          "dS0": torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)}
     if workspace is None:
         workspace = torch.empty(osdn_bwd_workspace_size(p), dtype=torch.uint8, device=dev)
-    osdn_bwd(p, q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, g["dq"], g["dk"], g["dv"], g["dbeta"], g["dr"],
-             g["dd0"], g["dS0"], workspace, stream)
+    if alpha is None:
+        osdn_bwd(p, q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, g["dq"], g["dk"], g["dv"], g["dbeta"],
+                 g["dr"], g["dd0"], g["dS0"], workspace, stream)
+        g["dalpha"] = None
+    else:
+        g["dalpha"] = torch.empty_like(alpha)
+        osdn_bwd_gated(p, q, k, v, beta, r, alpha, d0, S0, dout, dS_final, dd_final, g["dq"], g["dk"], g["dv"],
+                       g["dbeta"], g["dr"], g["dalpha"], g["dd0"], g["dS0"], workspace, stream)
     return g
 
 

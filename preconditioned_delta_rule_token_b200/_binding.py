@@ -105,6 +105,8 @@ def lib():
         L.osdn_bwd_workspace_size.restype = ctypes.c_int
         L.osdn_bwd.argtypes = [P] + [vp] * 17 + [vp, sz, vp]
         L.osdn_bwd.restype = ctypes.c_int
+        L.osdn_bwd_gated.argtypes = [P] + [vp] * 20 + [sz, vp]
+        L.osdn_bwd_gated.restype = ctypes.c_int
         L.osdn_sync_status.argtypes = [vp]
         L.osdn_sync_status.restype = ctypes.c_int
         L.osdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
@@ -271,6 +273,15 @@ def osdn_bwd(params, q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, dq, dk,
                           _ptr(dout), _ptr(dS_final), _ptr(dd_final), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta),
                           _ptr(dr), _ptr(dd0), _ptr(dS0), _ptr(workspace), ctypes.c_size_t(_ws_bytes(workspace)),
                           _stream(stream)))
+
+
+def osdn_bwd_gated(params, q, k, v, beta, r, alpha, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta, dr, dalpha,
+                   dd0, dS0, workspace, stream=None):
+    """Raw C-ABI call of the gated backward: as osdn_bwd plus alpha [B,T,H] and dalpha [B,T,H]."""
+    _check(lib().osdn_bwd_gated(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), _ptr(alpha),
+                                _ptr(d0), _ptr(S0), _ptr(dout), _ptr(dS_final), _ptr(dd_final), _ptr(dq), _ptr(dk),
+                                _ptr(dv), _ptr(dbeta), _ptr(dr), _ptr(dalpha), _ptr(dd0), _ptr(dS0), _ptr(workspace),
+                                ctypes.c_size_t(_ws_bytes(workspace)), _stream(stream)))
 
 
 def osdn_sync_status(stream=None) -> int:

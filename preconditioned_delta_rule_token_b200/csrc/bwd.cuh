@@ -29,13 +29,28 @@
 // chunk-block layout [unit][chunk][row][col], fp32):
 //   bwd_dtraj   d_t for every token (token-serial: one CTA per unit, a chain warp
 //               and three warps that stage the next slab of tokens);
-//   bwd_prep    per chunk: Kw, T, W, U0, P;
+//   bwd_prep    per chunk: Kw, T, W, U0, P (gated: and log2 gamma);
 //   bwd_state_f per (unit, dv tile): S at every chunk start, Vn;
 //   bwd_state_b per (unit, dv tile), chunks in reverse: dS' at every chunk end, dVn, dS0;
 //   bwd_grads   per chunk: dQ, dV (dv tiles in turn), then dA, dK, dKw, dD and the
-//               chunk part of dbeta;
+//               chunk part of dbeta (gated: and dalpha);
 //   bwd_dchain  token-serial reverse of the d recurrence, staged as bwd_dtraj:
 //               dk, dbeta, dr, dd0.
+// Gated OSDN (alpha given; the state decayed by alpha_t before token t's write):
+// with gamma the cumulative gate within the chunk, R_tj = gamma_t / gamma_j and
+// rho_j = gamma_C / gamma_j (every factor at most 1, taken as 2 to differences of
+// the in-chunk cumulative log2 alpha, each term clamped at -120, as in the forward),
+//   forward:  A = strict_tril(Kb Kw^T) (.) R, W = T diag(gamma) Kb, P = tril(Q Kw^T) (.) R,
+//             O = diag(gamma) Q S^T + P Vn, S' = gamma_C S + Vn^T diag(rho) Kw;
+//   backward: dVn = P^T dO + diag(rho) Kw dS'^T, dS = gamma_C dS' + dO^T diag(gamma) Q - dVn^T W,
+//             dQ = diag(gamma) dO S + (dP (.) R) Kw, dKw = diag(rho) Vn dS' + (dP (.) R)^T Q + ...,
+//             dT = dW (diag(gamma) Kb)^T + ..., dA (.) R in place of dA downstream,
+//             dK = diag(beta gamma) T^T dW + ..., dbeta gets gamma (.) rowdot(T^T dW, K),
+//   and the adjoint of G = ln gamma,
+//     dG_t = gamma_t <(dO S)_t, Q_t> + gamma_t beta_t <(T^T dW)_t, K_t> + sum_j X_tj - sum_j X_jt
+//            - Y_t + [t = last] (gamma_C <dS', S> + sum_j Y_j),
+//     X = dA (.) diag(beta) K Kw^T (.) R + dP (.) P,  Y_j = rho_j <(Vn dS')_j, Kw_j>,
+//   gives dalpha_m = (sum_{t >= m} dG_t) / alpha_m (chunk-local: gamma restarts every chunk).
 // Rows of S are independent given the chunk matrices, so the two state passes
 // split dv into tiles with no exchange.  The contractions run on mma.sync
 // m16n8k8 tf32 with fp32 accumulation; for fp32 inputs every product uses the
@@ -213,7 +228,7 @@ __device__ __forceinline__ void prefetch_rows(const void* p, size_t stride_bytes
 
 // Workspace layout of one backward call (fp32 regions, 256-byte aligned).
 struct Layout {
-    size_t d_all, kw, tinv, w, u0, p, ckS, ckdS, vn, dvn, dd, dkp, dbp, total;
+    size_t d_all, kw, tinv, w, u0, p, ckS, ckdS, vn, dvn, dd, dkp, dbp, lg, total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -237,12 +252,46 @@ inline Layout make_layout(int B, int T, int H, int DK, int DV) {
     L.dd = take(f * ch * C * DK);
     L.dkp = take(f * ch * C * DK);
     L.dbp = take(f * ch * C);
+    L.lg = take(f * ch * C);   // gated: log2 gamma_t of every chunk
     L.total = o;
     return L;
 }
 
 template <typename Tin>
 __device__ __forceinline__ float ld_or0(const Tin* p, size_t i, bool ok) { return ok ? to_f32(p[i]) : 0.f; }
+
+// 2^x (the special-function unit; results below the normal range flush to 0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Warp 0 of the CTA: gs[t] = sum_{m <= t} max(log2 alpha_m, -120) over the C tokens of a chunk
+// (alpha = 1 past its Tc valid tokens), the in-chunk cumulative log2 gate of the forward.
+template <typename Tin>
+__device__ __forceinline__ void chunk_log2_gates(float* gs, const Tin* alpha, size_t tok0, size_t tstride, int Tc,
+                                                 int lane, float* ls = nullptr) {
+    static_assert(C == 64, "two tokens per lane");
+    float l[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int t = 2 * lane + e;
+        l[e] = t < Tc ? fmaxf(log2f(to_f32(alpha[tok0 + t * tstride])), -120.f) : 0.f;
+    }
+    float x = l[0] + l[1];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    gs[2 * lane] = x - l[1];
+    gs[2 * lane + 1] = x;
+    if (ls) {   // and the clamped log2 alpha_t of every token
+        ls[2 * lane] = l[0];
+        ls[2 * lane + 1] = l[1];
+    }
+}
 
 // 16-byte vector load of 4 fp32 or 8 bf16 values as fp32.
 __device__ __forceinline__ void load16(const float* p, float (&x)[4]) {
@@ -465,13 +514,14 @@ bwd_dtraj_kernel(const Tin* __restrict__ k, const Tin* __restrict__ beta, const 
 template <int DK, int DV>
 struct PrepSmem {
     static constexpr int LDK = DK + 4, LDX = (DK > DV ? DK : DV) + 4;
-    static constexpr size_t kBytes = sizeof(float) * (size_t)(2 * C * LDK + C * LDX + 2 * C * LDC + C);
+    static constexpr size_t kBytes = sizeof(float) * (size_t)(2 * C * LDK + C * LDX + 2 * C * LDC + 2 * C);
 };
 
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(NTHR, 1)
 bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
-                const Tin* __restrict__ beta, float* __restrict__ ws, Layout L, int B, int T, int H, int NC)
+                const Tin* __restrict__ beta, const Tin* __restrict__ alpha, float* __restrict__ ws, Layout L, int B,
+                int T, int H, int NC)
 {
     constexpr bool SPLIT = std::is_same<Tin, float>::value;
     using SM = PrepSmem<DK, DV>;
@@ -483,6 +533,8 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     float* As = X + C * LDX;         // [C][LDC] strict_tril(Kb Kw^T)
     float* Ts = As + C * LDC;        // [C][LDC] (I + A)^{-1}
     float* bs = Ts + C * LDC;        // [C] beta
+    float* gs = bs + C;              // [C] gated: log2 gamma_t
+    const bool gated = alpha != nullptr;
 
     const int tid = threadIdx.x;
     const size_t nchunks = (size_t)B * H * NC;
@@ -512,6 +564,12 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
         prefetch_rows(d_all + tokn * DK, tstride * DK * sizeof(float), tcn, DK * sizeof(float));
     }
     if (tid < C) bs[tid] = ld_or0(beta, tok0 + tid * tstride, tid < Tc);
+    if (gated && tid < 32) {
+        chunk_log2_gates(gs, alpha, tok0, tstride, Tc, tid);
+        __syncwarp();
+        ws[L.lg / sizeof(float) + cid * C + 2 * tid] = gs[2 * tid];
+        ws[L.lg / sizeof(float) + cid * C + 2 * tid + 1] = gs[2 * tid + 1];
+    }
     async_tile<C, DK>(Kw, LDK, d_all + tok0 * DK, tstride * DK, Tc);     // d_t for now
     load_tile<C, DK>(Kb, LDK, k + tok0 * DK, tstride * DK, Tc);
     cp_async_wait_all();
@@ -527,6 +585,10 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     store_rows<C, DK>(kw_g, DK, Kw, LDK);
     cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{Kb}, Mat<1, LDK>{Kw},
                     [&](int m, int n, float x0, float x1) {
+                        if (gated) {   // x R_mn = gamma_m / gamma_n
+                            x0 *= ex2(gs[m] - gs[n]);
+                            x1 *= ex2(gs[m] - gs[n + 1]);
+                        }
                         store2(As + m * LDC + n, n < m ? x0 : 0.f, n + 1 < m ? x1 : 0.f);
                     });
     __syncthreads();
@@ -551,6 +613,8 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
         static_assert(LDC == tri::LD, "the blocked inverse takes the 68-float row stride");
         tri::tril_inv64_inplace(As, tid >> 5, tid & 31, [] { asm volatile("bar.sync 1, 128;" ::: "memory"); });
     }
+    if (gated)   // W = T diag(gamma) Kb: Kb rows x gamma_t (the Gram above used them unscaled)
+        for (int idx = tid; idx < C * DK; idx += NTHR) Kb[(idx / DK) * LDK + idx % DK] *= ex2(gs[idx / DK]);
     __syncthreads();
     store_rows<C, C>(t_g, C, Tm, LDC);
     cta_gemm<SPLIT>(C, DK, C, Mat<LDC, 1>{Tm}, Mat<LDK, 1>{Kb},
@@ -562,6 +626,10 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     __syncthreads();
     cta_gemm<SPLIT>(C, C, DK, Mat<LDX, 1>{X}, Mat<1, LDK>{Kw},
                     [&](int m, int n, float x0, float x1) {
+                        if (gated) {
+                            x0 *= ex2(gs[m] - gs[n]);
+                            x1 *= ex2(gs[m] - gs[n + 1]);
+                        }
                         store2(p_g + m * C + n, n <= m ? x0 : 0.f, n + 1 <= m ? x1 : 0.f);
                     });
     }
@@ -572,13 +640,13 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
 template <int DK, int DVT>
 struct StateSmem {
     static constexpr int LDK = DK + 4, LDT = DVT + 4;
-    static constexpr size_t kFwdBytes = sizeof(float) * (size_t)(DVT * LDK + 2 * C * LDK + C * LDT);
-    static constexpr size_t kBwdBytes = sizeof(float) * (size_t)(DVT * LDK + C * LDC + 2 * C * LDT + 2 * C * LDK);
+    static constexpr size_t kFwdBytes = sizeof(float) * (size_t)(DVT * LDK + 2 * C * LDK + C * LDT + C);
+    static constexpr size_t kBwdBytes = sizeof(float) * (size_t)(DVT * LDK + C * LDC + 2 * C * LDT + 2 * C * LDK + C);
 };
 
 template <int DK, int DV, int DVT, typename Tin>
 __global__ void __launch_bounds__(NTHR, 1)
-bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout L, int NC)
+bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout L, int NC, int gated)
 {
     constexpr bool SPLIT = std::is_same<Tin, float>::value;
     using SM = StateSmem<DK, DVT>;
@@ -588,6 +656,7 @@ bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout 
     float* Ws = Ss + DVT * LDK;      // [C][LDK] W
     float* Kws = Ws + C * LDK;       // [C][LDK] Kw
     float* Vs = Kws + C * LDK;       // [C][LDT] U0, then Vn (columns of the tile)
+    float* gs = Vs + C * LDT;        // [C] gated: log2 gamma_t
 
     const int tid = threadIdx.x;
     const int unit = blockIdx.x / NTILE, v0 = (blockIdx.x % NTILE) * DVT;
@@ -612,6 +681,7 @@ bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout 
         async_block<C, DK>(Ws, LDK, w_g);
         async_block<C, DK>(Kws, LDK, kw_g);
         async_tile<C, DVT>(Vs, LDT, u_g + v0, (size_t)DV);
+        if (gated && tid < C) gs[tid] = ws[L.lg / sizeof(float) + cid * C + tid];
         cp_async_wait_all();
         __syncthreads();
         cta_gemm<SPLIT>(C, DVT, DK, Mat<LDK, 1>{Ws}, Mat<1, LDK>{Ss}, [&](int m, int n, float x0, float x1) {
@@ -621,6 +691,12 @@ bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout 
             store2(vn_g + m * DV + v0 + n, vn0, vn1);
         });
         __syncthreads();
+        if (gated) {   // S' = gamma_C S + Vn^T diag(rho) Kw
+            const float gl = gs[C - 1], gc = ex2(gl);
+            for (int idx = tid; idx < DVT * DK; idx += NTHR) Ss[(idx / DK) * LDK + idx % DK] *= gc;
+            for (int idx = tid; idx < C * DK; idx += NTHR) Kws[(idx / DK) * LDK + idx % DK] *= ex2(gl - gs[idx / DK]);
+            __syncthreads();
+        }
         cta_gemm<SPLIT>(DVT, DK, C, Mat<1, LDT>{Vs}, Mat<LDK, 1>{Kws},
                         [&](int m, int n, float x0, float x1) { add2(Ss + m * LDK + n, x0, x1); });
     }
@@ -630,7 +706,7 @@ bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout 
 template <int DK, int DV, int DVT, typename Tin>
 __global__ void __launch_bounds__(NTHR, 1)
 bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, const float* __restrict__ dS_final,
-                   float* __restrict__ dS0, float* __restrict__ ws, Layout L, int B, int T, int H, int NC)
+                   float* __restrict__ dS0, float* __restrict__ ws, Layout L, int B, int T, int H, int NC, int gated)
 {
     constexpr bool SPLIT = std::is_same<Tin, float>::value;
     using SM = StateSmem<DK, DVT>;
@@ -642,6 +718,7 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
     float* dVs = dOs + C * LDT;      // [C][LDT] -dVn
     float* B1 = dVs + C * LDT;       // [C][LDK] Kw, then W
     float* B2 = B1 + C * LDK;        // [C][LDK] Q
+    float* gs = B2 + C * LDK;        // [C] gated: log2 gamma_t
 
     const int tid = threadIdx.x;
     const int unit = blockIdx.x / NTILE, v0 = (blockIdx.x % NTILE) * DVT, b = unit / H, h = unit % H;
@@ -672,9 +749,19 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
         async_block<C, DK>(B1, LDK, kw_g);
         load_tile<C, DVT>(dOs, LDT, dout + tok0 * DV + v0, (size_t)H * DV, Tc);
         load_tile<C, DK>(B2, LDK, q + tok0 * DK, (size_t)H * DK, Tc);
+        if (gated && tid < C) gs[tid] = ws[L.lg / sizeof(float) + cid * C + tid];
         cp_async_wait_all();
         __syncthreads();
-        // dVn = P^T dO + Kw dS'^T
+        if (gated) {   // Kw rows x rho_t and Q rows x gamma_t
+            const float gl = gs[C - 1];
+            for (int idx = tid; idx < C * DK; idx += NTHR) {
+                const int t = idx / DK, i = idx % DK;
+                B1[t * LDK + i] *= ex2(gl - gs[t]);
+                B2[t * LDK + i] *= ex2(gs[t]);
+            }
+            __syncthreads();
+        }
+        // dVn = P^T dO + diag(rho) Kw dS'^T
         cta_gemm2<SPLIT>(C, DVT, C, Mat<1, LDC>{Ps}, Mat<LDT, 1>{dOs}, DK, Mat<LDK, 1>{B1}, Mat<1, LDK>{dSs},
                          [&](int m, int n, float x0, float x1) {
                              dVs[m * LDT + n] = -x0;
@@ -683,9 +770,13 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
                          });
         __syncthreads();
         async_block<C, DK>(B1, LDK, w_g);
+        if (gated) {   // gamma_C dS'
+            const float gc = ex2(gs[C - 1]);
+            for (int idx = tid; idx < DVT * DK; idx += NTHR) dSs[(idx / DK) * LDK + idx % DK] *= gc;
+        }
         cp_async_wait_all();
         __syncthreads();
-        // dS = dS' + dO^T Q + (-dVn)^T W
+        // dS = gamma_C dS' + dO^T diag(gamma) Q + (-dVn)^T W
         cta_gemm2<SPLIT>(DVT, DK, C, Mat<1, LDT>{dOs}, Mat<LDK, 1>{B2}, C, Mat<1, LDT>{dVs}, Mat<LDK, 1>{B1},
                          [&](int m, int n, float x0, float x1) { add2(dSs + m * LDK + n, x0, x1); });
     }
@@ -700,6 +791,13 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
 // dKw += dP^T Q once. Key side, as written below. dQ, dKw, dW and dK stay in
 // registers: warp w (of 16) owns rows 16 (w % 4) .. + 15 and columns
 // (DK / 4) (w / 4) .. + DK / 4 - 1 of each.
+// Gated: the gate factors enter as the header states, and dalpha_m is taken as the sum of
+// the terms whose gate product holds alpha_m, each divided by alpha_m in the exponent
+// (2^(sum of the other clamped log2 alphas)): the pair (t, j) of A and P for j < m <= t,
+// the rows t >= m of dO S and of T^T dW, the rows j < m of Vn dS', and <dS', S>. No
+// difference of large terms is taken, so dalpha keeps its relative accuracy for gates
+// near 0 (where the chunk-local dG form, a reverse cumulative sum over 1 / alpha_m,
+// cancels).
 constexpr int J = 32;           // dv tile of the gradient kernel
 constexpr int LDJ = J + 4;
 
@@ -707,14 +805,15 @@ template <int DK>
 struct GradSmem {
     static constexpr int LDK = DK + 4;
     static constexpr size_t kBytes =
-        sizeof(float) * (size_t)(2 * C * LDK + 3 * C * LDC + 4 * C * LDJ + 2 * J * LDK + 2 * C);
+        sizeof(float) * (size_t)(2 * C * LDK + 4 * C * LDC + 4 * C * LDJ + 2 * J * LDK + 8 * C);
 };
 
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(NTHR, 1)
 bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
-                 const Tin* __restrict__ beta, const Tin* __restrict__ dout, Tin* __restrict__ dq,
-                 Tin* __restrict__ dv, float* __restrict__ ws, Layout L, int B, int T, int H, int NC)
+                 const Tin* __restrict__ beta, const Tin* __restrict__ alpha, const Tin* __restrict__ dout,
+                 Tin* __restrict__ dq, Tin* __restrict__ dv, Tin* __restrict__ dalpha, float* __restrict__ ws,
+                 Layout L, int B, int T, int H, int NC)
 {
     constexpr bool SPLIT = std::is_same<Tin, float>::value;
     constexpr int LDK = GradSmem<DK>::LDK, NT = DK / 32;
@@ -732,6 +831,15 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     float* dSJ = SJ + J * LDK;       // [J][LDK] rows of dS' (chunk end)
     float* bs = dSJ + J * LDK;       // [C] beta
     float* dbs = bs + C;             // [C] dbeta (the chunk part)
+    // gated only:
+    float* Xg = dbs + C;             // [C][LDC] the pair terms of d log gamma with R divided out
+    float* gsm = Xg + C * LDC;       // [C] log2 gamma_t
+    float* lsm = gsm + C;            // [C] clamped log2 alpha_t
+    float* gam = lsm + C;            // [C] gamma_t
+    float* av = gam + C;             // [C] <(dO S)_t, Q_t> + beta_t <(T^T dW)_t, K_t>
+    float* yr = av + C;              // [C] <(Vn dS')_t, Kw_t>
+    float* csd = yr + C;             // [1] <dS', S>
+    const bool gated = alpha != nullptr;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t nchunks = (size_t)B * H * NC;
@@ -762,7 +870,16 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     if (tid < C) {
         bs[tid] = ld_or0(beta, tok(tid), tid < Tc);
         dbs[tid] = 0.f;
+        av[tid] = 0.f;
+        yr[tid] = 0.f;
     }
+    if (gated) {
+        if (tid < 32) chunk_log2_gates(gsm, alpha, tok0, (size_t)H, Tc, tid, lsm);
+        if (tid == 0) *csd = 0.f;
+        __syncthreads();
+        if (tid < C) gam[tid] = ex2(gsm[tid]);
+    }
+    float sds = 0.f;   // gated: this thread's part of <dS', S>
 
     const int m0 = 16 * (warp & 3), n0 = (DK / 4) * (warp >> 2);
     float aQ[NT][4], aKw[NT][4], aW[NT][4];
@@ -808,8 +925,56 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         warp_mma<NT, SPLIT>(aQ, Mat<LDJ, 1>{dOs}, Mat<LDK, 1>{SJ}, m0, n0, J, lane);     // dO S
         warp_mma<NT, SPLIT>(aKw, Mat<LDJ, 1>{Vns}, Mat<LDK, 1>{dSJ}, m0, n0, J, lane);   // Vn dS'
         warp_mma<NT, SPLIT>(aW, Mat<LDJ, 1>{dVns}, Mat<LDK, 1>{SJ}, m0, n0, J, lane);    // dVn S
+        if (gated)
+            for (int idx = tid; idx < J * DK; idx += NTHR)
+                sds = fmaf(SJ[(idx / DK) * LDK + idx % DK], dSJ[(idx / DK) * LDK + idx % DK], sds);
     }
     __syncthreads();
+    if (gated) {
+        // <dS', S>; the rows of the ungated dO S and Vn dS' against Q and Kw; then
+        // dQ's dO S part x gamma_t and dKw's Vn dS' part x rho_t = gamma_C / gamma_t
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sds += __shfl_xor_sync(0xffffffffu, sds, off);
+        if (lane == 0) atomicAdd(csd, sds);
+        const int t4 = lane & 3;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int m = m0 + (lane >> 2) + 8 * hh;
+            const float gm = gam[m], rho = ex2(gsm[C - 1] - gsm[m]);
+            float pq = 0.f, pk = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < NT; ++jj) {
+                const int n = n0 + 8 * jj + 2 * t4;
+                pq = fmaf(aQ[jj][2 * hh], Qs[m * LDK + n], pq);
+                pq = fmaf(aQ[jj][2 * hh + 1], Qs[m * LDK + n + 1], pq);
+                pk = fmaf(aKw[jj][2 * hh], Kws[m * LDK + n], pk);
+                pk = fmaf(aKw[jj][2 * hh + 1], Kws[m * LDK + n + 1], pk);
+                aQ[jj][2 * hh] *= gm;
+                aQ[jj][2 * hh + 1] *= gm;
+                aKw[jj][2 * hh] *= rho;
+                aKw[jj][2 * hh + 1] *= rho;
+            }
+            pq += __shfl_xor_sync(0xffffffffu, pq, 1);
+            pq += __shfl_xor_sync(0xffffffffu, pq, 2);
+            pk += __shfl_xor_sync(0xffffffffu, pk, 1);
+            pk += __shfl_xor_sync(0xffffffffu, pk, 2);
+            if (t4 == 0) {
+                atomicAdd(&av[m], pq);
+                atomicAdd(&yr[m], pk);
+            }
+        }
+        // the P pair terms dP (.) strict_tril(Q Kw^T), then dP <- dP (.) R
+        cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{Qs}, Mat<1, LDK>{Kws}, [&](int m, int n, float x0, float x1) {
+            store2(Xg + m * LDC + n, n < m ? dPs[m * LDC + n] * x0 : 0.f,
+                   n + 1 < m ? dPs[m * LDC + n + 1] * x1 : 0.f);
+        });
+        __syncthreads();
+        for (int idx = tid; idx < C * C; idx += NTHR) {
+            const int m = idx / C, n = idx % C;
+            if (n <= m) dPs[m * LDC + n] *= ex2(gsm[m] - gsm[n]);
+        }
+        __syncthreads();
+    }
     warp_mma<NT, SPLIT>(aQ, Mat<LDC, 1>{dPs}, Mat<LDK, 1>{Kws}, m0, n0, C, lane);        // dP Kw
     warp_mma<NT, SPLIT>(aKw, Mat<1, LDC>{dPs}, Mat<LDK, 1>{Qs}, m0, n0, C, lane);        // dP^T Q
     frag_each(aQ, m0, n0, lane, [&](int m, int n, float x0, float x1) {
@@ -846,8 +1011,11 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     frag_each(aW, m0, n0, lane, [&](int m, int n, float x0, float x1) { store2(dWs + m * LDK + n, -x0, -x1); });
     load_tile<C, DK>(Ks, LDK, k + tok0 * DK, (size_t)H * DK, Tc);
     __syncthreads();
-    cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{dWs}, Mat<1, LDK>{Ks},
-                    [&](int m, int n, float x0, float x1) { add2(dTs + m * LDC + n, bs[n] * x0, bs[n + 1] * x1); });
+    cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{dWs}, Mat<1, LDK>{Ks}, [&](int m, int n, float x0, float x1) {
+        // x diag(beta gamma) (W = T diag(beta gamma) K when gated)
+        const float f0 = gated ? bs[n] * gam[n] : bs[n], f1 = gated ? bs[n + 1] * gam[n + 1] : bs[n + 1];
+        add2(dTs + m * LDC + n, f0 * x0, f1 * x1);
+    });
     cta_gemm<SPLIT>(C, C, DK, Mat<LDK, 1>{Ks}, Mat<1, LDK>{Kws},
                     [&](int m, int n, float x0, float x1) { store2(Gs + m * LDC + n, x0, x1); });
     __syncthreads();
@@ -855,7 +1023,14 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
                     [&](int m, int n, float x0, float x1) { store2(Xs + m * LDC + n, x0, x1); });
     __syncthreads();
     cta_gemm<SPLIT>(C, C, C, Mat<1, LDC>{Ts}, Mat<LDC, 1>{Xs}, [&](int m, int n, float x0, float x1) {
-        const float a0 = n < m ? -x0 : 0.f, a1 = n + 1 < m ? -x1 : 0.f;   // dA (strictly lower)
+        float a0 = n < m ? -x0 : 0.f, a1 = n + 1 < m ? -x1 : 0.f;   // dA (strictly lower)
+        if (gated && n < m) {   // the A pair terms beta_m dA (.) K Kw^T, then dA <- dA (.) R
+            // (R only below the diagonal: above it the ratio may overflow)
+            Xg[m * LDC + n] += bs[m] * a0 * Gs[m * LDC + n];
+            Xg[m * LDC + n + 1] += bs[m] * a1 * Gs[m * LDC + n + 1];
+            a0 *= ex2(gsm[m] - gsm[n]);
+            if (n + 1 < m) a1 *= ex2(gsm[m] - gsm[n + 1]);
+        }
         if (n < m) atomicAdd(&dbs[m], a0 * Gs[m * LDC + n] + a1 * Gs[m * LDC + n + 1]);
         dTs[m * LDC + n] = bs[m] * a0;                                    // diag(beta) dA
         dTs[m * LDC + n + 1] = bs[m] * a1;
@@ -864,23 +1039,28 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     float aK[NT][4];
     frag_zero(aK);
     warp_mma<NT, SPLIT>(aK, Mat<1, LDC>{Ts}, Mat<LDK, 1>{dWs}, m0, n0, C, lane);        // T^T dW
-    {   // dbeta += rowdot(T^T dW, K): the 4 lanes that share a row reduce before one atomic
+    {   // dbeta += gamma_m rowdot(T^T dW, K): the 4 lanes that share a row reduce before one
+        // atomic (gamma = 1 ungated); gated, the row's d log gamma term beta_m rowdot(T^T dW, K)
         const int t4 = lane & 3;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             const int m = m0 + (lane >> 2) + 8 * hh;
+            const float gm = gated ? gam[m] : 1.f, fk = bs[m] * gm;
             float part = 0.f;
 #pragma unroll
             for (int jj = 0; jj < NT; ++jj) {
                 const int n = n0 + 8 * jj + 2 * t4;
                 part = fmaf(aK[jj][2 * hh], Ks[m * LDK + n], part);
                 part = fmaf(aK[jj][2 * hh + 1], Ks[m * LDK + n + 1], part);
-                aK[jj][2 * hh] *= bs[m];
-                aK[jj][2 * hh + 1] *= bs[m];
+                aK[jj][2 * hh] *= fk;
+                aK[jj][2 * hh + 1] *= fk;
             }
             part += __shfl_xor_sync(0xffffffffu, part, 1);
             part += __shfl_xor_sync(0xffffffffu, part, 2);
-            if (t4 == 0) atomicAdd(&dbs[m], part);
+            if (t4 == 0) {
+                atomicAdd(&dbs[m], gm * part);
+                if (gated) atomicAdd(&av[m], bs[m] * part);
+            }
         }
     }
     warp_mma<NT, SPLIT>(aK, Mat<LDC, 1>{dTs}, Mat<LDK, 1>{Kws}, m0, n0, C, lane);       // + dAb Kw
@@ -898,6 +1078,22 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         }
     __syncthreads();
     if (tid < C) dbp_g[tid] = dbs[tid];
+    if (gated) {   // dalpha_m, warp w taking tokens w, w + 16, ..: lanes split each sum
+        const float gl = gsm[C - 1];
+        for (int m = warp; m < Tc; m += NTHR / 32) {
+            const float lm = lsm[m];
+            float s = 0.f;
+            for (int t = m + lane; t < C; t += 32) s = fmaf(av[t], ex2(gsm[t] - lm), s);
+            for (int j = lane; j < m; j += 32) s = fmaf(yr[j], ex2(gl - gsm[j] - lm), s);
+            for (int e = lane; e < (C - m) * m; e += 32) {   // rows t >= m, columns j < m
+                const int t = m + e / m, j = e % m;
+                s = fmaf(Xg[t * LDC + j], ex2(gsm[t] - gsm[j] - lm), s);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            if (lane == 0) dalpha[tok(m)] = from_f32<Tin>(fmaf(*csd, ex2(gl - lm), s));
+        }
+    }
     }
 }
 

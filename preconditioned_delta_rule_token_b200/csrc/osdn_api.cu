@@ -340,7 +340,7 @@ int launch_step(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, 
 // Forward and reverse state passes of the backward with a dv tile of DVT rows.
 template <typename Tin, int DK, int DV, int DVT>
 int launch_state_passes(const osdn_params* p, const Tin* q, const Tin* dout, const float* S0, const float* dS_final,
-                        float* dS0, float* ws, const osdn::bwd::Layout& L, int NC, cudaStream_t st) {
+                        float* dS0, float* ws, const osdn::bwd::Layout& L, int NC, int gated, cudaStream_t st) {
     namespace B = osdn::bwd;
     const unsigned ntiles = (unsigned)(p->B * p->H * (DV / DVT));
     const size_t s_sf = B::StateSmem<DK, DVT>::kFwdBytes, s_sb = B::StateSmem<DK, DVT>::kBwdBytes;
@@ -348,23 +348,24 @@ int launch_state_passes(const osdn_params* p, const Tin* q, const Tin* dout, con
     if ((e = cudaFuncSetAttribute(B::bwd_state_f_kernel<DK, DV, DVT, Tin>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_sf)) != cudaSuccess)
         return cuda_fail(e, "backward state attribute");
-    B::bwd_state_f_kernel<DK, DV, DVT, Tin><<<ntiles, B::NTHR, s_sf, st>>>(S0, ws, L, NC);
+    B::bwd_state_f_kernel<DK, DV, DVT, Tin><<<ntiles, B::NTHR, s_sf, st>>>(S0, ws, L, NC, gated);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward state launch");
     if ((e = cudaFuncSetAttribute(B::bwd_state_b_kernel<DK, DV, DVT, Tin>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_sb)) != cudaSuccess)
         return cuda_fail(e, "backward adjoint state attribute");
     B::bwd_state_b_kernel<DK, DV, DVT, Tin><<<ntiles, B::NTHR, s_sb, st>>>(dout, q, dS_final, dS0, ws, L, p->B,
-                                                                           p->T, p->H, NC);
+                                                                           p->T, p->H, NC, gated);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward adjoint state launch");
     return OSDN_OK;
 }
 
-// Backward: six launches on one stream (see bwd.cuh for what each computes).
+// Backward: six launches on one stream (see bwd.cuh for what each computes); alpha
+// non-NULL selects the gated form inside the same kernels.
 template <typename Tin, int DK, int DV>
 int launch_bwd_t(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, const Tin* beta, const Tin* r,
                  const float* d0, const float* S0, const Tin* dout, const float* dS_final, const float* dd_final,
                  Tin* dq, Tin* dk, Tin* dv, Tin* dbeta, Tin* dr, float* dd0, float* dS0, float* ws,
-                 cudaStream_t st) {
+                 const Tin* alpha, Tin* dalpha, cudaStream_t st) {
     namespace B = osdn::bwd;
     const B::Layout L = B::make_layout(p->B, p->T, p->H, DK, DV);
     const int units = p->B * p->H, NC = (p->T + B::C - 1) / B::C, an = anchor_of(p);
@@ -386,7 +387,8 @@ int launch_bwd_t(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v,
     const size_t s_prep = B::PrepSmem<DK, DV>::kBytes;
     if ((e = attr((const void*)B::bwd_prep_kernel<DK, DV, Tin>, s_prep)) != cudaSuccess)
         return cuda_fail(e, "backward prep attribute");
-    B::bwd_prep_kernel<DK, DV, Tin><<<pgrid, B::NTHR, s_prep, st>>>(q, k, v, beta, ws, L, p->B, p->T, p->H, NC);
+    B::bwd_prep_kernel<DK, DV, Tin><<<pgrid, B::NTHR, s_prep, st>>>(q, k, v, beta, alpha, ws, L, p->B, p->T, p->H,
+                                                                  NC);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward prep launch");
 
     // The two state passes are serial over the chunks; their dv tile is the widest of
@@ -395,16 +397,18 @@ int launch_bwd_t(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v,
     int dvt = DV;
     while (dvt > 32 && (long long)units * (DV / dvt) * 2 <= sms) dvt /= 2;
     int rcs;
-    if (dvt == 32) rcs = launch_state_passes<Tin, DK, DV, 32>(p, q, dout, S0, dS_final, dS0, ws, L, NC, st);
-    else if (dvt == 64) rcs = launch_state_passes<Tin, DK, DV, 64>(p, q, dout, S0, dS_final, dS0, ws, L, NC, st);
-    else rcs = launch_state_passes<Tin, DK, DV, DV>(p, q, dout, S0, dS_final, dS0, ws, L, NC, st);
+    const int gated = alpha != nullptr;
+    if (dvt == 32) rcs = launch_state_passes<Tin, DK, DV, 32>(p, q, dout, S0, dS_final, dS0, ws, L, NC, gated, st);
+    else if (dvt == 64)
+        rcs = launch_state_passes<Tin, DK, DV, 64>(p, q, dout, S0, dS_final, dS0, ws, L, NC, gated, st);
+    else rcs = launch_state_passes<Tin, DK, DV, DV>(p, q, dout, S0, dS_final, dS0, ws, L, NC, gated, st);
     if (rcs) return rcs;
 
     const size_t s_g = B::GradSmem<DK>::kBytes;
     if ((e = attr((const void*)B::bwd_grads_kernel<DK, DV, Tin>, s_g)) != cudaSuccess)
         return cuda_fail(e, "backward gradient attribute");
-    B::bwd_grads_kernel<DK, DV, Tin><<<pgrid, B::NTHR, s_g, st>>>(q, k, v, beta, dout, dq, dv, ws, L, p->B, p->T,
-                                                                   p->H, NC);
+    B::bwd_grads_kernel<DK, DV, Tin><<<pgrid, B::NTHR, s_g, st>>>(q, k, v, beta, alpha, dout, dq, dv, dalpha, ws, L,
+                                                                   p->B, p->T, p->H, NC);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward gradient launch");
 
     if ((e = attr((const void*)B::bwd_dchain_kernel<DK, Tin>, s_dc)) != cudaSuccess)
@@ -419,10 +423,11 @@ template <typename Tin>
 int launch_bwd(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
                const float* d0, const float* S0, const void* dout, const float* dS_final, const float* dd_final,
                void* dq, void* dk, void* dv, void* dbeta, void* dr, float* dd0, float* dS0, float* ws,
-               cudaStream_t st) {
+               const void* alpha, void* dalpha, cudaStream_t st) {
 #define OSDN_BWD_ARGS                                                                                        \
     p, (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)beta, (const Tin*)r, d0, S0, (const Tin*)dout, \
-        dS_final, dd_final, (Tin*)dq, (Tin*)dk, (Tin*)dv, (Tin*)dbeta, (Tin*)dr, dd0, dS0, ws, st
+        dS_final, dd_final, (Tin*)dq, (Tin*)dk, (Tin*)dv, (Tin*)dbeta, (Tin*)dr, dd0, dS0, ws, (const Tin*)alpha, \
+        (Tin*)dalpha, st
     if (p->dk == 128 && p->dv == 128) return launch_bwd_t<Tin, 128, 128>(OSDN_BWD_ARGS);
     if (p->dk == 128) return launch_bwd_t<Tin, 128, 64>(OSDN_BWD_ARGS);
     if (p->dv == 128) return launch_bwd_t<Tin, 64, 128>(OSDN_BWD_ARGS);
@@ -694,16 +699,19 @@ int osdn_bwd_workspace_size(const osdn_params* p, size_t* bytes) {
     return OSDN_OK;
 }
 
-int osdn_bwd(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
-             const float* d0, const float* S0, const void* dout, const float* dS_final, const float* dd_final,
-             void* dq, void* dk, void* dv, void* dbeta, void* dr, float* dd0, float* dS0, void* workspace,
-             size_t workspace_bytes, void* cuda_stream) {
+}  // extern "C"
+
+namespace {
+int bwd_impl(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
+             const void* alpha, const float* d0, const float* S0, const void* dout, const float* dS_final,
+             const float* dd_final, void* dq, void* dk, void* dv, void* dbeta, void* dr, void* dalpha, float* dd0,
+             float* dS0, void* workspace, size_t workspace_bytes, void* cuda_stream, bool gated) {
     t_last_error.clear();
     int rc = check_params(p, true);
     if (rc) return rc;
     if (!dense_layout(p)) return fail(OSDN_ERR_UNSUPPORTED, "the backward takes dense tensors only");
-    const void* ptrs[] = {q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta, dr, dd0, dS0,
-                          workspace};
+    const void* ptrs[] = {q, k, v, beta, r, alpha, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta, dr, dalpha,
+                          dd0, dS0, workspace};
     for (const void* x : ptrs)
         if (x && !aligned16(x)) return fail(OSDN_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
@@ -726,6 +734,7 @@ int osdn_bwd(const osdn_params* p, const void* q, const void* k, const void* v, 
     }
     if (!q || !k || !v || !beta || !dout || !dq || !dk || !dv || !dbeta)
         return fail(OSDN_ERR_INVALID_ARG, "q, k, v, beta, dout, dq, dk, dv and dbeta must not be NULL");
+    if (gated && (!alpha || !dalpha)) return fail(OSDN_ERR_INVALID_ARG, "alpha and dalpha must not be NULL");
     if (!workspace) return fail(OSDN_ERR_INVALID_ARG, "workspace is NULL");
     const size_t need = bwd_workspace_bytes(p);
     if (workspace_bytes < need)
@@ -733,11 +742,31 @@ int osdn_bwd(const osdn_params* p, const void* q, const void* k, const void* v, 
     if ((double)units * (double)((p->T + 63) / 64) > 2147483647.0)
         return fail(OSDN_ERR_INVALID_ARG, "B * H * ceil(T / 64) exceeds the grid limit");
     float* ws = reinterpret_cast<float*>(workspace);
+    if (!gated) alpha = dalpha = nullptr;
     if (p->dtype == OSDN_BF16)
         return launch_bwd<__nv_bfloat16>(p, q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta,
-                                         dr, dd0, dS0, ws, st);
+                                         dr, dd0, dS0, ws, alpha, dalpha, st);
     return launch_bwd<float>(p, q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta, dr, dd0, dS0,
-                             ws, st);
+                             ws, alpha, dalpha, st);
+}
+}  // namespace
+
+extern "C" {
+
+int osdn_bwd(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
+             const float* d0, const float* S0, const void* dout, const float* dS_final, const float* dd_final,
+             void* dq, void* dk, void* dv, void* dbeta, void* dr, float* dd0, float* dS0, void* workspace,
+             size_t workspace_bytes, void* cuda_stream) {
+    return bwd_impl(p, q, k, v, beta, r, nullptr, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta, dr, nullptr,
+                    dd0, dS0, workspace, workspace_bytes, cuda_stream, false);
+}
+
+int osdn_bwd_gated(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta,
+                   const void* r, const void* alpha, const float* d0, const float* S0, const void* dout,
+                   const float* dS_final, const float* dd_final, void* dq, void* dk, void* dv, void* dbeta, void* dr,
+                   void* dalpha, float* dd0, float* dS0, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    return bwd_impl(p, q, k, v, beta, r, alpha, d0, S0, dout, dS_final, dd_final, dq, dk, dv, dbeta, dr, dalpha,
+                    dd0, dS0, workspace, workspace_bytes, cuda_stream, true);
 }
 
 int osdn_sync_status(void* cuda_stream) {

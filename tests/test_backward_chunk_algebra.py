@@ -65,50 +65,105 @@ def _d_trajectory(k, beta, r, d0, eta, anchor):
     return D, d
 
 
-def chunk_backward(q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, eta, anchor, C):
-    """Gradients of one (b, h) unit by the chunk-form adjoint. q, k: [T, dk]; v, dout: [T, dv]."""
+def chunk_backward(q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, eta, anchor, C, alpha=None,
+                   dalpha_form="direct"):
+    """Gradients of one (b, h) unit by the chunk-form adjoint. q, k: [T, dk]; v, dout: [T, dv].
+
+    alpha [T] (gated OSDN, the state decayed by alpha_t before token t's write) takes the
+    chunk form with every decay factor a ratio of the in-chunk cumulative gate gamma:
+    R_tj = gamma_t / gamma_j, rho_j = gamma_C / gamma_j,
+        A = strict_tril(Kb Kw^T (.) R), W = T diag(beta gamma) K, P = tril(Q Kw^T) (.) R,
+        O = diag(gamma) Q S^T + P Vn, S' = gamma_C S + Vn^T diag(rho) Kw,
+    and its reverse
+        dVn = P^T dO + diag(rho) Kw dS'^T,  dS = gamma_C dS' + dO^T diag(gamma) Q - dVn^T W,
+        dPr = tril(dO Vn^T) (.) R,  dQ = diag(gamma) dO S + dPr Kw,
+        dW = -dVn S,  dT = dW (diag(beta gamma) K)^T + dVn (diag(beta) V)^T,
+        dA = -strict_tril(T^T dT T^T),  dAr = dA (.) R,
+        dKw = diag(rho) Vn dS' + dPr^T Q + dAr^T Kb,
+        dK = diag(beta) dAr Kw + diag(beta gamma) T^T dW + dKw (.) D,
+        dbeta = rowdot(dAr Kw, K) + gamma (.) rowdot(T^T dW, K) + rowdot(T^T dVn, V),
+    with the adjoint of G = log gamma collected from every place gamma enters,
+        dG_t = gamma_t <dO_t, (Q S^T)_t> + gamma_t beta_t <(T^T dW)_t, K_t> + sum_j X_tj - sum_j X_jt
+               - Y_t + [t = last] (gamma_C <dS', S> + sum_j Y_j),
+        X = (dA (.) Kb Kw^T + tril(dO Vn^T) (.) Q Kw^T) (.) R,  Y_j = rho_j <Vn_j, dS' Kw_j>,
+    and dalpha_m = (sum_{t >= m} dG_t) / alpha_m (G_t is the sum of log alpha up to t): the
+    "cumsum" form, which needs alpha > 0. The "direct" form (the CUDA kernel's) sums only the
+    terms whose gate product holds alpha_m and divides alpha_m out in the exponent:
+        dalpha_m = sum_{t >= m} a_t 2^(L_t - l_m) + sum_{j < m} y_j 2^(L_C - L_j - l_m)
+                   + c 2^(L_C - l_m) + sum_{t >= m > j} X'_tj 2^(L_t - L_j - l_m),
+    l = log2 alpha (clamped at -120, so alpha = 0 is allowed), L its in-chunk cumulative sum,
+    a_t = <dO_t, (Q S^T)_t> + beta_t <(T^T dW)_t, K_t>, y_j = <Vn_j, dS' Kw_j>, c = <dS', S>,
+    X' = X with R divided out. Gamma and every ratio are taken as 2^(differences of L)."""
     T, dk = k.shape
     dv = v.shape[1]
     r = np.ones(T) if r is None else r
+    gated = alpha is not None
+    alpha = np.ones(T) if alpha is None else alpha
     D, _ = _d_trajectory(k, beta, r, d0, eta, anchor)
     Kw_all = D * k
     starts = list(range(0, T, C))
     # forward over the chunks: the state at every chunk start and the chunk matrices
     S = S0.copy()
     saved = []
+    lg2 = np.maximum(np.log2(np.maximum(alpha, 1e-300)), -120.0)
     for c0 in starts:
         sl = slice(c0, min(T, c0 + C))
         K, Kw, Q, V, be = k[sl], Kw_all[sl], q[sl], v[sl], beta[sl]
         n = len(K)
+        L = np.cumsum(lg2[sl])
+        g = 2.0 ** L
+        R = np.tril(2.0 ** np.minimum(L[:, None] - L[None, :], 0.0))
+        rho = 2.0 ** (L[-1] - L)
         Kb = be[:, None] * K
-        A = np.tril(Kb @ Kw.T, -1)
+        A = np.tril(Kb @ Kw.T, -1) * R
         Tm = np.linalg.inv(np.eye(n) + A)
-        W = Tm @ Kb
+        W = Tm @ (g[:, None] * Kb)
         U0 = Tm @ (be[:, None] * V)
         Vn = U0 - W @ S.T
-        P = np.tril(Q @ Kw.T)
-        saved.append((sl, S.copy(), Tm, W, Vn, P))
-        S = S + Vn.T @ Kw
+        P = np.tril(Q @ Kw.T) * R
+        saved.append((sl, S.copy(), Tm, W, Vn, P, g, R, rho, L))
+        S = g[-1] * S + Vn.T @ (rho[:, None] * Kw)
     # reverse over the chunks
     dS = dS_final.copy()
     dq, dk_, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
-    dbeta, dD = np.zeros(T), np.zeros((T, dk))
-    for sl, Sc, Tm, W, Vn, P in reversed(saved):
+    dbeta, dD, dalpha = np.zeros(T), np.zeros((T, dk)), np.zeros(T)
+    for sl, Sc, Tm, W, Vn, P, g, R, rho, L in reversed(saved):
         K, Kw, Q, V, be, dO, Dc = k[sl], Kw_all[sl], q[sl], v[sl], beta[sl], dout[sl], D[sl]
-        dVn = P.T @ dO + Kw @ dS.T
-        dS_prev = dS + dO.T @ Q - dVn.T @ W
-        dP = np.tril(dO @ Vn.T)
-        dq[sl] = dO @ Sc + dP @ Kw
+        Kb = be[:, None] * K
+        dVn = P.T @ dO + (rho[:, None] * Kw) @ dS.T
+        dS_prev = g[-1] * dS + dO.T @ (g[:, None] * Q) - dVn.T @ W
+        dPm = np.tril(dO @ Vn.T)                  # adjoint of P
+        dPr = dPm * R                             # adjoint of the unmasked Q Kw^T
+        dq[sl] = g[:, None] * (dO @ Sc) + dPr @ Kw
         dW = -dVn @ Sc
-        dT = (dW @ K.T + dVn @ V.T) * be[None, :]
-        dA = -np.tril(Tm.T @ dT @ Tm.T, -1)
-        dAb = be[:, None] * dA
-        dKw = Vn @ dS + dP.T @ Q + dAb.T @ K
+        dT = dW @ (g[:, None] * Kb).T + dVn @ (be[:, None] * V).T
+        dA = -np.tril(Tm.T @ dT @ Tm.T, -1)       # adjoint of A
+        dAr = dA * R                              # adjoint of the unmasked Kb Kw^T
+        dKw = rho[:, None] * (Vn @ dS) + dPr.T @ Q + dAr.T @ Kb
         TdW, TdVn = Tm.T @ dW, Tm.T @ dVn
         dvv[sl] = be[:, None] * TdVn
-        dk_[sl] = be[:, None] * TdW + dAb @ Kw + dKw * Dc
-        dbeta[sl] = (TdW * K).sum(1) + (TdVn * V).sum(1) + (dA * (K @ Kw.T)).sum(1)
+        dk_[sl] = be[:, None] * (dAr @ Kw) + (be * g)[:, None] * TdW + dKw * Dc
+        dbeta[sl] = ((dAr @ Kw) * K).sum(1) + g * (TdW * K).sum(1) + (TdVn * V).sum(1)
         dD[sl] = dKw * K
+        if gated and dalpha_form == "cumsum":
+            # adjoint of G = log gamma, then of log alpha (reverse cumulative sum), then of alpha
+            X = (dA * (Kb @ Kw.T) + dPm * (Q @ Kw.T)) * R
+            Yr = rho * ((Vn @ dS) * Kw).sum(1)    # rho_j <Vn_j, dS' Kw_j>
+            dG = g * (dO * (Q @ Sc.T)).sum(1) + g * be * (TdW * K).sum(1) + X.sum(1) - X.sum(0) - Yr
+            dG[-1] += g[-1] * (dS * Sc).sum() + Yr.sum()
+            dalpha[sl] = np.cumsum(dG[::-1])[::-1] / alpha[sl]
+        elif gated:
+            Xp = np.tril(dA * (Kb @ Kw.T) + dPm * (Q @ Kw.T), -1)
+            a = (dO * (Q @ Sc.T)).sum(1) + be * (TdW * K).sum(1)
+            y = ((Vn @ dS) * Kw).sum(1)
+            cs = (dS * Sc).sum()
+            l = lg2[sl]
+            da = np.zeros(len(l))
+            for m in range(len(l)):
+                da[m] = ((a[m:] * 2.0 ** (L[m:] - l[m])).sum() + (y[:m] * 2.0 ** (L[-1] - L[:m] - l[m])).sum()
+                         + cs * 2.0 ** (L[-1] - l[m])
+                         + (Xp[m:, :m] * 2.0 ** (L[m:, None] - L[None, :m] - l[m])).sum())
+            dalpha[sl] = da
         dS = dS_prev
     # reverse of the preconditioner recurrence
     Ld = dd_final.copy()
@@ -129,7 +184,7 @@ def chunk_backward(q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, eta, anch
             ds = -dx * eta * beta[t] ** 2 / n
             dk_[t] += 2 * k[t] * (x * Ld + ds * d - dx * x / n)
         Ld = r[t] * Ld + dD[t] + ds * a
-    return dict(dq=dq, dk=dk_, dv=dvv, dbeta=dbeta, dr=dr, dd0=Ld + dd_anchor, dS0=dS)
+    return dict(dq=dq, dk=dk_, dv=dvv, dbeta=dbeta, dr=dr, dd0=Ld + dd_anchor, dS0=dS, dalpha=dalpha)
 
 
 @pytest.mark.parametrize("T,C,anchor,apf", [(150, 64, False, True), (150, 64, True, True), (64, 64, False, True),
@@ -149,6 +204,64 @@ def test_chunk_adjoint_matches_the_token_gradients(T, C, anchor, apf):
     for name, want in pairs:
         np.testing.assert_allclose(got[name], want, rtol=1e-9, atol=1e-10 * max(1.0, np.abs(want).max()),
                                    err_msg=name)
+
+
+@pytest.mark.parametrize("T,C,anchor,lo", [(150, 64, False, 0.85), (150, 64, True, 0.3), (97, 16, False, 0.05),
+                                            (64, 64, True, 0.6)])
+def test_gated_chunk_adjoint_matches_the_token_gradients(T, C, anchor, lo):
+    """Gated OSDN: the chunk-form adjoint above, with the decay as ratios of the in-chunk
+    cumulative gate, equals the oracle's token-by-token gradients (dalpha included), for
+    gates down to 0.05 and a run of small gates over a whole chunk."""
+    c, cot = _case(T + C + 1, T)
+    rng = np.random.default_rng(T * 3 + C)
+    alpha = rng.uniform(lo, 1.0, (1, T, 1))
+    alpha[0, C:min(T, 2 * C), 0] = max(lo, 0.2)
+    eta = 0.3
+    ref = oracle.bwd(c["q"], c["k"], c["v"], c["beta"], cot["dout"], c["r"], c["d0"], c["S0"], cot["dS_final"],
+                     cot["dd_final"], eta=eta, anchor=anchor, alpha=alpha)
+    u = lambda x: None if x is None else x[0, :, 0]
+    got = chunk_backward(u(c["q"]), u(c["k"]), u(c["v"]), u(c["beta"]), u(c["r"]), c["d0"][0, 0], c["S0"][0, 0],
+                         u(cot["dout"]), cot["dS_final"][0, 0], cot["dd_final"][0, 0], eta, anchor, C,
+                         alpha=u(alpha))
+    for name in ("dq", "dk", "dv", "dbeta", "dr", "dalpha"):
+        want = u(ref[name])
+        np.testing.assert_allclose(got[name], want, rtol=1e-8, atol=1e-9 * max(1.0, np.abs(want).max()),
+                                   err_msg=name)
+    for name in ("dd0", "dS0"):
+        want = ref[name][0, 0]
+        np.testing.assert_allclose(got[name], want, rtol=1e-8, atol=1e-9 * max(1.0, np.abs(want).max()),
+                                   err_msg=name)
+    got_c = chunk_backward(u(c["q"]), u(c["k"]), u(c["v"]), u(c["beta"]), u(c["r"]), c["d0"][0, 0], c["S0"][0, 0],
+                           u(cot["dout"]), cot["dS_final"][0, 0], cot["dd_final"][0, 0], eta, anchor, C,
+                           alpha=u(alpha), dalpha_form="cumsum")
+    want = u(ref["dalpha"])
+    np.testing.assert_allclose(got_c["dalpha"], want, rtol=1e-7, atol=1e-8 * max(1.0, np.abs(want).max()))
+
+
+@pytest.mark.parametrize("T,C", [(150, 64), (97, 16)])
+def test_gated_chunk_adjoint_with_zero_gates(T, C):
+    """alpha = 0 at a chunk start, inside a chunk, twice in one chunk, and gates of 1e-6 and
+    1e-30: the direct form of dalpha (no division by alpha) equals the oracle's gradients,
+    every element at rtol 1e-7, where the reverse cumulative sum over 1 / alpha is undefined
+    or cancels."""
+    c, cot = _case(T + 2 * C, T)
+    rng = np.random.default_rng(T + 5 * C)
+    alpha = rng.uniform(0.3, 1.0, (1, T, 1))
+    for t, val in ((0, 0.0), (C, 0.0), (C + 5, 0.0), (C + 9, 0.0), (3, 1e-6), (2 * C + 7, 1e-30), (T - 1, 0.0)):
+        if t < T:
+            alpha[0, t, 0] = val
+    eta = 0.3
+    ref = oracle.bwd(c["q"], c["k"], c["v"], c["beta"], cot["dout"], c["r"], c["d0"], c["S0"], cot["dS_final"],
+                     cot["dd_final"], eta=eta, anchor=False, alpha=alpha)
+    u = lambda x: None if x is None else x[0, :, 0]
+    got = chunk_backward(u(c["q"]), u(c["k"]), u(c["v"]), u(c["beta"]), u(c["r"]), c["d0"][0, 0], c["S0"][0, 0],
+                         u(cot["dout"]), cot["dS_final"][0, 0], cot["dd_final"][0, 0], eta, False, C,
+                         alpha=u(alpha))
+    for name in ("dq", "dk", "dv", "dbeta", "dr", "dalpha"):
+        want = u(ref[name])
+        np.testing.assert_allclose(got[name], want, rtol=1e-7, atol=1e-9 * max(1.0, np.abs(want).max()),
+                                   err_msg=name)
+    assert np.all(np.isfinite(got["dalpha"]))
 
 
 def chunk_dchain(k, beta, r, dD, dd_final, eta, L):
