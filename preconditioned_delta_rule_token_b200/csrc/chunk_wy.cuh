@@ -160,15 +160,24 @@ __device__ __forceinline__ float sfu_log2(float x) {
     return y;
 }
 
-// Eight bf16 values at p (16-byte aligned shared memory) multiplied by s in place.
-__device__ __forceinline__ void scale_bf16x8(uint8_t* p, float s) {
+// A scale factor as the sum of two bf16 values, hi = bf16(s) and lo = bf16(s - hi), so that
+// x * s is x * lo + x * hi with one fused rounding at the end.
+struct Bf16Scale {
+    __nv_bfloat162 hi, lo;
+    __device__ __forceinline__ explicit Bf16Scale(float s) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(s);
+        hi = __bfloat162bfloat162(h);
+        lo = __bfloat162bfloat162(__float2bfloat16_rn(s - __bfloat162float(h)));
+    }
+};
+
+// Eight bf16 values at p (16-byte aligned shared memory) multiplied by s in place, in packed
+// bf16x2 arithmetic.
+__device__ __forceinline__ void scale_bf16x8(uint8_t* p, const Bf16Scale& s) {
     uint4 u = *reinterpret_cast<uint4*>(p);
     __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(e[q]);
-        e[q] = __floats2bfloat162_rn(s * f.x, s * f.y);
-    }
+    for (int q = 0; q < 4; ++q) e[q] = __hfma2(e[q], s.hi, __hmul2(e[q], s.lo));
     *reinterpret_cast<uint4*>(p) = u;
 }
 
@@ -561,7 +570,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int i = 0; i < 4; ++i) {
                     const int t = (et >> 3) + 16 * i;
                     const float gt = g.at(t);
-                    const float sq = sfu_exp2(gt), sk = sfu_exp2(gl - gt);
+                    const Bf16Scale sq(sfu_exp2(gt)), sk(sfu_exp2(gl - gt));
                     const uint32_t row = (t >> 3) * 1024 + (t & 7) * 128 + ch * 16;
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
