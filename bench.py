@@ -364,9 +364,10 @@ def backward_flops(w):
     return 2.0 * mac * nch
 
 
-def run_backward(w, g, stream, hbm, tf_peak, steps=5, warmup=2):
-    """osdn_bwd on the same layer with inputs and upstream gradients resident in HBM and
-    the workspace preallocated; CUDA events on the launching stream."""
+def run_backward(w, g, stream, hbm, tf_peak, steps=5, warmup=2, gated=False):
+    """osdn_bwd (gated: osdn_bwd_gated with alpha ~ U(0.9, 1)) on the same layer with inputs
+    and upstream gradients resident in HBM and the workspace preallocated; CUDA events on the
+    launching stream."""
     import preconditioned_delta_rule_token_b200 as pk
     dev = g["k"].device
     cot = {k_: (None if v_ is None else v_.to(dev)) for k_, v_ in W.make_backward_cotangents(w).items()}
@@ -376,11 +377,21 @@ def run_backward(w, g, stream, hbm, tf_peak, steps=5, warmup=2):
     grads["dr"] = None if g["r"] is None else torch.empty_like(g["r"])
     dd0 = torch.empty((w.B, w.H, w.dk), dtype=torch.float32, device=dev)
     dS0 = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+    alpha = dalpha = None
+    if gated:
+        alpha = (0.9 + 0.1 * torch.rand((w.B, w.T, w.H), generator=torch.Generator().manual_seed(w.seed + 77))).to(
+            g["k"].dtype).to(dev)
+        dalpha = torch.empty_like(alpha)
 
     def call():
-        pk.osdn_bwd(p, g["q"], g["k"], g["v"], g["beta"], g["r"], None, None, cot["dout"], cot["dS_final"],
-                    cot["dd_final"], grads["dq"], grads["dk"], grads["dv"], grads["dbeta"], grads["dr"], dd0, dS0,
-                    ws, stream)
+        if gated:
+            pk.osdn_bwd_gated(p, g["q"], g["k"], g["v"], g["beta"], g["r"], alpha, None, None, cot["dout"],
+                              cot["dS_final"], cot["dd_final"], grads["dq"], grads["dk"], grads["dv"], grads["dbeta"],
+                              grads["dr"], dalpha, dd0, dS0, ws, stream)
+        else:
+            pk.osdn_bwd(p, g["q"], g["k"], g["v"], g["beta"], g["r"], None, None, cot["dout"], cot["dS_final"],
+                        cot["dd_final"], grads["dq"], grads["dk"], grads["dv"], grads["dbeta"], grads["dr"], dd0,
+                        dS0, ws, stream)
 
     for _ in range(warmup):
         call()
@@ -393,11 +404,12 @@ def run_backward(w, g, stream, hbm, tf_peak, steps=5, warmup=2):
     torch.cuda.synchronize()
     assert pk.osdn_sync_status(stream) == 0
     ms = e0.elapsed_time(e1) / steps
-    nbytes, F = backward_bytes(w), backward_flops(w)
+    nbytes, F = backward_bytes(w) + (2 * w.B * w.T * w.H * elem(w) if gated else 0), backward_flops(w)
     t_hbm, t_tc = nbytes / (hbm * 1e9), F / (tf_peak * 1e12)
     t_roof = max(t_hbm, t_tc)
     del ws
-    return {"call": "osdn_bwd (6 kernel launches)", "ms": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),
+    return {"call": "osdn_bwd_gated (6 kernel launches), alpha ~ U(0.9, 1)" if gated else
+            "osdn_bwd (6 kernel launches)", "ms": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),
             "algorithmic_bytes": nbytes, "flops": F, "t_roofline_us": t_roof * 1e6,
             "bound": "tensor" if t_tc >= t_hbm else "hbm", "frac": t_roof / (ms / 1e3),
             "tflops": F / (ms / 1e3) / 1e12, "gbs": nbytes / (ms / 1e3) / 1e9,
@@ -542,6 +554,7 @@ def run_ours(args, world, rank, local):
         line["gated"] = run_gated(w, g, p, ws, out, Sf, stream, hbm)
     if world == 1 and not args.no_backward:
         line["backward"] = run_backward(w, g, stream, hbm, tf_peak)
+        line["backward_gated"] = run_backward(w, g, stream, hbm, tf_peak, gated=True)
     if world == 1 and not args.no_cpu_baseline:
         v_, desc, cores = oracle_sample(w, seconds=12.0)
         line["cpu_baseline"] = {"value": v_, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
