@@ -541,7 +541,9 @@ def run_ours(args, world, rank, local):
                      "step_traffic": step_traffic,
                      "step_traffic_over_method_bytes": None if step_traffic is None else step_traffic / path_bytes(w)},
         "kernels_ms": {k_: v_["ms"] for k_, v_ in kernels.items()},
-        "gpu_launches": 2 * args.steps,
+        # per step: the scan, then the chunk kernel, or (sequences split into segments) the identity
+        # fill, three chunk-kernel passes and the combine
+        "gpu_launches": (2 if pk.osdn_fwd_segments(p) == 1 else 6) * args.steps,
         "clocks": clocks.summary(),
         "wall_s_timed_region": t_wall,
     }

@@ -90,10 +90,30 @@ typedef struct {
 
 /* Bytes of device workspace osdn_fwd needs for these parameters (written to
  * *bytes). The workspace holds the scaled write keys d_t (.) k_t in the input
- * dtype plus a small status block; it is scratch owned by the caller, needs no
- * initialisation, and may be reused by the next call on the same stream.
+ * dtype [B, T, H, dk] and, when phase 2 splits the sequences into segments
+ * (osdn_fwd_segments > 1), three fp32 states per segment and head (start
+ * state, own end state, transfer; 3 * B * P * H * dv * dk * 4 bytes) and a
+ * 16 KiB tile of zeros. It is scratch owned by the caller, needs no
+ * initialisation, and may be reused by the next call on the same stream. The
+ * size depends on the SM count of the current device.
  * Returns OSDN_OK, OSDN_ERR_INVALID_ARG or OSDN_ERR_UNSUPPORTED. */
 int osdn_fwd_workspace_size(const osdn_params *p, size_t *bytes);
+
+/* Number of segments P that phase 2 (osdn_fwd, osdn_fwd_chunk and their gated
+ * forms) cuts every sequence into, written to *segments; 1 means no split.
+ * Phase 2 carries the state serially through the chunks of a sequence, so
+ * with few (b, h) units most SMs would idle. On the tensor-core path (bf16,
+ * dk = dv = 128, dense tensors) P is the largest power of two up to 16 with
+ * B * H * P <= the SM count, lowered until T is a multiple of 64 P with
+ * T / P >= 512; P < 4 is not used. Each chunk update is affine in the state
+ * (technical summary section 2.1: S <- S (I - W^T Kw) + U0^T Kw), so a
+ * segment's end state is S_start E + L, with L its end state from S = 0 and E
+ * its end state from S = I with V = 0. A split call runs the chunk kernel
+ * three times over the B * P segments (for L, for E, and for the outputs from
+ * the combined start states) plus two small kernels (identity fill,
+ * combine). The outputs equal the unsplit ones up to rounding.
+ * Errors: OSDN_ERR_INVALID_ARG (bad params, NULL segments), OSDN_ERR_UNSUPPORTED. */
+int osdn_fwd_segments(const osdn_params *p, int *segments);
 
 /* Chunkwise-parallel OSDN forward over T tokens for every (b, h).
  *   Phase 1 (preconditioner scan, section 2.2 "two phases"): d_t for every
@@ -148,11 +168,13 @@ int osdn_fwd_scan_diag(const osdn_params *p,
 /* Phase 2 of osdn_fwd alone: the chunked delta rule with the scaled write
  * keys that a preceding osdn_fwd_scan with the same parameters left in the
  * workspace (ordered before this call on the stream). Writes out and
- * final_S (nullable). Same arguments and rules as osdn_fwd. */
+ * final_S (nullable); when it splits the sequences (osdn_fwd_segments > 1)
+ * it also writes the segment scratch after the scaled keys, which it leaves
+ * unchanged. Same arguments and rules as osdn_fwd. */
 int osdn_fwd_chunk(const osdn_params *p,
                    const void *q, const void *k, const void *v, const void *beta,
                    const float *S0, void *out, float *final_S,
-                   const void *workspace, size_t workspace_bytes,
+                   void *workspace, size_t workspace_bytes,
                    void *cuda_stream);
 
 /* One recurrent decode token for every (b, h), in place (constant memory):
@@ -187,7 +209,8 @@ int osdn_step_ex(const osdn_params *p,
  * a 64-token chunk, so every gate value in [0, 1] stays in range.
  * osdn_fwd_gated: as osdn_fwd plus alpha (not NULL when T > 0); bf16 inputs
  * with dk = dv = 128 only (else OSDN_ERR_UNSUPPORTED).
- * osdn_fwd_chunk_gated: phase 2 alone, after osdn_fwd_scan on the same stream.
+ * osdn_fwd_chunk_gated: phase 2 alone, after osdn_fwd_scan on the same stream
+ * (splitting into segments as osdn_fwd_chunk does).
  * osdn_step_gated: osdn_step_ex with the decay (alpha [B, H], not NULL); every
  * dtype and width osdn_step accepts. */
 int osdn_fwd_gated(const osdn_params *p,
@@ -202,7 +225,7 @@ int osdn_fwd_chunk_gated(const osdn_params *p,
                          const void *q, const void *k, const void *v,
                          const void *beta, const void *alpha,
                          const float *S0, void *out, float *final_S,
-                         const void *workspace, size_t workspace_bytes,
+                         void *workspace, size_t workspace_bytes,
                          void *cuda_stream);
 
 int osdn_step_gated(const osdn_params *p,

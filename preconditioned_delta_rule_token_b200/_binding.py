@@ -81,6 +81,8 @@ def lib():
         P = ctypes.POINTER(osdn_params)
         L.osdn_fwd_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
         L.osdn_fwd_workspace_size.restype = ctypes.c_int
+        L.osdn_fwd_segments.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
+        L.osdn_fwd_segments.restype = ctypes.c_int
         L.osdn_fwd.argtypes = [P] + [vp] * 10 + [vp, sz, vp]
         L.osdn_fwd.restype = ctypes.c_int
         L.osdn_fwd_scan.argtypes = [P] + [vp] * 5 + [vp, sz, vp]
@@ -177,6 +179,13 @@ def _stream(stream):
 def osdn_fwd_workspace_size(params: osdn_params) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().osdn_fwd_workspace_size(ctypes.byref(params), ctypes.byref(n)))
+    return n.value
+
+
+def osdn_fwd_segments(params: osdn_params) -> int:
+    """Segments per sequence that phase 2 splits into (1: none)."""
+    n = ctypes.c_int(0)
+    _check(lib().osdn_fwd_segments(ctypes.byref(params), ctypes.byref(n)))
     return n.value
 
 

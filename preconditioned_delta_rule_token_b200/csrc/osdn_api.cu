@@ -21,6 +21,7 @@
 #include "chunk_wy.cuh"
 #include "scan_ws.cuh"
 #include "scan_seq.cuh"
+#include "segments.cuh"
 #include "step.cuh"
 
 namespace {
@@ -110,15 +111,49 @@ int check_params(const osdn_params* p, bool need_T) {
     return OSDN_OK;
 }
 
+// Number of segments phase 2 cuts each sequence into (1: none). Only the tensor-core path
+// (bf16, dk = dv = 128, dense tensors) splits, and only when the (b, h) units leave most SMs idle:
+// P is the largest power of two up to 16 with units * P <= SMs, then lowered until the segments
+// are whole 64-token chunks of at least 512 tokens; below 4 segments the three passes cost more
+// than they save.
+int seg_count(const osdn_params* p) {
+    if (p->dtype != OSDN_BF16 || p->dk != 128 || p->dv != 128 || p->T <= 0 || !dense_layout(p)) return 1;
+    int sms = 148, dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+        sms = n;
+    else
+        (void)cudaGetLastError();   // no device (host-only use): keep the B200 count
+    const long long units = (long long)p->B * p->H;
+    int P = 1;
+    while (P < 16 && units * P * 2 <= sms) P *= 2;
+    while (P >= 4 && (p->T % (64 * P) != 0 || p->T / P < 512)) P /= 2;
+    return P >= 4 ? P : 1;
+}
+
+// The forward's workspace: the scaled write keys, then (segmented phase 2 only) the start
+// states, end states and transfers of every segment, fp32 [B P, H, dv, dk] each, and a 64-token
+// tile of zeros that the transfer pass reads as V.
 struct WorkspaceLayout {
     size_t kw_off, kw_bytes, total;
+    int seg;                       // segments per sequence (1: phase 2 is not split)
+    size_t seg_S, seg_L, seg_E, seg_Z;
 };
 
 WorkspaceLayout layout_of(const osdn_params* p) {
-    WorkspaceLayout L;
+    WorkspaceLayout L{};
     L.kw_off = 0;
     L.kw_bytes = (size_t)p->B * (size_t)p->T * (size_t)p->H * (size_t)p->dk * elem_size(p->dtype);
     L.total = round_up(L.kw_bytes, 256);
+    L.seg = seg_count(p);
+    if (L.seg > 1) {
+        const size_t st = (size_t)p->B * L.seg * p->H * p->dv * p->dk * sizeof(float);
+        L.seg_S = L.total;
+        L.seg_L = L.seg_S + st;
+        L.seg_E = L.seg_L + st;
+        L.seg_Z = L.seg_E + st;
+        L.total = L.seg_Z + 64 * 128 * sizeof(__nv_bfloat16);
+    }
     if (L.total == 0) L.total = 256;
     return L;
 }
@@ -187,9 +222,12 @@ int make_token_map(CUtensorMap* m, const void* base, int B, int T, int H, int wi
 }
 
 // Phase 2 on the tensor cores (WY form, state chain fed by prepared W and U0): bf16, dk = dv = 128.
+// v_zero: v is one 64-token tile of zeros [64][128] and V is read as zeros everywhere (the map
+// covers only that tile; every other chunk and head lies outside it and is filled with zeros).
 int launch_chunk_wy(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                     const __nv_bfloat16* beta, const float* S0, __nv_bfloat16* out, float* final_S,
-                    const __nv_bfloat16* kw, cudaStream_t st, const __nv_bfloat16* alpha = nullptr) {
+                    const __nv_bfloat16* kw, cudaStream_t st, const __nv_bfloat16* alpha = nullptr,
+                    bool v_zero = false) {
     CUtensorMap mq, mk, mkw, mv, mo;
     const TokStrides s = strides_of(p);
     const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -197,7 +235,9 @@ int launch_chunk_wy(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfl
     if ((rc = make_token_map(&mq, q, p->B, p->T, p->H, 128, 64, sw, 64, s.q))) return rc;
     if ((rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, sw, 64, s.k))) return rc;
     if ((rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, sw, 64, dense_tok3(p, 128)))) return rc;
-    if ((rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 64, sw, 64, s.v))) return rc;
+    if (v_zero) rc = make_token_map(&mv, v, 1, 64, 1, 128, 64, sw, 64, osdn::Tok3{64 * 128, 128, 128});
+    else rc = make_token_map(&mv, v, p->B, p->T, p->H, 128, 64, sw, 64, s.v);
+    if (rc) return rc;
     if ((rc = make_token_map(&mo, out, p->B, p->T, p->H, 128, 64, sw, 64, s.o))) return rc;
     auto kern = alpha ? osdn::chunk_wy_kernel<true> : osdn::chunk_wy_kernel<false>;
     const size_t smem = osdn::WyLayout::kBytes;
@@ -208,6 +248,43 @@ int launch_chunk_wy(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfl
                                          g_wait_limit_ns.load());
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core chunk launch");
     return OSDN_OK;
+}
+
+// Phase 2 on the tensor cores with each sequence cut into L.seg segments (segments.cuh): the
+// chunk kernel over [B P, T / P] for the segments' own end states (S0 = 0) and transfers
+// (S0 = I, V = 0), the combine of the start states and final states, and the chunk kernel
+// again from those start states for the outputs. The first two passes also write out; the
+// last one overwrites it.
+int launch_chunk_wy_segmented(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                              const __nv_bfloat16* v, const __nv_bfloat16* beta, const __nv_bfloat16* alpha,
+                              const float* S0, __nv_bfloat16* out, float* final_S, const __nv_bfloat16* kw,
+                              char* ws, const WorkspaceLayout& L, cudaStream_t st) {
+    const int P = L.seg;
+    osdn_params ps = *p;                       // the segments as B P sequences of T / P tokens (dense)
+    ps.B = p->B * P;
+    ps.T = p->T / P;
+    if (ps.struct_size >= sizeof(osdn_params))
+        for (int i = 0; i < 3; ++i) ps.stride_q[i] = ps.stride_k[i] = ps.stride_v[i] = ps.stride_o[i] = 0;
+    float* Sst = reinterpret_cast<float*>(ws + L.seg_S);
+    float* Lb = reinterpret_cast<float*>(ws + L.seg_L);
+    float* Eb = reinterpret_cast<float*>(ws + L.seg_E);
+    auto* Z = reinterpret_cast<__nv_bfloat16*>(ws + L.seg_Z);
+    const size_t units_s = (size_t)ps.B * ps.H;
+    cudaError_t e = cudaMemsetAsync(Z, 0, 64 * 128 * sizeof(__nv_bfloat16), st);
+    if (e != cudaSuccess) return cuda_fail(e, "segment zero tile");
+    osdn::seg::identity_kernel<<<1024, 256, 0, st>>>(Sst, units_s, 128);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "segment identity launch");
+    int rc;
+    if ((rc = launch_chunk_wy(&ps, q, k, v, beta, nullptr, out, Lb, kw, st, alpha))) return rc;
+    if ((rc = launch_chunk_wy(&ps, q, k, Z, beta, Sst, out, Eb, kw, st, alpha, true))) return rc;
+    auto comb = osdn::seg::combine_kernel<128>;
+    const size_t smem = osdn::seg::CombineSmem<128>::kBytes;
+    if ((e = cudaFuncSetAttribute(comb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return cuda_fail(e, "segment combine attribute");
+    comb<<<dim3((unsigned)(p->B * p->H), 128 / osdn::seg::kRows), osdn::seg::kThreads, smem, st>>>(
+        S0, Eb, Lb, Sst, final_S, p->H, P);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "segment combine launch");
+    return launch_chunk_wy(&ps, q, k, v, beta, Sst, out, nullptr, kw, st, alpha);
 }
 
 // Phase 1 in chunk form on the tensor cores: bf16, dk = 128.
@@ -261,12 +338,18 @@ int launch_scan(const osdn_params* p, const Tin* k, const Tin* beta, const Tin* 
 }
 
 // Phase 2: chunkwise delta rule with the scaled write key.
+// ws: the whole workspace when phase 2 may use its segment scratch (NULL: never split).
 template <typename Tin>
 int launch_chunk(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v, const Tin* beta, const float* S0,
-                 Tin* out, float* final_S, const Tin* kw, cudaStream_t st) {
+                 Tin* out, float* final_S, const Tin* kw, cudaStream_t st, char* ws = nullptr) {
     if (p->T == 0) return copy_initial_state(p, nullptr, S0, final_S, nullptr, true, false, st);
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
-        if (p->dk == 128 && p->dv == 128) return launch_chunk_wy(p, q, k, v, beta, S0, out, final_S, kw, st);
+        if (p->dk == 128 && p->dv == 128) {
+            const WorkspaceLayout L = layout_of(p);
+            if (ws && L.seg > 1)
+                return launch_chunk_wy_segmented(p, q, k, v, beta, nullptr, S0, out, final_S, kw, ws, L, st);
+            return launch_chunk_wy(p, q, k, v, beta, S0, out, final_S, kw, st);
+        }
     }
     const int units = p->B * p->H;
     constexpr int DVT = 64;
@@ -293,18 +376,25 @@ int launch_chunk(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v,
 
 // Phase 2 of the gated variant: the tensor-core kernel only (bf16, dk = dv = 128).
 int launch_chunk_gated(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta,
-                       const void* alpha, const float* S0, void* out, float* final_S, const void* kw, cudaStream_t st) {
+                       const void* alpha, const float* S0, void* out, float* final_S, const void* kw, cudaStream_t st,
+                       char* ws = nullptr) {
     if (p->dtype != OSDN_BF16 || p->dk != 128 || p->dv != 128)
         return fail(OSDN_ERR_UNSUPPORTED, "the gated forward needs bf16 inputs with dk = dv = 128");
     if (p->T == 0) return copy_initial_state(p, nullptr, S0, final_S, nullptr, true, false, st);
     using T = __nv_bfloat16;
+    const WorkspaceLayout L = layout_of(p);
+    if (ws && L.seg > 1)
+        return launch_chunk_wy_segmented(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)alpha,
+                                         S0, (T*)out, final_S, (const T*)kw, ws, L, st);
     return launch_chunk_wy(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S,
                            (const T*)kw, st, (const T*)alpha);
 }
 
 // Pointer and workspace checks shared by the forward entry points.
+// keys_only: the workspace needs to hold only the scaled keys (phase 2 is never split).
 int check_fwd_args(const osdn_params* p, std::initializer_list<const void*> required,
-                   std::initializer_list<const void*> all, const void* workspace, size_t ws_bytes) {
+                   std::initializer_list<const void*> all, const void* workspace, size_t ws_bytes,
+                   bool keys_only = false) {
     if (p->T > 0) {
         for (const void* x : required)
             if (!x) return fail(OSDN_ERR_INVALID_ARG, "a required pointer (q, k, v, beta, out) is NULL");
@@ -313,7 +403,8 @@ int check_fwd_args(const osdn_params* p, std::initializer_list<const void*> requ
     for (const void* x : all)
         if (x && !aligned16(x)) return fail(OSDN_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
     if (workspace && !aligned16(workspace)) return fail(OSDN_ERR_INVALID_ARG, "every pointer must be 16-byte aligned");
-    const size_t need = layout_of(p).total;
+    const WorkspaceLayout L = layout_of(p);
+    const size_t need = keys_only ? L.kw_bytes : L.total;
     if (p->T > 0 && ws_bytes < need)
         return fail(OSDN_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
     return OSDN_OK;
@@ -492,6 +583,15 @@ int osdn_fwd_workspace_size(const osdn_params* p, size_t* bytes) {
     return OSDN_OK;
 }
 
+int osdn_fwd_segments(const osdn_params* p, int* segments) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    if (!segments) return fail(OSDN_ERR_INVALID_ARG, "segments is NULL");
+    *segments = layout_of(p).seg;
+    return OSDN_OK;
+}
+
 int osdn_fwd(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
              const float* d0, const float* S0, void* out, float* final_S, float* final_d, void* workspace,
              size_t workspace_bytes, void* cuda_stream) {
@@ -509,7 +609,8 @@ int osdn_fwd(const osdn_params* p, const void* q, const void* k, const void* v, 
         T* kw = (T*)(ws ? ws + kw_off : nullptr);
         rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
         if (rc) return rc;
-        return launch_chunk<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S, kw, st);
+        return launch_chunk<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S, kw, st,
+                               ws);
     }
     using T = float;
     T* kw = (T*)(ws ? ws + kw_off : nullptr);
@@ -535,11 +636,11 @@ int osdn_fwd_gated(const osdn_params* p, const void* q, const void* k, const voi
     T* kw = (T*)(workspace ? reinterpret_cast<char*>(workspace) + layout_of(p).kw_off : nullptr);
     rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
     if (rc) return rc;
-    return launch_chunk_gated(p, q, k, v, beta, alpha, S0, out, final_S, kw, st);
+    return launch_chunk_gated(p, q, k, v, beta, alpha, S0, out, final_S, kw, st, reinterpret_cast<char*>(workspace));
 }
 
 int osdn_fwd_chunk_gated(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta,
-                         const void* alpha, const float* S0, void* out, float* final_S, const void* workspace,
+                         const void* alpha, const float* S0, void* out, float* final_S, void* workspace,
                          size_t workspace_bytes, void* cuda_stream) {
     t_last_error.clear();
     int rc = check_params(p, true);
@@ -548,8 +649,9 @@ int osdn_fwd_chunk_gated(const osdn_params* p, const void* q, const void* k, con
     rc = check_fwd_args(p, {q, k, v, beta, out}, {q, k, v, beta, alpha, S0, out, final_S}, workspace, workspace_bytes);
     if (rc) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
-    const char* ws = reinterpret_cast<const char*>(workspace) + layout_of(p).kw_off;
-    return launch_chunk_gated(p, q, k, v, beta, alpha, S0, out, final_S, ws, st);
+    char* ws = reinterpret_cast<char*>(workspace);
+    return launch_chunk_gated(p, q, k, v, beta, alpha, S0, out, final_S, ws ? ws + layout_of(p).kw_off : nullptr, st,
+                              ws);
 }
 
 int osdn_fwd_scan(const osdn_params* p, const void* k, const void* beta, const void* r, const float* d0,
@@ -587,7 +689,7 @@ int osdn_fwd_scan_diag(const osdn_params* p, const void* k, const void* beta, co
 }
 
 int osdn_fwd_chunk(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta,
-                   const float* S0, void* out, float* final_S, const void* workspace, size_t workspace_bytes,
+                   const float* S0, void* out, float* final_S, void* workspace, size_t workspace_bytes,
                    void* cuda_stream) {
     t_last_error.clear();
     int rc = check_params(p, true);
@@ -595,11 +697,12 @@ int osdn_fwd_chunk(const osdn_params* p, const void* q, const void* k, const voi
     rc = check_fwd_args(p, {q, k, v, beta, out}, {q, k, v, beta, S0, out, final_S}, workspace, workspace_bytes);
     if (rc) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
-    const char* ws = reinterpret_cast<const char*>(workspace) + layout_of(p).kw_off;
+    char* wsb = reinterpret_cast<char*>(workspace);
+    const char* ws = wsb ? wsb + layout_of(p).kw_off : nullptr;
     if (p->dtype == OSDN_BF16) {
         using T = __nv_bfloat16;
         return launch_chunk<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S,
-                               (const T*)ws, st);
+                               (const T*)ws, st, wsb);
     }
     return launch_chunk<float>(p, (const float*)q, (const float*)k, (const float*)v, (const float*)beta, S0,
                                (float*)out, final_S, (const float*)ws, st);
@@ -621,7 +724,7 @@ int osdn_fwd_noalloc(const osdn_params* p, const void* q, const void* k, const v
         if (rc) return rc;
     }
     rc = check_fwd_args(p, {q, k, v, beta, out}, {q, k, v, beta, r, d0, S0, out, final_S, final_d}, scratch,
-                        (size_t)OSDN_NOALLOC_SCRATCH_BYTES);
+                        (size_t)OSDN_NOALLOC_SCRATCH_BYTES, true);
     if (rc) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
     if (p->dtype == OSDN_BF16) {
