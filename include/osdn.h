@@ -115,6 +115,18 @@ int osdn_fwd_workspace_size(const osdn_params *p, size_t *bytes);
  * Errors: OSDN_ERR_INVALID_ARG (bad params, NULL segments), OSDN_ERR_UNSUPPORTED. */
 int osdn_fwd_segments(const osdn_params *p, int *segments);
 
+/* Kernel launches one osdn_fwd (or osdn_fwd_gated) call makes, written to
+ * *launches: 2 without segments (scan, chunk); 6 with segments (scan, identity
+ * fill, three chunk passes, combine). With segments and one sequence (B = 1,
+ * anchored APF off) osdn_fwd overlaps the scan with phase 2: the scan runs as
+ * P launches on cuda_stream, one per segment, each from the d the previous one
+ * ended with, while two library-owned non-blocking streams (created on first
+ * use, forked from and joined back to cuda_stream by events) run the chunk
+ * passes of the first half of the segments and then of all but the last:
+ * P + 9 launches. T = 0: at most one (d filled with ones).
+ * Errors: OSDN_ERR_INVALID_ARG (bad params, NULL launches), OSDN_ERR_UNSUPPORTED. */
+int osdn_fwd_launches(const osdn_params *p, int *launches);
+
 /* Chunkwise-parallel OSDN forward over T tokens for every (b, h).
  *   Phase 1 (preconditioner scan, section 2.2 "two phases"): d_t for every
  *   token from k, beta, r and d0; the scaled write keys d_t (.) k_t go to the

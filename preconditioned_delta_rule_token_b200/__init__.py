@@ -17,11 +17,11 @@ import torch
 from ._binding import (OSDN_BF16, OSDN_ERR_CUDA, OSDN_ERR_INVALID_ARG, OSDN_ERR_TIMEOUT, OSDN_ERR_UNSUPPORTED,
                        OSDN_FP32, OSDN_OK, LIB_PATH, OsdnError, build, get_last_error, make_params, osdn_fwd,
                        osdn_fwd_chunk, osdn_fwd_scan, osdn_fwd_scan_diag,
-                       osdn_fwd_workspace_size, osdn_fwd_segments, osdn_params, osdn_set_wait_limit_ns, osdn_step, osdn_step_ex,
+                       osdn_fwd_workspace_size, osdn_fwd_segments, osdn_fwd_launches, osdn_params, osdn_set_wait_limit_ns, osdn_step, osdn_step_ex,
                        osdn_fwd_gated, osdn_fwd_chunk_gated, osdn_step_gated,
                        osdn_bwd, osdn_bwd_gated, osdn_bwd_workspace_size, osdn_sync_status)
 
-__all__ = ["forward", "backward", "step", "osdn_bwd", "osdn_bwd_gated", "osdn_bwd_workspace_size", "residual_ratio", "osdn_fwd_scan_diag", "osdn_fwd", "osdn_fwd_scan", "osdn_fwd_chunk", "osdn_step", "osdn_fwd_workspace_size", "osdn_fwd_segments", "osdn_sync_status",
+__all__ = ["forward", "backward", "step", "osdn_bwd", "osdn_bwd_gated", "osdn_bwd_workspace_size", "residual_ratio", "osdn_fwd_scan_diag", "osdn_fwd", "osdn_fwd_scan", "osdn_fwd_chunk", "osdn_step", "osdn_fwd_workspace_size", "osdn_fwd_segments", "osdn_fwd_launches", "osdn_sync_status",
            "osdn_set_wait_limit_ns", "osdn_step_ex",
            "osdn_fwd_gated", "osdn_fwd_chunk_gated", "osdn_step_gated",
            "osdn_params", "make_params", "get_last_error", "OsdnError", "build", "LIB_PATH",

@@ -83,6 +83,8 @@ def lib():
         L.osdn_fwd_workspace_size.restype = ctypes.c_int
         L.osdn_fwd_segments.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
         L.osdn_fwd_segments.restype = ctypes.c_int
+        L.osdn_fwd_launches.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
+        L.osdn_fwd_launches.restype = ctypes.c_int
         L.osdn_fwd.argtypes = [P] + [vp] * 10 + [vp, sz, vp]
         L.osdn_fwd.restype = ctypes.c_int
         L.osdn_fwd_scan.argtypes = [P] + [vp] * 5 + [vp, sz, vp]
@@ -179,6 +181,13 @@ def _stream(stream):
 def osdn_fwd_workspace_size(params: osdn_params) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().osdn_fwd_workspace_size(ctypes.byref(params), ctypes.byref(n)))
+    return n.value
+
+
+def osdn_fwd_launches(params: osdn_params) -> int:
+    """Kernel launches of one osdn_fwd call with these parameters."""
+    n = ctypes.c_int(0)
+    _check(lib().osdn_fwd_launches(ctypes.byref(params), ctypes.byref(n)))
     return n.value
 
 

@@ -133,11 +133,15 @@ int seg_count(const osdn_params* p) {
 
 // The forward's workspace: the scaled write keys, then (segmented phase 2 only) the start
 // states, end states and transfers of every segment, fp32 [B P, H, dv, dk] each, and a 64-token
-// tile of zeros that the transfer pass reads as V.
+// tile of zeros that the transfer pass reads as V. When osdn_fwd also overlaps the scan with
+// phase 2 (one sequence, plain APF): identity start states for the transfer passes, d after
+// every segment, and an output tile for the transfer passes of half the segments.
 struct WorkspaceLayout {
     size_t kw_off, kw_bytes, total;
     int seg;                       // segments per sequence (1: phase 2 is not split)
     size_t seg_S, seg_L, seg_E, seg_Z;
+    bool overlap;                  // osdn_fwd runs the scan segment by segment, phase 2 alongside
+    size_t ov_I, ov_D, ov_O;
 };
 
 WorkspaceLayout layout_of(const osdn_params* p) {
@@ -153,6 +157,14 @@ WorkspaceLayout layout_of(const osdn_params* p) {
         L.seg_E = L.seg_L + st;
         L.seg_Z = L.seg_E + st;
         L.total = L.seg_Z + 64 * 128 * sizeof(__nv_bfloat16);
+        L.overlap = p->B == 1 && !anchor_of(p);
+        if (L.overlap) {
+            const size_t seg_tokens = (size_t)p->T / L.seg * p->H;
+            L.ov_I = round_up(L.total, 256);
+            L.ov_D = L.ov_I + st;
+            L.ov_O = round_up(L.ov_D + (size_t)L.seg * p->H * p->dk * sizeof(float), 256);
+            L.total = L.ov_O + (size_t)(L.seg / 2) * seg_tokens * p->dv * sizeof(__nv_bfloat16);
+        }
     }
     if (L.total == 0) L.total = 256;
     return L;
@@ -282,9 +294,153 @@ int launch_chunk_wy_segmented(const osdn_params* p, const __nv_bfloat16* q, cons
     if ((e = cudaFuncSetAttribute(comb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
         return cuda_fail(e, "segment combine attribute");
     comb<<<dim3((unsigned)(p->B * p->H), 128 / osdn::seg::kRows), osdn::seg::kThreads, smem, st>>>(
-        S0, Eb, Lb, Sst, final_S, p->H, P);
+        S0, Eb, Lb, Sst, final_S, p->H, P, 0, P);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "segment combine launch");
     return launch_chunk_wy(&ps, q, k, v, beta, Sst, out, nullptr, kw, st, alpha);
+}
+
+// Two non-blocking streams per device for the overlapped forward, created on first use and
+// kept for the life of the process (a fork from and a join back to the caller's stream by
+// events around every use).
+int side_streams(cudaStream_t out[2]) {
+    static std::mutex mu;
+    static cudaStream_t streams[64][2] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "current device");
+    if (dev < 0 || dev >= 64) return fail(OSDN_ERR_UNSUPPORTED, "device index %d above 63", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < 2; ++i)
+        if (!streams[dev][i] && (e = cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "side stream");
+    out[0] = streams[dev][0];
+    out[1] = streams[dev][1];
+    return OSDN_OK;
+}
+
+template <typename Tin>
+int launch_scan(const osdn_params* p, const Tin* k, const Tin* beta, const Tin* r, const float* d0, float* final_d,
+                Tin* kw, cudaStream_t st, float* rho = nullptr, float* q_geo = nullptr);
+
+// osdn_fwd for one sequence (B = 1) split into P segments, with the scan overlapped with phase 2
+// (segments.cuh). The caller's stream runs the scan segment by segment, each from the d the
+// previous one ended with. The first half of the segments, then all but the last, go through the
+// passes for their own end states and transfers on two side streams as soon as the scan has
+// covered them, and through the combine and the output pass on the first side stream; the output
+// pass of the second half also covers the last segment, whose end state is the final state.
+// Consecutive segments of one sequence are a dense [n, T / P, H, d] tensor, so every launch is
+// the existing scan or chunk kernel on such a view.
+int launch_fwd_overlapped(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                          const __nv_bfloat16* v, const __nv_bfloat16* beta, const __nv_bfloat16* r,
+                          const __nv_bfloat16* alpha, const float* d0, const float* S0, __nv_bfloat16* out,
+                          float* final_S, float* final_d, char* ws, const WorkspaceLayout& L, cudaStream_t st) {
+    using T = __nv_bfloat16;
+    const int P = L.seg, half = P / 2, H = p->H, D = 128;
+    const int Ls = p->T / P;
+    const size_t segtok = (size_t)Ls * H;                 // token-heads per segment
+    const size_t sstate = (size_t)H * D * D;               // floats of one segment's states
+    auto view = [&](int nseg) {                            // nseg consecutive segments as a dense tensor
+        osdn_params v_ = *p;
+        v_.B = nseg;
+        v_.T = Ls;
+        if (v_.struct_size >= sizeof(osdn_params))
+            for (int i = 0; i < 3; ++i) v_.stride_q[i] = v_.stride_k[i] = v_.stride_v[i] = v_.stride_o[i] = 0;
+        return v_;
+    };
+    T* kw = reinterpret_cast<T*>(ws + L.kw_off);
+    float* Sst = reinterpret_cast<float*>(ws + L.seg_S);
+    float* Lb = reinterpret_cast<float*>(ws + L.seg_L);
+    float* Eb = reinterpret_cast<float*>(ws + L.seg_E);
+    T* Z = reinterpret_cast<T*>(ws + L.seg_Z);
+    float* Sid = reinterpret_cast<float*>(ws + L.ov_I);
+    float* dseg = reinterpret_cast<float*>(ws + L.ov_D);
+    T* Oe = reinterpret_cast<T*>(ws + L.ov_O);
+    auto at = [&](auto* base, int seg, int width) { return base + (size_t)seg * segtok * width; };
+    auto tok = [&](const T* base, int seg) { return base ? base + (size_t)seg * segtok : nullptr; };
+
+    cudaStream_t side[2];
+    int rc = side_streams(side);
+    if (rc) return rc;
+    cudaEvent_t ev[6];   // fork, first half scanned, all but the last scanned, all scanned, transfers, done
+    cudaError_t e = cudaSuccess;
+    int made = 0;
+    for (; made < 6 && e == cudaSuccess; ++made) e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+        for (int i = 0; i < made - 1; ++i) cudaEventDestroy(ev[i]);
+        return cuda_fail(e, "event");
+    }
+    auto chk = [&](cudaError_t x, const char* what) { return x == cudaSuccess ? OSDN_OK : cuda_fail(x, what); };
+    do {
+        // fork: the side streams start after everything before this call on the caller's stream
+        if ((rc = chk(cudaEventRecord(ev[0], st), "fork"))) break;
+        if ((rc = chk(cudaStreamWaitEvent(side[0], ev[0], 0), "fork"))) break;
+        if ((rc = chk(cudaStreamWaitEvent(side[1], ev[0], 0), "fork"))) break;
+        if ((rc = chk(cudaMemsetAsync(Z, 0, 64 * 128 * sizeof(T), side[1]), "segment zero tile"))) break;
+        osdn::seg::identity_kernel<<<1024, 256, 0, side[1]>>>(Sid, (size_t)(P - 1) * H, D);
+        if ((rc = chk(cudaGetLastError(), "segment identity launch"))) break;
+        // the scan, segment by segment, on the caller's stream
+        const osdn_params one = view(1);
+        for (int sg = 0; sg < P && !rc; ++sg) {
+            const float* din = sg == 0 ? d0 : dseg + (size_t)(sg - 1) * H * D;
+            float* dout = sg == P - 1 ? final_d : dseg + (size_t)sg * H * D;
+            rc = launch_scan<T>(&one, at(k, sg, D), tok(beta, sg), tok(r, sg), din, dout, at(kw, sg, D), st);
+            if (!rc && sg == half - 1) rc = chk(cudaEventRecord(ev[1], st), "scan event");
+            if (!rc && sg == P - 2) rc = chk(cudaEventRecord(ev[2], st), "scan event");
+        }
+        if (rc) break;
+        if ((rc = chk(cudaEventRecord(ev[3], st), "scan event"))) break;
+        auto comb = osdn::seg::combine_kernel<128>;
+        const size_t csm = osdn::seg::CombineSmem<128>::kBytes;
+        if ((rc = chk(cudaFuncSetAttribute(comb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csm),
+                      "segment combine attribute")))
+            break;
+        // segments [s0, s1): own end states (side 0) and transfers (side 1) once scanned (event ev_in),
+        // then their start states from S_in and the state after them (side 0)
+        auto halfpass = [&](int s0, int s1, cudaEvent_t ev_in, const float* S_in, float* S_after) -> int {
+            const osdn_params vw = view(s1 - s0);
+            int rr;
+            if ((rr = chk(cudaStreamWaitEvent(side[0], ev_in, 0), "segment wait"))) return rr;
+            if ((rr = chk(cudaStreamWaitEvent(side[1], ev_in, 0), "segment wait"))) return rr;
+            if ((rr = launch_chunk_wy(&vw, at(q, s0, D), at(k, s0, D), at(v, s0, D), tok(beta, s0), nullptr,
+                                      at(out, s0, D), Lb + s0 * sstate, at(kw, s0, D), side[0], tok(alpha, s0))))
+                return rr;
+            if ((rr = launch_chunk_wy(&vw, at(q, s0, D), at(k, s0, D), Z, tok(beta, s0), Sid, Oe,
+                                      Eb + s0 * sstate, at(kw, s0, D), side[1], tok(alpha, s0), true)))
+                return rr;
+            if ((rr = chk(cudaEventRecord(ev[4], side[1]), "segment event"))) return rr;
+            if ((rr = chk(cudaStreamWaitEvent(side[0], ev[4], 0), "segment wait"))) return rr;
+            comb<<<dim3((unsigned)H, D / osdn::seg::kRows), osdn::seg::kThreads, csm, side[0]>>>(
+                S_in, Eb, Lb, Sst, S_after, H, P, s0, s1 - s0);
+            return chk(cudaGetLastError(), "segment combine launch");
+        };
+        // first half: start states from S0, then its outputs
+        if ((rc = halfpass(0, half, ev[1], S0, Sst + half * sstate))) break;
+        {
+            const osdn_params vw = view(half);
+            if ((rc = launch_chunk_wy(&vw, q, k, v, beta, Sst, out, nullptr, kw, side[0], alpha))) break;
+        }
+        // segments half .. P - 2, then the outputs of half .. P - 1 once the scan is done; their end
+        // states land over the consumed own end states, and the last one is the final state
+        if ((rc = halfpass(half, P - 1, ev[2], Sst + half * sstate, Sst + (P - 1) * sstate))) break;
+        if ((rc = chk(cudaStreamWaitEvent(side[0], ev[3], 0), "segment wait"))) break;
+        {
+            const osdn_params vw = view(P - half);
+            if ((rc = launch_chunk_wy(&vw, at(q, half, D), at(k, half, D), at(v, half, D), tok(beta, half),
+                                      Sst + half * sstate, at(out, half, D), Lb + half * sstate, at(kw, half, D),
+                                      side[0], tok(alpha, half))))
+                break;
+        }
+        if (final_S &&
+            (rc = chk(cudaMemcpyAsync(final_S, Lb + (P - 1) * sstate, sstate * sizeof(float),
+                                      cudaMemcpyDeviceToDevice, side[0]),
+                      "final state copy")))
+            break;
+        // join: the caller's stream waits for both side streams (side 1 ends before ev[4], which side 0 waited for)
+        if ((rc = chk(cudaEventRecord(ev[5], side[0]), "join"))) break;
+        rc = chk(cudaStreamWaitEvent(st, ev[5], 0), "join");
+    } while (false);
+    for (int i = 0; i < 6; ++i) cudaEventDestroy(ev[i]);
+    return rc;
 }
 
 // Phase 1 in chunk form on the tensor cores: bf16, dk = 128.
@@ -310,7 +466,7 @@ int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bflo
 // Phase 1: preconditioner scan -> scaled write keys (workspace) and final d.
 template <typename Tin>
 int launch_scan(const osdn_params* p, const Tin* k, const Tin* beta, const Tin* r, const float* d0, float* final_d,
-                Tin* kw, cudaStream_t st, float* rho = nullptr, float* q_geo = nullptr) {
+                Tin* kw, cudaStream_t st, float* rho, float* q_geo) {
     if (p->T == 0) {
         if (q_geo) {   // empty sequences: the geometric mean of no ratios is 1
             const size_t n = (size_t)p->B * p->H, blocks = (n + 255) / 256;
@@ -592,6 +748,19 @@ int osdn_fwd_segments(const osdn_params* p, int* segments) {
     return OSDN_OK;
 }
 
+int osdn_fwd_launches(const osdn_params* p, int* launches) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    if (!launches) return fail(OSDN_ERR_INVALID_ARG, "launches is NULL");
+    const WorkspaceLayout L = layout_of(p);
+    if (p->T == 0) *launches = 1;                    // at most the fill of d with ones
+    else if (L.seg == 1) *launches = 2;              // scan, chunk
+    else if (!L.overlap) *launches = 6;              // scan, identity, three chunk passes, combine
+    else *launches = L.seg + 9;                      // P scans, identity, 2 x (two passes, combine, output pass)
+    return OSDN_OK;
+}
+
 int osdn_fwd(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
              const float* d0, const float* S0, void* out, float* final_S, float* final_d, void* workspace,
              size_t workspace_bytes, void* cuda_stream) {
@@ -607,6 +776,10 @@ int osdn_fwd(const osdn_params* p, const void* q, const void* k, const void* v, 
     if (p->dtype == OSDN_BF16) {
         using T = __nv_bfloat16;
         T* kw = (T*)(ws ? ws + kw_off : nullptr);
+        const WorkspaceLayout L = layout_of(p);
+        if (L.overlap)
+            return launch_fwd_overlapped(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)r,
+                                         nullptr, d0, S0, (T*)out, final_S, final_d, ws, L, st);
         rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
         if (rc) return rc;
         return launch_chunk<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S, kw, st,
@@ -634,6 +807,11 @@ int osdn_fwd_gated(const osdn_params* p, const void* q, const void* k, const voi
     cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
     using T = __nv_bfloat16;
     T* kw = (T*)(workspace ? reinterpret_cast<char*>(workspace) + layout_of(p).kw_off : nullptr);
+    const WorkspaceLayout L = layout_of(p);
+    if (L.overlap)
+        return launch_fwd_overlapped(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)r,
+                                     (const T*)alpha, d0, S0, (T*)out, final_S, final_d,
+                                     reinterpret_cast<char*>(workspace), L, st);
     rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
     if (rc) return rc;
     return launch_chunk_gated(p, q, k, v, beta, alpha, S0, out, final_S, kw, st, reinterpret_cast<char*>(workspace));

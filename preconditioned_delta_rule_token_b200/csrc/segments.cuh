@@ -11,6 +11,9 @@
 // [B P, T / P, H, d]), so the chunk kernel runs all segments at once, three
 // times: for L (S0 = 0), for E (S0 = I, V read as zeros) and, once the start
 // states S_start(p + 1) = S_start(p) E_p + L_p are combined, for the outputs.
+// With one sequence (B = 1) any run of consecutive segments is itself a dense
+// [n, T / P, H, d] tensor, so the passes can also go batch by batch while the
+// scan is still working on later segments.
 #pragma once
 #include <cstddef>
 #include <cstdint>
@@ -33,16 +36,17 @@ struct CombineSmem {
     static constexpr size_t kBytes = sizeof(float) * (size_t)(D * D + kRows * D);
 };
 
-// Start state of every segment and the final state of every sequence:
-//   S_start(0) = S0 (zeros when NULL),  S_start(p + 1) = S_start(p) E_p + L_p,
-//   final_S = S_start(P - 1) E_{P-1} + L_{P-1}  (skipped when NULL).
-// S0 and final_S are [B, H, D, D]; E, L and S_start are [B P, H, D, D] with segment p of
-// sequence b at index b P + p. Rows of S are independent, so CTA (unit, y) takes rows
-// 16 y .. 16 y + 15 of unit b H + h; every thread owns one row and 8 columns of the product.
+// Start states of segments p0 .. p0 + n - 1 of every sequence and the state after them:
+//   S_start(p0) = S0 (zeros when NULL),  S_start(p + 1) = S_start(p) E_p + L_p,
+//   S_after = S_start(p0 + n - 1) E + L of that segment  (skipped when NULL).
+// S0 and S_after are [B, H, D, D]; E, L and S_start are [B P, H, D, D] with segment p of
+// sequence b at index b P + p. (p0 = 0, n = P: every start state and the final state.)
+// Rows of S are independent, so CTA (unit, y) takes rows 16 y .. 16 y + 15 of unit b H + h;
+// every thread owns one row and 8 columns of the product.
 template <int D>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const float* __restrict__ S0, const float* __restrict__ E, const float* __restrict__ L,
-               float* __restrict__ S_start, float* __restrict__ final_S, int H, int P)
+               float* __restrict__ S_start, float* __restrict__ S_after, int H, int P, int p0, int n)
 {
     static_assert(kThreads == kRows * (D / 8), "one thread per row and 8 columns");
     extern __shared__ float sm[];
@@ -52,7 +56,7 @@ combine_kernel(const float* __restrict__ S0, const float* __restrict__ E, const 
     const int tid = threadIdx.x, r = tid / (D / 8), c0 = (tid % (D / 8)) * 8;
     for (int i = tid; i < kRows * D; i += kThreads)
         Ss[i] = S0 ? S0[((size_t)unit * D + r0 + i / D) * D + i % D] : 0.f;
-    for (int p = 0; p < P; ++p) {
+    for (int p = p0; p < p0 + n; ++p) {
         const size_t su = ((size_t)b * P + p) * H + h;
         __syncthreads();             // Ss holds S_start(p); every thread is done with Es
         for (int i = tid; i < kRows * D; i += kThreads) S_start[(su * D + r0 + i / D) * D + i % D] = Ss[i];
@@ -78,8 +82,8 @@ combine_kernel(const float* __restrict__ S0, const float* __restrict__ E, const 
         for (int j = 0; j < 8; ++j) Ss[r * D + c0 + j] = acc[j];
     }
     __syncthreads();
-    if (final_S)
-        for (int i = tid; i < kRows * D; i += kThreads) final_S[((size_t)unit * D + r0 + i / D) * D + i % D] = Ss[i];
+    if (S_after)
+        for (int i = tid; i < kRows * D; i += kThreads) S_after[((size_t)unit * D + r0 + i / D) * D + i % D] = Ss[i];
 }
 
 }  // namespace seg

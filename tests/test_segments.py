@@ -91,10 +91,15 @@ def test_segment_plan(B, T, H, dtype, dk, want):
     assert P == want
     kw = B * T * H * dk * (2 if dtype == torch.bfloat16 else 4)
     ws = pk.osdn_fwd_workspace_size(p)
+    up = lambda x: -(-x // 256) * 256
     if P == 1:
-        assert ws == max(256, -(-kw // 256) * 256)
+        assert ws == max(256, up(kw))
     else:
-        assert ws == -(-kw // 256) * 256 + 3 * B * P * H * 128 * 128 * 4 + 64 * 128 * 2
+        st = B * P * H * 128 * 128 * 4
+        want_ws = up(kw) + 3 * st + 64 * 128 * 2          # start states, own end states, transfers, zeros
+        if B == 1:   # one sequence: the scan overlaps phase 2 in osdn_fwd
+            want_ws = up(up(want_ws) + st + P * H * 128 * 4) + (P // 2) * (T // P) * H * 128 * 2
+        assert ws == want_ws
 
 
 def test_segment_plan_needs_dense_tensors():
@@ -164,3 +169,55 @@ def test_gpu_split_gated_forward_matches_oracle(lo):
         torch.bfloat16)
     _check_against_oracle(w, alpha=alpha)
     _check_against_oracle(w, alpha=alpha, split_phases=True)
+
+
+@pytest.mark.gpu
+def test_gpu_overlapped_forward_joins_the_callers_stream():
+    """One sequence: osdn_fwd overlaps the scan with phase 2 on two library streams. Called
+    twice on a non-default stream, each result read after synchronizing that stream alone:
+    both bit-identical (every launch is joined back to the caller's stream), and equal to the
+    oracle."""
+    import preconditioned_delta_rule_token_b200 as pk
+    w = _few_units(1, 2, 4096, seed=67)
+    inp = W.make_forward_inputs(w)
+    p = pk.make_params(w.B, w.T, w.H, w.dk, w.dv, inp["k"].dtype, w.eta)
+    assert pk.osdn_fwd_segments(p) == 8 and pk.osdn_fwd_launches(p) == 17
+    g = {n: _dev(x) for n, x in inp.items()}
+    s = torch.cuda.Stream()
+    res = []
+    for _ in range(2):
+        with torch.cuda.stream(s):
+            out, S, d = pk.forward(g["q"], g["k"], g["v"], g["beta"], g["r"], g["d0"], g["S0"], eta=w.eta,
+                                   stream=s)
+        s.synchronize()
+        res.append((out.cpu(), S.cpu(), d.cpu()))
+    assert pk.osdn_sync_status() == 0
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
+    f = W.to_f64
+    ro, rS, rd = oracle.fwd(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["beta"]), f(inp["r"]), f(inp["d0"]),
+                            f(inp["S0"]), eta=w.eta)
+    out, S, d = res[0]
+    errs = (slice_rel_err(out.float().numpy(), ro, (0, 2)), slice_rel_err(S.numpy(), rS, (0, 1)),
+            slice_rel_err(d.numpy(), rd, (0, 1)))
+    assert max(errs) <= BF16_TOL, errs
+
+
+@pytest.mark.gpu
+def test_gpu_split_anchored_single_sequence():
+    # anchored APF: one sequence splits phase 2 but does not overlap the scan (its segments would
+    # each need the anchor d0 separately)
+    import preconditioned_delta_rule_token_b200 as pk
+    w = _few_units(1, 2, 4096, seed=68)
+    inp = W.make_forward_inputs(w)
+    p = pk.make_params(w.B, w.T, w.H, w.dk, w.dv, inp["k"].dtype, w.eta, 64, True)
+    assert pk.osdn_fwd_segments(p) == 8 and pk.osdn_fwd_launches(p) == 6
+    g = {n: _dev(x) for n, x in inp.items()}
+    out, S, d = pk.forward(g["q"], g["k"], g["v"], g["beta"], g["r"], g["d0"], g["S0"], eta=w.eta, apf_anchor=True)
+    assert pk.osdn_sync_status() == 0
+    f = W.to_f64
+    ro, rS, rd = oracle.fwd(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["beta"]), f(inp["r"]), f(inp["d0"]),
+                            f(inp["S0"]), eta=w.eta, anchor=True)
+    errs = (slice_rel_err(out.float().cpu().numpy(), ro, (0, 2)), slice_rel_err(S.cpu().numpy(), rS, (0, 1)),
+            slice_rel_err(d.cpu().numpy(), rd, (0, 1)))
+    assert max(errs) <= BF16_TOL, errs
