@@ -330,6 +330,8 @@ int osdn_bwd_gated(const osdn_params *p,
  * scan overwrites every scratch entry the chunk phase reads, so stale contents
  * from an earlier call are never used. Two calls that overlap on the GPU (for
  * example on two streams) race on the array: order them on one stream.
+ * It never splits sequences into segments (osdn_fwd_segments): where
+ * osdn_fwd splits, the two agree up to rounding; elsewhere bit for bit.
  * Errors: those of osdn_fwd; OSDN_ERR_INVALID_ARG when the scratch needed
  * exceeds OSDN_NOALLOC_SCRATCH_BYTES; OSDN_ERR_CUDA when the address lookup
  * fails. */
