@@ -105,7 +105,10 @@ int osdn_fwd_workspace_size(const osdn_params *p, size_t *bytes);
  * with few (b, h) units most SMs would idle. On the tensor-core path (bf16,
  * dk = dv = 128, dense tensors) P is the largest power of two up to 16 with
  * B * H * P <= the SM count, lowered until T is a multiple of 64 P with
- * T / P >= 512; P < 4 is not used. Each chunk update is affine in the state
+ * T / P >= 512; P < 4 is not used. One sequence (B = 1, anchored APF off)
+ * with T a multiple of 1024, T >= 8192 and 3 H <= the SM count takes P = 16:
+ * osdn_fwd then overlaps the scan with phase 2 (osdn_fwd_launches), where
+ * short segments keep the work left after the scan short. Each chunk update is affine in the state
  * (technical summary section 2.1: S <- S (I - W^T Kw) + U0^T Kw), so a
  * segment's end state is S_start E + L, with L its end state from S = 0 and E
  * its end state from S = I with V = 0. A split call runs the chunk kernel
@@ -118,12 +121,15 @@ int osdn_fwd_segments(const osdn_params *p, int *segments);
 /* Kernel launches one osdn_fwd (or osdn_fwd_gated) call makes, written to
  * *launches: 2 without segments (scan, chunk); 6 with segments (scan, identity
  * fill, three chunk passes, combine). With segments and one sequence (B = 1,
- * anchored APF off) osdn_fwd overlaps the scan with phase 2: the scan runs as
- * P launches on cuda_stream, one per segment, each from the d the previous one
- * ended with, while two library-owned non-blocking streams (created on first
- * use, forked from and joined back to cuda_stream by events) run the chunk
- * passes of the first half of the segments and then of all but the last:
- * P + 9 launches. T = 0: at most one (d filled with ones).
+ * anchored APF off) osdn_fwd overlaps the scan with phase 2. Segments
+ * 0 .. P - 2 go in batches of nb = min(P / 2, (SMs - H) / (2 H)); the scan
+ * runs on cuda_stream as one launch per batch and one for the last segment,
+ * each from the d the previous one ended with, while two library-owned
+ * non-blocking streams (created on first use, forked from and joined back to
+ * cuda_stream by events) run each batch's chunk passes as soon as the scan
+ * has covered it, and the last segment's output pass after the scan:
+ * 2 + 5 ceil((P - 1) / nb) launches.
+ * T = 0: at most one (d filled with ones).
  * Errors: OSDN_ERR_INVALID_ARG (bad params, NULL launches), OSDN_ERR_UNSUPPORTED. */
 int osdn_fwd_launches(const osdn_params *p, int *launches);
 

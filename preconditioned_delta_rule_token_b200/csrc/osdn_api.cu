@@ -116,14 +116,28 @@ int check_params(const osdn_params* p, bool need_T) {
 // P is the largest power of two up to 16 with units * P <= SMs, then lowered until the segments
 // are whole 64-token chunks of at least 512 tokens; below 4 segments the three passes cost more
 // than they save.
-int seg_count(const osdn_params* p) {
-    if (p->dtype != OSDN_BF16 || p->dk != 128 || p->dv != 128 || p->T <= 0 || !dense_layout(p)) return 1;
+int sm_count() {
     int sms = 148, dev = 0, n = 0;
     if (cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
         sms = n;
     else
         (void)cudaGetLastError();   // no device (host-only use): keep the B200 count
+    return sms;
+}
+
+// Segments per batch of the overlapped forward (one sequence, H heads): its own-end-state and
+// transfer passes run side by side next to the scan, so 2 n H + H CTAs must fit the SMs.
+int overlap_batch(int H, int P) {
+    const int nb = (sm_count() - H) / (2 * H);
+    return nb < P / 2 ? nb : P / 2;
+}
+
+int seg_count(const osdn_params* p) {
+    if (p->dtype != OSDN_BF16 || p->dk != 128 || p->dv != 128 || p->T <= 0 || !dense_layout(p)) return 1;
+    const int sms = sm_count();
+    if (p->B == 1 && !anchor_of(p) && p->T % 1024 == 0 && p->T / 16 >= 512 && overlap_batch(p->H, 16) >= 1)
+        return 16;   // one sequence, overlapped with the scan: short segments keep the tail after the scan short
     const long long units = (long long)p->B * p->H;
     int P = 1;
     while (P < 16 && units * P * 2 <= sms) P *= 2;
@@ -134,13 +148,14 @@ int seg_count(const osdn_params* p) {
 // The forward's workspace: the scaled write keys, then (segmented phase 2 only) the start
 // states, end states and transfers of every segment, fp32 [B P, H, dv, dk] each, and a 64-token
 // tile of zeros that the transfer pass reads as V. When osdn_fwd also overlaps the scan with
-// phase 2 (one sequence, plain APF): identity start states for the transfer passes, d after
-// every segment, and an output tile for the transfer passes of half the segments.
+// phase 2 (one sequence, plain APF): identity start states for the transfer passes of one batch,
+// d after every segment, and an output tile for the transfer passes of one batch.
 struct WorkspaceLayout {
     size_t kw_off, kw_bytes, total;
     int seg;                       // segments per sequence (1: phase 2 is not split)
     size_t seg_S, seg_L, seg_E, seg_Z;
     bool overlap;                  // osdn_fwd runs the scan segment by segment, phase 2 alongside
+    int ov_batch;                  // segments per batch of the overlapped passes
     size_t ov_I, ov_D, ov_O;
 };
 
@@ -157,13 +172,15 @@ WorkspaceLayout layout_of(const osdn_params* p) {
         L.seg_E = L.seg_L + st;
         L.seg_Z = L.seg_E + st;
         L.total = L.seg_Z + 64 * 128 * sizeof(__nv_bfloat16);
-        L.overlap = p->B == 1 && !anchor_of(p);
+        L.ov_batch = p->B == 1 && !anchor_of(p) ? overlap_batch(p->H, L.seg) : 0;
+        L.overlap = L.ov_batch >= 1;
         if (L.overlap) {
             const size_t seg_tokens = (size_t)p->T / L.seg * p->H;
+            const size_t batch_states = (size_t)L.ov_batch * p->H * p->dv * p->dk * sizeof(float);
             L.ov_I = round_up(L.total, 256);
-            L.ov_D = L.ov_I + st;
+            L.ov_D = L.ov_I + batch_states;
             L.ov_O = round_up(L.ov_D + (size_t)L.seg * p->H * p->dk * sizeof(float), 256);
-            L.total = L.ov_O + (size_t)(L.seg / 2) * seg_tokens * p->dv * sizeof(__nv_bfloat16);
+            L.total = L.ov_O + (size_t)L.ov_batch * seg_tokens * p->dv * sizeof(__nv_bfloat16);
         }
     }
     if (L.total == 0) L.total = 256;
@@ -323,19 +340,21 @@ int launch_scan(const osdn_params* p, const Tin* k, const Tin* beta, const Tin* 
                 Tin* kw, cudaStream_t st, float* rho = nullptr, float* q_geo = nullptr);
 
 // osdn_fwd for one sequence (B = 1) split into P segments, with the scan overlapped with phase 2
-// (segments.cuh). The caller's stream runs the scan segment by segment, each from the d the
-// previous one ended with. The first half of the segments, then all but the last, go through the
-// passes for their own end states and transfers on two side streams as soon as the scan has
-// covered them, and through the combine and the output pass on the first side stream; the output
-// pass of the second half also covers the last segment, whose end state is the final state.
-// Consecutive segments of one sequence are a dense [n, T / P, H, d] tensor, so every launch is
-// the existing scan or chunk kernel on such a view.
+// (segments.cuh). Segments 0 .. P - 2 go in batches of L.ov_batch. The caller's stream runs the
+// scan batch by batch and then over the last segment, each launch from the d the previous one
+// ended with. As soon as the scan has covered a batch, two side streams run its passes for the
+// own end states and the transfers
+// side by side, then the first side stream combines the batch's start states and runs its output
+// pass; the output pass of the last batch also covers the last segment, after the scan ends, and
+// that segment's end state is the final state. Consecutive segments of one sequence are a dense
+// [n, T / P, H, d] tensor, so every launch is the existing scan or chunk kernel on such a view.
 int launch_fwd_overlapped(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k,
                           const __nv_bfloat16* v, const __nv_bfloat16* beta, const __nv_bfloat16* r,
                           const __nv_bfloat16* alpha, const float* d0, const float* S0, __nv_bfloat16* out,
                           float* final_S, float* final_d, char* ws, const WorkspaceLayout& L, cudaStream_t st) {
     using T = __nv_bfloat16;
-    const int P = L.seg, half = P / 2, H = p->H, D = 128;
+    const int P = L.seg, nb = L.ov_batch, H = p->H, D = 128;
+    const int nbatch = (P - 1 + nb - 1) / nb;             // batches over segments 0 .. P - 2
     const int Ls = p->T / P;
     const size_t segtok = (size_t)Ls * H;                 // token-heads per segment
     const size_t sstate = (size_t)H * D * D;               // floats of one segment's states
@@ -361,85 +380,86 @@ int launch_fwd_overlapped(const osdn_params* p, const __nv_bfloat16* q, const __
     cudaStream_t side[2];
     int rc = side_streams(side);
     if (rc) return rc;
-    cudaEvent_t ev[6];   // fork, first half scanned, all but the last scanned, all scanned, transfers, done
+    // events: fork, scan end, join, and per batch: scanned, transfers done
+    const int nev = 3 + 2 * nbatch;
+    cudaEvent_t ev[3 + 2 * 16];
     cudaError_t e = cudaSuccess;
     int made = 0;
-    for (; made < 6 && e == cudaSuccess; ++made) e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming);
+    for (; made < nev; ++made)
+        if ((e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming)) != cudaSuccess) break;
     if (e != cudaSuccess) {
-        for (int i = 0; i < made - 1; ++i) cudaEventDestroy(ev[i]);
+        for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
         return cuda_fail(e, "event");
     }
+    cudaEvent_t ev_fork = ev[0], ev_scanned_all = ev[1], ev_join = ev[2];
+    auto ev_scanned = [&](int bt) { return ev[3 + 2 * bt]; };
+    auto ev_transfers = [&](int bt) { return ev[4 + 2 * bt]; };
     auto chk = [&](cudaError_t x, const char* what) { return x == cudaSuccess ? OSDN_OK : cuda_fail(x, what); };
     do {
         // fork: the side streams start after everything before this call on the caller's stream
-        if ((rc = chk(cudaEventRecord(ev[0], st), "fork"))) break;
-        if ((rc = chk(cudaStreamWaitEvent(side[0], ev[0], 0), "fork"))) break;
-        if ((rc = chk(cudaStreamWaitEvent(side[1], ev[0], 0), "fork"))) break;
+        if ((rc = chk(cudaEventRecord(ev_fork, st), "fork"))) break;
+        if ((rc = chk(cudaStreamWaitEvent(side[0], ev_fork, 0), "fork"))) break;
+        if ((rc = chk(cudaStreamWaitEvent(side[1], ev_fork, 0), "fork"))) break;
         if ((rc = chk(cudaMemsetAsync(Z, 0, 64 * 128 * sizeof(T), side[1]), "segment zero tile"))) break;
-        osdn::seg::identity_kernel<<<1024, 256, 0, side[1]>>>(Sid, (size_t)(P - 1) * H, D);
+        osdn::seg::identity_kernel<<<1024, 256, 0, side[1]>>>(Sid, (size_t)nb * H, D);
         if ((rc = chk(cudaGetLastError(), "segment identity launch"))) break;
-        // the scan, segment by segment, on the caller's stream
-        const osdn_params one = view(1);
-        for (int sg = 0; sg < P && !rc; ++sg) {
-            const float* din = sg == 0 ? d0 : dseg + (size_t)(sg - 1) * H * D;
-            float* dout = sg == P - 1 ? final_d : dseg + (size_t)sg * H * D;
-            rc = launch_scan<T>(&one, at(k, sg, D), tok(beta, sg), tok(r, sg), din, dout, at(kw, sg, D), st);
-            if (!rc && sg == half - 1) rc = chk(cudaEventRecord(ev[1], st), "scan event");
-            if (!rc && sg == P - 2) rc = chk(cudaEventRecord(ev[2], st), "scan event");
+        // the scan on the caller's stream: one launch per batch (its segments as one run of tokens),
+        // then one for the last segment; d after each launch goes to the next, an event after each batch
+        for (int bt = 0; bt <= nbatch && !rc; ++bt) {
+            const int s0 = bt == nbatch ? P - 1 : bt * nb;
+            const int s1 = bt == nbatch ? P : (s0 + nb < P - 1 ? s0 + nb : P - 1);
+            osdn_params run = view(1);
+            run.T = (s1 - s0) * Ls;
+            const float* din = bt == 0 ? d0 : dseg + (size_t)(bt - 1) * H * D;
+            float* dout = bt == nbatch ? final_d : dseg + (size_t)bt * H * D;
+            rc = launch_scan<T>(&run, at(k, s0, D), tok(beta, s0), tok(r, s0), din, dout, at(kw, s0, D), st);
+            if (!rc && bt < nbatch) rc = chk(cudaEventRecord(ev_scanned(bt), st), "scan event");
         }
         if (rc) break;
-        if ((rc = chk(cudaEventRecord(ev[3], st), "scan event"))) break;
+        if ((rc = chk(cudaEventRecord(ev_scanned_all, st), "scan event"))) break;
         auto comb = osdn::seg::combine_kernel<128>;
         const size_t csm = osdn::seg::CombineSmem<128>::kBytes;
         if ((rc = chk(cudaFuncSetAttribute(comb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csm),
                       "segment combine attribute")))
             break;
-        // segments [s0, s1): own end states (side 0) and transfers (side 1) once scanned (event ev_in),
-        // then their start states from S_in and the state after them (side 0)
-        auto halfpass = [&](int s0, int s1, cudaEvent_t ev_in, const float* S_in, float* S_after) -> int {
+        for (int bt = 0; bt < nbatch && !rc; ++bt) {
+            const int s0 = bt * nb, s1 = s0 + nb < P - 1 ? s0 + nb : P - 1;
             const osdn_params vw = view(s1 - s0);
-            int rr;
-            if ((rr = chk(cudaStreamWaitEvent(side[0], ev_in, 0), "segment wait"))) return rr;
-            if ((rr = chk(cudaStreamWaitEvent(side[1], ev_in, 0), "segment wait"))) return rr;
-            if ((rr = launch_chunk_wy(&vw, at(q, s0, D), at(k, s0, D), at(v, s0, D), tok(beta, s0), nullptr,
+            // own end states (side 0) and transfers (side 1) once the batch is scanned
+            if ((rc = chk(cudaStreamWaitEvent(side[0], ev_scanned(bt), 0), "segment wait"))) break;
+            if ((rc = chk(cudaStreamWaitEvent(side[1], ev_scanned(bt), 0), "segment wait"))) break;
+            if ((rc = launch_chunk_wy(&vw, at(q, s0, D), at(k, s0, D), at(v, s0, D), tok(beta, s0), nullptr,
                                       at(out, s0, D), Lb + s0 * sstate, at(kw, s0, D), side[0], tok(alpha, s0))))
-                return rr;
-            if ((rr = launch_chunk_wy(&vw, at(q, s0, D), at(k, s0, D), Z, tok(beta, s0), Sid, Oe,
-                                      Eb + s0 * sstate, at(kw, s0, D), side[1], tok(alpha, s0), true)))
-                return rr;
-            if ((rr = chk(cudaEventRecord(ev[4], side[1]), "segment event"))) return rr;
-            if ((rr = chk(cudaStreamWaitEvent(side[0], ev[4], 0), "segment wait"))) return rr;
-            comb<<<dim3((unsigned)H, D / osdn::seg::kRows), osdn::seg::kThreads, csm, side[0]>>>(
-                S_in, Eb, Lb, Sst, S_after, H, P, s0, s1 - s0);
-            return chk(cudaGetLastError(), "segment combine launch");
-        };
-        // first half: start states from S0, then its outputs
-        if ((rc = halfpass(0, half, ev[1], S0, Sst + half * sstate))) break;
-        {
-            const osdn_params vw = view(half);
-            if ((rc = launch_chunk_wy(&vw, q, k, v, beta, Sst, out, nullptr, kw, side[0], alpha))) break;
-        }
-        // segments half .. P - 2, then the outputs of half .. P - 1 once the scan is done; their end
-        // states land over the consumed own end states, and the last one is the final state
-        if ((rc = halfpass(half, P - 1, ev[2], Sst + half * sstate, Sst + (P - 1) * sstate))) break;
-        if ((rc = chk(cudaStreamWaitEvent(side[0], ev[3], 0), "segment wait"))) break;
-        {
-            const osdn_params vw = view(P - half);
-            if ((rc = launch_chunk_wy(&vw, at(q, half, D), at(k, half, D), at(v, half, D), tok(beta, half),
-                                      Sst + half * sstate, at(out, half, D), Lb + half * sstate, at(kw, half, D),
-                                      side[0], tok(alpha, half))))
                 break;
+            if ((rc = launch_chunk_wy(&vw, at(q, s0, D), at(k, s0, D), Z, tok(beta, s0), Sid, Oe, Eb + s0 * sstate,
+                                      at(kw, s0, D), side[1], tok(alpha, s0), true)))
+                break;
+            if ((rc = chk(cudaEventRecord(ev_transfers(bt), side[1]), "segment event"))) break;
+            if ((rc = chk(cudaStreamWaitEvent(side[0], ev_transfers(bt), 0), "segment wait"))) break;
+            // start states of the batch from S_start(s0) (S0 for the first), and S_start(s1) after it
+            comb<<<dim3((unsigned)H, D / osdn::seg::kRows), osdn::seg::kThreads, csm, side[0]>>>(
+                bt == 0 ? S0 : Sst + s0 * sstate, Eb, Lb, Sst, Sst + s1 * sstate, H, P, s0, s1 - s0);
+            if ((rc = chk(cudaGetLastError(), "segment combine launch"))) break;
+            // the batch's outputs; the last batch also takes the last segment once the scan is done,
+            // with end states over the consumed own end states (the last one is the final state)
+            const bool last = bt == nbatch - 1;
+            if (last && (rc = chk(cudaStreamWaitEvent(side[0], ev_scanned_all, 0), "segment wait"))) break;
+            const osdn_params vo = view(last ? P - s0 : s1 - s0);
+            rc = launch_chunk_wy(&vo, at(q, s0, D), at(k, s0, D), at(v, s0, D), tok(beta, s0), Sst + s0 * sstate,
+                                 at(out, s0, D), last ? Lb + s0 * sstate : nullptr, at(kw, s0, D), side[0],
+                                 tok(alpha, s0));
         }
+        if (rc) break;
         if (final_S &&
             (rc = chk(cudaMemcpyAsync(final_S, Lb + (P - 1) * sstate, sstate * sizeof(float),
                                       cudaMemcpyDeviceToDevice, side[0]),
                       "final state copy")))
             break;
-        // join: the caller's stream waits for both side streams (side 1 ends before ev[4], which side 0 waited for)
-        if ((rc = chk(cudaEventRecord(ev[5], side[0]), "join"))) break;
-        rc = chk(cudaStreamWaitEvent(st, ev[5], 0), "join");
+        // join: the caller's stream waits for side 0, which has waited for every event of side 1
+        if ((rc = chk(cudaEventRecord(ev_join, side[0]), "join"))) break;
+        rc = chk(cudaStreamWaitEvent(st, ev_join, 0), "join");
     } while (false);
-    for (int i = 0; i < 6; ++i) cudaEventDestroy(ev[i]);
+    for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
     return rc;
 }
 
@@ -757,7 +777,8 @@ int osdn_fwd_launches(const osdn_params* p, int* launches) {
     if (p->T == 0) *launches = 1;                    // at most the fill of d with ones
     else if (L.seg == 1) *launches = 2;              // scan, chunk
     else if (!L.overlap) *launches = 6;              // scan, identity, three chunk passes, combine
-    else *launches = L.seg + 9;                      // P scans, identity, 2 x (two passes, combine, output pass)
+    else   // identity, last-segment scan, per batch a scan, two passes, combine, output pass
+        *launches = 2 + 5 * ((L.seg - 1 + L.ov_batch - 1) / L.ov_batch);
     return OSDN_OK;
 }
 
