@@ -613,8 +613,11 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
         static_assert(LDC == tri::LD, "the blocked inverse takes the 68-float row stride");
         tri::tril_inv64_inplace(As, tid >> 5, tid & 31, [] { asm volatile("bar.sync 1, 128;" ::: "memory"); });
     }
-    if (gated)   // W = T diag(gamma) Kb: Kb rows x gamma_t (the Gram above used them unscaled)
-        for (int idx = tid; idx < C * DK; idx += NTHR) Kb[(idx / DK) * LDK + idx % DK] *= ex2(gs[idx / DK]);
+    if (gated) {   // W = T diag(gamma) Kb: Kb rows x gamma_t (the Gram above used them unscaled)
+        if (tid < C) bs[tid] = ex2(gs[tid]);   // beta is no longer needed: gamma_t in its place
+        __syncthreads();
+        for (int idx = tid; idx < C * DK; idx += NTHR) Kb[(idx / DK) * LDK + idx % DK] *= bs[idx / DK];
+    }
     __syncthreads();
     store_rows<C, C>(t_g, C, Tm, LDC);
     cta_gemm<SPLIT>(C, DK, C, Mat<LDC, 1>{Tm}, Mat<LDK, 1>{Kb},
@@ -640,8 +643,9 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
 template <int DK, int DVT>
 struct StateSmem {
     static constexpr int LDK = DK + 4, LDT = DVT + 4;
-    static constexpr size_t kFwdBytes = sizeof(float) * (size_t)(DVT * LDK + 2 * C * LDK + C * LDT + C);
-    static constexpr size_t kBwdBytes = sizeof(float) * (size_t)(DVT * LDK + C * LDC + 2 * C * LDT + 2 * C * LDK + C);
+    static constexpr size_t kFwdBytes = sizeof(float) * (size_t)(DVT * LDK + 2 * C * LDK + C * LDT + 2 * C);
+    static constexpr size_t kBwdBytes =
+        sizeof(float) * (size_t)(DVT * LDK + C * LDC + 2 * C * LDT + 2 * C * LDK + 3 * C);
 };
 
 template <int DK, int DV, int DVT, typename Tin>
@@ -657,6 +661,7 @@ bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout 
     float* Kws = Ws + C * LDK;       // [C][LDK] Kw
     float* Vs = Kws + C * LDK;       // [C][LDT] U0, then Vn (columns of the tile)
     float* gs = Vs + C * LDT;        // [C] gated: log2 gamma_t
+    float* rh = gs + C;              // [C] gated: rho_t = gamma_C / gamma_t
 
     const int tid = threadIdx.x;
     const int unit = blockIdx.x / NTILE, v0 = (blockIdx.x % NTILE) * DVT;
@@ -693,8 +698,10 @@ bwd_state_f_kernel(const float* __restrict__ S0, float* __restrict__ ws, Layout 
         __syncthreads();
         if (gated) {   // S' = gamma_C S + Vn^T diag(rho) Kw
             const float gl = gs[C - 1], gc = ex2(gl);
+            if (tid < C) rh[tid] = ex2(gl - gs[tid]);
             for (int idx = tid; idx < DVT * DK; idx += NTHR) Ss[(idx / DK) * LDK + idx % DK] *= gc;
-            for (int idx = tid; idx < C * DK; idx += NTHR) Kws[(idx / DK) * LDK + idx % DK] *= ex2(gl - gs[idx / DK]);
+            __syncthreads();
+            for (int idx = tid; idx < C * DK; idx += NTHR) Kws[(idx / DK) * LDK + idx % DK] *= rh[idx / DK];
             __syncthreads();
         }
         cta_gemm<SPLIT>(DVT, DK, C, Mat<1, LDT>{Vs}, Mat<LDK, 1>{Kws},
@@ -719,6 +726,8 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
     float* B1 = dVs + C * LDT;       // [C][LDK] Kw, then W
     float* B2 = B1 + C * LDK;        // [C][LDK] Q
     float* gs = B2 + C * LDK;        // [C] gated: log2 gamma_t
+    float* rh = gs + C;              // [C] gated: rho_t = gamma_C / gamma_t
+    float* gm = rh + C;              // [C] gated: gamma_t
 
     const int tid = threadIdx.x;
     const int unit = blockIdx.x / NTILE, v0 = (blockIdx.x % NTILE) * DVT, b = unit / H, h = unit % H;
@@ -753,11 +762,15 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
         cp_async_wait_all();
         __syncthreads();
         if (gated) {   // Kw rows x rho_t and Q rows x gamma_t
-            const float gl = gs[C - 1];
+            if (tid < C) {
+                rh[tid] = ex2(gs[C - 1] - gs[tid]);
+                gm[tid] = ex2(gs[tid]);
+            }
+            __syncthreads();
             for (int idx = tid; idx < C * DK; idx += NTHR) {
                 const int t = idx / DK, i = idx % DK;
-                B1[t * LDK + i] *= ex2(gl - gs[t]);
-                B2[t * LDK + i] *= ex2(gs[t]);
+                B1[t * LDK + i] *= rh[t];
+                B2[t * LDK + i] *= gm[t];
             }
             __syncthreads();
         }
@@ -797,7 +810,11 @@ bwd_state_b_kernel(const Tin* __restrict__ dout, const Tin* __restrict__ q, cons
 // the rows t >= m of dO S and of T^T dW, the rows j < m of Vn dS', and <dS', S>. No
 // difference of large terms is taken, so dalpha keeps its relative accuracy for gates
 // near 0 (where the chunk-local dG form, a reverse cumulative sum over 1 / alpha_m,
-// cancels).
+// cancels). With G the in-chunk cumulative clamped log2 alpha (G_{-1} = 0), the factor of
+// pair (t, j) is 2^(G_t - G_j - l_m) = 2^(G_t - G_m) 2^(G_{m-1} - G_j), both at most 1, so
+//   dalpha_m = sum_{t >= m} 2^(G_t - G_m) (Y_tm + a_t 2^G_{m-1})
+//              + 2^(G_C - G_m) (sum_{j < m} W_mj y_j + <dS', S> 2^G_{m-1}),
+// with W_mj = 2^(G_{m-1} - G_j) (j < m) and Y = X' W^T, one 64 x 64 x 64 product.
 constexpr int J = 32;           // dv tile of the gradient kernel
 constexpr int LDJ = J + 4;
 
@@ -1078,20 +1095,29 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         }
     __syncthreads();
     if (tid < C) dbp_g[tid] = dbs[tid];
-    if (gated) {   // dalpha_m, warp w taking tokens w, w + 16, ..: lanes split each sum
+    if (gated) {   // dalpha: W over the key-side buffers, Y = X' W^T, then warp w takes tokens w, w + 16, ..
+        float* Wm = Xs;              // [C][LDC] W_mj
+        float* Ym = Gs;              // [C][LDC] Y_tm
+        for (int idx = tid; idx < C * C; idx += NTHR) {
+            const int m = idx / C, j = idx % C;
+            Wm[m * LDC + j] = j < m ? ex2((m > 0 ? gsm[m - 1] : 0.f) - gsm[j]) : 0.f;
+        }
+        __syncthreads();
+        cta_gemm<SPLIT>(C, C, C, Mat<LDC, 1>{Xg}, Mat<1, LDC>{Wm},
+                        [&](int t, int m, float x0, float x1) { store2(Ym + t * LDC + m, x0, x1); });
+        __syncthreads();
         const float gl = gsm[C - 1];
         for (int m = warp; m < Tc; m += NTHR / 32) {
-            const float lm = lsm[m];
-            float s = 0.f;
-            for (int t = m + lane; t < C; t += 32) s = fmaf(av[t], ex2(gsm[t] - lm), s);
-            for (int j = lane; j < m; j += 32) s = fmaf(yr[j], ex2(gl - gsm[j] - lm), s);
-            for (int e = lane; e < (C - m) * m; e += 32) {   // rows t >= m, columns j < m
-                const int t = m + e / m, j = e % m;
-                s = fmaf(Xg[t * LDC + j], ex2(gsm[t] - gsm[j] - lm), s);
-            }
+            const float gmm = gsm[m], gp = ex2(m > 0 ? gsm[m - 1] : 0.f);
+            float s = 0.f, u = 0.f;
+            for (int t = m + lane; t < C; t += 32) s = fmaf(ex2(gsm[t] - gmm), fmaf(av[t], gp, Ym[t * LDC + m]), s);
+            for (int j = lane; j < m; j += 32) u = fmaf(Wm[m * LDC + j], yr[j], u);
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-            if (lane == 0) dalpha[tok(m)] = from_f32<Tin>(fmaf(*csd, ex2(gl - lm), s));
+            for (int off = 16; off > 0; off >>= 1) {
+                s += __shfl_xor_sync(0xffffffffu, s, off);
+                u += __shfl_xor_sync(0xffffffffu, u, off);
+            }
+            if (lane == 0) dalpha[tok(m)] = from_f32<Tin>(fmaf(ex2(gl - gmm), fmaf(*csd, gp, u), s));
         }
     }
     }

@@ -93,7 +93,12 @@ def chunk_backward(q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, eta, anch
                    + c 2^(L_C - l_m) + sum_{t >= m > j} X'_tj 2^(L_t - L_j - l_m),
     l = log2 alpha (clamped at -120, so alpha = 0 is allowed), L its in-chunk cumulative sum,
     a_t = <dO_t, (Q S^T)_t> + beta_t <(T^T dW)_t, K_t>, y_j = <Vn_j, dS' Kw_j>, c = <dS', S>,
-    X' = X with R divided out. Gamma and every ratio are taken as 2^(differences of L)."""
+    X' = X with R divided out. Gamma and every ratio are taken as 2^(differences of L).
+    The "factorized" form (the kernel's) splits each exponent into two non-positive parts,
+    L_t - L_j - l_m = (L_t - L_m) + (L_{m-1} - L_j), so the pair sums are one matrix product
+    Y = X' W^T with W_mj = 2^(L_{m-1} - L_j) (j < m):
+        dalpha_m = sum_{t >= m} 2^(L_t - L_m) (Y_tm + a_t 2^L_{m-1})
+                   + 2^(L_C - L_m) (sum_{j < m} W_mj y_j + c 2^L_{m-1})."""
     T, dk = k.shape
     dv = v.shape[1]
     r = np.ones(T) if r is None else r
@@ -152,6 +157,20 @@ def chunk_backward(q, k, v, beta, r, d0, S0, dout, dS_final, dd_final, eta, anch
             dG = g * (dO * (Q @ Sc.T)).sum(1) + g * be * (TdW * K).sum(1) + X.sum(1) - X.sum(0) - Yr
             dG[-1] += g[-1] * (dS * Sc).sum() + Yr.sum()
             dalpha[sl] = np.cumsum(dG[::-1])[::-1] / alpha[sl]
+        elif gated and dalpha_form == "factorized":
+            Xp = np.tril(dA * (Kb @ Kw.T) + dPm * (Q @ Kw.T), -1)
+            a = (dO * (Q @ Sc.T)).sum(1) + be * (TdW * K).sum(1)
+            y = ((Vn @ dS) * Kw).sum(1)
+            cs = (dS * Sc).sum()
+            n = len(L)
+            Lm1 = np.concatenate([[0.0], L[:-1]])                 # L_{m-1}, with L_{-1} = 0
+            Wf = np.tril(2.0 ** np.minimum(Lm1[:, None] - L[None, :], 0.0), -1)
+            Y = Xp @ Wf.T
+            da = np.zeros(n)
+            for m in range(n):
+                da[m] = ((2.0 ** (L[m:] - L[m]) * (Y[m:, m] + a[m:] * 2.0 ** Lm1[m])).sum()
+                         + 2.0 ** (L[-1] - L[m]) * ((Wf[m, :m] * y[:m]).sum() + cs * 2.0 ** Lm1[m]))
+            dalpha[sl] = da
         elif gated:
             Xp = np.tril(dA * (Kb @ Kw.T) + dPm * (Q @ Kw.T), -1)
             a = (dO * (Q @ Sc.T)).sum(1) + be * (TdW * K).sum(1)
@@ -262,6 +281,11 @@ def test_gated_chunk_adjoint_with_zero_gates(T, C):
         np.testing.assert_allclose(got[name], want, rtol=1e-7, atol=1e-9 * max(1.0, np.abs(want).max()),
                                    err_msg=name)
     assert np.all(np.isfinite(got["dalpha"]))
+    got_f = chunk_backward(u(c["q"]), u(c["k"]), u(c["v"]), u(c["beta"]), u(c["r"]), c["d0"][0, 0], c["S0"][0, 0],
+                           u(cot["dout"]), cot["dS_final"][0, 0], cot["dd_final"][0, 0], eta, False, C,
+                           alpha=u(alpha), dalpha_form="factorized")
+    want = u(ref["dalpha"])
+    np.testing.assert_allclose(got_f["dalpha"], want, rtol=1e-7, atol=1e-9 * max(1.0, np.abs(want).max()))
 
 
 def chunk_dchain(k, beta, r, dD, dd_final, eta, L):
