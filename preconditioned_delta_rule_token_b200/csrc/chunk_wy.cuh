@@ -138,7 +138,7 @@ struct ColsToRows {
     // both halves of a 64-column block (tokens 0..63), one after the other
     __device__ __forceinline__ void copy64(uint32_t taddr, uint8_t* tile, uint32_t half_stride, int m0, float s,
                                            int lane) {
-#pragma unroll
+#pragma unroll 1
         for (int part = 0; part < 2; ++part) {
             load(taddr + 32 * part);
             tc::tmem_wait_ld();
@@ -354,7 +354,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // Vn^T = U0^T - S W^T (D columns 0-63) -> bf16 over columns 0-31 (A operand of GBS and GBO)
             if (tc::named_sync_or(BAR_STATE, 128, !wait(L::BA, c & 1))) break;
             tc::tc_fence_after();
-#pragma unroll
+#pragma unroll 1
             for (int hv = 0; hv < 2; ++hv) {   // in place, 32 columns at a time (the bf16 half lands on consumed columns)
                 uint32_t x[32], w[16];
                 tc::tmem_ld32(tl + COL_D + 32 * hv, x);
@@ -375,7 +375,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (tc::named_sync_or(BAR_STATE, 128, !wait(L::BS, c & 1))) break;
             tc::tc_fence_after();
             const float gnext = (GATED && c + 1 < nchunks) ? sfu_exp2(nxt.last()) : 1.f;
-#pragma unroll
+#pragma unroll 1
             for (int qt = 0; qt < 4; ++qt) {
                 uint32_t x[32];
                 tc::tmem_ld32(tl + COL_S + qt * 32, x);
@@ -454,41 +454,29 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             if (GATED) tc::named_sync(BAR_PREP, 128);
             const float gt = GATED ? glog[gtid & 63] : 0.f;
-            {
-                uint32_t r[64];
-                tc::tmem_ld32(tl + COL_R1 + (c % 3) * 64, *reinterpret_cast<uint32_t(*)[32]>(r));
-                tc::tmem_ld32(tl + COL_R1 + (c % 3) * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+            // 8 columns per TMEM load in a rolled loop (small code: the four roles share an instruction cache)
+#pragma unroll 1
+            for (int jb = 0; jb < 64; jb += 8) {
+                uint32_t r8[8];
+                tc::tmem_ld8(tl + COL_R1 + (c % 3) * 64 + jb, r8);
                 tc::tmem_wait_ld();
-                if (gtid < C) {   // A[t][j] = beta_t <k_t, kw_j> for j < t, zero elsewhere (full rows); gated x gamma_t / gamma_j
+                float sj[8], x[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) sj[u] = GATED ? sfu_exp2(gt - glog[jb + u]) : 1.f;
+                if (gtid < C) {   // A[t][j] = beta_t <k_t, kw_j> for j < t, zero elsewhere; gated x gamma_t / gamma_j
                     const int t = gtid;
 #pragma unroll
-                    for (int j = 0; j < 64; j += 4) {
-                        float a4[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            float sj = bt;
-                            if (GATED) sj *= sfu_exp2(gt - glog[j + u]);
-                            a4[u] = (j + u < t) ? sj * __uint_as_float(r[j + u]) : 0.f;
-                        }
-                        *reinterpret_cast<float4*>(AF + t * L::LDF + j) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-                    }
+                    for (int u = 0; u < 8; ++u) x[u] = (jb + u < t) ? bt * sj[u] * __uint_as_float(r8[u]) : 0.f;
+                    *reinterpret_cast<float4*>(AF + t * L::LDF + jb) = make_float4(x[0], x[1], x[2], x[3]);
+                    *reinterpret_cast<float4*>(AF + t * L::LDF + jb + 4) = make_float4(x[4], x[5], x[6], x[7]);
                 } else {          // P[t][j] = <q_t, kw_j> for j <= t; gated x gamma_t / gamma_j
                     const int t = gtid - C;
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        float x[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int j = cc * 8 + e;
-                            float sj = 1.f;
-                            if (GATED) sj = sfu_exp2(gt - glog[j]);
-                            x[e] = (j <= t) ? sj * __uint_as_float(r[j]) : 0.f;
-                        }
-                        uint4 pk;
-                        pk.x = tc::pack_bf16(x[0], x[1]); pk.y = tc::pack_bf16(x[2], x[3]);
-                        pk.z = tc::pack_bf16(x[4], x[5]); pk.w = tc::pack_bf16(x[6], x[7]);
-                        *reinterpret_cast<uint4*>(sm + L::PB + s2 * 8192 + tc::sw128_off(t, cc)) = pk;
-                    }
+                    for (int u = 0; u < 8; ++u) x[u] = (jb + u <= t) ? sj[u] * __uint_as_float(r8[u]) : 0.f;
+                    uint4 pk;
+                    pk.x = tc::pack_bf16(x[0], x[1]); pk.y = tc::pack_bf16(x[2], x[3]);
+                    pk.z = tc::pack_bf16(x[4], x[5]); pk.w = tc::pack_bf16(x[6], x[7]);
+                    *reinterpret_cast<uint4*>(sm + L::PB + s2 * 8192 + tc::sw128_off(t, jb >> 3)) = pk;
                 }
             }
             if (GATED && gtid < C) betag[gtid] = bt * sfu_exp2(gt);   // beta_j gamma_j (read after the inverse's syncs)
@@ -566,7 +554,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int ch = et & 7;
                 const float gl = g.last();
                 uint8_t* kw = sm + (c % 3) * L::STAGE + L::KW;
-#pragma unroll
+#pragma unroll 1
                 for (int i = 0; i < 4; ++i) {
                     const int t = (et >> 3) + 16 * i;
                     const float gt = g.at(t);

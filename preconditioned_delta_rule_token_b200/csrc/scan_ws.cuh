@@ -254,8 +254,8 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                     const int cidx = (i & 63) >> 3;
                     const float da = s_da[i];
                     float d = s_d[i];   // the carry e = d - d_anchor
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll 1
+                    for (int hh = 0; hh < 2; ++hh) {   // rolled: smaller code
                         const int tb = s * SUB + hh * 32;   // multiple of 8
                         uint8_t* rowbase = colbase + (tb >> 3) * 1024;
                         float kk[32], rr[32], xx[32];
