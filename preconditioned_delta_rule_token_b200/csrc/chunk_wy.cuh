@@ -55,10 +55,11 @@
 //   S <- gamma_C S + sum_j (gamma_C / gamma_j) u_j kw_j^T.
 // The ratios are exp2 of differences of the in-chunk cumulative log2(alpha) (each log2 clamped at
 // -120, so alpha = 0 restarts the state to within 2^-120), which keeps every gate value in [0, 1]
-// in range. The kernel applies them in the prep (A_g, P_g and the second operand T diag(beta gamma)
-// of GW), in the epilogue group (the chunk's Q rows x gamma_t and its Kw rows x gamma_C / gamma_t, so
-// that GBS adds U^T diag(gamma_C / gamma) Kw; done two chunks ahead, once G1 has read both tiles), and
-// in the state group (the fp32 state x gamma_C of the next chunk when it is converted to bf16).
+// in range. The kernel applies them in the prep (A_g and P_g), in the epilogue group (the chunk's K
+// and Q rows x gamma_t, so that GW forms W^T = (diag(gamma) K)^T (T diag(beta))^T from the same T
+// tile as GU and GA forms diag(gamma) Q S^T, and its Kw rows x gamma_C / gamma_t, so that GBS adds
+// U^T diag(gamma_C / gamma) Kw; done two chunks ahead, once G1 has read the three tiles), and in the
+// state group (the fp32 state x gamma_C of the next chunk when it is converted to bf16).
 #pragma once
 #include "tc_ptx.cuh"
 #include "tril_inv.cuh"
@@ -69,15 +70,12 @@ struct WyLayout {
     static constexpr uint32_t STAGE = 49152, NSTAGE = 3;   // [K0|Q0|K1|Q1] (8 KB each) + [Kw0|Kw1]
     static constexpr uint32_t QK = 0, KW = 32768;
     static constexpr uint32_t VB = NSTAGE * STAGE;          // two V tiles [V0|V1], 16 KB each
-    static constexpr uint32_t TB = VB + 2 * 16384;          // T diag(beta) bf16 [64 t][64 j] (B operand of GU, GW);
-                                                            // ungated: two of them, by chunk parity (TB, TB2)
-    static constexpr uint32_t TB2 = TB + 8192;              // gated: T diag(beta gamma) bf16 (B operand of GW)
-    static constexpr uint32_t PB = TB2 + 8192;              // two P tiles bf16 [64 t][64 j]
+    static constexpr uint32_t TB = VB + 2 * 16384;          // two T diag(beta) tiles bf16 (B of GU, GW), by parity
+    static constexpr uint32_t PB = TB + 2 * 8192;           // two P tiles bf16 [64 t][64 j]
     static constexpr int LDF = tri::LD;
     static constexpr uint32_t AF = PB + 2 * 8192;           // A, then T, fp32 [64][LDF]
     static constexpr uint32_t BETA = AF + 64 * LDF * 4;     // prep: beta of its chunk
-    static constexpr uint32_t BETAG = BETA + 256;           // prep, gated: beta_j gamma_j of its chunk
-    static constexpr uint32_t GLOG = BETAG + 256;           // prep, gated: log2 gamma_t of its chunk
+    static constexpr uint32_t GLOG = BETA + 256;            // prep, gated: log2 gamma_t of its chunk
     static constexpr uint32_t BAR = GLOG + 256;
     enum {
         FULLQ = 0,   // 3: K, Q, Kw of a stage landed
@@ -93,7 +91,7 @@ struct WyLayout {
         EVN = 16,    // state: bf16 Vn written
         EOR = 17,    // epilogue: O^T columns read and zeroed
         BAP = 18,    // 2: GA done (by chunk parity; the prep reuses T diag(beta) tile c % 2)
-        ESC = 20,    // 2, gated, epilogue: Q and Kw of a chunk scaled by its gates (by chunk parity: the
+        ESC = 20,    // 2, gated, epilogue: K, Q and Kw of a chunk scaled by its gates (by chunk parity: the
                      // epilogue may finish chunk c + 2 before the issuer has consumed chunk c + 1)
         DRAIN = 22,
         NBAR = 23
@@ -416,7 +414,6 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int gtid = tid - 128;                // 0..127; also the TMEM lane (R1 row) it reads
         const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
         float* betas = reinterpret_cast<float*>(sm + L::BETA);
-        float* betag = reinterpret_cast<float*>(sm + L::BETAG);
         float* glog = reinterpret_cast<float*>(sm + L::GLOG);
         float* AF = reinterpret_cast<float*>(sm + L::AF);
         auto load_beta = [&](int c) -> float {
@@ -479,20 +476,17 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     *reinterpret_cast<uint4*>(sm + L::PB + s2 * 8192 + tc::sw128_off(t, jb >> 3)) = pk;
                 }
             }
-            if (GATED && gtid < C) betag[gtid] = bt * sfu_exp2(gt);   // beta_j gamma_j (read after the inverse's syncs)
             tc::tc_fence_before();
             tc::named_sync(BAR_PREP, 128);
-            // T = (I + A)^{-1}, written as bf16 T diag(beta) (gated also T diag(beta gamma)) straight into the B
-            // operands of GU and GW, once GW and GU of the chunk that last used those tiles have read them:
-            // ungated tile c % 2 (GA(c - 2) completes after both), gated the single pair (GA(c - 1)).
+            // T = (I + A)^{-1}, written as bf16 T diag(beta) straight into tile c % 2, the B operand of GU and
+            // GW, once GW and GU of chunk c - 2, the tile's last readers, have read it (GA(c - 2) completes
+            // after both).
             auto tiles_free = [&]() -> bool {
-                bool f = false;
-                if (GATED) f = c >= 1 && !wait(L::BA, (c - 1) & 1);
-                else f = c >= 2 && !wait(L::BAP + s2, ((c - 2) >> 1) & 1);
+                const bool f = c >= 2 && !wait(L::BAP + s2, ((c - 2) >> 1) & 1);
                 return tc::named_sync_or(BAR_PREP, 128, f);
             };
-            uint8_t* tb = sm + L::TB + (GATED ? 0u : (uint32_t)s2 * 8192u);
-            if (!tri::tril_inv64_to_bf16(AF, tb, betas, GATED ? sm + L::TB2 : nullptr, betag, q4, lane,
+            uint8_t* tb = sm + L::TB + (uint32_t)s2 * 8192u;
+            if (!tri::tril_inv64_to_bf16(AF, tb, betas, q4, lane,
                                          [] { tc::named_sync(BAR_PREP, 128); }, tiles_free))
                 break;
             tc::fence_proxy_async_smem();   // P and the T tiles -> the tensor core (async proxy)
@@ -541,8 +535,9 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (nchunks > 3) prefetch_l2(3);
             if (nchunks > 4) prefetch_l2(4);
         }
-        // gated: chunk c's Q rows x gamma_t and Kw rows x gamma_C / gamma_t (GBS then adds U^T diag(gamma_C /
-        // gamma) Kw), once G1(c), their other reader, has completed; the issuer waits for it before GA(c)
+        // gated: chunk c's K and Q rows x gamma_t (GW then forms (diag(gamma) K)^T (T diag(beta))^T, GA
+        // diag(gamma) Q S^T) and Kw rows x gamma_C / gamma_t (GBS then adds U^T diag(gamma_C / gamma) Kw), once
+        // G1(c), their other reader, has completed; the issuer waits for it before GW(c)
         auto gate_scale = [&](int c) -> bool {
             if (tc::named_sync_or(BAR_EPI, 128, !wait(L::D1 + c % 3, (c / 3) & 1))) return false;
             ChunkGates g;
@@ -562,6 +557,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const uint32_t row = (t >> 3) * 1024 + (t & 7) * 128 + ch * 16;
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
+                        scale_bf16x8(st + half * 16384 + row, sq);          // K
                         scale_bf16x8(st + half * 16384 + 8192 + row, sq);   // Q
                         scale_bf16x8(kw + half * 8192 + row, sk);           // Kw
                     }
@@ -623,9 +619,8 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     } else {
         // ================================================================ issuer warp
         if (lane == 0) {
-            // T diag(beta) of chunk c (B operand of GU; of GW ungated) and gated T diag(beta gamma) (B of GW)
-            auto dTB = [&](int c) { return tc::sdesc_sw128(sb + L::TB + (GATED ? 0u : (uint32_t)(c & 1) * 8192u), 16, 1024); };
-            auto dTBW = [&](int c) { return GATED ? tc::sdesc_sw128(sb + L::TB2, 16, 1024) : dTB(c); };
+            // T diag(beta) of chunk c, the B operand of GU and GW
+            auto dTB = [&](int c) { return tc::sdesc_sw128(sb + L::TB + (uint32_t)(c & 1) * 8192u, 16, 1024); };
             auto st = [&](int c) { return sb + (uint32_t)(c % 3) * L::STAGE; };
             auto G1 = [&](int c) {   // R1[c%3] = [K; Q] Kw^T
                 const uint64_t a = tc::sdesc_sw128(st(c) + L::QK, 16, 1024), bk = tc::sdesc_sw128(st(c) + L::KW, 16, 1024);
@@ -641,7 +636,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint64_t a = tc::sdesc_sw128(st(c) + L::QK, 16384, 1024);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::umma_bf16(tmem + COL_R1 + (c % 3) * 64, a + ((ks * 2048) >> 4), dTBW(c) + ((ks * 32) >> 4),
+                    tc::umma_bf16(tmem + COL_R1 + (c % 3) * 64, a + ((ks * 2048) >> 4), dTB(c) + ((ks * 32) >> 4),
                                   ID_N64_AMN, ks > 0);
                 tc::umma_commit(bars + L::BW);
             };
@@ -682,6 +677,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             };
             auto issue_gw = [&](int c) -> bool {
                 if (!wait(L::ETB, c & 1)) return false;
+                if (GATED && !wait(L::ESC + (c & 1), (c >> 1) & 1)) return false;
                 tc::tc_fence_after();
                 GW(c);
                 return true;
@@ -698,14 +694,14 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                       (issue_g1(0) && (nchunks < 2 || issue_g1(1)) && issue_gw(0) && issue_gu(0));
             for (int c = 0; ok && c < nchunks; ++c) {
                 // GA(c) needs bf16 S_c, -W(c) and (c > 0) the O^T columns read out and zeroed
-                ok = wait(L::ESB, c & 1) && wait(L::EWE, c & 1) && (c == 0 || wait(L::EOR, (c - 1) & 1)) &&
-                     (!GATED || wait(L::ESC + (c & 1), (c >> 1) & 1));
+                ok = wait(L::ESB, c & 1) && wait(L::EWE, c & 1) && (c == 0 || wait(L::EOR, (c - 1) & 1));
                 if (!ok) break;
                 tc::tc_fence_after();
                 GA(c);
                 // window while the state group converts Vn: GW(c+1), G1(c+2) when their inputs are ready
                 bool gw_done = c + 1 >= nchunks, g1_done = c + 2 >= nchunks;
-                if (!gw_done && tc::mbar_test(bars + L::ETB, (c + 1) & 1)) {
+                if (!gw_done && tc::mbar_test(bars + L::ETB, (c + 1) & 1) &&
+                    (!GATED || tc::mbar_test(bars + L::ESC + ((c + 1) & 1), ((c + 1) >> 1) & 1))) {
                     tc::tc_fence_after();
                     GW(c + 1);
                     gw_done = true;

@@ -300,9 +300,8 @@ __device__ __forceinline__ void blk_convert_bf16(uint8_t* tile, const float* T, 
 }
 
 // T = (I + A)^{-1} for a strictly lower 64 x 64 A (fp32, stride LD, 16-byte aligned rows), written
-// only as bf16 tiles: tb = T diag(sc) and, when tb2 is not null, tb2 = T diag(sc2) (128-byte-swizzled
-// K-major, row t, column j; 16 x 16 blocks above the diagonal blocks are not written and must hold
-// zeros). A's lower blocks are overwritten by intermediates. The same blocking as tril_inv64 in three
+// only as the bf16 tile tb = T diag(sc) (128-byte-swizzled K-major, row t, column j; 16 x 16 blocks
+// above the diagonal blocks are not written and must hold zeros). A's lower blocks are overwritten by intermediates. The same blocking as tril_inv64 in three
 // barrier-separated phases after the diagonal blocks:
 //   phase 0: T_ii = (I + A_ii)^{-1}, right-looking forward substitution, one warp per block;
 //   phase 1: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22) (warps 0, 1);
@@ -315,9 +314,8 @@ __device__ __forceinline__ void blk_convert_bf16(uint8_t* tile, const float* T, 
 // as a barrier of the group and return true on every thread when the group is to stop (the
 // function then returns false right away). Returns true after a final sync().
 template <class Sync, class TilesFree>
-__device__ __forceinline__ bool tril_inv64_to_bf16(float* A, uint8_t* tb, const float* sc, uint8_t* tb2,
-                                                   const float* sc2, int warp, int lane, Sync sync,
-                                                   TilesFree tiles_free) {
+__device__ __forceinline__ bool tril_inv64_to_bf16(float* A, uint8_t* tb, const float* sc, int warp, int lane,
+                                                   Sync sync, TilesFree tiles_free) {
     auto blk = [&](int i, int j) { return A + (i * 16) * LD + j * 16; };
     {   // phase 0: column j of T_ww by right-looking substitution (lanes 16-31 repeat lanes 0-15)
         const int j = lane & 15;
@@ -366,11 +364,6 @@ __device__ __forceinline__ bool tril_inv64_to_bf16(float* A, uint8_t* tb, const 
         blk_convert_bf16(tb, A, sc, o, o, lane);
         blk_convert_bf16(tb, A, sc, o + 1, o, lane);
         blk_convert_bf16(tb, A, sc, o + 1, o + 1, lane);
-        if (tb2) {
-            blk_convert_bf16(tb2, A, sc2, o, o, lane);
-            blk_convert_bf16(tb2, A, sc2, o + 1, o, lane);
-            blk_convert_bf16(tb2, A, sc2, o + 1, o + 1, lane);
-        }
     }
     sync();
     {                 // phase 3: block (a, b) of T, a = 2 + warp / 2, b = warp % 2
@@ -380,7 +373,6 @@ __device__ __forceinline__ bool tril_inv64_to_bf16(float* A, uint8_t* tb, const 
         blk_mma_trunc(c, blk(a, 2), blk(2, bb), lane);
         if (a == 3) blk_mma_trunc(c, blk(3, 3), blk(3, bb), lane);
         blk_store_bf16(tb, c, -1.f, sc, a, bb, lane);
-        if (tb2) blk_store_bf16(tb2, c, -1.f, sc2, a, bb, lane);
     }
     sync();
     return true;
