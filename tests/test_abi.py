@@ -151,3 +151,28 @@ def test_backward_workspace_and_argument_checks(osdn_lib):
     assert rc == osdn_lib.OSDN_ERR_INVALID_ARG and "aligned" in osdn_lib.get_last_error()
     bad = _params(osdn_lib, dk=96)
     assert L.osdn_bwd_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == osdn_lib.OSDN_ERR_UNSUPPORTED
+
+
+def test_new_entry_points_check_their_arguments_on_the_host(osdn_lib):
+    """osdn_bwd_gated refuses a NULL alpha or dalpha (T > 0) before touching the device;
+    osdn_fwd_segments and osdn_fwd_launches refuse NULL outputs and report the plan."""
+    L = osdn_lib.lib()
+    fake = ctypes.c_void_p(1 << 20)             # never dereferenced: checks fail first
+    p = _params(osdn_lib)
+    args = [ctypes.byref(p)] + [fake] * 5        # q, k, v, beta, r
+    tail = [None, None, fake, None, None, fake, fake, fake, fake, None]   # d0, S0, dout, dS_f, dd_f, dq..dbeta, dr
+    for alpha, dalpha in ((None, fake), (fake, None)):
+        rc = L.osdn_bwd_gated(*args, alpha, *tail, dalpha, None, None, fake, ctypes.c_size_t(1 << 40), None)
+        assert rc == osdn_lib.OSDN_ERR_INVALID_ARG
+        assert b"alpha" in L.osdn_get_last_error()
+    n = ctypes.c_int(0)
+    assert L.osdn_fwd_segments(ctypes.byref(p), None) == osdn_lib.OSDN_ERR_INVALID_ARG
+    assert L.osdn_fwd_launches(ctypes.byref(p), None) == osdn_lib.OSDN_ERR_INVALID_ARG
+    assert L.osdn_fwd_launches(ctypes.byref(p), ctypes.byref(n)) == 0 and n.value >= 1
+    one_seq = osdn_lib.make_params(1, 32768, 16, 128, 128, __import__("torch").bfloat16, 1e-2)
+    assert osdn_lib.osdn_fwd_segments(one_seq) == 16
+    assert osdn_lib.osdn_fwd_launches(one_seq) == 2 + 5 * 4      # batches of 4 segments over 0 .. 14
+    anchored = osdn_lib.make_params(1, 32768, 16, 128, 128, __import__("torch").bfloat16, 1e-2, 64, True)
+    assert osdn_lib.osdn_fwd_launches(anchored) == 6              # split, not overlapped
+    layer = osdn_lib.make_params(8, 4096, 16, 128, 128, __import__("torch").bfloat16, 1e-2)
+    assert osdn_lib.osdn_fwd_segments(layer) == 1 and osdn_lib.osdn_fwd_launches(layer) == 2
