@@ -222,3 +222,15 @@ def test_gpu_split_anchored_single_sequence():
     errs = (slice_rel_err(out.float().cpu().numpy(), ro, (0, 2)), slice_rel_err(S.cpu().numpy(), rS, (0, 1)),
             slice_rel_err(d.cpu().numpy(), rd, (0, 1)))
     assert max(errs) <= BF16_TOL, errs
+
+
+@pytest.mark.gpu
+def test_gpu_split_gated_several_sequences():
+    # B = 2: phase 2 split into segments without the overlap (gated, alpha down to 0.05)
+    import preconditioned_delta_rule_token_b200 as pk
+    w = _few_units(2, 3, 2048, seed=69)
+    p = pk.make_params(w.B, w.T, w.H, w.dk, w.dv, torch.bfloat16, w.eta)
+    assert pk.osdn_fwd_segments(p) == 4 and pk.osdn_fwd_launches(p) == 6
+    alpha = (0.05 + 0.95 * torch.rand((w.B, w.T, w.H), generator=torch.Generator().manual_seed(70))).to(
+        torch.bfloat16)
+    _check_against_oracle(w, alpha=alpha)
