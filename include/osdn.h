@@ -93,7 +93,10 @@ typedef struct {
  * dtype [B, T, H, dk] and, when phase 2 splits the sequences into segments
  * (osdn_fwd_segments > 1), three fp32 states per segment and head (start
  * state, own end state, transfer; 3 * B * P * H * dv * dk * 4 bytes) and a
- * 16 KiB tile of zeros. It is scratch owned by the caller, needs no
+ * 16 KiB tile of zeros. When osdn_fwd pipelines the scan with phase 2
+ * (osdn_fwd_launches) it also holds beta, r and alpha reordered by segment
+ * (3 * B * T * H * 2 bytes) and two fp32 states and two d vectors per (b, h)
+ * handed from segment to segment. It is scratch owned by the caller, needs no
  * initialisation, and may be reused by the next call on the same stream. The
  * size depends on the SM count of the current device.
  * Returns OSDN_OK, OSDN_ERR_INVALID_ARG or OSDN_ERR_UNSUPPORTED. */
@@ -129,6 +132,16 @@ int osdn_fwd_segments(const osdn_params *p, int *segments);
  * cuda_stream by events) run each batch's chunk passes as soon as the scan
  * has covered it, and the last segment's output pass after the scan:
  * 2 + 5 ceil((P - 1) / nb) launches.
+ * Without segments, when B * H is at most half the SM count (tensor-core path,
+ * dense tensors, anchored APF off), osdn_fwd instead pipelines the two phases
+ * over Q = 4 segments of each sequence when each keeps at least 1024 tokens
+ * (else 2 of at least 512, else none): one launch reorders beta, r and alpha by
+ * segment, then cuda_stream scans segment after segment (each scan from the
+ * d the previous one ended with) while a library-owned stream runs phase 2 of
+ * each segment once it is scanned, from the state the previous segment ended
+ * with: 1 + 2 Q launches, with phase 2 of segment s beside the scan of s + 1
+ * on other SMs. Segments end on chunk boundaries and hand over d and S in
+ * fp32, so the results equal the unpipelined ones bit for bit.
  * T = 0: at most one (d filled with ones).
  * Errors: OSDN_ERR_INVALID_ARG (bad params, NULL launches), OSDN_ERR_UNSUPPORTED. */
 int osdn_fwd_launches(const osdn_params *p, int *launches);

@@ -9,6 +9,7 @@
 #include <cstddef>
 #include <cstdarg>
 #include <cstdio>
+#include <cstring>
 #include <initializer_list>
 #include <mutex>
 #include <string>
@@ -145,11 +146,31 @@ int seg_count(const osdn_params* p) {
     return P >= 4 ? P : 1;
 }
 
+// Segments of the pipelined forward (1: none). When phase 2 is not split and the (b, h) units
+// take at most half the SMs, osdn_fwd cuts each sequence into P segments and runs the scan of
+// segment s + 1 beside phase 2 of segment s, each on its own SMs; phase 2 of a segment starts
+// from the state the previous one ended with, so no transfer passes are needed. Every launch of
+// phase 2 pays its own pipeline fill and drain (about three chunks), so segments stay long: four
+// when each keeps at least 1024 tokens, else two of at least 512. Not with the anchored
+// preconditioner (its anchor is the d of the whole sequence's start).
+constexpr int kMaxPipe = 4;
+int pipe_count(const osdn_params* p) {
+    if (p->dtype != OSDN_BF16 || p->dk != 128 || p->dv != 128 || p->T <= 0 || !dense_layout(p) || anchor_of(p))
+        return 1;
+    if (seg_count(p) > 1 || 2LL * p->B * p->H > sm_count()) return 1;
+    for (int P = kMaxPipe; P >= 2; P /= 2)
+        if (p->T % (64 * P) == 0 && p->T / P >= (P > 2 ? 1024 : 512)) return P;
+    return 1;
+}
+
 // The forward's workspace: the scaled write keys, then (segmented phase 2 only) the start
 // states, end states and transfers of every segment, fp32 [B P, H, dv, dk] each, and a 64-token
 // tile of zeros that the transfer pass reads as V. When osdn_fwd also overlaps the scan with
 // phase 2 (one sequence, plain APF): identity start states for the transfer passes of one batch,
-// d after every segment, and an output tile for the transfer passes of one batch.
+// d after every segment, and an output tile for the transfer passes of one batch. When it
+// pipelines the scan with phase 2 instead (few units, phase 2 not split): beta, r and alpha
+// segment-major, and two buffers each for the state and d handed from segment to segment (the
+// scaled write keys are then segment-major too).
 struct WorkspaceLayout {
     size_t kw_off, kw_bytes, total;
     int seg;                       // segments per sequence (1: phase 2 is not split)
@@ -157,6 +178,9 @@ struct WorkspaceLayout {
     bool overlap;                  // osdn_fwd runs the scan segment by segment, phase 2 alongside
     int ov_batch;                  // segments per batch of the overlapped passes
     size_t ov_I, ov_D, ov_O;
+    int pipe;                      // segments of the pipelined forward (1: not pipelined)
+    size_t pp_in[3];               // beta, r, alpha segment-major [P][B][T / P][H]
+    size_t pp_S, pp_D;             // two state and two d buffers [B, H, dv, dk], [B, H, dk] fp32
 };
 
 WorkspaceLayout layout_of(const osdn_params* p) {
@@ -182,6 +206,17 @@ WorkspaceLayout layout_of(const osdn_params* p) {
             L.ov_O = round_up(L.ov_D + (size_t)L.seg * p->H * p->dk * sizeof(float), 256);
             L.total = L.ov_O + (size_t)L.ov_batch * seg_tokens * p->dv * sizeof(__nv_bfloat16);
         }
+    }
+    L.pipe = pipe_count(p);
+    if (L.pipe > 1) {
+        const size_t units = (size_t)p->B * p->H;
+        for (int a = 0; a < 3; ++a) {
+            L.pp_in[a] = L.total;
+            L.total = round_up(L.total + (size_t)p->B * p->T * p->H * sizeof(__nv_bfloat16), 256);
+        }
+        L.pp_S = L.total;
+        L.pp_D = L.pp_S + 2 * units * p->dv * p->dk * sizeof(float);
+        L.total = round_up(L.pp_D + 2 * units * p->dk * sizeof(float), 256);
     }
     if (L.total == 0) L.total = 256;
     return L;
@@ -458,6 +493,86 @@ int launch_fwd_overlapped(const osdn_params* p, const __nv_bfloat16* q, const __
         // join: the caller's stream waits for side 0, which has waited for every event of side 1
         if ((rc = chk(cudaEventRecord(ev_join, side[0]), "join"))) break;
         rc = chk(cudaStreamWaitEvent(st, ev_join, 0), "join");
+    } while (false);
+    for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
+    return rc;
+}
+
+// osdn_fwd with each sequence cut into L.pipe segments (pipe_count): the caller's stream
+// reorders beta, r and alpha segment-major and scans segment after segment, each launch from
+// the d the previous one ended with; a side stream runs phase 2 of each segment once its scan
+// is done, from the state the previous segment ended with. Phase 2 of segment s thus runs
+// beside the scan of segment s + 1. Segment s of q, k, v and out is the [B, T / P, H, 128] view
+// at token s T / P with the whole sequence's strides; its scaled write keys, beta, r and alpha
+// are dense blocks of the workspace, so every launch is the existing scan or chunk kernel.
+int launch_fwd_pipelined(const osdn_params* p, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                         const __nv_bfloat16* v, const __nv_bfloat16* beta, const __nv_bfloat16* r,
+                         const __nv_bfloat16* alpha, const float* d0, const float* S0, __nv_bfloat16* out,
+                         float* final_S, float* final_d, char* ws, const WorkspaceLayout& L, cudaStream_t st) {
+    using T = __nv_bfloat16;
+    const int P = L.pipe, H = p->H, D = 128;
+    const int Ls = p->T / P;
+    const size_t segtok = (size_t)p->B * Ls * H;           // token-heads of one segment of every sequence
+    const size_t units = (size_t)p->B * H;
+    osdn_params vw{};                                      // one segment of every sequence
+    std::memcpy(&vw, p, p->struct_size < sizeof(vw) ? p->struct_size : sizeof(vw));
+    vw.struct_size = sizeof(vw);
+    vw.T = Ls;
+    const int64_t full[3] = {(int64_t)p->T * H * D, (int64_t)H * D, D};
+    for (int i = 0; i < 3; ++i) vw.stride_q[i] = vw.stride_k[i] = vw.stride_v[i] = vw.stride_o[i] = full[i];
+    auto view_at = [&](auto* base, int seg) { return base + (size_t)seg * Ls * H * D; };
+    T* kw = reinterpret_cast<T*>(ws + L.kw_off);
+    T* in[3] = {reinterpret_cast<T*>(ws + L.pp_in[0]), r ? reinterpret_cast<T*>(ws + L.pp_in[1]) : nullptr,
+                alpha ? reinterpret_cast<T*>(ws + L.pp_in[2]) : nullptr};
+    auto seg_of = [&](T* base, int seg) { return base ? base + (size_t)seg * segtok : nullptr; };
+    float* Sb = reinterpret_cast<float*>(ws + L.pp_S);
+    float* db = reinterpret_cast<float*>(ws + L.pp_D);
+
+    cudaStream_t side[2];
+    int rc = side_streams(side);
+    if (rc) return rc;
+    if (P < 2 || P > kMaxPipe) return fail(OSDN_ERR_UNSUPPORTED, "%d pipelined segments", P);
+    const int nev = 2 + P;                                 // fork, join, per segment: scanned
+    cudaEvent_t ev[2 + kMaxPipe];
+    cudaError_t e = cudaSuccess;
+    int made = 0;
+    for (; made < nev; ++made)
+        if ((e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming)) != cudaSuccess) break;
+    if (e != cudaSuccess) {
+        for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+        return cuda_fail(e, "event");
+    }
+    auto chk = [&](cudaError_t x, const char* what) { return x == cudaSuccess ? OSDN_OK : cuda_fail(x, what); };
+    do {
+        osdn::seg::SegGather g{};
+        const void* src[3] = {beta, r, alpha};
+        for (int a = 0; a < 3; ++a) {
+            g.src[a] = in[a] ? reinterpret_cast<const uint4*>(src[a]) : nullptr;
+            g.dst[a] = reinterpret_cast<uint4*>(in[a]);
+        }
+        const size_t words = (size_t)p->B * p->T * H / 8, blocks = (words + 255) / 256;
+        osdn::seg::gather_kernel<<<(unsigned)(blocks > 1024 ? 1024 : blocks), 256, 0, st>>>(g, p->B, p->T, H, P);
+        if ((rc = chk(cudaGetLastError(), "segment gather launch"))) break;
+        // fork after the gather: the side stream reads the reordered beta and alpha
+        if ((rc = chk(cudaEventRecord(ev[0], st), "fork"))) break;
+        if ((rc = chk(cudaStreamWaitEvent(side[0], ev[0], 0), "fork"))) break;
+        // enqueued segment by segment, so that phase 2 of a segment is queued as soon as its scan is
+        for (int sg = 0; sg < P && !rc; ++sg) {
+            const float* din = sg == 0 ? d0 : db + (size_t)((sg - 1) & 1) * units * D;
+            float* dout = sg == P - 1 ? final_d : db + (size_t)(sg & 1) * units * D;
+            if ((rc = launch_scan<T>(&vw, view_at(k, sg), seg_of(in[0], sg), seg_of(in[1], sg), din, dout,
+                                     kw + (size_t)sg * segtok * D, st)))
+                break;
+            if ((rc = chk(cudaEventRecord(ev[2 + sg], st), "scan event"))) break;
+            if ((rc = chk(cudaStreamWaitEvent(side[0], ev[2 + sg], 0), "segment wait"))) break;
+            const float* sin = sg == 0 ? S0 : Sb + (size_t)((sg - 1) & 1) * units * D * D;
+            float* sout = sg == P - 1 ? final_S : Sb + (size_t)(sg & 1) * units * D * D;
+            rc = launch_chunk_wy(&vw, view_at(q, sg), view_at(k, sg), view_at(v, sg), seg_of(in[0], sg), sin,
+                                 view_at(out, sg), sout, kw + (size_t)sg * segtok * D, side[0], seg_of(in[2], sg));
+        }
+        if (rc) break;
+        if ((rc = chk(cudaEventRecord(ev[1], side[0]), "join"))) break;
+        rc = chk(cudaStreamWaitEvent(st, ev[1], 0), "join");
     } while (false);
     for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
     return rc;
@@ -775,6 +890,7 @@ int osdn_fwd_launches(const osdn_params* p, int* launches) {
     if (!launches) return fail(OSDN_ERR_INVALID_ARG, "launches is NULL");
     const WorkspaceLayout L = layout_of(p);
     if (p->T == 0) *launches = 1;                    // at most the fill of d with ones
+    else if (L.pipe > 1) *launches = 1 + 2 * L.pipe; // gather, per segment a scan and a chunk pass
     else if (L.seg == 1) *launches = 2;              // scan, chunk
     else if (!L.overlap) *launches = 6;              // scan, identity, three chunk passes, combine
     else   // identity, last-segment scan, per batch a scan, two passes, combine, output pass
@@ -801,6 +917,9 @@ int osdn_fwd(const osdn_params* p, const void* q, const void* k, const void* v, 
         if (L.overlap)
             return launch_fwd_overlapped(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)r,
                                          nullptr, d0, S0, (T*)out, final_S, final_d, ws, L, st);
+        if (L.pipe > 1)
+            return launch_fwd_pipelined(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)r,
+                                        nullptr, d0, S0, (T*)out, final_S, final_d, ws, L, st);
         rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
         if (rc) return rc;
         return launch_chunk<T>(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, S0, (T*)out, final_S, kw, st,
@@ -833,6 +952,10 @@ int osdn_fwd_gated(const osdn_params* p, const void* q, const void* k, const voi
         return launch_fwd_overlapped(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)r,
                                      (const T*)alpha, d0, S0, (T*)out, final_S, final_d,
                                      reinterpret_cast<char*>(workspace), L, st);
+    if (L.pipe > 1)
+        return launch_fwd_pipelined(p, (const T*)q, (const T*)k, (const T*)v, (const T*)beta, (const T*)r,
+                                    (const T*)alpha, d0, S0, (T*)out, final_S, final_d,
+                                    reinterpret_cast<char*>(workspace), L, st);
     rc = launch_scan<T>(p, (const T*)k, (const T*)beta, (const T*)r, d0, final_d, kw, st);
     if (rc) return rc;
     return launch_chunk_gated(p, q, k, v, beta, alpha, S0, out, final_S, kw, st, reinterpret_cast<char*>(workspace));

@@ -13,7 +13,11 @@
 // states S_start(p + 1) = S_start(p) E_p + L_p are combined, for the outputs.
 // With one sequence (B = 1) any run of consecutive segments is itself a dense
 // [n, T / P, H, d] tensor, so the passes can also go batch by batch while the
-// scan is still working on later segments.
+// scan is still working on later segments. With enough SMs for both phases at
+// once, the phases can also simply alternate over the segments on two streams
+// (phase 2 of a segment from the state the previous one ended with, beside the
+// scan of the next): no transfer passes, only the per-token tensors [B, T, H]
+// reordered so that each segment of every sequence is one dense block.
 #pragma once
 #include <cstddef>
 #include <cstdint>
@@ -26,6 +30,26 @@ __global__ void identity_kernel(float* __restrict__ S, size_t units, int D) {
     const size_t n = units * (size_t)D * D;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
         S[i] = ((i / D) % D == i % D) ? 1.f : 0.f;
+}
+
+// Up to three per-token tensors [B, T, H] (bf16) reordered segment-major, [P][B][T / P][H], so that
+// segment s of every sequence is the dense [B, T / P, H] block at s B (T / P) H. Rows of T / P H
+// elements are whole 16-byte words (T / P a multiple of 64): copied as uint4.
+struct SegGather {
+    const uint4* src[3];   // NULL entries are skipped
+    uint4* dst[3];
+};
+__global__ void gather_kernel(SegGather g, int B, int T, int H, int P) {
+    const size_t row = (size_t)(T / P) * H / 8;           // words of one (segment, sequence) row
+    const size_t n = (size_t)B * T * H / 8;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t r = i / row, w = i % row;            // destination row r = s B + b
+        const size_t s = r / B, b = r % B;
+        const size_t j = (b * P + s) * row + w;           // word w of segment s of sequence b in [B, T, H]
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+            if (g.src[a]) g.dst[a][i] = g.src[a][j];
+    }
 }
 
 constexpr int kRows = 16;       // rows of S per CTA of the combine

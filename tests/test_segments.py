@@ -75,7 +75,12 @@ def _params(B, T, H, dk=128, dv=128, dtype=torch.bfloat16):
 @pytest.mark.parametrize("B,T,H,dtype,dk,want", [
     (1, 32768, 16, torch.bfloat16, 128, 16),   # long context, one sequence: overlapped, short segments
     (8, 4096, 16, torch.bfloat16, 128, 1),     # 128 units fill the SMs
-    (8, 2048, 8, torch.bfloat16, 128, 1),      # 64 units: 2 segments would not pay
+    (8, 2048, 8, torch.bfloat16, 128, 1),      # 64 units: 2 segments would not pay (pipelined instead)
+    (4, 1024, 16, torch.bfloat16, 128, 1),     # 64 units, pipelined in 2 segments of 512 tokens
+    (2, 8192, 16, torch.bfloat16, 128, 4),     # 32 units: split (4 segments), not pipelined
+    (2, 4096, 20, torch.bfloat16, 128, 1),     # 40 units, pipelined in 4 segments of 1024 tokens
+    (2, 1536, 8, torch.bfloat16, 128, 1),      # 16 units, 2 pipelined segments (4 would be 384 tokens)
+    (8, 2048, 10, torch.bfloat16, 128, 1),     # 80 units: more than half the SMs, not pipelined
     (1, 4096, 1, torch.bfloat16, 128, 8),      # 16 capped by T / P >= 512
     (1, 4096, 2, torch.bfloat16, 128, 8),
     (1, 4000, 2, torch.bfloat16, 128, 1),      # T not a multiple of 64 P for any P >= 4
@@ -93,7 +98,13 @@ def test_segment_plan(B, T, H, dtype, dk, want):
     ws = pk.osdn_fwd_workspace_size(p)
     up = lambda x: -(-x // 256) * 256
     if P == 1:
-        assert ws == max(256, up(kw))
+        pipe = _pipe_count(B, T, H, dtype, dk)
+        want_ws = max(256, up(kw))
+        if pipe > 1:   # beta, r, alpha segment-major; two states and two d handed between segments
+            units = B * H
+            want_ws = up(up(kw) + 3 * up(B * T * H * 2) + 2 * units * 128 * 128 * 4 + 2 * units * 128 * 4)
+        assert ws == want_ws
+        assert pk.osdn_fwd_launches(p) == (1 + 2 * pipe if pipe > 1 else 2)
     else:
         st = B * P * H * 128 * 128 * 4
         want_ws = up(kw) + 3 * st + 64 * 128 * 2          # start states, own end states, transfers, zeros
@@ -101,6 +112,17 @@ def test_segment_plan(B, T, H, dtype, dk, want):
             nb = min((148 - H) // (2 * H), P // 2)
             want_ws = up(up(want_ws) + nb * H * 128 * 128 * 4 + P * H * 128 * 4) + nb * (T // P) * H * 128 * 2
         assert ws == want_ws
+
+
+def _pipe_count(B, T, H, dtype, dk, sms=148):
+    """The pipelined forward's segment count: phase 2 not split, the units at most half the SMs,
+    four segments of at least 1024 tokens, else two of at least 512, else none."""
+    if dtype != torch.bfloat16 or dk != 128 or T <= 0 or 2 * B * H > sms:
+        return 1
+    for P, least in ((4, 1024), (2, 512)):
+        if T % (64 * P) == 0 and T // P >= least:
+            return P
+    return 1
 
 
 def test_segment_plan_needs_dense_tensors():
@@ -234,3 +256,60 @@ def test_gpu_split_gated_several_sequences():
     alpha = (0.05 + 0.95 * torch.rand((w.B, w.T, w.H), generator=torch.Generator().manual_seed(70))).to(
         torch.bfloat16)
     _check_against_oracle(w, alpha=alpha)
+
+
+def _pipelined_case(w, alpha=None):
+    """osdn_fwd (or osdn_fwd_gated) on a pipelined shape against the oracle, and bit for bit
+    against the two phases called one after the other (osdn_fwd_scan, then osdn_fwd_chunk: the
+    same kernels over whole sequences). Segments end on scan blocks and chunk boundaries and
+    hand over d and S in fp32, so the two orders do the same arithmetic."""
+    import preconditioned_delta_rule_token_b200 as pk
+    inp = W.make_forward_inputs(w)
+    p = pk.make_params(w.B, w.T, w.H, w.dk, w.dv, inp["k"].dtype, w.eta)
+    P = _pipe_count(w.B, w.T, w.H, torch.bfloat16, 128)
+    assert P > 1 and pk.osdn_fwd_segments(p) == 1 and pk.osdn_fwd_launches(p) == 1 + 2 * P
+    g = {n: _dev(x) for n, x in inp.items()}
+    a = _dev(alpha)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out, S, d = pk.forward(g["q"], g["k"], g["v"], g["beta"], g["r"], g["d0"], g["S0"], eta=w.eta, alpha=a,
+                               stream=s)
+    s.synchronize()
+    out2 = torch.empty_like(g["v"])
+    S2 = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device="cuda")
+    d2 = torch.empty((w.B, w.H, w.dk), dtype=torch.float32, device="cuda")
+    ws = torch.empty(pk.osdn_fwd_workspace_size(p), dtype=torch.uint8, device="cuda")
+    pk.osdn_fwd_scan(p, g["k"], g["beta"], g["r"], g["d0"], d2, ws)
+    if a is None:
+        pk.osdn_fwd_chunk(p, g["q"], g["k"], g["v"], g["beta"], g["S0"], out2, S2, ws)
+    else:
+        pk.osdn_fwd_chunk_gated(p, g["q"], g["k"], g["v"], g["beta"], a, g["S0"], out2, S2, ws)
+    torch.cuda.synchronize()
+    assert pk.osdn_sync_status() == 0
+    f = W.to_f64
+    ro, rS, rd = oracle.fwd(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["beta"]), f(inp["r"]), f(inp["d0"]),
+                            f(inp["S0"]), eta=w.eta, alpha=None if alpha is None else f(alpha))
+    errs = (slice_rel_err(out.float().cpu().numpy(), ro, (0, 2)), slice_rel_err(S.cpu().numpy(), rS, (0, 1)),
+            slice_rel_err(d.cpu().numpy(), rd, (0, 1)))
+    assert max(errs) <= BF16_TOL, errs
+    assert torch.equal(out, out2) and torch.equal(S, S2) and torch.equal(d, d2)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,H,T,apf", [(2, 2, 1024, True), (4, 10, 2048, True), (2, 20, 4096, False)])
+def test_gpu_pipelined_forward_matches_oracle(B, H, T, apf):
+    # 4 units with segments too short to split, and 40 units (more than 148 / 4, so not split
+    # either): 2, 2 and 4 pipelined segments; from a nonzero initial state
+    w = W.Workload("few units", B, H, T, 128, 128, 64, W.BF16, apf, "gaussian", eta=1e-2, seed=71 + T // 512,
+                   d0="uniform", S0="normal")
+    _pipelined_case(w)
+
+
+@pytest.mark.gpu
+def test_gpu_pipelined_gated_forward_matches_oracle():
+    # alpha down to 0.05 with exact zeros (restarts) on both sides of segment boundaries
+    w = _few_units(4, 10, 2048, seed=75)
+    alpha = 0.05 + 0.95 * torch.rand((w.B, w.T, w.H), generator=torch.Generator().manual_seed(76))
+    alpha[:, 510:514] = 0.0
+    alpha[1, 1024] = 0.0
+    _pipelined_case(w, alpha=alpha.to(torch.bfloat16))
