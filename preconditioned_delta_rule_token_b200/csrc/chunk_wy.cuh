@@ -184,10 +184,11 @@ __device__ __forceinline__ void scale_bf16x8(uint8_t* p, const Bf16Scale& s) {
 // computed by every lane of a warp.
 struct ChunkGates {
     float g0, g1;   // log2 gamma of tokens 2 lane, 2 lane + 1
-    __device__ __forceinline__ static float log2_alpha(const __nv_bfloat16* alpha, size_t idx, bool valid) {
-        return valid ? fmaxf(sfu_log2(__bfloat162float(alpha[idx])), -120.f) : 0.f;
+    // log2 alpha of one token from its raw value (RawAlpha); tokens past T count as alpha = 1
+    __device__ __forceinline__ static float log2_of(__nv_bfloat16 a, bool valid) {
+        return valid ? fmaxf(sfu_log2(__bfloat162float(a)), -120.f) : 0.f;
     }
-    // la0, la1: log2 alpha of the lane's two tokens (from log2_alpha)
+    // la0, la1: log2 alpha of the lane's two tokens (from log2_of)
     __device__ __forceinline__ void scan(float la0, float la1, int lane) {
         float x = la0 + la1;
 #pragma unroll
@@ -204,6 +205,12 @@ struct ChunkGates {
         return (t & 1) ? b : a;
     }
     __device__ __forceinline__ float last() const { return __shfl_sync(0xffffffffu, g1, 31); }
+};
+
+// alpha of a lane's two tokens of one chunk as loaded (bf16 bits): loaded a chunk or more ahead and
+// first used by ChunkGates::log2_of, so that the load's latency is not waited for where it is issued.
+struct RawAlpha {
+    __nv_bfloat16 a0, a1;
 };
 
 template <bool GATED>
@@ -275,24 +282,25 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     };
     auto alpha_idx = [&](int t) { return ((size_t)b * T + t) * H + h; };
+    auto load_raw = [&](int cc) -> RawAlpha {   // gated: alpha of tokens 2 lane, 2 lane + 1 of chunk cc
+        const int t = cc * C + 2 * lane;
+        const __nv_bfloat16 one = __float2bfloat16(1.f);
+        return RawAlpha{t < T ? alpha[alpha_idx(t)] : one, t + 1 < T ? alpha[alpha_idx(t + 1)] : one};
+    };
+    auto gates_from = [&](const RawAlpha& ra, int cc, ChunkGates& g) {   // gated: the gates of chunk cc
+        const int t = cc * C + 2 * lane;
+        g.scan(ChunkGates::log2_of(ra.a0, t < T), ChunkGates::log2_of(ra.a1, t + 1 < T), lane);
+    };
 
     if (warp < 4) {
         // ================================================================ state group
         const int v = tid;                                   // TMEM lane: value row of S / key feature
         const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
         // gated: gates of the current chunk (cur) and of the next one (nxt), every warp all 64 tokens;
-        // log2 alpha of the chunk after nxt is loaded an iteration ahead (pa0, pa1)
+        // alpha of the chunk after nxt is loaded an iteration ahead (pa)
         ChunkGates cur{0.f, 0.f}, nxt{0.f, 0.f};
-        float pa0 = 0.f, pa1 = 0.f;
-        auto load_la = [&](int cc) {
-            const int t = cc * C + 2 * lane;
-            pa0 = ChunkGates::log2_alpha(alpha, alpha_idx(t), t < T);
-            pa1 = ChunkGates::log2_alpha(alpha, alpha_idx(t + 1), t + 1 < T);
-        };
-        auto gates_of = [&](int cc, ChunkGates& g) {
-            load_la(cc);
-            g.scan(pa0, pa1, lane);
-        };
+        RawAlpha pa{};
+        auto gates_of = [&](int cc, ChunkGates& g) { gates_from(load_raw(cc), cc, g); };
         if (GATED && nchunks > 0) gates_of(0, nxt);
         {   // initial state: fp32 S (gated: x gamma_C of chunk 0), its bf16 copy (A operand of GA), zeroed O^T
             const float* srow = S0 ? S0 + ((size_t)unit * DV + v) * DK : nullptr;
@@ -343,7 +351,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             cur = nxt;
             if (GATED) {
                 if (nchunks > 1) gates_of(1, nxt);
-                if (nchunks > 2) load_la(2);
+                if (nchunks > 2) pa = load_raw(2);
             }
             ok = w_epilogue(0);
         }
@@ -403,8 +411,8 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (tid == 0 && c + 1 < nchunks) tc::mbar_arrive1(bars + L::ESB);
             if (GATED) {
                 cur = nxt;
-                if (c + 2 < nchunks) nxt.scan(pa0, pa1, lane);
-                if (c + 3 < nchunks) load_la(c + 3);
+                if (c + 2 < nchunks) gates_from(pa, c + 2, nxt);
+                if (c + 3 < nchunks) pa = load_raw(c + 3);
             }
         }
         tc::tc_fence_before();
@@ -421,14 +429,9 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             return (gtid < C && t < T) ? __bfloat162float(beta[((size_t)b * T + t) * H + h]) : 0.f;
         };
         float bnext = nchunks > 0 ? load_beta(0) : 0.f;
-        // gated: log2 alpha of tokens 2 lane, 2 lane + 1 of the next chunk (every prep warp)
-        auto load_la = [&](int c, float& a0, float& a1) {
-            const int t = c * C + 2 * lane;
-            a0 = ChunkGates::log2_alpha(alpha, alpha_idx(t), t < T);
-            a1 = ChunkGates::log2_alpha(alpha, alpha_idx(t + 1), t + 1 < T);
-        };
-        float la0 = 0.f, la1 = 0.f;
-        if (GATED && nchunks > 0) load_la(0, la0, la1);
+        // gated: alpha of the next chunk, loaded a chunk ahead (every prep warp)
+        RawAlpha la{};
+        if (GATED && nchunks > 0) la = load_raw(0);
         for (int i = gtid; i < 2 * 8192 / 16; i += 128)   // the T tiles' blocks above the diagonal stay zero
             reinterpret_cast<uint4*>(sm + L::TB)[i] = make_uint4(0u, 0u, 0u, 0u);
         for (int c = 0; c < nchunks; ++c) {
@@ -437,8 +440,8 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (c + 1 < nchunks) bnext = load_beta(c + 1);
             ChunkGates g{0.f, 0.f};
             if (GATED) {
-                g.scan(la0, la1, lane);
-                if (c + 1 < nchunks) load_la(c + 1, la0, la1);
+                gates_from(la, c, g);
+                if (c + 1 < nchunks) la = load_raw(c + 1);
             }
             bool fail = !wait(L::D1 + c % 3, (c / 3) & 1);
             if (!fail && c >= 2) fail = !wait(L::BO + s2, ((c - 2) >> 1) & 1);   // GBO(c-2) has read P tile s2
@@ -538,12 +541,14 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // gated: chunk c's K and Q rows x gamma_t (GW then forms (diag(gamma) K)^T (T diag(beta))^T, GA
         // diag(gamma) Q S^T) and Kw rows x gamma_C / gamma_t (GBS then adds U^T diag(gamma_C / gamma) Kw), once
         // G1(c), their other reader, has completed; the issuer waits for it before GW(c)
+        RawAlpha ea{};   // gated: alpha of the next chunk to scale, loaded a call ahead
+        if (GATED && nchunks > 0) ea = load_raw(0);
         auto gate_scale = [&](int c) -> bool {
+            const RawAlpha ra = ea;
+            if (c + 1 < nchunks) ea = load_raw(c + 1);
             if (tc::named_sync_or(BAR_EPI, 128, !wait(L::D1 + c % 3, (c / 3) & 1))) return false;
             ChunkGates g;
-            const int t0 = c * C + 2 * lane;
-            g.scan(ChunkGates::log2_alpha(alpha, alpha_idx(t0), t0 < T),
-                   ChunkGates::log2_alpha(alpha, alpha_idx(t0 + 1), t0 + 1 < T), lane);
+            gates_from(ra, c, g);
             uint8_t* st = sm + (c % 3) * L::STAGE + L::QK;
             {   // thread (et % 8) takes 16-byte chunk et % 8 of rows t = et / 8 + 16 i of each tile
                 const int ch = et & 7;
