@@ -424,11 +424,12 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         float* betas = reinterpret_cast<float*>(sm + L::BETA);
         float* glog = reinterpret_cast<float*>(sm + L::GLOG);
         float* AF = reinterpret_cast<float*>(sm + L::AF);
-        auto load_beta = [&](int c) -> float {
+        // beta of the next chunk, loaded a chunk ahead as bf16 and converted where it is used
+        auto load_beta = [&](int c) -> __nv_bfloat16 {
             const int t = c * C + gtid;
-            return (gtid < C && t < T) ? __bfloat162float(beta[((size_t)b * T + t) * H + h]) : 0.f;
+            return (gtid < C && t < T) ? beta[((size_t)b * T + t) * H + h] : __float2bfloat16(0.f);
         };
-        float bnext = nchunks > 0 ? load_beta(0) : 0.f;
+        __nv_bfloat16 bnext = nchunks > 0 ? load_beta(0) : __float2bfloat16(0.f);
         // gated: alpha of the next chunk, loaded a chunk ahead (every prep warp)
         RawAlpha la{};
         if (GATED && nchunks > 0) la = load_raw(0);
@@ -436,7 +437,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             reinterpret_cast<uint4*>(sm + L::TB)[i] = make_uint4(0u, 0u, 0u, 0u);
         for (int c = 0; c < nchunks; ++c) {
             const int s2 = c & 1;
-            const float bt = bnext;
+            const __nv_bfloat16 braw = bnext;
             if (c + 1 < nchunks) bnext = load_beta(c + 1);
             ChunkGates g{0.f, 0.f};
             if (GATED) {
@@ -447,6 +448,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!fail && c >= 2) fail = !wait(L::BO + s2, ((c - 2) >> 1) & 1);   // GBO(c-2) has read P tile s2
             if (tc::named_sync_or(BAR_PREP, 128, fail)) break;
             tc::tc_fence_after();
+            const float bt = __bfloat162float(braw);
             if (gtid < C) betas[gtid] = bt;
             if (GATED && q4 == 0) {
                 glog[2 * lane] = g.g0;

@@ -315,13 +315,15 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         const int row = tp & 127;              // token of the block and TMEM lane this thread serves
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         float* np = reinterpret_cast<float*>(sm + L::NP);
-        auto load_pv = [&](int blk) -> float {   // group 0: beta, group 1: r (1 past T or without APF)
+        // group 0: beta, group 1: r (1 past T or without APF); loaded a block ahead as bf16 and
+        // converted where it is used, so that the load is not waited for where it is issued
+        auto load_pv = [&](int blk) -> __nv_bfloat16 {
             const int tok = blk * BLK + row;
             const size_t gi = ((size_t)b * T + tok) * H + h;
-            if (g == 0) return tok < T ? __bfloat162float(beta[gi]) : 0.f;
-            return (tok < T && r) ? __bfloat162float(r[gi]) : 1.f;
+            if (g == 0) return tok < T ? beta[gi] : __float2bfloat16(0.f);
+            return (tok < T && r) ? r[gi] : __float2bfloat16(1.f);
         };
-        float pv = nblk > 0 ? load_pv(0) : 0.f;
+        __nv_bfloat16 pv = nblk > 0 ? load_pv(0) : __float2bfloat16(0.f);
         for (int blk = 0; blk < nblk; ++blk) {
             uint8_t* KS = kblock(blk);
             float* vb = vecs(blk);
@@ -329,7 +331,7 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             if (!fail && blk >= 2) fail = !wait(L::MFREE + (blk & 1), ((blk - 2) >> 1) & 1);
             if (tc::named_sync_or(BAR_PREP, 256, fail)) break;
             // beta (group 0) or r (group 1) of token `row`, loaded one block ahead
-            const float bt = pv;
+            const float bt = __bfloat162float(pv);
             if (g == 0) vb[L::V_BETA + row] = bt;
             else vb[L::V_R + row] = bt;
             if (blk + 1 < nblk) pv = load_pv(blk + 1);
