@@ -17,8 +17,9 @@
  * normalisation or 1/sqrt(dk) scale is applied to q or k inside the op.
  *
  * Conventions for every entry point
- *   - All tensor pointers are DEVICE pointers owned by the caller. The library
- *     never allocates device memory and never frees anything.
+ *   - All tensor pointers are DEVICE pointers owned by the caller (except the
+ *     host buffers of osdn_fwd_host). The library never allocates device memory
+ *     and never frees anything.
  *   - Layouts are row-major (last dimension contiguous), dense unless the
  *     strides of osdn_params say otherwise (forward only):
  *       q, k   [B, T, H, dk]     v, out [B, T, H, dv]
@@ -360,6 +361,38 @@ int osdn_fwd_noalloc(const osdn_params *p,
                      const float *d0, const float *S0,
                      void *out, float *final_S, float *final_d,
                      void *cuda_stream);
+
+/* osdn_fwd on HOST buffers, with the transfers pipelined against the compute.
+ * q, k, v, beta, r (nullable), d0, S0 (nullable) and out, final_S, final_d
+ * (nullable) are dense host tensors in the layouts of osdn_fwd; page-locked
+ * memory (cudaHostAlloc, cudaHostRegister) lets the copies run asynchronously and
+ * overlap, pageable memory works but serialises them. device_buffer is
+ * caller-owned device memory of at least osdn_fwd_host_buffer_size() bytes
+ * (16-byte aligned): it holds the whole problem's device copies and one
+ * workspace. The B sequences are cut into `groups` groups of consecutive
+ * sequences (0: min(B, 8); at most 16). A library-owned non-blocking stream
+ * copies each group's inputs in; cuda_stream runs osdn_fwd on the group once
+ * they are in; a second library-owned stream copies its results back. So the
+ * upload of one group, the compute of another and the download of a third
+ * overlap (the link is full duplex). The call forks from cuda_stream and joins
+ * back to it by events; the host results are complete once cuda_stream has
+ * reached the point of the call. Sequences are independent, so the results
+ * equal osdn_fwd's on the whole batch up to the rounding of the segment plan
+ * a smaller batch may choose (osdn_fwd_segments). Dense tensors only (the
+ * strides of osdn_params must be zero or dense).
+ * Errors: OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED, OSDN_ERR_CUDA. */
+int osdn_fwd_host(const osdn_params *p,
+                  const void *q, const void *k, const void *v,
+                  const void *beta, const void *r,
+                  const float *d0, const float *S0,
+                  void *out, float *final_S, float *final_d,
+                  void *device_buffer, size_t device_bytes,
+                  int groups, void *cuda_stream);
+
+/* Bytes of device_buffer that osdn_fwd_host needs for these parameters and
+ * `groups` (as in osdn_fwd_host), written to *bytes.
+ * Errors: OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED. */
+int osdn_fwd_host_buffer_size(const osdn_params *p, int groups, size_t *bytes);
 
 /* Waits for the work queued on cuda_stream, then reports whether any bounded
  * device-side wait of the library's kernels gave up since the last call

@@ -19,12 +19,13 @@ from ._binding import (OSDN_BF16, OSDN_ERR_CUDA, OSDN_ERR_INVALID_ARG, OSDN_ERR_
                        osdn_fwd_chunk, osdn_fwd_scan, osdn_fwd_scan_diag,
                        osdn_fwd_workspace_size, osdn_fwd_segments, osdn_fwd_launches, osdn_params, osdn_set_wait_limit_ns, osdn_step, osdn_step_ex,
                        osdn_fwd_gated, osdn_fwd_chunk_gated, osdn_step_gated,
-                       osdn_bwd, osdn_bwd_gated, osdn_bwd_workspace_size, osdn_sync_status)
+                       osdn_bwd, osdn_bwd_gated, osdn_bwd_workspace_size, osdn_sync_status,
+                       osdn_fwd_host, osdn_fwd_host_buffer_size)
 
 __all__ = ["forward", "backward", "step", "osdn_bwd", "osdn_bwd_gated", "osdn_bwd_workspace_size", "residual_ratio", "osdn_fwd_scan_diag", "osdn_fwd", "osdn_fwd_scan", "osdn_fwd_chunk", "osdn_step", "osdn_fwd_workspace_size", "osdn_fwd_segments", "osdn_fwd_launches", "osdn_sync_status",
            "osdn_set_wait_limit_ns", "osdn_step_ex",
-           "osdn_fwd_gated", "osdn_fwd_chunk_gated", "osdn_step_gated",
-           "osdn_params", "make_params", "get_last_error", "OsdnError", "build", "LIB_PATH",
+           "osdn_fwd_gated", "osdn_fwd_chunk_gated", "osdn_step_gated", "osdn_fwd_host", "osdn_fwd_host_buffer_size",
+           "forward_host", "osdn_params", "make_params", "get_last_error", "OsdnError", "build", "LIB_PATH",
            "OSDN_OK", "OSDN_ERR_INVALID_ARG", "OSDN_ERR_UNSUPPORTED", "OSDN_ERR_CUDA", "OSDN_ERR_TIMEOUT",
            "OSDN_BF16", "OSDN_FP32"]
 
@@ -49,6 +50,25 @@ def forward(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, chunk=64, workspa
         osdn_fwd(p, q, k, v, beta, r, d0, S0, out, final_S, final_d, workspace, stream)
     else:
         osdn_fwd_gated(p, q, k, v, beta, r, alpha, d0, S0, out, final_S, final_d, workspace, stream)
+    return out, final_S, final_d
+
+
+def forward_host(q, k, v, beta, r=None, d0=None, S0=None, eta=1e-2, chunk=64, groups=0, device_buffer=None,
+                 stream=None, apf_anchor=False):
+    """forward() on HOST tensors (page-locked for overlapped copies): the library copies each group of
+    sequences in, runs the forward on it and copies its results back, with the copies of one group
+    overlapping the compute of its neighbours (osdn_fwd_host). groups = 0: the library's default.
+    Returns host tensors (out, final_S, final_d); the call is asynchronous on `stream`."""
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    p = make_params(B, T, H, dk, dv, k.dtype, eta, chunk, apf_anchor)
+    pin = q.is_pinned()
+    out = torch.empty((B, T, H, dv), dtype=k.dtype, pin_memory=pin)
+    final_S = torch.empty((B, H, dv, dk), dtype=torch.float32, pin_memory=pin)
+    final_d = torch.empty((B, H, dk), dtype=torch.float32, pin_memory=pin)
+    if device_buffer is None:
+        device_buffer = torch.empty(osdn_fwd_host_buffer_size(p, groups), dtype=torch.uint8, device="cuda")
+    osdn_fwd_host(p, q, k, v, beta, r, d0, S0, out, final_S, final_d, device_buffer, groups, stream)
     return out, final_S, final_d
 
 

@@ -105,6 +105,10 @@ def lib():
         L.osdn_fwd_gated.restype = ctypes.c_int
         L.osdn_fwd_chunk_gated.argtypes = [P] + [vp] * 8 + [vp, sz, vp]
         L.osdn_fwd_chunk_gated.restype = ctypes.c_int
+        L.osdn_fwd_host_buffer_size.argtypes = [P, ctypes.c_int, ctypes.POINTER(sz)]
+        L.osdn_fwd_host_buffer_size.restype = ctypes.c_int
+        L.osdn_fwd_host.argtypes = [P] + [vp] * 10 + [vp, sz, ctypes.c_int, vp]
+        L.osdn_fwd_host.restype = ctypes.c_int
         L.osdn_bwd_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
         L.osdn_bwd_workspace_size.restype = ctypes.c_int
         L.osdn_bwd.argtypes = [P] + [vp] * 17 + [vp, sz, vp]
@@ -164,6 +168,17 @@ def _ptr_tok(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _host_ptr(t):
+    """Pointer of a dense host tensor (page-locked memory lets its copies overlap; pageable works too)."""
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise OsdnError(OSDN_ERR_INVALID_ARG, "osdn_fwd_host takes host tensors (the device data lives in device_buffer)")
+    if not t.is_contiguous():
+        raise OsdnError(OSDN_ERR_INVALID_ARG, "tensor is not contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
 def _set_strides(params, q=None, k=None, v=None, out=None):
     """Copy the (b, t, h) element strides of q, k, v, out into params (zeros: dense)."""
     for name, t in (("stride_q", q), ("stride_k", k), ("stride_v", v), ("stride_o", out)):
@@ -209,6 +224,22 @@ def osdn_fwd(params, q, k, v, beta, r, d0, S0, out, final_S, final_d, workspace,
 
 def _ws_bytes(workspace):
     return 0 if workspace is None else workspace.numel() * workspace.element_size()
+
+
+def osdn_fwd_host_buffer_size(params: osdn_params, groups: int = 0) -> int:
+    """Bytes of the device buffer osdn_fwd_host needs for these parameters and group count."""
+    n = ctypes.c_size_t(0)
+    _check(lib().osdn_fwd_host_buffer_size(ctypes.byref(params), ctypes.c_int(int(groups)), ctypes.byref(n)))
+    return n.value
+
+
+def osdn_fwd_host(params, q, k, v, beta, r, d0, S0, out, final_S, final_d, device_buffer, groups=0, stream=None):
+    """Raw C-ABI call: inputs and outputs are dense HOST tensors, device_buffer a CUDA tensor of at
+    least osdn_fwd_host_buffer_size bytes."""
+    _check(lib().osdn_fwd_host(ctypes.byref(params), _host_ptr(q), _host_ptr(k), _host_ptr(v), _host_ptr(beta),
+                               _host_ptr(r), _host_ptr(d0), _host_ptr(S0), _host_ptr(out), _host_ptr(final_S),
+                               _host_ptr(final_d), _ptr(device_buffer), ctypes.c_size_t(_ws_bytes(device_buffer)),
+                               ctypes.c_int(int(groups)), _stream(stream)))
 
 
 def osdn_fwd_scan(params, k, beta, r, d0, final_d, workspace, stream=None):

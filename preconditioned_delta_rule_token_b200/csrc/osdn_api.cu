@@ -1209,3 +1209,183 @@ int osdn_sync_status(void* cuda_stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------- host buffers
+namespace {
+
+// Two non-blocking copy streams per device (host to device, device to host) for osdn_fwd_host,
+// apart from the streams the forward itself forks to, so that copies never queue behind its
+// kernels. Created on first use and kept for the life of the process.
+int copy_streams(cudaStream_t out[2]) {
+    static std::mutex mu;
+    static cudaStream_t streams[64][2] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "current device");
+    if (dev < 0 || dev >= 64) return fail(OSDN_ERR_UNSUPPORTED, "device index %d above 63", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < 2; ++i)
+        if (!streams[dev][i] && (e = cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "copy stream");
+    out[0] = streams[dev][0];
+    out[1] = streams[dev][1];
+    return OSDN_OK;
+}
+
+constexpr int kMaxHostGroups = 16;
+
+// The device region of osdn_fwd_host: the whole problem's inputs, outputs and initial states,
+// then the forward workspace of the largest group, each 256-byte aligned.
+struct HostLayout {
+    int groups, per;   // groups of `per` consecutive sequences (the last may hold fewer)
+    size_t q, k, v, beta, r, out, S, d, d0, S0, ws, ws_bytes, total;
+};
+
+osdn_params full_params(const osdn_params* p) {   // a version-3 copy of any accepted version
+    osdn_params f{};
+    std::memcpy(&f, p, p->struct_size < sizeof(f) ? p->struct_size : sizeof(f));
+    f.struct_size = sizeof(f);
+    return f;
+}
+
+HostLayout host_layout_of(const osdn_params* p, int groups) {
+    HostLayout L{};
+    int g = groups <= 0 ? 8 : groups;
+    if (g > p->B) g = p->B;
+    if (g > kMaxHostGroups) g = kMaxHostGroups;
+    L.per = (p->B + g - 1) / g;
+    L.groups = (p->B + L.per - 1) / L.per;
+    const size_t es = elem_size(p->dtype), tok = (size_t)p->B * p->T * p->H, units = (size_t)p->B * p->H;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = round_up(off + bytes, 256);
+        return o;
+    };
+    L.q = take(tok * p->dk * es);
+    L.k = take(tok * p->dk * es);
+    L.v = take(tok * p->dv * es);
+    L.beta = take(tok * es);
+    L.r = take(tok * es);
+    L.out = take(tok * p->dv * es);
+    L.S = take(units * p->dv * p->dk * sizeof(float));
+    L.d = take(units * p->dk * sizeof(float));
+    L.S0 = take(units * p->dv * p->dk * sizeof(float));
+    L.d0 = take(units * p->dk * sizeof(float));
+    osdn_params gp = full_params(p);
+    gp.B = L.per;
+    size_t ws = layout_of(&gp).total;
+    const int last = p->B - (L.groups - 1) * L.per;   // the last group's sequences
+    if (last != L.per) {
+        gp.B = last;
+        const size_t w2 = layout_of(&gp).total;
+        if (w2 > ws) ws = w2;
+    }
+    L.ws_bytes = ws;
+    L.ws = take(ws);
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+int osdn_fwd_host_buffer_size(const osdn_params* p, int groups, size_t* bytes) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    if (!bytes) return fail(OSDN_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = host_layout_of(p, groups).total;
+    return OSDN_OK;
+}
+
+int osdn_fwd_host(const osdn_params* p, const void* q, const void* k, const void* v, const void* beta, const void* r,
+                  const float* d0, const float* S0, void* out, float* final_S, float* final_d, void* device_buffer,
+                  size_t device_bytes, int groups, void* cuda_stream) {
+    t_last_error.clear();
+    int rc = check_params(p, true);
+    if (rc) return rc;
+    if (!dense_layout(p)) return fail(OSDN_ERR_UNSUPPORTED, "osdn_fwd_host takes dense host tensors only");
+    if (p->T > 0 && (!q || !k || !v || !beta || !out))
+        return fail(OSDN_ERR_INVALID_ARG, "a required pointer (q, k, v, beta, out) is NULL");
+    if (!device_buffer) return fail(OSDN_ERR_INVALID_ARG, "device_buffer is NULL");
+    if (!aligned16(device_buffer)) return fail(OSDN_ERR_INVALID_ARG, "device_buffer must be 16-byte aligned");
+    const HostLayout L = host_layout_of(p, groups);
+    if (device_bytes < L.total)
+        return fail(OSDN_ERR_INVALID_ARG, "device_buffer too small: %zu bytes given, %zu needed", device_bytes, L.total);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    cudaStream_t cs[2];
+    if ((rc = copy_streams(cs))) return rc;
+    char* dbuf = reinterpret_cast<char*>(device_buffer);
+    const size_t es = elem_size(p->dtype);
+    const size_t seq_tok = (size_t)p->T * p->H;               // token-heads of one sequence
+    const size_t seq_S = (size_t)p->H * p->dv * p->dk, seq_d = (size_t)p->H * p->dk;
+
+    const int nev = 2 + 2 * L.groups;                          // fork, join, per group: inputs in, computed
+    cudaEvent_t ev[2 + 2 * kMaxHostGroups];
+    cudaError_t e = cudaSuccess;
+    int made = 0;
+    for (; made < nev; ++made)
+        if ((e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming)) != cudaSuccess) break;
+    if (e != cudaSuccess) {
+        for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+        return cuda_fail(e, "event");
+    }
+    auto chk = [&](cudaError_t x, const char* what) -> int { return x == cudaSuccess ? OSDN_OK : cuda_fail(x, what); };
+    // n bytes from host src + off to device region dst + off (or back), on stream s; src may be NULL
+    auto h2d = [&](size_t dst, const void* src, size_t off, size_t n, cudaStream_t s) -> int {
+        if (!src || n == 0) return OSDN_OK;
+        return chk(cudaMemcpyAsync(dbuf + dst + off, static_cast<const char*>(src) + off, n, cudaMemcpyHostToDevice, s),
+                   "host to device copy");
+    };
+    auto d2h = [&](void* dst, size_t src, size_t off, size_t n, cudaStream_t s) -> int {
+        if (!dst || n == 0) return OSDN_OK;
+        return chk(cudaMemcpyAsync(static_cast<char*>(dst) + off, dbuf + src + off, n, cudaMemcpyDeviceToHost, s),
+                   "device to host copy");
+    };
+    do {
+        if ((rc = chk(cudaEventRecord(ev[0], st), "fork"))) break;
+        if ((rc = chk(cudaStreamWaitEvent(cs[0], ev[0], 0), "fork"))) break;
+        if ((rc = chk(cudaStreamWaitEvent(cs[1], ev[0], 0), "fork"))) break;
+        for (int gi = 0; gi < L.groups && !rc; ++gi) {
+            const int b0 = gi * L.per, nb = p->B - b0 < L.per ? p->B - b0 : L.per;
+            const size_t t0 = (size_t)b0 * seq_tok, tn = (size_t)nb * seq_tok;
+            // inputs of the group's sequences (contiguous in every [B, ...] tensor) on the copy-in stream
+            if ((rc = h2d(L.q, q, t0 * p->dk * es, tn * p->dk * es, cs[0]))) break;
+            if ((rc = h2d(L.k, k, t0 * p->dk * es, tn * p->dk * es, cs[0]))) break;
+            if ((rc = h2d(L.v, v, t0 * p->dv * es, tn * p->dv * es, cs[0]))) break;
+            if ((rc = h2d(L.beta, beta, t0 * es, tn * es, cs[0]))) break;
+            if ((rc = h2d(L.r, r, t0 * es, tn * es, cs[0]))) break;
+            if ((rc = h2d(L.S0, S0, (size_t)b0 * seq_S * 4, (size_t)nb * seq_S * 4, cs[0]))) break;
+            if ((rc = h2d(L.d0, d0, (size_t)b0 * seq_d * 4, (size_t)nb * seq_d * 4, cs[0]))) break;
+            if ((rc = chk(cudaEventRecord(ev[2 + 2 * gi], cs[0]), "inputs event"))) break;
+            // the group's forward on the caller's stream, once its inputs are in
+            if ((rc = chk(cudaStreamWaitEvent(st, ev[2 + 2 * gi], 0), "inputs wait"))) break;
+            osdn_params gp = full_params(p);
+            gp.B = nb;
+            auto at = [&](size_t base, size_t off) { return static_cast<void*>(dbuf + base + off); };
+            rc = osdn_fwd(&gp, at(L.q, t0 * p->dk * es), at(L.k, t0 * p->dk * es), at(L.v, t0 * p->dv * es),
+                          at(L.beta, t0 * es), r ? at(L.r, t0 * es) : nullptr,
+                          d0 ? static_cast<const float*>(at(L.d0, (size_t)b0 * seq_d * 4)) : nullptr,
+                          S0 ? static_cast<const float*>(at(L.S0, (size_t)b0 * seq_S * 4)) : nullptr,
+                          at(L.out, t0 * p->dv * es), static_cast<float*>(at(L.S, (size_t)b0 * seq_S * 4)),
+                          static_cast<float*>(at(L.d, (size_t)b0 * seq_d * 4)), dbuf + L.ws, L.ws_bytes, st);
+            if (rc) break;
+            if ((rc = chk(cudaEventRecord(ev[3 + 2 * gi], st), "compute event"))) break;
+            // its results back on the copy-out stream
+            if ((rc = chk(cudaStreamWaitEvent(cs[1], ev[3 + 2 * gi], 0), "compute wait"))) break;
+            if ((rc = d2h(out, L.out, t0 * p->dv * es, tn * p->dv * es, cs[1]))) break;
+            if ((rc = d2h(final_S, L.S, (size_t)b0 * seq_S * 4, (size_t)nb * seq_S * 4, cs[1]))) break;
+            if ((rc = d2h(final_d, L.d, (size_t)b0 * seq_d * 4, (size_t)nb * seq_d * 4, cs[1]))) break;
+        }
+        if (rc) break;
+        // join: the caller's stream waits for the last copies back (it already waited for every copy in)
+        if ((rc = chk(cudaEventRecord(ev[1], cs[1]), "join"))) break;
+        rc = chk(cudaStreamWaitEvent(st, ev[1], 0), "join");
+    } while (false);
+    for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
+    return rc;
+}
+
+}  // extern "C"

@@ -176,3 +176,30 @@ def test_new_entry_points_check_their_arguments_on_the_host(osdn_lib):
     assert osdn_lib.osdn_fwd_launches(anchored) == 6              # split, not overlapped
     layer = osdn_lib.make_params(8, 4096, 16, 128, 128, __import__("torch").bfloat16, 1e-2)
     assert osdn_lib.osdn_fwd_segments(layer) == 1 and osdn_lib.osdn_fwd_launches(layer) == 2
+
+
+def test_fwd_host_checks_on_the_host():
+    """osdn_fwd_host and its buffer size: argument checks that finish before any device call."""
+    import ctypes
+    import torch
+    import preconditioned_delta_rule_token_b200 as pk
+    from preconditioned_delta_rule_token_b200 import _binding as b
+    L = b.lib()
+    p = pk.make_params(8, 4096, 16, 128, 128, torch.bfloat16, 1e-2)
+    sizes = {g: pk.osdn_fwd_host_buffer_size(p, g) for g in (0, 1, 2, 4, 8, 64)}
+    tok = 8 * 4096 * 16
+    inputs = tok * 128 * 2 * 4 + tok * 2 * 2          # q, k, v, out; beta, r
+    for g, n in sizes.items():
+        assert n >= inputs and n % 256 == 0, (g, n)
+    assert sizes[0] == sizes[8]                         # the default is min(B, 8) groups
+    assert sizes[64] == sizes[8]                        # at most one group per sequence
+    dummy = ctypes.c_void_p(1 << 20)
+    args = [ctypes.byref(p)] + [dummy] * 5 + [None, None] + [dummy, None, None]
+    rc = L.osdn_fwd_host(*args, None, ctypes.c_size_t(sizes[0]), 0, None)
+    assert rc == pk.OSDN_ERR_INVALID_ARG and "device_buffer" in pk.get_last_error()
+    rc = L.osdn_fwd_host(*args, ctypes.c_void_p(1 << 21), ctypes.c_size_t(sizes[0] - 256), 0, None)
+    assert rc == pk.OSDN_ERR_INVALID_ARG and "too small" in pk.get_last_error()
+    ps = pk.make_params(8, 4096, 16, 128, 128, torch.bfloat16, 1e-2)
+    ps.stride_q[0], ps.stride_q[1], ps.stride_q[2] = 4096 * 16 * 384, 16 * 384, 384
+    rc = L.osdn_fwd_host(ctypes.byref(ps), *args[1:], ctypes.c_void_p(1 << 21), ctypes.c_size_t(sizes[0]), 0, None)
+    assert rc == pk.OSDN_ERR_UNSUPPORTED
