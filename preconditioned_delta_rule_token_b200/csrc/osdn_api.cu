@@ -579,20 +579,21 @@ int launch_fwd_pipelined(const osdn_params* p, const __nv_bfloat16* q, const __n
 }
 
 // Phase 1 in chunk form on the tensor cores: bf16, dk = 128.
+// d_traj non-NULL: the instance that also writes d_t of every token (fp32 [B, T, H, 128]).
 int launch_scan_tc(const osdn_params* p, const __nv_bfloat16* k, const __nv_bfloat16* beta,
                    const __nv_bfloat16* r, const float* d0, float* final_d, __nv_bfloat16* kw, float* rho,
-                   float* q_geo, cudaStream_t st) {
+                   float* q_geo, cudaStream_t st, float* d_traj = nullptr) {
     CUtensorMap mk, mkw;
     int rc = make_token_map(&mk, k, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128, strides_of(p).k);
     if (rc) return rc;
     rc = make_token_map(&mkw, kw, p->B, p->T, p->H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128, dense_tok3(p, 128));
     if (rc) return rc;
-    auto kern = osdn::scan_ws_kernel<0>;
+    auto kern = d_traj ? osdn::scan_ws_kernel<1> : osdn::scan_ws_kernel<0>;
     const size_t smem = osdn::ScanLayout::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan kernel attribute");
-    kern<<<p->B * p->H, 384, smem, st>>>(mk, mkw, beta, r, d0, final_d, rho, q_geo, p->B, p->T, p->H, p->eta, anchor_of(p),
-                                         g_wait_limit_ns.load());
+    kern<<<p->B * p->H, 384, smem, st>>>(mk, mkw, beta, r, d0, final_d, rho, q_geo, d_traj, p->B, p->T, p->H, p->eta,
+                                         anchor_of(p), g_wait_limit_ns.load());
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");
     return OSDN_OK;
 }
@@ -760,11 +761,23 @@ int launch_bwd_t(const osdn_params* p, const Tin* q, const Tin* k, const Tin* v,
         return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     };
     const size_t s_dt = B::DtrajSmem<DK, Tin>::kBytes, s_dc = B::DchainSmem<DK, Tin>::kBytes;
-    if ((e = attr((const void*)B::bwd_dtraj_kernel<DK, Tin>, s_dt)) != cudaSuccess)
-        return cuda_fail(e, "backward d trajectory attribute");
-    B::bwd_dtraj_kernel<DK, Tin><<<(unsigned)units, B::SERIAL_THREADS, s_dt, st>>>(
-        k, beta, r, d0, ws + L.d_all / sizeof(float), p->B, p->T, p->H, p->eta, an);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward d trajectory launch");
+    bool traj_done = false;
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value && DK == 128) {
+        // d_t of every token from the forward's chunk-form scan on the tensor cores; its scaled keys
+        // (bf16) land in the Kw region, which bwd_prep writes next
+        const int rc = launch_scan_tc(p, k, beta, r, d0, nullptr,
+                                      reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(ws) + L.kw), nullptr,
+                                      nullptr, st, ws + L.d_all / sizeof(float));
+        if (rc) return rc;
+        traj_done = true;
+    }
+    if (!traj_done) {   // token-serial trajectory (fp32 inputs, dk = 64)
+        if ((e = attr((const void*)B::bwd_dtraj_kernel<DK, Tin>, s_dt)) != cudaSuccess)
+            return cuda_fail(e, "backward d trajectory attribute");
+        B::bwd_dtraj_kernel<DK, Tin><<<(unsigned)units, B::SERIAL_THREADS, s_dt, st>>>(
+            k, beta, r, d0, ws + L.d_all / sizeof(float), p->B, p->T, p->H, p->eta, an);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "backward d trajectory launch");
+    }
 
     const size_t s_prep = B::PrepSmem<DK, DV>::kBytes;
     if ((e = attr((const void*)B::bwd_prep_kernel<DK, DV, Tin>, s_prep)) != cudaSuccess)

@@ -77,12 +77,14 @@ struct ScanLayout {
     static constexpr uint32_t kTx = 2 * 16384;
 };
 
-template <int kUnused = 0>
+// TRAJ = 1 also writes d_t (fp32, before token t's own update) of every token to
+// d_traj [B, T, H, DK], the trajectory the backward differentiates through.
+template <int TRAJ = 0>
 __global__ void __launch_bounds__(384, 1)
 scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kw,
                const __nv_bfloat16* __restrict__ beta, const __nv_bfloat16* __restrict__ r,
                const float* __restrict__ d0, float* __restrict__ d_final, float* __restrict__ rho,
-               float* __restrict__ q_geo, int B, int T, int H, float eta, int anchor,
+               float* __restrict__ q_geo, float* __restrict__ d_traj, int B, int T, int H, float eta, int anchor,
                unsigned long long wait_limit_ns)
 {
     constexpr int DK = 128, BLK = 128, SUB = 64;
@@ -273,6 +275,10 @@ scan_ws_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const float kv = kk[j];
+                            if constexpr (TRAJ != 0) {
+                                const int t = blk * BLK + tb + j;
+                                if (t < T) d_traj[(((size_t)b * T + t) * H + h) * DK + i] = d + da;
+                            }
                             kk[j] = (d + da) * kv;                           // scaled key, with d before token j
                             d = fmaf(rr[j], d, xx[j] * (kv * kv));
                         }
