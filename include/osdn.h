@@ -289,6 +289,9 @@ int osdn_step_gated(const osdn_params *p,
  * i.e. about (5 dk + 3 dv + 130) * 4 bytes per token and head plus
  * 8 dv dk bytes per chunk and head (3.5 GB at B8 T4096 H16 dk = dv = 128).
  * T = 0 copies dS_final to dS0 and dd_final to dd0 (zeros when NULL).
+ * Some per-row sums of a chunk are reduced with shared-memory atomic adds, so
+ * two calls on the same inputs can differ in the last bits (the forward
+ * entry points are bitwise reproducible).
  * Errors: OSDN_ERR_INVALID_ARG, OSDN_ERR_UNSUPPORTED, OSDN_ERR_CUDA. */
 int osdn_bwd_workspace_size(const osdn_params *p, size_t *bytes);
 
