@@ -52,3 +52,23 @@ def test_gpu_fwd_host_equals_the_device_forward_per_group(groups, pinned):
 def test_gpu_fwd_host_fp32_without_apf():
     w = W.Workload("host buffers fp32", 3, 2, 200, 64, 64, 64, W.FP32, False, "gaussian", eta=1e-2, seed=81)
     _check(w, 2, True, FP32_TOL)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("with_init", [True, False])
+def test_gpu_fwd_host_empty_sequences(with_init):
+    """T = 0: no tokens; the final state is the initial one (zeros and ones when none is given)."""
+    import preconditioned_delta_rule_token_b200 as pk
+    B, H, dk, dv = 3, 2, 128, 128
+    q = torch.empty((B, 0, H, dk), dtype=torch.bfloat16).pin_memory()
+    v = torch.empty((B, 0, H, dv), dtype=torch.bfloat16).pin_memory()
+    beta = torch.empty((B, 0, H), dtype=torch.bfloat16).pin_memory()
+    g = torch.Generator().manual_seed(82)
+    d0 = (0.5 + torch.rand((B, H, dk), generator=g)).pin_memory() if with_init else None
+    S0 = torch.randn((B, H, dv, dk), generator=g).pin_memory() if with_init else None
+    s = torch.cuda.Stream()
+    out, S, d = pk.forward_host(q, q, v, beta, None, d0, S0, groups=2, stream=s)
+    s.synchronize()
+    assert out.shape == (B, 0, H, dv) and pk.osdn_sync_status() == 0
+    assert torch.equal(S, S0 if with_init else torch.zeros_like(S))
+    assert torch.equal(d, d0 if with_init else torch.ones_like(d))
